@@ -1,0 +1,56 @@
+"""Helpers shared by the tests: run a PagedBatch step through the CPU oracle, compare results."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from pagedattention_block_table_b200.inputs import PagedBatch, bf16_bits
+
+ATOL_MAX = 1e-2      # attention max-abs error vs the oracle (bf16 inputs, bf16 output)
+ATOL_MEAN = 1e-3     # attention mean-abs error vs the oracle
+FP8_MAX = 5e-2       # fp8 cache, vs the oracle on the original bf16 K/V
+
+
+def oracle_step(batch: PagedBatch, O, keep_pre_step=False):
+    """Fill the history, then run the step (forks, append, decode, prefill) in the oracle."""
+    nb, hkv, d = batch.num_blocks, batch.num_kv_heads, batch.head_dim
+    dt = np.uint8 if batch.kv_dtype else np.uint16
+    kc = np.zeros((nb, hkv, 16, d), dt)
+    vc = np.zeros((nb, hkv, 16, d), dt)
+    tk = bf16_bits(batch.tok_k)
+    tv = bf16_bits(batch.tok_v)
+    ks = None if batch.k_scale is None else batch.k_scale.cpu().numpy()
+    vs = None if batch.v_scale is None else batch.v_scale.cpu().numpy()
+    O.kv_append(kc, vc, tk, tv, batch.setup_slots, batch.kv_dtype, ks, vs)
+    res = {}
+    if keep_pre_step:
+        res["k_pre"], res["v_pre"] = kc.copy(), vc.copy()
+    O.copy_blocks(kc, vc, batch.cow_pairs)
+    if keep_pre_step:
+        res["k_forked"], res["v_forked"] = kc.copy(), vc.copy()
+    rows = batch.step_rows()
+    O.kv_append(kc, vc, tk[rows], tv[rows], batch.step_slots, batch.kv_dtype, ks, vs)
+    res["k_cache"], res["v_cache"] = kc, vc
+    ctx = batch.context_lens
+    nd = batch.num_decode
+    if nd:
+        res["decode"] = O.paged_decode(bf16_bits(batch.q_decode), kc, vc, batch.decode_tables, ctx[:nd],
+                                       batch.scale, batch.kv_dtype, ks, vs)
+    if batch.num_seqs > nd:
+        res["prefill"] = O.paged_prefill(bf16_bits(batch.q_prefill), batch.cu_q_lens, kc, vc, batch.prefill_tables,
+                                         ctx[nd:], batch.scale, batch.kv_dtype, ks, vs)
+    return res
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, max_tol=ATOL_MAX, mean_tol=ATOL_MEAN, what=""):
+    err = np.abs(got - ref)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    mx, mn = float(err.max()) if err.size else 0.0, float(err.mean()) if err.size else 0.0
+    assert mx <= max_tol, f"{what}: max abs err {mx:.3e} > {max_tol:.1e}"
+    if mean_tol is not None:
+        assert mn <= mean_tol, f"{what}: mean abs err {mn:.3e} > {mean_tol:.1e}"
+    return mx, mn
