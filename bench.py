@@ -1,0 +1,394 @@
+"""Benchmark of one paged-attention serving step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the hot path over one batch: copy-on-write forks (when the workload
+has shared prefixes), kv_append of every new token, paged decode attention (split-K + LSE
+reduce) and paged prefill (when the workload has prefill chunks).  The default workload is the
+Llama-3-8B-shaped decode batch (64 sequences, 32 query / 8 KV heads, head_dim 128, 16-token
+blocks, contexts uniform in [513, 4097] after the append, blocks shuffled over a pool 1.25x the
+need).  Inputs are seeded synthetic data; every input is resident in HBM before timing and
+the KV pool (about 1.2 GB) is larger than L2, so every step streams the cache from HBM.
+
+metric: KV-read HBM GB/s = algorithmic bytes of the decode attention (every cached K and V
+element once, plus q, out, tables and lengths) / step time, summed over ranks.
+One JSON line on rank 0.  With --impl reference the CPU oracle is timed instead on a bounded
+sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged-attn decode: KV-read HBM GB/s (% of peak), sequence-steps/s"
+DEFAULT_WORKLOAD = "llama3_8b_decode"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_bytes(batch) -> int:
+    """Algorithmic bytes of one decode-attention call: each cached K/V element of every decoding
+    sequence once, the queries, the outputs, the block-table entries used and the lengths."""
+    nd = batch.num_decode
+    ctx = batch.context_lens[:nd].astype(np.int64)
+    e = 1 if batch.kv_dtype else 2
+    kv = int(ctx.sum()) * 2 * batch.num_kv_heads * batch.head_dim * e
+    qo = 2 * nd * batch.num_q_heads * batch.head_dim * 2
+    tables = int(((ctx + 15) // 16).sum()) * 4 + 4 * nd
+    return kv + qo + tables
+
+
+def kv_bytes(batch) -> int:
+    nd = batch.num_decode
+    e = 1 if batch.kv_dtype else 2
+    return int(batch.context_lens[:nd].astype(np.int64).sum()) * 2 * batch.num_kv_heads * batch.head_dim * e
+
+
+class ClockSampler:
+    """Polls SM clock, max clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML unavailable: report no clocks rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+def traffic_record(kernel_tag: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f).get(kernel_tag)
+        if not d:
+            return None
+        from pagedattention_block_table_b200.build import source_digest
+        if d.get("source_digest") != source_digest():
+            return None
+        return d
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    from pagedattention_block_table_b200 import binding as B
+    from pagedattention_block_table_b200.inputs import make_batch
+    from pagedattention_block_table_b200.runner import DeviceStep
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B.lib()
+    batch = make_batch(args.workload, device=dev)
+    st = DeviceStep(batch, device=dev, split_tokens=args.split or None)
+    st.fill_history()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    launches = (1 if batch.cow_pairs.shape[0] else 0) + 1 + (1 if batch.num_decode else 0) \
+        + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0)
+
+    for _ in range(max(3, args.warmup)):
+        st.step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+
+    K = args.steps
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    with ClockSampler(local_rank) as clk:
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for i in range(K):
+            st.fork()
+            st.append()
+            d0[i].record(stream)
+            st.decode()
+            d1[i].record(stream)
+            st.prefill()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = ev0.elapsed_time(ev1) / K
+    dec_ms = sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K
+    if B.pa_get_device_error() != B.PA_OK:
+        raise RuntimeError("device error flagged during the timed region")
+
+    # end to end: inputs from pinned host memory, result back to the host, every step
+    host = {
+        "q": st.q_dec.cpu().pin_memory(), "k": st.k_new.cpu().pin_memory(), "v": st.v_new.cpu().pin_memory(),
+        "slots": st.step_slots.cpu().pin_memory(), "tables": st.dec_tables.cpu().pin_memory(),
+        "lens": st.dec_lens.cpu().pin_memory(),
+    }
+    if st.max_q:
+        host["qp"] = st.q_pre.cpu().pin_memory()
+    dst = {"q": st.q_dec, "k": st.k_new, "v": st.v_new, "slots": st.step_slots, "tables": st.dec_tables,
+           "lens": st.dec_lens, "qp": st.q_pre}
+    out_host = torch.empty_like(st.out_dec, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    if st.max_q:
+        out_pre_host = torch.empty_like(st.out_pre, device="cpu").pin_memory()
+        d2h += out_pre_host.numel() * out_pre_host.element_size()
+
+    def e2e_step():
+        for k, t in host.items():
+            dst[k].copy_(t, non_blocking=True)
+        st.step()
+        out_host.copy_(st.out_dec, non_blocking=True)
+        if st.max_q:
+            out_pre_host.copy_(st.out_pre, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    K2 = max(1, min(K, 500))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K2):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / K2
+
+    t = torch.tensor([step_ms, dec_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    step_ms, dec_ms, e2e_ms = (float(x) for x in t.tolist())
+
+    dbytes = decode_bytes(batch)
+    kvb = kv_bytes(batch)
+    peak, peak_kind = peaks()
+    value = world * dbytes / (step_ms * 1e-3) / 1e9
+    achieved = dbytes / (dec_ms * 1e-3) / 1e9
+    tr = traffic_record(f"decode/{args.workload}")
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8_e4m3 KV, bf16 q/out, fp32 accumulate" if batch.kv_dtype else "bf16",
+        "data": "synthetic",
+        "config": {
+            "workload": args.workload,
+            "num_seqs": batch.num_decode, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
+            "head_dim": batch.head_dim, "block_size": 16, "num_blocks": batch.num_blocks,
+            "context_tokens": int(batch.context_lens[:batch.num_decode].sum()),
+            "prefill_chunks": int(batch.num_seqs - batch.num_decode), "cow_pairs": int(batch.cow_pairs.shape[0]),
+            "split_tokens": st.split_tokens,
+            "l2": "inputs larger than L2: KV pool %.2f GB vs 126 MB" % (2 * st.k_cache.numel() * st.k_cache.element_size() / 1e9),
+            "parallelism": f"replicas x{world}",
+        },
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "seq_steps_per_s": round(world * batch.num_decode / (step_ms * 1e-3), 1),
+        "decode_kv_bytes_per_step": kvb,
+        "roofline": {
+            "kernel": "pa_paged_attention (paged_decode_kernel + lse_reduce_kernel)",
+            "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+            "traffic": None if tr is None else tr.get("bytes_per_launch"),
+            "algorithmic_bytes": dbytes, "avg_launch_ms": round(dec_ms, 5),
+        },
+        "e2e": {"value": round(world * dbytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": launches * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(batch, args.cpu_sample_seqs)
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle legs
+
+def _oracle_sample(batch, nseq):
+    """Host inputs of the oracle for the first `nseq` decoding sequences, in a contiguous cache."""
+    from pagedattention_block_table_b200.inputs import bf16_bits
+    ctx = batch.context_lens
+    seqs = list(range(min(nseq, batch.num_decode)))
+    k_rows, v_rows, slots, tables, lens = [], [], [], [], []
+    base = 0
+    mb = max((int(ctx[s]) + 15) // 16 for s in seqs)
+    for s in seqs:
+        L = int(ctx[s])
+        rows = torch.from_numpy(batch.seq_rows(s)[:L]).to(batch.tok_k.device)
+        k_rows.append(bf16_bits(batch.tok_k.index_select(0, rows)))
+        v_rows.append(bf16_bits(batch.tok_v.index_select(0, rows)))
+        nb = (L + 15) // 16
+        slots.append(base * 16 + np.arange(L, dtype=np.int64))
+        t = np.full(mb, -1, np.int32)
+        t[:nb] = base + np.arange(nb)
+        tables.append(t)
+        lens.append(L)
+        base += nb
+    q = bf16_bits(batch.q_decode[: len(seqs)])
+    ks = vs = None
+    if batch.kv_dtype:
+        ks, vs = batch.k_scale.cpu().numpy(), batch.v_scale.cpu().numpy()
+    return dict(k=np.concatenate(k_rows), v=np.concatenate(v_rows), slots=np.concatenate(slots),
+                tables=np.stack(tables), lens=np.array(lens, np.int32), q=q, nb=base, ks=ks, vs=vs,
+                kv_bytes=int(sum(lens)) * 2 * batch.num_kv_heads * batch.head_dim * (1 if batch.kv_dtype else 2))
+
+
+def _oracle_run(batch, smp):
+    from oracle import oracle as O
+    dt = np.uint8 if batch.kv_dtype else np.uint16
+    kc = np.zeros((smp["nb"], batch.num_kv_heads, 16, batch.head_dim), dt)
+    vc = np.zeros_like(kc)
+    t0 = time.perf_counter()
+    O.kv_append(kc, vc, smp["k"], smp["v"], smp["slots"], batch.kv_dtype, smp["ks"], smp["vs"])
+    O.paged_decode(smp["q"], kc, vc, smp["tables"], smp["lens"], batch.scale, batch.kv_dtype, smp["ks"], smp["vs"])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(batch, nseq):
+    from oracle import oracle as O
+    smp = _oracle_sample(batch, nseq)
+    secs = _oracle_run(batch, smp)
+    return {"value": round(smp["kv_bytes"] / secs / 1e9, 4), "unit": "GB/s", "cores": O.num_threads(),
+            "kind": "oracle",
+            "sample": f"append + decode of the first {len(smp['lens'])} of {batch.num_decode} sequences "
+                      f"({int(smp['lens'].sum())} context tokens), fp64, one run of {secs:.2f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    from oracle import oracle as O
+    from pagedattention_block_table_b200.inputs import make_batch
+    batch = make_batch(args.workload, device="cpu")
+    smp = _oracle_sample(batch, args.ref_sample_seqs)
+    for _ in range(max(0, min(args.warmup, 1))):
+        _oracle_run(batch, smp)
+    K = max(1, min(args.steps, args.ref_max_steps))
+    secs = sum(_oracle_run(batch, smp) for _ in range(K)) / K
+    value = smp["kv_bytes"] / secs / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(secs * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample_seqs": len(smp["lens"])},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
+                         "sample": f"append + decode of {len(smp['lens'])} of {batch.num_decode} sequences per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--split", type=int, default=0, help="split_tokens (0 = library default)")
+    ap.add_argument("--cpu-sample-seqs", type=int, default=16)
+    ap.add_argument("--ref-sample-seqs", type=int, default=4)
+    ap.add_argument("--ref-max-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks have nothing to do
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn.so, the B200 (sm_100a) PagedAttention hot path.
+ *
+ * Pages this follows (cited by title and section):
+ *   [Core Concepts]    "3、核心概念：LLM推理原理、KV Cache、PagedAttention、连续批处理（Continuous
+ *                      Batching）机制", §3.1 (decode step: only the new token's K/V are computed,
+ *                      its query attends over the cached K/V) and §3.2 (KV cache cut into fixed
+ *                      blocks of 16 or 32 tokens; a block table maps logical to physical blocks;
+ *                      prefill writes the prompt's K/V into blocks; each decode step writes the new
+ *                      token at the end of the current block, taking a new block when it is full;
+ *                      the attention kernel reads the non-contiguous K/V through the block table).
+ *   [vLLM overview]    uml.org.cn vLLM page, section 二 "PagedAttention" (16-token pages, one page
+ *                      table per request, pages stitched together for attention), "Prefix Sharing"
+ *                      (shared pages, copy-on-write on divergence), "Continuous Batching" (prefill
+ *                      and decode requests in one batch).
+ *   [KV Cache to vLLM] "从KV Cache到vLLM：大模型推理提速与显存优化实战", §1.2 (new query against all
+ *                      cached keys), §2.1 (KV size formula), §2.2 (1-byte KV elements; GQA: several
+ *                      query heads share one KV head).
+ *
+ * Common conventions
+ *   - Block size is 16 tokens (PA_BLOCK_SIZE).  A KV cache is two device arrays, K and V, each
+ *     laid out [num_blocks][num_kv_heads][16][head_dim] ("HND"): one (block, KV head) tile is
+ *     16*head_dim contiguous elements.  Elements are bf16 (PA_KV_BF16) or OCP FP8 E4M3
+ *     (PA_KV_FP8_E4M3) with one fp32 scale per KV head for K and one for V: value = code * scale.
+ *   - head_dim is 64 or 128.  num_q_heads must be a multiple of num_kv_heads; query head h uses
+ *     KV head h / (num_q_heads / num_kv_heads).  The group size must be 1, 2, 4, 8 or a multiple of 8.
+ *   - bf16 tensors (q, k, v, out) are row-major with the last dimension contiguous.
+ *   - A block table is int32 [num_seqs][max_blocks_per_seq]: entry i is the physical block holding
+ *     tokens 16*i .. 16*i+15 of that sequence; entries past ceil(context_len/16) are never read.
+ *   - All pointers are DEVICE pointers unless stated; all buffers are owned by the caller; the
+ *     library never allocates device memory.  Every call is asynchronous on `stream` (0 = the
+ *     legacy default stream) and returns after launching.
+ *   - Device pointers must be 16-byte aligned.
+ *
+ * Errors
+ *   Arguments are checked on the host before anything is launched; a bad one returns PA_EINVAL
+ *   or PA_EUNSUPPORTED and launches nothing.  A failed launch returns PA_ECUDA.  Values that only
+ *   the device sees (a block id outside [0, num_blocks), a slot outside the pool, a context length
+ *   beyond the table or beyond max_context_len) are not trusted: the kernel clamps the access into
+ *   the pool, sets a per-device error word and carries on; pa_get_device_error() reports it.  No
+ *   kernel traps, asserts or waits without a bound.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pa_stream_t; /* same handle as cudaStream_t */
+typedef int pa_status;
+
+#define PA_OK 0
+#define PA_EINVAL (-1)        /* malformed argument (size, null pointer, misalignment) */
+#define PA_EUNSUPPORTED (-2)  /* valid but not built: head_dim, group size, dtype */
+#define PA_ECUDA (-3)         /* a CUDA launch or query failed */
+#define PA_EDEVICE_OOB (-4)   /* a kernel met a block id / slot / length outside its bounds */
+#define PA_EWORKSPACE (-5)    /* workspace missing or smaller than required */
+
+#define PA_BLOCK_SIZE 16
+#define PA_KV_BF16 0
+#define PA_KV_FP8_E4M3 1
+
+/*
+ * pa_kv_append -- write new tokens' K and V into their slots [Core Concepts §3.2: each new token is
+ * written at the end of its sequence's current block; prefill writes all prompt tokens].
+ *   k_cache, v_cache : the cache (see conventions), written in place.
+ *   k, v             : bf16 [num_tokens][num_kv_heads][head_dim], the new tokens.
+ *   slot_mapping     : int64 [num_tokens]; token n goes to block slot/16, offset slot%16.  A negative
+ *                      slot means "padding, write nothing".  Slots must be distinct.
+ *   kv_dtype         : PA_KV_BF16 (bit copy) or PA_KV_FP8_E4M3: code = E4M3(x / scale[h]), the
+ *                      binary32 quotient rounded to nearest even and saturated to +-448.
+ *   k_scale, v_scale : fp32 [num_kv_heads] device arrays; read only for FP8, may be NULL for bf16.
+ * num_tokens == 0 launches nothing and returns PA_OK.
+ */
+pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *v,
+                       const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
+                       int head_dim, int64_t num_blocks, int kv_dtype, const float *k_scale,
+                       const float *v_scale, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write fork [vLLM overview, Prefix Sharing: after divergence the new token
+ * is written into a copied page; the shared page stays unchanged].  For each pair p the whole physical
+ * block src_dst_pairs[2p] (all KV heads, 16 slots, K and V) is copied to block src_dst_pairs[2p+1].
+ *   src_dst_pairs : int32 [num_pairs][2] on the device.  Preconditions: destinations are distinct and
+ *                   no destination is also a source in the same call (copies run concurrently).
+ */
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, int num_pairs,
+                         int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
+                         pa_stream_t stream);
+
+/*
+ * pa_paged_attention_workspace_size -- bytes of fp32 scratch pa_paged_attention needs for the given
+ * split.  0 when every sequence fits one split (no workspace needed).  split_tokens as below.
+ */
+size_t pa_paged_attention_workspace_size(int num_seqs, int num_q_heads, int head_dim,
+                                         int max_context_len, int split_tokens);
+
+/*
+ * pa_paged_attention_auto_split -- the split length pa_paged_attention picks for split_tokens == 0.
+ */
+int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int max_context_len, int kv_dtype);
+
+/*
+ * pa_paged_attention -- decode attention over the paged cache [Core Concepts §3.2: the kernel reads
+ * non-contiguous K/V through the block table; KV Cache to vLLM §1.2: the new token's query attends
+ * over all cached keys and takes the weighted sum of values; §2.2 GQA].  For every sequence b and
+ * query head h:  out[b][h] = softmax_t(scale * q[b][h] . K_b[t]) . V_b[t]  over t < context_lens[b],
+ * K_b[t] = k_cache[block_tables[b][t/16]][h/G][t%16].  context_lens counts the newest token (append
+ * first, then attend).  A context length of 0 gives a zero row.
+ *   out          : bf16 [num_seqs][num_q_heads][head_dim]
+ *   q            : bf16 [num_seqs][num_q_heads][head_dim]
+ *   block_tables : int32 [num_seqs][max_blocks_per_seq];  context_lens : int32 [num_seqs]
+ *   max_context_len : host-side upper bound of context_lens (sizes the launch and the workspace).
+ *   split_tokens : tokens per split-K partition (a multiple of 16); 0 = pa_paged_attention_auto_split.
+ *                  When a sequence spans several splits each writes a partial (max, sum, unnormalised
+ *                  output) to the workspace and a log-sum-exp reduce combines them.
+ *   workspace    : device scratch of at least pa_paged_attention_workspace_size(...) bytes, or NULL
+ *                  when that is 0.  Its contents need no initialisation and are clobbered.
+ */
+pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq,
+                             const int32_t *context_lens, int num_seqs, int num_q_heads,
+                             int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+                             int kv_dtype, const float *k_scale, const float *v_scale,
+                             int max_context_len, int split_tokens, void *workspace,
+                             size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_paged_prefill -- causal attention of prefill chunks over their paged history [vLLM overview,
+ * Continuous Batching: requests in prefill share the batch with decoding ones; Core Concepts §3.2:
+ * prefill writes the prompt's K/V into blocks].  Chunk c owns query rows cu_q_lens[c] ..
+ * cu_q_lens[c+1]-1 (C_c rows) and its context_lens[c] = H_c + C_c tokens are in the cache (append the
+ * chunk first).  Row i of the chunk is position H_c + i and attends to positions t <= H_c + i.
+ *   out, q       : bf16 [cu_q_lens[num_chunks]][num_q_heads][head_dim]
+ *   cu_q_lens    : int32 [num_chunks + 1] on the device, non-decreasing, cu_q_lens[0] = 0
+ *   block_tables : int32 [num_chunks][max_blocks_per_seq];  context_lens : int32 [num_chunks]
+ *   max_q_len    : host-side upper bound of C_c;  max_context_len : upper bound of context_lens.
+ * bf16 caches only (kv_dtype must be PA_KV_BF16).  Runs on the tcgen05 tensor cores.
+ */
+pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks,
+                           const void *k_cache, const void *v_cache, const int32_t *block_tables,
+                           int max_blocks_per_seq, const int32_t *context_lens, int num_q_heads,
+                           int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+                           int kv_dtype, int max_q_len, int max_context_len, pa_stream_t stream);
+
+/*
+ * pa_get_device_error -- synchronise `stream`, then return PA_EDEVICE_OOB if any kernel of this library
+ * on the current device has met an out-of-range block id, slot or length since the last call (and
+ * clear the flag), else PA_OK (or PA_ECUDA if the synchronisation failed).
+ */
+pa_status pa_get_device_error(pa_stream_t stream);
+
+/* pa_status_string -- static text for a status code. */
+const char *pa_status_string(pa_status status);
+
+/*
+ * pa_kv_cache_bytes -- bytes of a KV cache [KV Cache to vLLM §2.1]:
+ *   2 (K and V) * layers * kv_heads * head_dim * seq_len * batch * elem_bytes.  -1 on negative input.
+ */
+int64_t pa_kv_cache_bytes(int64_t layers, int64_t kv_heads, int64_t head_dim, int64_t seq_len,
+                          int64_t batch, int64_t elem_bytes);
+
+/* pa_version -- library version string. */
+const char *pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

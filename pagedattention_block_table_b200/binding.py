@@ -1,0 +1,211 @@
+"""Thin ctypes binding of ``libpagedattn.so`` (declared in ``include/pagedattn.h``).
+
+Each function has the name of the C entry point it calls and only marshals arguments:
+torch CUDA tensors become device pointers, sizes are read off tensor shapes, the stream
+defaults to torch's current stream, and a non-zero status raises :class:`PagedAttnError`.
+Every step of the computation runs in the library's CUDA kernels; there is no fallback.
+If the library is missing this module raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libpagedattn.so")
+
+PA_OK = 0
+PA_EINVAL = -1
+PA_EUNSUPPORTED = -2
+PA_ECUDA = -3
+PA_EDEVICE_OOB = -4
+PA_EWORKSPACE = -5
+PA_BLOCK_SIZE = 16
+PA_KV_BF16 = 0
+PA_KV_FP8_E4M3 = 1
+
+# every entry point include/pagedattn.h declares
+EXPORTED = (
+    "pa_kv_append", "pa_copy_blocks", "pa_paged_attention_workspace_size",
+    "pa_paged_attention_auto_split", "pa_paged_attention", "pa_paged_prefill",
+    "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
+)
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {pa_status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libpagedattn.so not built ({LIB_PATH}); run "
+                              "`python -m pagedattention_block_table_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.pa_kv_append.restype = I
+        L.pa_kv_append.argtypes = [P, P, P, P, P, I64, I, I, I64, I, P, P, P]
+        L.pa_copy_blocks.restype = I
+        L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I64, I, P]
+        L.pa_paged_attention_workspace_size.restype = SZ
+        L.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I]
+        L.pa_paged_attention_auto_split.restype = I
+        L.pa_paged_attention_auto_split.argtypes = [I, I, I, I, I, I]
+        L.pa_paged_attention.restype = I
+        L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P, SZ, P]
+        L.pa_paged_prefill.restype = I
+        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, F, I, I, I, P]
+        L.pa_get_device_error.restype = I
+        L.pa_get_device_error.argtypes = [P]
+        L.pa_status_string.restype = ctypes.c_char_p
+        L.pa_status_string.argtypes = [I]
+        L.pa_kv_cache_bytes.restype = I64
+        L.pa_kv_cache_bytes.argtypes = [I64] * 6
+        L.pa_version.restype = ctypes.c_char_p
+        L.pa_version.argtypes = []
+        _lib = L
+    return _lib
+
+
+# ------------------------------------------------------------------------------ helpers
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtypes=None, cuda=True):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, what: str):
+    if status != PA_OK:
+        raise PagedAttnError(status, what)
+
+
+_CACHE_DTYPES = {PA_KV_BF16: (torch.bfloat16,), PA_KV_FP8_E4M3: (torch.uint8, torch.float8_e4m3fn)}
+
+
+def _cache_geometry(k_cache: torch.Tensor):
+    if k_cache.dim() != 4 or k_cache.shape[2] != PA_BLOCK_SIZE:
+        raise ValueError("cache must be [num_blocks][num_kv_heads][16][head_dim]")
+    nb, hkv, _, d = k_cache.shape
+    return int(nb), int(hkv), int(d)
+
+
+# ------------------------------------------------------------------------------ entry points
+
+def pa_version() -> str:
+    return lib().pa_version().decode()
+
+
+def pa_status_string(status: int) -> str:
+    return lib().pa_status_string(int(status)).decode()
+
+
+def pa_kv_cache_bytes(layers, kv_heads, head_dim, seq_len, batch, elem_bytes) -> int:
+    return int(lib().pa_kv_cache_bytes(layers, kv_heads, head_dim, seq_len, batch, elem_bytes))
+
+
+def pa_kv_append(k_cache, v_cache, k, v, slot_mapping, kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None,
+                 stream=None):
+    nb, hkv, d = _cache_geometry(k_cache)
+    cd = _CACHE_DTYPES[kv_dtype]
+    if k.shape != (slot_mapping.shape[0], hkv, d) or v.shape != k.shape:
+        raise ValueError("k/v must be [num_tokens][num_kv_heads][head_dim]")
+    st = lib().pa_kv_append(
+        _ptr(k_cache, "k_cache", cd), _ptr(v_cache, "v_cache", cd), _ptr(k, "k", (torch.bfloat16,)),
+        _ptr(v, "v", (torch.bfloat16,)), _ptr(slot_mapping, "slot_mapping", (torch.int64,)),
+        int(slot_mapping.shape[0]), hkv, d, nb, int(kv_dtype),
+        _ptr(k_scale, "k_scale", (torch.float32,)), _ptr(v_scale, "v_scale", (torch.float32,)), _stream(stream))
+    _check(st, "pa_kv_append")
+
+
+def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, kv_dtype=PA_KV_BF16, stream=None):
+    nb, hkv, d = _cache_geometry(k_cache)
+    cd = _CACHE_DTYPES[kv_dtype]
+    pairs = src_dst_pairs
+    n = int(pairs.numel() // 2)
+    st = lib().pa_copy_blocks(_ptr(k_cache, "k_cache", cd), _ptr(v_cache, "v_cache", cd),
+                              _ptr(pairs, "src_dst_pairs", (torch.int32,)), n, hkv, d, nb, int(kv_dtype),
+                              _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def pa_paged_attention_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, split_tokens) -> int:
+    return int(lib().pa_paged_attention_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                       split_tokens))
+
+
+def pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                  kv_dtype=PA_KV_BF16) -> int:
+    return int(lib().pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                   max_context_len, kv_dtype))
+
+
+def pa_paged_attention(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                       kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, split_tokens=0, workspace=None,
+                       stream=None):
+    nb, hkv, d = _cache_geometry(k_cache)
+    cd = _CACHE_DTYPES[kv_dtype]
+    b, hq, dq = q.shape
+    if dq != d or out.shape != q.shape:
+        raise ValueError("q/out must be [num_seqs][num_q_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != b or context_lens.shape != (b,):
+        raise ValueError("block_tables [num_seqs][max_blocks] / context_lens [num_seqs] mismatch")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib().pa_paged_attention(
+        _ptr(out, "out", (torch.bfloat16,)), _ptr(q, "q", (torch.bfloat16,)), _ptr(k_cache, "k_cache", cd),
+        _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
+        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), b, hq, hkv, d, nb,
+        float(scale), int(kv_dtype), _ptr(k_scale, "k_scale", (torch.float32,)),
+        _ptr(v_scale, "v_scale", (torch.float32,)), int(max_context_len), int(split_tokens),
+        _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
+    _check(st, "pa_paged_attention")
+
+
+def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, max_q_len,
+                     max_context_len, kv_dtype=PA_KV_BF16, stream=None):
+    nb, hkv, d = _cache_geometry(k_cache)
+    cd = _CACHE_DTYPES[kv_dtype]
+    tq, hq, dq = q.shape
+    n = int(cu_q_lens.shape[0]) - 1
+    if dq != d or out.shape != q.shape:
+        raise ValueError("q/out must be [total_q][num_q_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != n or context_lens.shape != (n,):
+        raise ValueError("block_tables [num_chunks][max_blocks] / context_lens [num_chunks] mismatch")
+    st = lib().pa_paged_prefill(
+        _ptr(out, "out", (torch.bfloat16,)), _ptr(q, "q", (torch.bfloat16,)),
+        _ptr(cu_q_lens, "cu_q_lens", (torch.int32,)), n, _ptr(k_cache, "k_cache", cd),
+        _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
+        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), hq, hkv, d, nb,
+        float(scale), int(kv_dtype), int(max_q_len), int(max_context_len), _stream(stream))
+    _check(st, "pa_paged_prefill")
+
+
+def pa_get_device_error(stream=None) -> int:
+    """Synchronise the stream; return PA_EDEVICE_OOB (and clear it) if a kernel flagged a bad index."""
+    return int(lib().pa_get_device_error(_stream(stream)))

@@ -1,0 +1,56 @@
+"""Build ``libpagedattn.so`` (the CUDA kernels and their C ABI) in-tree with nvcc for sm_100a.
+
+The whole library is one translation unit (``csrc/api.cu`` includes every kernel header).
+Run ``python -m pagedattention_block_table_b200.build`` or call :func:`build`.
+"""
+from __future__ import annotations
+
+import glob
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libpagedattn.so")
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+              "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr"]
+
+
+def _sources():
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
+                  + [os.path.join(ROOT, "include", "pagedattn.h")])
+
+
+def source_digest() -> str:
+    """sha256 of the library's sources: identifies which kernels a profile was taken on."""
+    import hashlib
+    h = hashlib.sha256()
+    for src in _sources():
+        with open(src, "rb") as f:
+            h.update(os.path.basename(src).encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), "/usr/local/cuda/bin/nvcc", "nvcc"):
+        if cand and (os.path.isabs(cand) and os.path.exists(cand) or not os.path.isabs(cand)):
+            return cand
+    return "nvcc"
+
+
+def build(force: bool = False, out: str = LIB, extra=()) -> str:
+    """Compile if any source is newer than the library (or ``force``).  Returns the .so path."""
+    if not force and os.path.exists(out):
+        t = os.path.getmtime(out)
+        if all(os.path.getmtime(s) <= t for s in _sources()) and not extra:
+            return out
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", out + ".tmp", os.path.join(CSRC, "api.cu")]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    return out
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv))

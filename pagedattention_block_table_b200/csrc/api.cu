@@ -1,0 +1,313 @@
+// api.cu -- the extern "C" boundary of libpagedattn.so: host-side argument checks, launch
+// configuration, and the per-device error word.  Declarations and argument contracts are in
+// include/pagedattn.h.  Everything runs asynchronously on the caller's stream; nothing here
+// allocates device memory.
+#include <math.h>
+#include <stdio.h>
+
+#include <atomic>
+
+#include "../../include/pagedattn.h"
+#include "decode.cuh"
+#include "kv_append.cuh"
+#include "prefill.cuh"
+
+// Launch shapes of the decode kernel (warps per CTA, pipeline stages per warp); overridable
+// at build time for tuning sweeps.
+#ifndef PA_DEC_NW
+#define PA_DEC_NW 4
+#endif
+#ifndef PA_DEC_STAGES_BF16_128
+#define PA_DEC_STAGES_BF16_128 2
+#endif
+#ifndef PA_DEC_STAGES_SMALL
+#define PA_DEC_STAGES_SMALL 4
+#endif
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev >= kMaxDevices) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+  }
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev].store(n, std::memory_order_relaxed);
+    v = n;
+  }
+  return v;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+pa_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    fprintf(stderr, "pagedattn: launch failed: %s\n", cudaGetErrorString(e));
+    return PA_ECUDA;
+  }
+  return PA_OK;
+}
+
+int queries_per_cta(int group) {
+  if (group % 4 == 0) return 4;
+  if (group % 2 == 0) return 2;
+  return 1;
+}
+
+template <typename K>
+pa_status set_smem(K kernel, int bytes) {
+  // cudaFuncSetAttribute applies to the current device; cheap to repeat.
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return launch_status();
+  return PA_OK;
+}
+
+template <int KT, int D, int QPB>
+constexpr int stages_for() {
+  return (KT == 0 && D == 128) ? PA_DEC_STAGES_BF16_128 : PA_DEC_STAGES_SMALL;
+}
+
+template <int KT, int D, int QPB>
+int decode_smem() {
+  return pa::DecodeCfg<KT, D, QPB, PA_DEC_NW, stages_for<KT, D, QPB>()>::SMEM;
+}
+
+int decode_smem_rt(int kt, int d, int qpb) {
+#define PA_SM(KT, D, Q) \
+  if (kt == KT && d == D && qpb == Q) return decode_smem<KT, D, Q>();
+  PA_SM(0, 64, 1) PA_SM(0, 64, 2) PA_SM(0, 64, 4) PA_SM(0, 128, 1) PA_SM(0, 128, 2) PA_SM(0, 128, 4)
+  PA_SM(1, 64, 1) PA_SM(1, 64, 2) PA_SM(1, 64, 4) PA_SM(1, 128, 1) PA_SM(1, 128, 2) PA_SM(1, 128, 4)
+#undef PA_SM
+  return 0;
+}
+
+template <int KT, int D, int QPB>
+pa_status launch_decode(const pa::DecodeParams &P, dim3 grid, cudaStream_t st) {
+  constexpr int S = stages_for<KT, D, QPB>();
+  using C = pa::DecodeCfg<KT, D, QPB, PA_DEC_NW, S>;
+  auto kern = pa::paged_decode_kernel<KT, D, QPB, PA_DEC_NW, S>;
+  pa_status s = set_smem(kern, C::SMEM);
+  if (s != PA_OK) return s;
+  kern<<<grid, PA_DEC_NW * 32, C::SMEM, st>>>(P);
+  return launch_status();
+}
+
+pa_status dispatch_decode(int kt, int d, int qpb, const pa::DecodeParams &P, dim3 grid, cudaStream_t st) {
+#define PA_DD(KT, D, Q) \
+  if (kt == KT && d == D && qpb == Q) return launch_decode<KT, D, Q>(P, grid, st);
+  PA_DD(0, 64, 1) PA_DD(0, 64, 2) PA_DD(0, 64, 4) PA_DD(0, 128, 1) PA_DD(0, 128, 2) PA_DD(0, 128, 4)
+  PA_DD(1, 64, 1) PA_DD(1, 64, 2) PA_DD(1, 64, 4) PA_DD(1, 128, 1) PA_DD(1, 128, 2) PA_DD(1, 128, 4)
+#undef PA_DD
+  return PA_EUNSUPPORTED;
+}
+
+int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+extern "C" {
+
+const char *pa_version(void) { return "pagedattn-b200 0.1.0 (sm_100a)"; }
+
+const char *pa_status_string(pa_status s) {
+  switch (s) {
+    case PA_OK: return "ok";
+    case PA_EINVAL: return "invalid argument";
+    case PA_EUNSUPPORTED: return "unsupported configuration";
+    case PA_ECUDA: return "CUDA error";
+    case PA_EDEVICE_OOB: return "device-side out-of-range block id, slot or length";
+    case PA_EWORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int64_t pa_kv_cache_bytes(int64_t layers, int64_t kv_heads, int64_t head_dim, int64_t seq_len,
+                          int64_t batch, int64_t elem_bytes) {
+  if (layers < 0 || kv_heads < 0 || head_dim < 0 || seq_len < 0 || batch < 0 || elem_bytes < 0) return -1;
+  return 2 * layers * kv_heads * head_dim * seq_len * batch * elem_bytes;
+}
+
+pa_status pa_get_device_error(pa_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return launch_status();
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, pa::g_error_word, sizeof v) != cudaSuccess) return launch_status();
+  if (v == 0) return PA_OK;
+  const unsigned zero = 0;
+  if (cudaMemcpyToSymbol(pa::g_error_word, &zero, sizeof zero) != cudaSuccess) return launch_status();
+  return PA_EDEVICE_OOB;
+}
+
+pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *v,
+                       const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
+                       int64_t num_blocks, int kv_dtype, const float *k_scale, const float *v_scale,
+                       pa_stream_t stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_EUNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k_cache || !v_cache || !k || !v || !slot_mapping) return PA_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v) || !aligned16(slot_mapping))
+    return PA_EINVAL;
+  if (kv_dtype == PA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return PA_EINVAL;
+  if (num_blocks > (int64_t(1) << 40)) return PA_EINVAL;
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int chunks = head_dim / 8;  // 8 elements per thread
+  const int64_t total = num_tokens * num_kv_heads * chunks;
+  const int threads = 256;
+  const int64_t want = ceil_div64(total, threads);
+  const int grid = static_cast<int>(want < 65536 ? want : 65536);
+  if (kv_dtype == PA_KV_BF16) {
+    pa::kv_append_bf16_kernel<<<grid, threads, 0, st>>>(
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), static_cast<const uint4 *>(k),
+        static_cast<const uint4 *>(v), slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock);
+  } else {
+    pa::kv_append_fp8_kernel<<<grid, threads, 0, st>>>(
+        static_cast<uint2 *>(k_cache), static_cast<uint2 *>(v_cache), static_cast<const uint4 *>(k),
+        static_cast<const uint4 *>(v), slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock,
+        k_scale, v_scale);
+  }
+  return launch_status();
+}
+
+pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, int num_pairs,
+                         int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype, pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_EUNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (num_pairs > 65535) return PA_EINVAL;
+  if (!k_cache || !v_cache || !src_dst_pairs) return PA_EINVAL;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
+  const int elem = kv_dtype == PA_KV_BF16 ? 2 : 1;
+  const int64_t vecs = (int64_t)num_kv_heads * pa::kBlock * head_dim * elem / 16;
+  const int threads = 256;
+  const int64_t gx = ceil_div64(vecs, threads);
+  dim3 grid(static_cast<unsigned>(gx < 64 ? gx : 64), static_cast<unsigned>(num_pairs));
+  pa::copy_blocks_kernel<<<grid, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), src_dst_pairs, vecs, num_blocks);
+  return launch_status();
+}
+
+int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                  int max_context_len, int kv_dtype) {
+  if (num_seqs <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 16;
+  const int group = num_q_heads / num_kv_heads;
+  const int qpb = queries_per_cta(group > 0 ? group : 1);
+  const int64_t units = (int64_t)num_seqs * num_kv_heads * (group / qpb > 0 ? group / qpb : 1);
+  const int smem = decode_smem_rt(kv_dtype, head_dim, qpb);
+  int per_sm = smem > 0 ? (227 * 1024) / (smem + 1024) : 1;
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 8) per_sm = 8;
+  const int64_t slots = (int64_t)device_sm_count() * per_sm;
+  // Split only as far as needed for ~4 waves of work units of at least 256 tokens.
+  int64_t S = ceil_div64(max_context_len, 16) * 16;
+  while (S > 256 && units * ceil_div64(max_context_len, S) < 4 * slots) S = ceil_div64(S / 2, 16) * 16;
+  if (S < 256) S = 256;
+  return static_cast<int>(S);
+}
+
+size_t pa_paged_attention_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                         int split_tokens) {
+  if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 || split_tokens <= 0) return 0;
+  const int64_t ms = ceil_div64(max_context_len, split_tokens);
+  if (ms <= 1) return 0;
+  return static_cast<size_t>((int64_t)num_seqs * num_q_heads * ms * (head_dim + 2) * 4);
+}
+
+pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, const void *v_cache,
+                             const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
+                             int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int64_t num_blocks,
+                             float scale, int kv_dtype, const float *k_scale, const float *v_scale,
+                             int max_context_len, int split_tokens, void *workspace, size_t workspace_bytes,
+                             pa_stream_t stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return PA_EINVAL;
+  if (num_q_heads % num_kv_heads != 0) return PA_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_EUNSUPPORTED;
+  if (max_context_len < 0 || split_tokens < 0 || split_tokens % pa::kBlock != 0) return PA_EINVAL;
+  if (!(scale == scale) || isinf(scale)) return PA_EINVAL;
+  if (num_seqs == 0) return PA_OK;
+  if (num_seqs > 65535) return PA_EINVAL;
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
+  if (kv_dtype == PA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return PA_EINVAL;
+  const int group = num_q_heads / num_kv_heads;
+  const int qpb = queries_per_cta(group);
+  if ((int64_t)num_kv_heads * (group / qpb) > 65535) return PA_EINVAL;
+  int S = split_tokens;
+  if (S == 0) S = pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, kv_dtype);
+  const int64_t max_splits = max_context_len > 0 ? ceil_div64(max_context_len, S) : 1;
+  if (max_splits > 65535) return PA_EINVAL;
+  const size_t need = pa_paged_attention_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, S);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_EWORKSPACE;
+
+  pa::DecodeParams P;
+  P.out = static_cast<__nv_bfloat16 *>(out);
+  P.q = static_cast<const __nv_bfloat16 *>(q);
+  P.k_cache = static_cast<const uint8_t *>(k_cache);
+  P.v_cache = static_cast<const uint8_t *>(v_cache);
+  P.block_tables = block_tables;
+  P.context_lens = context_lens;
+  P.k_scale = k_scale;
+  P.v_scale = v_scale;
+  P.num_blocks = num_blocks;
+  P.max_blocks_per_seq = max_blocks_per_seq;
+  P.num_q_heads = num_q_heads;
+  P.num_kv_heads = num_kv_heads;
+  P.group = group;
+  P.split_tokens = S;
+  P.max_splits = static_cast<int>(max_splits);
+  P.max_context_len = max_context_len;
+  P.qscale = scale * 1.4426950408889634f;
+  if (need > 0) {
+    P.ws_o = static_cast<float *>(workspace);
+    P.ws_ml = P.ws_o + (int64_t)num_seqs * num_q_heads * max_splits * head_dim;
+  } else {
+    P.ws_o = nullptr;
+    P.ws_ml = nullptr;
+  }
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(static_cast<unsigned>(max_splits), static_cast<unsigned>(num_kv_heads * (group / qpb)),
+            static_cast<unsigned>(num_seqs));
+  pa_status s = dispatch_decode(kv_dtype, head_dim, qpb, P, grid, st);
+  if (s != PA_OK || max_splits <= 1) return s;
+  dim3 rgrid(static_cast<unsigned>((num_q_heads + 3) / 4), static_cast<unsigned>(num_seqs));
+  if (head_dim == 128)
+    pa::lse_reduce_kernel<128><<<rgrid, 128, 0, st>>>(P);
+  else
+    pa::lse_reduce_kernel<64><<<rgrid, 128, 0, st>>>(P);
+  return launch_status();
+}
+
+pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
+                           const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
+                           const int32_t *context_lens, int num_q_heads, int num_kv_heads, int head_dim,
+                           int64_t num_blocks, float scale, int kv_dtype, int max_q_len, int max_context_len,
+                           pa_stream_t stream) {
+  if (num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+    return PA_EINVAL;
+  if (num_q_heads % num_kv_heads != 0) return PA_EINVAL;
+  if (head_dim != 128 && head_dim != 64) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16) return PA_EUNSUPPORTED;
+  if (max_q_len < 0 || max_context_len < 0) return PA_EINVAL;
+  if (!(scale == scale) || isinf(scale)) return PA_EINVAL;
+  if (num_chunks == 0 || max_q_len == 0) return PA_OK;
+  if (!out || !q || !cu_q_lens || !k_cache || !v_cache || !block_tables || !context_lens) return PA_EINVAL;
+  if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
+  return pa::launch_prefill(out, q, cu_q_lens, num_chunks, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                            context_lens, num_q_heads, num_kv_heads, head_dim, num_blocks, scale, max_q_len,
+                            max_context_len, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,457 @@
+// decode.cuh -- paged decode attention (split-K) and its log-sum-exp reduce, sm_100a.
+//
+// What it computes (Core Concepts page §3.2; KV Cache to vLLM page §1.2, §2.2): for each
+// sequence b and query head h, out = softmax(scale * q . K^T) V over the sequence's context,
+// where token t's K/V row is read through the block table: physical block table[b][t/16],
+// slot t%16, KV head h / G (GQA: G query heads share one KV head).
+//
+// Design (B200): the work unit is (sequence, KV head, split of `split_tokens` tokens).  One
+// CTA per unit; its warps take the split's 16-token blocks round-robin and each warp runs its
+// own pipeline: lane 0 pulls the (block, head) K tile and V tile -- each one contiguous
+// 16*head_dim run in the [block][head][16][D] layout -- into shared memory with 1-D bulk async
+// copies (cp.async.bulk, mbarrier completion, no multicast), STAGES blocks ahead.  All query
+// heads of the group are processed against each tile, so every KV byte crosses HBM once.
+// Scores use an fp32 online softmax in base 2 (q is pre-scaled by scale*log2(e)); partial
+// sums are combined with warp shuffles.  Warps of a CTA merge their (max, sum, output) in
+// shared memory; a sequence covering several splits writes fp32 partials that
+// `lse_reduce_kernel` combines:  out = sum_p 2^(m_p-M) o_p / sum_p 2^(m_p-M) l_p.
+#pragma once
+#include "pa_common.cuh"
+
+namespace pa {
+
+struct DecodeParams {
+  __nv_bfloat16 *out;
+  const __nv_bfloat16 *q;
+  const uint8_t *k_cache;
+  const uint8_t *v_cache;
+  const int32_t *block_tables;
+  const int32_t *context_lens;
+  const float *k_scale;
+  const float *v_scale;
+  float *ws_o;   // [B][Hq][max_splits][D] partial outputs (unnormalised)
+  float *ws_ml;  // [B][Hq][max_splits][2]  partial (max in log2 units, sum)
+  int64_t num_blocks;
+  int max_blocks_per_seq;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;        // Hq / Hkv
+  int split_tokens; // multiple of 16
+  int max_splits;   // ceil(max_context_len / split_tokens)
+  int max_context_len;
+  float qscale;     // scale * log2(e)
+};
+
+template <int KT, int D, int QPB, int NW, int STAGES>
+struct DecodeCfg {
+  static constexpr int E = KT == 0 ? 2 : 1;          // bytes per cache element
+  static constexpr int RB = D * E;                   // bytes per token row of one head
+  static constexpr int TILE = kBlock * RB;           // bytes of one (block, head) K or V tile
+  static constexpr int LPT = (RB / 16) >= 8 ? 8 : RB / 16;  // lanes per token in QK
+  static constexpr int TPP = 32 / LPT;               // tokens per QK pass
+  static constexpr int NP = kBlock / TPP;            // QK passes per block
+  static constexpr int CPL = RB / 16 / LPT;          // 16-byte chunks per lane per token
+  static constexpr int CE = 16 / E;                  // elements per 16-byte chunk
+  static constexpr int DPL = CPL * CE;               // dims per lane in QK
+  static constexpr int LPV = D / 8;                  // lanes per V row in PV (8 elements each)
+  static constexpr int RPL = 32 / LPV;               // V rows per PV step
+  static constexpr int NU = kBlock / RPL;            // PV steps per block
+  static constexpr int P_BYTES = kBlock * QPB * 4;
+  static constexpr int A_BYTES = 16;                 // alpha[QPB], padded
+  static constexpr int BAR_BYTES = STAGES * 8;
+  static constexpr int WARP_BYTES = ((2 * STAGES * TILE + P_BYTES + A_BYTES + BAR_BYTES) + 127) / 128 * 128;
+  static constexpr int SMEM = NW * WARP_BYTES;
+  static constexpr int MERGE_FLOATS = QPB * (D + 2);
+  static_assert(QPB == 1 || QPB == 2 || QPB == 4, "queries per CTA");
+  static_assert(QPB <= LPT, "one query per lane after the reduce-scatter");
+  static_assert(MERGE_FLOATS * 4 <= 2 * STAGES * TILE, "merge area fits in the warp's tiles");
+};
+
+// Sum `acc[0..N)` over the LPT lanes of a token group, leaving lane-dependent query `qsel`'s
+// full sum in acc[0] (reduce-scatter: each butterfly step halves the values a lane keeps).
+template <int N, int LPT>
+__device__ __forceinline__ float group_reduce_scatter(float (&acc)[N], int lane) {
+  int nv = N;
+#pragma unroll
+  for (int off = LPT / 2; off >= 1; off >>= 1) {
+    if (nv > 1) {
+      const int half = nv / 2;
+      const bool up = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        if (i < half) {
+          const float send = up ? acc[i] : acc[i + half];
+          const float keep = up ? acc[i + half] : acc[i];
+          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+        }
+      }
+      nv = half;
+    } else {
+      acc[0] += __shfl_xor_sync(0xffffffffu, acc[0], off);
+    }
+  }
+  return acc[0];
+}
+
+// Query index (within the CTA's QPB) whose sum group_reduce_scatter leaves in this lane.
+template <int N, int LPT>
+__device__ __forceinline__ int group_reduce_qsel(int lane) {
+  int nv = N, qb = 0;
+#pragma unroll
+  for (int off = LPT / 2; off >= 1; off >>= 1) {
+    if (nv > 1) {
+      const int half = nv / 2;
+      if (lane & off) qb += half;
+      nv = half;
+    }
+  }
+  return qb;
+}
+
+template <int KT, int D, int QPB, int NW, int STAGES>
+__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams P) {
+  using C = DecodeCfg<KT, D, QPB, NW, STAGES>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int sub_groups = P.group / QPB;
+  const int g = blockIdx.y / sub_groups;
+  const int h0 = g * P.group + (blockIdx.y % sub_groups) * QPB;  // first query head of this CTA
+  const int b = blockIdx.z;
+
+  // ---- context length, validated: never read past the table row or the launch bound
+  int L = P.context_lens[b];
+  {
+    const int lim = min(P.max_blocks_per_seq * kBlock, P.max_context_len);
+    if (L < 0 || L > lim) {
+      if (threadIdx.x == 0 && split == 0) flag_error(kErrLength);
+      L = L < 0 ? 0 : lim;
+    }
+  }
+  const int n_splits = (L + P.split_tokens - 1) / P.split_tokens;
+  if (split >= (n_splits > 1 ? n_splits : 1)) return;
+  const bool final_out = n_splits <= 1;
+  const int t0 = split * P.split_tokens;
+  const int t1 = min(L, t0 + P.split_tokens);
+  const int nblk = t1 > t0 ? (t1 - t0 + kBlock - 1) / kBlock : 0;
+  const int blk0 = t0 / kBlock;
+
+  uint8_t *wbase = smem + warp * C::WARP_BYTES;
+  float *p_s = reinterpret_cast<float *>(wbase + 2 * STAGES * C::TILE);
+  float *alpha_s = p_s + kBlock * QPB;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(alpha_s) + C::A_BYTES);
+
+  const int nwb = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;  // blocks of this warp
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // ---- query registers: the dims this lane multiplies in QK, pre-scaled
+  const int r = lane / C::LPT, j = lane % C::LPT;
+  float qf[QPB][C::DPL];
+  {
+    float qs = P.qscale;
+    if (KT == 1) qs *= P.k_scale[g];
+#pragma unroll
+    for (int qi = 0; qi < QPB; ++qi) {
+      const __nv_bfloat16 *qrow = P.q + ((int64_t)b * P.num_q_heads + h0 + qi) * D;
+#pragma unroll
+      for (int k = 0; k < C::CPL; ++k) {
+        const int d0 = (k * C::LPT + j) * C::CE;
+#pragma unroll
+        for (int e8 = 0; e8 < C::CE; e8 += 8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(qrow + d0 + e8);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            qf[qi][k * C::CE + e8 + 2 * t] = bf16lo(ww[t]) * qs;
+            qf[qi][k * C::CE + e8 + 2 * t + 1] = bf16hi(ww[t]) * qs;
+          }
+        }
+      }
+    }
+  }
+  const int qsel = group_reduce_qsel<QPB, C::LPT>(lane);
+
+  // ---- block-table window: lane k holds the entry of this warp's block (win*32 + k)
+  const int32_t *trow = P.block_tables + (int64_t)b * P.max_blocks_per_seq;
+  auto load_window = [&](int win) -> int {
+    const int i = win * 32 + lane;
+    int e = 0;
+    if (i < nwb) {
+      e = __ldg(trow + blk0 + warp + NW * i);
+      if (e < 0 || e >= P.num_blocks) {
+        flag_error(kErrBlockId);
+        e = 0;
+      }
+    }
+    return e;
+  };
+  int tw = load_window(0);
+  const uint64_t pol = l2_evict_first_policy();
+  const int64_t head_stride = (int64_t)C::TILE;
+  auto issue = [&](int i) {  // warp-uniform call
+    if (i >= nwb) return;
+    if ((i & 31) == 0 && i > 0) tw = load_window(i >> 5);
+    const int e = __shfl_sync(0xffffffffu, tw, i & 31);
+    if (lane == 0) {
+      const int s = i % STAGES;
+      const int64_t off = ((int64_t)e * P.num_kv_heads + g) * head_stride;
+      mbar_arrive_expect_tx(&bars[s], 2 * C::TILE);
+      bulk_g2s(wbase + s * C::TILE, P.k_cache + off, C::TILE, &bars[s], pol);
+      bulk_g2s(wbase + (STAGES + s) * C::TILE, P.v_cache + off, C::TILE, &bars[s], pol);
+    }
+  };
+
+  // ---- running state: this lane's query qsel (m, l); o[q][8 dims] for all queries
+  float m_run = -INFINITY, l_run = 0.f;
+  float o[QPB][8];
+#pragma unroll
+  for (int qi = 0; qi < QPB; ++qi)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[qi][e] = 0.f;
+
+  const int c = lane % C::LPV, hv = lane / C::LPV;
+  int issued = 0;
+  for (; issued < STAGES && issued < nwb; ++issued) issue(issued);
+  bool ok = true;
+  int i = 0;
+  for (; i < nwb; ++i) {
+    const int s = i % STAGES;
+    const bool got = mbar_wait(&bars[s], (i / STAGES) & 1);
+    if (__any_sync(0xffffffffu, !got)) {
+      ok = false;
+      break;
+    }
+    const int jb = warp + NW * i;                       // block index within the split
+    const int nvalid = min(kBlock, t1 - (t0 + jb * kBlock));
+    const uint8_t *Kt = wbase + s * C::TILE;
+    const uint8_t *Vt = wbase + (STAGES + s) * C::TILE;
+
+    // -- scores: token t = pp*TPP + r, LPT lanes per token
+    float sc[C::NP];
+#pragma unroll
+    for (int pp = 0; pp < C::NP; ++pp) {
+      const int t = pp * C::TPP + r;
+      float acc[QPB];
+#pragma unroll
+      for (int qi = 0; qi < QPB; ++qi) acc[qi] = 0.f;
+#pragma unroll
+      for (int k = 0; k < C::CPL; ++k) {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(Kt + t * C::RB + (k * C::LPT + j) * 16);
+        const uint32_t ww[4] = {raw.x, raw.y, raw.z, raw.w};
+        if constexpr (KT == 0) {
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            const float lo = bf16lo(ww[t2]), hi = bf16hi(ww[t2]);
+#pragma unroll
+            for (int qi = 0; qi < QPB; ++qi) {
+              acc[qi] = fmaf(qf[qi][k * C::CE + 2 * t2], lo, acc[qi]);
+              acc[qi] = fmaf(qf[qi][k * C::CE + 2 * t2 + 1], hi, acc[qi]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] & 0xffffu));
+            const float2 bq = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] >> 16));
+#pragma unroll
+            for (int qi = 0; qi < QPB; ++qi) {
+              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 0], a.x, acc[qi]);
+              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 1], a.y, acc[qi]);
+              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 2], bq.x, acc[qi]);
+              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 3], bq.y, acc[qi]);
+            }
+          }
+        }
+      }
+      const float sv = group_reduce_scatter<QPB, C::LPT>(acc, lane);
+      sc[pp] = t < nvalid ? sv : -INFINITY;
+    }
+
+    // -- online softmax for query qsel over this block's 16 tokens
+    float mb = sc[0];
+#pragma unroll
+    for (int pp = 1; pp < C::NP; ++pp) mb = fmaxf(mb, sc[pp]);
+#pragma unroll
+    for (int off = C::LPT; off < 32; off <<= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+    const float m_new = fmaxf(m_run, mb);
+    const float alpha = exp2f(m_run - m_new);
+    float ps = 0.f;
+#pragma unroll
+    for (int pp = 0; pp < C::NP; ++pp) {
+      const float pv = exp2f(sc[pp] - m_new);
+      ps += pv;
+      p_s[(pp * C::TPP + r) * QPB + qsel] = pv;
+    }
+#pragma unroll
+    for (int off = C::LPT; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+    l_run = l_run * alpha + ps;
+    m_run = m_new;
+    if (r == 0) alpha_s[qsel] = alpha;
+    __syncwarp();
+
+    // -- o = alpha*o + P V: lane owns dims [8c, 8c+8) and tokens u*RPL + hv
+#pragma unroll
+    for (int qi = 0; qi < QPB; ++qi) {
+      const float a = alpha_s[qi];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[qi][e] *= a;
+    }
+#pragma unroll
+    for (int u = 0; u < C::NU; ++u) {
+      const int t = u * C::RPL + hv;
+      if (t < nvalid) {
+        float v[8];
+        if constexpr (KT == 0) {
+          const uint4 raw = *reinterpret_cast<const uint4 *>(Vt + t * C::RB + c * 16);
+          const uint32_t ww[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int t2 = 0; t2 < 4; ++t2) {
+            v[2 * t2] = bf16lo(ww[t2]);
+            v[2 * t2 + 1] = bf16hi(ww[t2]);
+          }
+        } else {
+          const uint2 raw = *reinterpret_cast<const uint2 *>(Vt + t * C::RB + c * 8);
+          const uint32_t ww[2] = {raw.x, raw.y};
+#pragma unroll
+          for (int t2 = 0; t2 < 2; ++t2) {
+            const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] & 0xffffu));
+            const float2 bq = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] >> 16));
+            v[4 * t2 + 0] = a.x;
+            v[4 * t2 + 1] = a.y;
+            v[4 * t2 + 2] = bq.x;
+            v[4 * t2 + 3] = bq.y;
+          }
+        }
+        float pq[QPB];
+        if constexpr (QPB == 4) {
+          const float4 p4 = *reinterpret_cast<const float4 *>(p_s + t * QPB);
+          pq[0] = p4.x;
+          pq[1] = p4.y;
+          pq[2] = p4.z;
+          pq[3] = p4.w;
+        } else {
+#pragma unroll
+          for (int qi = 0; qi < QPB; ++qi) pq[qi] = p_s[t * QPB + qi];
+        }
+#pragma unroll
+        for (int qi = 0; qi < QPB; ++qi)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[qi][e] = fmaf(pq[qi], v[e], o[qi][e]);
+      }
+    }
+    __syncwarp();
+    if (issued < nwb) issue(issued++);
+  }
+  if (!ok) {
+    // a wait gave up: give the copies this warp still has in flight a bounded chance to land,
+    // then drop this warp's state (the error word already says why)
+    for (int k = i; k < issued; ++k) (void)mbar_wait(&bars[k % STAGES], (k / STAGES) & 1);
+    m_run = -INFINITY;
+    l_run = 0.f;
+#pragma unroll
+    for (int qi = 0; qi < QPB; ++qi)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[qi][e] = 0.f;
+  }
+
+  // ---- merge the RPL token-parity lane groups, then the warps
+#pragma unroll
+  for (int off = C::LPV; off < 32; off <<= 1)
+#pragma unroll
+    for (int qi = 0; qi < QPB; ++qi)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[qi][e] += __shfl_xor_sync(0xffffffffu, o[qi][e], off);
+  __syncwarp();
+  float *mrg = reinterpret_cast<float *>(wbase);  // this warp's tiles are all consumed
+  if (hv == 0) {
+#pragma unroll
+    for (int qi = 0; qi < QPB; ++qi)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mrg[qi * D + c * 8 + e] = o[qi][e];
+  }
+  if (r == 0) {
+    mrg[QPB * D + 2 * qsel] = m_run;
+    mrg[QPB * D + 2 * qsel + 1] = l_run;
+  }
+  __syncthreads();
+
+  const float vs = KT == 1 ? P.v_scale[g] : 1.f;
+  for (int idx = threadIdx.x; idx < QPB * D; idx += NW * 32) {
+    const int qi = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w)
+      M = fmaxf(M, reinterpret_cast<const float *>(smem + w * C::WARP_BYTES)[QPB * D + 2 * qi]);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float *mw = reinterpret_cast<const float *>(smem + w * C::WARP_BYTES);
+        const float sc_w = exp2f(mw[QPB * D + 2 * qi] - M);
+        Lsum += sc_w * mw[QPB * D + 2 * qi + 1];
+        O += sc_w * mw[qi * D + d];
+      }
+    }
+    const int h = h0 + qi;
+    if (final_out) {
+      const float val = Lsum > 0.f ? O / Lsum * vs : 0.f;
+      P.out[((int64_t)b * P.num_q_heads + h) * D + d] = __float2bfloat16_rn(val);
+    } else {
+      const int64_t row = ((int64_t)b * P.num_q_heads + h) * P.max_splits + split;
+      P.ws_o[row * D + d] = O * vs;
+      if (d == 0) {
+        P.ws_ml[row * 2] = M;
+        P.ws_ml[row * 2 + 1] = Lsum;
+      }
+    }
+  }
+}
+
+// Combine the split partials of every (sequence, query head) whose context spans more than one
+// split: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p.
+// One warp per (sequence, query head); lane owns D/32 dims.
+template <int D>
+__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
+  const int h = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  if (h >= P.num_q_heads) return;
+  int L = P.context_lens[b];
+  const int lim = min(P.max_blocks_per_seq * kBlock, P.max_context_len);
+  L = L < 0 ? 0 : (L > lim ? lim : L);
+  const int n = (L + P.split_tokens - 1) / P.split_tokens;
+  if (n <= 1) return;  // written directly by the decode kernel
+  const int64_t row0 = ((int64_t)b * P.num_q_heads + h) * P.max_splits;
+  float M = -INFINITY;
+  for (int p = 0; p < n; ++p) M = fmaxf(M, P.ws_ml[(row0 + p) * 2]);
+  constexpr int DPL = D / 32;
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  float den = 0.f;
+  for (int p = 0; p < n; ++p) {
+    const float w = M == -INFINITY ? 0.f : exp2f(P.ws_ml[(row0 + p) * 2] - M);
+    den += w * P.ws_ml[(row0 + p) * 2 + 1];
+    const float *op = P.ws_o + (row0 + p) * D + lane * DPL;
+    if constexpr (DPL == 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(op);
+      acc[0] += w * v.x;
+      acc[1] += w * v.y;
+      acc[2] += w * v.z;
+      acc[3] += w * v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] += w * op[e];
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  __nv_bfloat16 *orow = P.out + ((int64_t)b * P.num_q_heads + h) * D + lane * DPL;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) orow[e] = __float2bfloat16_rn(acc[e] * inv);
+}
+
+}  // namespace pa

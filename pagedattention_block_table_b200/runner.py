@@ -1,0 +1,107 @@
+"""One serving step over a paged KV cache, on the device, through the C ABI.
+
+A step is what the pages describe for one iteration of a continuously batched engine
+(vLLM overview page, "Continuous Batching"; Core Concepts page §3.2): forks of shared
+pages are copied (copy-on-write), every request's new tokens are appended at the end of
+its current block, decoding requests attend over their whole context and prefill chunks
+attend causally over their history plus themselves.  This module only places tensors on
+the device and calls the binding; all arithmetic runs in libpagedattn's kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import numpy as np
+import torch
+
+from . import binding as B
+from .inputs import PagedBatch
+
+
+class DeviceStep:
+    """Device-resident state (cache, tables, inputs) of one :class:`PagedBatch` step."""
+
+    def __init__(self, batch: PagedBatch, device="cuda", split_tokens: Optional[int] = None,
+                 zero_cache: bool = True):
+        self.batch = batch
+        self.device = torch.device(device)
+        dev = self.device
+        nb, hkv, d = batch.num_blocks, batch.num_kv_heads, batch.head_dim
+        self.kv_dtype = B.PA_KV_FP8_E4M3 if batch.kv_dtype else B.PA_KV_BF16
+        cdt = torch.uint8 if batch.kv_dtype else torch.bfloat16
+        alloc = torch.zeros if zero_cache else torch.empty
+        self.k_cache = alloc((nb, hkv, 16, d), dtype=cdt, device=dev)
+        self.v_cache = alloc((nb, hkv, 16, d), dtype=cdt, device=dev)
+        self.k_scale = None if batch.k_scale is None else batch.k_scale.to(dev, torch.float32).contiguous()
+        self.v_scale = None if batch.v_scale is None else batch.v_scale.to(dev, torch.float32).contiguous()
+
+        nd = batch.num_decode
+        ctx = batch.context_lens
+        self.dec_tables = torch.from_numpy(batch.decode_tables).to(dev)
+        self.dec_lens = torch.from_numpy(np.ascontiguousarray(ctx[:nd])).to(dev)
+        self.dec_max_len = int(ctx[:nd].max()) if nd else 0
+        self.pre_tables = torch.from_numpy(batch.prefill_tables).to(dev)
+        self.pre_lens = torch.from_numpy(np.ascontiguousarray(ctx[nd:])).to(dev)
+        self.pre_max_len = int(ctx[nd:].max()) if ctx.shape[0] > nd else 0
+        self.cu_q = torch.from_numpy(batch.cu_q_lens).to(dev)
+        self.max_q = int(batch.new_lens[nd:].max()) if ctx.shape[0] > nd else 0
+        self.q_dec = batch.q_decode.to(dev).contiguous()
+        self.q_pre = batch.q_prefill.to(dev).contiguous()
+        self.out_dec = torch.empty_like(self.q_dec)
+        self.out_pre = torch.empty_like(self.q_pre)
+        self.cow = torch.from_numpy(np.ascontiguousarray(batch.cow_pairs)).to(dev)
+        rows = torch.from_numpy(batch.step_rows()).to(batch.tok_k.device)
+        self.k_new = batch.tok_k.index_select(0, rows).to(dev).contiguous()
+        self.v_new = batch.tok_v.index_select(0, rows).to(dev).contiguous()
+        self.step_slots = torch.from_numpy(batch.step_slots).to(dev)
+
+        hq = batch.num_q_heads
+        if split_tokens is None:
+            split_tokens = batch.split_tokens or 0
+        if split_tokens == 0 and nd:
+            split_tokens = B.pa_paged_attention_auto_split(nd, hq, hkv, d, self.dec_max_len, self.kv_dtype)
+        self.split_tokens = split_tokens
+        ws = B.pa_paged_attention_workspace_size(nd, hq, d, self.dec_max_len, split_tokens) if nd else 0
+        self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=dev) if ws else None
+
+    # ------------------------------------------------------------------ set-up (not part of a step)
+    def fill_history(self, chunk_tokens: int = 1 << 16):
+        """Write every sequence's history into the cache (the earlier prefills and decodes)."""
+        b = self.batch
+        slots = torch.from_numpy(b.setup_slots)
+        n = slots.shape[0]
+        for lo in range(0, n, chunk_tokens):
+            hi = min(n, lo + chunk_tokens)
+            k = b.tok_k[lo:hi].to(self.device).contiguous()
+            v = b.tok_v[lo:hi].to(self.device).contiguous()
+            B.pa_kv_append(self.k_cache, self.v_cache, k, v, slots[lo:hi].to(self.device).contiguous(),
+                           self.kv_dtype, self.k_scale, self.v_scale)
+
+    # ------------------------------------------------------------------ the step
+    def fork(self, stream=None):
+        if self.cow.shape[0]:
+            B.pa_copy_blocks(self.k_cache, self.v_cache, self.cow, self.kv_dtype, stream)
+
+    def append(self, stream=None):
+        B.pa_kv_append(self.k_cache, self.v_cache, self.k_new, self.v_new, self.step_slots, self.kv_dtype,
+                       self.k_scale, self.v_scale, stream)
+
+    def decode(self, stream=None, split_tokens: Optional[int] = None):
+        if self.batch.num_decode == 0:
+            return
+        B.pa_paged_attention(self.out_dec, self.q_dec, self.k_cache, self.v_cache, self.dec_tables, self.dec_lens,
+                             self.batch.scale, self.dec_max_len, self.kv_dtype, self.k_scale, self.v_scale,
+                             self.split_tokens if split_tokens is None else split_tokens, self.workspace, stream)
+
+    def prefill(self, stream=None):
+        if self.max_q == 0:
+            return
+        B.pa_paged_prefill(self.out_pre, self.q_pre, self.cu_q, self.k_cache, self.v_cache, self.pre_tables,
+                           self.pre_lens, self.batch.scale, self.max_q, self.pre_max_len, self.kv_dtype, stream)
+
+    def step(self, stream=None):
+        """copy-on-write forks -> append -> decode attention -> prefill attention."""
+        self.fork(stream)
+        self.append(stream)
+        self.decode(stream)
+        self.prefill(stream)

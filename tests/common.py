@@ -54,3 +54,24 @@ def assert_close(got: np.ndarray, ref: np.ndarray, max_tol=ATOL_MAX, mean_tol=AT
     if mean_tol is not None:
         assert mn <= mean_tol, f"{what}: mean abs err {mn:.3e} > {mean_tol:.1e}"
     return mx, mn
+
+
+def oracle_decode_one(batch: PagedBatch, s: int, O, kv_dtype=None):
+    """Oracle decode of sequence s alone (all query heads) from its token rows, in a fresh
+    contiguous cache; used to check sampled outputs of full-size runs."""
+    kv_dtype = batch.kv_dtype if kv_dtype is None else kv_dtype
+    L = int(batch.context_lens[s])
+    rows = torch.from_numpy(batch.seq_rows(s)[:L]).to(batch.tok_k.device)
+    tk = bf16_bits(batch.tok_k.index_select(0, rows))
+    tv = bf16_bits(batch.tok_v.index_select(0, rows))
+    nblk = max(1, (L + 15) // 16)
+    dt = np.uint8 if kv_dtype else np.uint16
+    kc = np.zeros((nblk, batch.num_kv_heads, 16, batch.head_dim), dt)
+    vc = np.zeros_like(kc)
+    ks = vs = None
+    if kv_dtype:
+        ks, vs = batch.k_scale.cpu().numpy(), batch.v_scale.cpu().numpy()
+    O.kv_append(kc, vc, tk, tv, np.arange(L, dtype=np.int64), kv_dtype, ks, vs)
+    q = bf16_bits(batch.q_decode[s:s + 1])
+    return O.paged_decode(q, kc, vc, np.arange(nblk, dtype=np.int32)[None], np.array([L], np.int32), batch.scale,
+                          kv_dtype, ks, vs)[0]

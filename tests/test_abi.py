@@ -1,0 +1,106 @@
+"""The C-ABI library loads and exports every entry point include/pagedattn.h declares; host-only
+calls and host-side argument checks (no kernel is launched, so no GPU is needed)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from pagedattention_block_table_b200 import binding as B
+from pagedattention_block_table_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return B.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_set():
+    assert sorted(B.EXPORTED) == _declared()
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(pa_\w+)", out))
+    missing = [s for s in _declared() if s not in exported]
+    assert not missing, missing
+    for s in _declared():
+        assert hasattr(L, s)
+
+
+def test_library_is_sm100a_only():
+    """The build passes exactly one target, sm_100a (no PTX for other archs to JIT)."""
+    assert "arch=compute_100a,code=sm_100a" in build.NVCC_FLAGS
+
+
+def test_kv_cache_bytes_host_function(L):
+    assert B.pa_kv_cache_bytes(32, 8, 128, 4096, 1, 2) == 536870912
+    assert B.pa_kv_cache_bytes(32, 8, 128, 4096, 8, 1) == 2 * 1024 ** 3
+    assert B.pa_kv_cache_bytes(-1, 8, 128, 4096, 8, 1) == -1
+
+
+def test_status_strings(L):
+    for s in (B.PA_OK, B.PA_EINVAL, B.PA_EUNSUPPORTED, B.PA_ECUDA, B.PA_EDEVICE_OOB, B.PA_EWORKSPACE):
+        assert B.pa_status_string(s) and B.pa_status_string(s) != "unknown status"
+    assert "sm_100a" in B.pa_version()
+
+
+def test_workspace_size(L):
+    assert B.pa_paged_attention_workspace_size(8, 32, 128, 32768, 512) == 8 * 32 * 64 * 130 * 4
+    assert B.pa_paged_attention_workspace_size(8, 32, 128, 512, 512) == 0
+    assert B.pa_paged_attention_workspace_size(8, 32, 128, 513, 512) == 8 * 32 * 2 * 130 * 4
+
+
+def _raw_attention(L, **kw):
+    args = dict(out=16, q=16, k=16, v=16, bt=16, mbs=4, cl=16, ns=2, hq=8, hkv=2, d=128, nb=10, scale=0.1,
+                dt=0, ks=None, vs=None, maxl=64, split=0, ws=None, wsb=0)
+    args.update(kw)
+    P = ctypes.c_void_p
+    return L.pa_paged_attention(P(args["out"]), P(args["q"]), P(args["k"]), P(args["v"]), P(args["bt"]), args["mbs"],
+                                P(args["cl"]), args["ns"], args["hq"], args["hkv"], args["d"], args["nb"],
+                                args["scale"], args["dt"], P(args["ks"]) if args["ks"] else None,
+                                P(args["vs"]) if args["vs"] else None, args["maxl"], args["split"],
+                                P(args["ws"]) if args["ws"] else None, args["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(hq=7), B.PA_EINVAL),                 # not a multiple of the KV heads
+    (dict(d=96), B.PA_EUNSUPPORTED),           # head_dim
+    (dict(dt=3), B.PA_EUNSUPPORTED),           # dtype
+    (dict(dt=1), B.PA_EINVAL),                 # fp8 without scales
+    (dict(split=24), B.PA_EINVAL),             # split not a multiple of 16
+    (dict(q=0), B.PA_EINVAL),                  # null pointer
+    (dict(out=8), B.PA_EINVAL),                # misaligned
+    (dict(maxl=4096, split=512), B.PA_EWORKSPACE),  # needs a workspace, none given
+    (dict(nb=0), B.PA_EINVAL),
+    (dict(scale=float("nan")), B.PA_EINVAL),
+])
+def test_attention_rejects_bad_arguments_before_launch(L, bad, status):
+    assert _raw_attention(L, **bad) == status
+
+
+def test_empty_batch_is_a_no_op(L):
+    assert _raw_attention(L, ns=0, q=0, out=0) == B.PA_OK
+    P = ctypes.c_void_p
+    assert L.pa_kv_append(None, None, None, None, None, 0, 8, 128, 10, 0, None, None, None) == B.PA_OK
+    assert L.pa_copy_blocks(None, None, None, 0, 8, 128, 10, 0, None) == B.PA_OK
+    assert L.pa_kv_append(P(16), P(16), P(16), P(16), P(16), 4, 8, 96, 10, 0, None, None, None) == B.PA_EUNSUPPORTED
+    assert L.pa_kv_append(P(16), P(16), P(16), P(16), None, 4, 8, 128, 10, 0, None, None, None) == B.PA_EINVAL
+
+
+def test_prefill_rejects_fp8_and_bad_heads(L):
+    P = ctypes.c_void_p
+    f = L.pa_paged_prefill
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 0.1, 1, 16, 64, None) == B.PA_EUNSUPPORTED
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 0.1, 0, 16, 64, None) == B.PA_EINVAL

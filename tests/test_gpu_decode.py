@@ -1,0 +1,148 @@
+"""GPU parity of paged decode attention (bf16 and FP8 caches, split-K) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from pagedattention_block_table_b200.inputs import make_batch
+from tests.common import ATOL_MAX, ATOL_MEAN, FP8_MAX, assert_close, oracle_decode_one, oracle_step, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_decode(batch, split_tokens=None):
+    from pagedattention_block_table_b200.runner import DeviceStep
+    st = DeviceStep(batch, split_tokens=split_tokens)
+    st.fill_history()
+    st.step()
+    torch.cuda.synchronize()
+    return st
+
+
+SMALL = {
+    # the tiny workload exactly as specified
+    "tiny": ("tiny_decode", {}),
+    # 8B shapes, ragged lengths spanning several tiles, splits and a ragged tail
+    "gqa4_d128": ("llama3_8b_decode", dict(num_seqs=6, hist=("fixed", [0, 15, 16, 511, 1023, 1700]))),
+    "gqa8_d128": ("llama3_8b_decode", dict(num_seqs=3, num_q_heads=64, num_kv_heads=8, hist=("uniform", 30, 900))),
+    "gqa2_d64": ("tiny_decode", dict(num_seqs=5, num_q_heads=4, num_kv_heads=2, hist=("uniform", 1, 700),
+                                     num_blocks=None)),
+    "mha_d64": ("tiny_decode", dict(num_seqs=3, num_q_heads=3, num_kv_heads=3, hist=("uniform", 200, 600),
+                                    num_blocks=None)),
+    "gqa3_d128": ("llama3_8b_decode", dict(num_seqs=2, num_q_heads=6, num_kv_heads=2, hist=("uniform", 40, 300))),
+}
+
+
+@pytest.mark.parametrize("case", sorted(SMALL))
+@pytest.mark.parametrize("split", [None, 64, 256])
+def test_decode_bf16_matches_oracle(O, cuda_lib, case, split):
+    name, ov = SMALL[case]
+    batch = make_batch(name, seed=41, overrides=ov)
+    ref = oracle_step(batch, O)["decode"]
+    st = _gpu_decode(batch, split)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(st.out_dec), ref, what=f"{case} split={split}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("split", [None, 128])
+def test_decode_fp8_matches_oracle(O, cuda_lib, d, split):
+    batch = make_batch("mha_fp8_decode", seed=42, overrides=dict(num_seqs=4, num_q_heads=8, num_kv_heads=8,
+                                                               head_dim=d, hist=("uniform", 1, 700)))
+    st = _gpu_decode(batch, split)
+    got = to_f64(st.out_dec)
+    # against the oracle on the dequantised cache: kernel arithmetic only
+    assert_close(got, oracle_step(batch, O)["decode"], what="fp8 vs dequantised")
+    # against the oracle on the original bf16 K/V: includes the quantisation error
+    b16 = make_batch("mha_fp8_decode", seed=42, overrides=dict(num_seqs=4, num_q_heads=8, num_kv_heads=8,
+                                                             head_dim=d, hist=("uniform", 1, 700), kv_dtype=None))
+    assert_close(got, oracle_step(b16, O)["decode"], max_tol=FP8_MAX, mean_tol=None, what="fp8 vs bf16")
+
+
+def test_decode_fp8_with_gqa(O, cuda_lib):
+    batch = make_batch("mha_fp8_decode", seed=43, overrides=dict(num_seqs=3, num_q_heads=16, num_kv_heads=4,
+                                                               hist=("uniform", 10, 400)))
+    assert_close(to_f64(_gpu_decode(batch).out_dec), oracle_step(batch, O)["decode"], what="fp8 gqa4")
+
+
+def test_placement_invariance_bit_identical(cuda_lib):
+    kw = dict(seed=44, overrides=dict(num_seqs=5, hist=("uniform", 100, 1200)))
+    outs = [_gpu_decode(make_batch("llama3_8b_decode", perm_seed=p, **kw), 256).out_dec for p in (1, 2, -1)]
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+def test_split_and_unsplit_agree(O, cuda_lib):
+    batch = make_batch("llama3_8b_decode", seed=45, overrides=dict(num_seqs=4, hist=("uniform", 1000, 3000)))
+    ref = oracle_step(batch, O)["decode"]
+    a = to_f64(_gpu_decode(batch, 4096).out_dec)
+    b = to_f64(_gpu_decode(batch, 512).out_dec)
+    assert_close(a, ref, what="unsplit")
+    assert_close(b, ref, what="split 512")
+    assert_close(a, b, max_tol=ATOL_MAX, mean_tol=ATOL_MEAN, what="split vs unsplit")
+
+
+def test_one_token_context_returns_v_exactly(cuda_lib):
+    batch = make_batch("llama3_8b_decode", seed=46, overrides=dict(num_seqs=3, hist=("fixed", [0, 0, 0])))
+    st = _gpu_decode(batch)
+    g = batch.num_q_heads // batch.num_kv_heads
+    for s in range(3):
+        v0 = st.v_new[s]                                   # the only token: [Hkv][D]
+        assert torch.equal(st.out_dec[s], v0.repeat_interleave(g, 0))
+
+
+def test_zero_length_sequence_gives_zero_row(cuda_lib):
+    from pagedattention_block_table_b200 import binding as B
+    batch = make_batch("llama3_8b_decode", seed=47, overrides=dict(num_seqs=3, hist=("fixed", [5, 40, 9])))
+    from pagedattention_block_table_b200.runner import DeviceStep
+    st = DeviceStep(batch)
+    st.fill_history()
+    st.append()
+    lens = st.dec_lens.clone()
+    lens[1] = 0
+    out = torch.full_like(st.out_dec, 7.0)
+    B.pa_paged_attention(out, st.q_dec, st.k_cache, st.v_cache, st.dec_tables, lens, batch.scale, st.dec_max_len)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out[1]) == 0
+    assert torch.isfinite(out.float()).all()
+
+
+def test_bad_block_id_is_flagged_and_stays_in_pool(cuda_lib):
+    from pagedattention_block_table_b200 import binding as B
+    batch = make_batch("tiny_decode", seed=48)
+    from pagedattention_block_table_b200.runner import DeviceStep
+    st = DeviceStep(batch)
+    st.fill_history()
+    st.append()
+    bad = st.dec_tables.clone()
+    bad[2, 1] = batch.num_blocks + 1000
+    B.pa_paged_attention(st.out_dec, st.q_dec, st.k_cache, st.v_cache, bad, st.dec_lens, batch.scale, st.dec_max_len)
+    assert B.pa_get_device_error() == B.PA_EDEVICE_OOB
+    lens = st.dec_lens.clone()
+    lens[0] = batch.max_blocks_per_seq * 16 + 5                     # beyond the table row
+    B.pa_paged_attention(st.out_dec, st.q_dec, st.k_cache, st.v_cache, st.dec_tables, lens, batch.scale,
+                         batch.max_blocks_per_seq * 16 + 5)
+    assert B.pa_get_device_error() == B.PA_EDEVICE_OOB
+    assert B.pa_get_device_error() == B.PA_OK
+
+
+# ----------------------------------------------------------------------------- full size, sampled
+
+FULL = [
+    ("llama3_8b_decode", None, [0, 17, 40, 63]),
+    ("long_context_decode", None, [0, 5]),
+    ("mha_fp8_decode", None, [0, 11, 31]),
+]
+
+
+@pytest.mark.parametrize("name,split,samples", FULL)
+def test_full_size_sampled(O, cuda_lib, name, split, samples):
+    batch = make_batch(name, device="cuda")
+    st = _gpu_decode(batch, split)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    got = to_f64(st.out_dec)
+    assert np.all(np.isfinite(got))
+    for s in samples:
+        ref = oracle_decode_one(batch, s, O)
+        assert_close(got[s], ref, what=f"{name} seq {s}")
+        if batch.kv_dtype:
+            ref16 = oracle_decode_one(batch, s, O, kv_dtype=0)
+            assert_close(got[s], ref16, max_tol=FP8_MAX, mean_tol=None, what=f"{name} seq {s} vs bf16")
