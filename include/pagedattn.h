@@ -131,6 +131,33 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
                              size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_paged_attention_noalloc -- pa_paged_attention for callers that cannot allocate device memory.
+ * The pages have no counterpart of this call.  It exists for callers that cannot call cudaMalloc
+ * themselves: a plugin inside a serving engine that has already reserved the GPU's memory for its
+ * own KV pool and forbids further allocations, or a latency-critical loop that must not take the
+ * device-wide synchronisation a cudaMalloc/cudaFree implies.  Arguments and results are those of
+ * pa_paged_attention without `workspace`; the caller still passes every input and output buffer.
+ *
+ * Instead of a caller workspace, the split-K partials go to one library-owned scratch array of
+ * PA_NOALLOC_SCRATCH_BYTES (a file-scope __device__ array: every GPU that loads the library holds
+ * it until the process exits).  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before any stream capture.
+ * All calls on a device share the one array and it keeps the last call's contents; the kernels
+ * write every partial they read, so nothing needs clearing between calls, but calls whose work
+ * overlaps on the GPU (two streams, two host threads) race on it and must be serialised by the caller.
+ * With split_tokens == 0 the split length is the auto choice, lengthened until the partials fit; an
+ * explicit split_tokens whose partials would exceed the array returns PA_EWORKSPACE and launches
+ * nothing.  Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+pa_status pa_paged_attention_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                     const int32_t *block_tables, int max_blocks_per_seq,
+                                     const int32_t *context_lens, int num_seqs, int num_q_heads,
+                                     int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+                                     int kv_dtype, const float *k_scale, const float *v_scale,
+                                     int max_context_len, int split_tokens, pa_stream_t stream);
+
+/*
  * pa_paged_prefill -- causal attention of prefill chunks over their paged history [vLLM overview,
  * Continuous Batching: requests in prefill share the batch with decoding ones; Core Concepts §3.2:
  * prefill writes the prompt's K/V into blocks].  Chunk c owns query rows cu_q_lens[c] ..

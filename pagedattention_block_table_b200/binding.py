@@ -32,6 +32,7 @@ EXPORTED = (
     "pa_kv_append", "pa_copy_blocks", "pa_paged_attention_workspace_size",
     "pa_paged_attention_auto_split", "pa_paged_attention", "pa_paged_prefill",
     "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
+    "pa_paged_attention_noalloc",
 )
 
 
@@ -63,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_attention_auto_split.argtypes = [I, I, I, I, I, I]
         L.pa_paged_attention.restype = I
         L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P, SZ, P]
+        L.pa_paged_attention_noalloc.restype = I
+        L.pa_paged_attention_noalloc.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P]
         L.pa_paged_prefill.restype = I
         L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, F, I, I, I, P]
         L.pa_get_device_error.restype = I
@@ -185,6 +188,26 @@ def pa_paged_attention(out, q, k_cache, v_cache, block_tables, context_lens, sca
         _ptr(v_scale, "v_scale", (torch.float32,)), int(max_context_len), int(split_tokens),
         _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
     _check(st, "pa_paged_attention")
+
+
+def pa_paged_attention_noalloc(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                               kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, split_tokens=0, stream=None):
+    """pa_paged_attention without a workspace argument, for callers that cannot allocate device memory:
+    the split partials go to the library's static per-device scratch (shared by every call)."""
+    nb, hkv, d = _cache_geometry(k_cache)
+    cd = _CACHE_DTYPES[kv_dtype]
+    b, hq, dq = q.shape
+    if dq != d or out.shape != q.shape:
+        raise ValueError("q/out must be [num_seqs][num_q_heads][head_dim]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != b or context_lens.shape != (b,):
+        raise ValueError("block_tables [num_seqs][max_blocks] / context_lens [num_seqs] mismatch")
+    st = lib().pa_paged_attention_noalloc(
+        _ptr(out, "out", (torch.bfloat16,)), _ptr(q, "q", (torch.bfloat16,)), _ptr(k_cache, "k_cache", cd),
+        _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
+        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), b, hq, hkv, d, nb,
+        float(scale), int(kv_dtype), _ptr(k_scale, "k_scale", (torch.float32,)),
+        _ptr(v_scale, "v_scale", (torch.float32,)), int(max_context_len), int(split_tokens), _stream(stream))
+    _check(st, "pa_paged_attention_noalloc")
 
 
 def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, max_q_len,

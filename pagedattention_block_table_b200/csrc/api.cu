@@ -311,3 +311,61 @@ pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, i
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// pa_paged_attention_noalloc: the decode call for callers that cannot allocate device memory.
+// Its split-K partials live in this file-scope array instead of a caller workspace.  Host code
+// must not pass `g_noalloc_scratch` itself to a kernel (on the host that name is only a stand-in
+// for the device symbol); it passes the device address looked up once per device below.
+static __device__ __align__(256) float g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES / sizeof(float)];
+
+namespace {
+std::atomic<void *> g_noalloc_addr[kMaxDevices];
+
+// Device address of g_noalloc_scratch on the current device (looked up on the first call per device).
+void *noalloc_scratch_address() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void *p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    void *addr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess || addr == nullptr) {
+      fprintf(stderr, "pagedattn: cudaGetSymbolAddress(scratch) failed: %s\n", cudaGetErrorString(e));
+      return nullptr;
+    }
+    g_noalloc_addr[dev].store(addr, std::memory_order_release);
+    p = addr;
+  }
+  return p;
+}
+}  // namespace
+
+extern "C" pa_status pa_paged_attention_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                                const int32_t *block_tables, int max_blocks_per_seq,
+                                                const int32_t *context_lens, int num_seqs, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
+                                                int kv_dtype, const float *k_scale, const float *v_scale,
+                                                int max_context_len, int split_tokens, pa_stream_t stream) {
+  const size_t cap = PA_NOALLOC_SCRATCH_BYTES;
+  int S = split_tokens;
+  if (S == 0 && num_seqs > 0 && num_q_heads > 0 && num_kv_heads > 0 && max_context_len > 0) {
+    S = pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, kv_dtype);
+    while (pa_paged_attention_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, S) > cap)
+      S = static_cast<int>(ceil_div64(2 * (int64_t)S, 16) * 16);
+  }
+  const size_t need = S > 0 ? pa_paged_attention_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, S) : 0;
+  if (need > cap) {
+    fprintf(stderr, "pagedattn: pa_paged_attention_noalloc needs %zu bytes of split partials, more than the "
+            "%zu-byte static scratch; use a longer split_tokens (or 0)\n", need, cap);
+    return PA_EWORKSPACE;
+  }
+  void *ws = nullptr;
+  if (need > 0 && num_seqs > 0) {
+    ws = noalloc_scratch_address();
+    if (ws == nullptr) return PA_ECUDA;
+  }
+  return pa_paged_attention(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                            num_q_heads, num_kv_heads, head_dim, num_blocks, scale, kv_dtype, k_scale, v_scale,
+                            max_context_len, S, ws, ws ? cap : 0, stream);
+}
