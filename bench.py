@@ -59,6 +59,25 @@ def decode_bytes(batch) -> int:
     return kv + qo + tables
 
 
+def prefill_flops(batch) -> int:
+    """4 * D * Hq * sum over chunk rows of the keys each row attends (QK^T and PV, causal)."""
+    tot = 0
+    ctx = batch.context_lens
+    for s in range(batch.num_decode, batch.num_seqs):
+        C = int(batch.new_lens[s])
+        H = int(ctx[s]) - C
+        tot += C * H + C * (C + 1) // 2
+    return 4 * batch.head_dim * batch.num_q_heads * tot
+
+
+def bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    return 1590.0, "fallback"
+
+
 def kv_bytes(batch) -> int:
     nd = batch.num_decode
     e = 1 if batch.kv_dtype else 2
@@ -135,6 +154,23 @@ def traffic_record(kernel_tag: str):
         return None
 
 
+def combine_over_ranks(times_ms: dict, bytes_per_step: int, world: int, device) -> dict:
+    """Whole-job figures from every rank's own timings: each time is the MAX over ranks (the job is
+    as slow as its slowest replica) and the work is the SUM of the ranks' bytes per step."""
+    keys = sorted(times_ms)
+    t = torch.tensor([float(times_ms[k]) for k in keys] + [float(bytes_per_step)], dtype=torch.float64,
+                     device=device)
+    if world > 1:
+        mx = t[:-1].clone()
+        torch.distributed.all_reduce(mx, op=torch.distributed.ReduceOp.MAX)
+        tot = t[-1:].clone()
+        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.SUM)
+        t = torch.cat([mx, tot])
+    out = {k: float(v) for k, v in zip(keys, t[:-1].tolist())}
+    out["bytes"] = float(t[-1])
+    return out
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -165,6 +201,7 @@ def run_ours(args, rank, world, local_rank):
     ev1 = torch.cuda.Event(enable_timing=True)
     d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    p1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     with ClockSampler(local_rank) as clk:
         torch.cuda.synchronize(dev)
         ev0.record(stream)
@@ -175,12 +212,14 @@ def run_ours(args, rank, world, local_rank):
             st.decode()
             d1[i].record(stream)
             st.prefill()
+            p1[i].record(stream)
         ev1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     step_ms = ev0.elapsed_time(ev1) / K
     dec_ms = sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K
+    pre_ms = sum(a.elapsed_time(b) for a, b in zip(d1, p1)) / K
     if B.pa_get_device_error() != B.PA_OK:
         raise RuntimeError("device error flagged during the timed region")
 
@@ -224,15 +263,12 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / K2
 
-    t = torch.tensor([step_ms, dec_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    step_ms, dec_ms, e2e_ms = (float(x) for x in t.tolist())
-
     dbytes = decode_bytes(batch)
     kvb = kv_bytes(batch)
+    agg = combine_over_ranks({"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms}, dbytes, world, dev)
+    step_ms, dec_ms, e2e_ms = agg["step_ms"], agg["dec_ms"], agg["e2e_ms"]
     peak, peak_kind = peaks()
-    value = world * dbytes / (step_ms * 1e-3) / 1e9
+    value = agg["bytes"] / (step_ms * 1e-3) / 1e9
     achieved = dbytes / (dec_ms * 1e-3) / 1e9
     tr = traffic_record(f"decode/{args.workload}")
     line = {
@@ -246,7 +282,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "fp8_e4m3 KV, bf16 q/out, fp32 accumulate" if batch.kv_dtype else "bf16",
+        "dtype": {0: "bf16", 1: "fp8_e4m3 KV, bf16 q/out, fp32 accumulate",
+                  2: "int8 KV, bf16 q/out, fp32 accumulate"}[batch.kv_dtype],
         "data": "synthetic",
         "config": {
             "workload": args.workload,
@@ -268,11 +305,18 @@ def run_ours(args, rank, world, local_rank):
             "traffic": None if tr is None else tr.get("bytes_per_launch"),
             "algorithmic_bytes": dbytes, "avg_launch_ms": round(dec_ms, 5),
         },
-        "e2e": {"value": round(world * dbytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(agg["bytes"] / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches * K,
         "clocks": clk.summary(),
     }
+    if st.max_q:
+        pf = prefill_flops(batch)
+        tf_peak = bf16_peak()
+        line["prefill"] = {"kernel": "paged_prefill_kernel (tcgen05)", "bound": "tensor", "unit": "TFLOP/s",
+                           "achieved": round(pf / (pre_ms * 1e-3) / 1e12, 2), "peak": tf_peak[0],
+                           "peak_kind": tf_peak[1], "frac": round(pf / (pre_ms * 1e-3) / 1e12 / tf_peak[0], 4),
+                           "flops": pf, "avg_launch_ms": round(pre_ms, 5)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(batch, args.cpu_sample_seqs)
     return line
@@ -280,19 +324,23 @@ def run_ours(args, rank, world, local_rank):
 
 # ----------------------------------------------------------------------------- oracle legs
 
-def _oracle_sample(batch, nseq):
-    """Host inputs of the oracle for the first `nseq` decoding sequences, in a contiguous cache."""
+def _oracle_sample(batch, nseq, first=0, kv_head=None):
+    """Host inputs of the oracle for decoding sequences first .. first+nseq-1 (all KV heads, or only
+    `kv_head` and its query-head group), laid out in a fresh contiguous cache."""
     from pagedattention_block_table_b200.inputs import bf16_bits
     ctx = batch.context_lens
-    seqs = list(range(min(nseq, batch.num_decode)))
+    seqs = list(range(first, min(first + nseq, batch.num_decode)))
+    G = batch.num_q_heads // batch.num_kv_heads
+    hsel = slice(None) if kv_head is None else slice(kv_head, kv_head + 1)
+    qsel = slice(None) if kv_head is None else slice(kv_head * G, (kv_head + 1) * G)
     k_rows, v_rows, slots, tables, lens = [], [], [], [], []
     base = 0
     mb = max((int(ctx[s]) + 15) // 16 for s in seqs)
     for s in seqs:
         L = int(ctx[s])
         rows = torch.from_numpy(batch.seq_rows(s)[:L]).to(batch.tok_k.device)
-        k_rows.append(bf16_bits(batch.tok_k.index_select(0, rows)))
-        v_rows.append(bf16_bits(batch.tok_v.index_select(0, rows)))
+        k_rows.append(bf16_bits(batch.tok_k.index_select(0, rows)[:, hsel]))
+        v_rows.append(bf16_bits(batch.tok_v.index_select(0, rows)[:, hsel]))
         nb = (L + 15) // 16
         slots.append(base * 16 + np.arange(L, dtype=np.int64))
         t = np.full(mb, -1, np.int32)
@@ -300,19 +348,21 @@ def _oracle_sample(batch, nseq):
         tables.append(t)
         lens.append(L)
         base += nb
-    q = bf16_bits(batch.q_decode[: len(seqs)])
+    q = bf16_bits(batch.q_decode[first:first + len(seqs)][:, qsel])
+    hkv = batch.num_kv_heads if kv_head is None else 1
     ks = vs = None
     if batch.kv_dtype:
-        ks, vs = batch.k_scale.cpu().numpy(), batch.v_scale.cpu().numpy()
+        ks = batch.k_scale.cpu().numpy()[hsel].copy()
+        vs = batch.v_scale.cpu().numpy()[hsel].copy()
     return dict(k=np.concatenate(k_rows), v=np.concatenate(v_rows), slots=np.concatenate(slots),
-                tables=np.stack(tables), lens=np.array(lens, np.int32), q=q, nb=base, ks=ks, vs=vs,
-                kv_bytes=int(sum(lens)) * 2 * batch.num_kv_heads * batch.head_dim * (1 if batch.kv_dtype else 2))
+                tables=np.stack(tables), lens=np.array(lens, np.int32), q=q, nb=base, ks=ks, vs=vs, hkv=hkv,
+                kv_bytes=int(sum(lens)) * 2 * hkv * batch.head_dim * (1 if batch.kv_dtype else 2))
 
 
 def _oracle_run(batch, smp):
     from oracle import oracle as O
-    dt = np.uint8 if batch.kv_dtype else np.uint16
-    kc = np.zeros((smp["nb"], batch.num_kv_heads, 16, batch.head_dim), dt)
+    dt = {0: np.uint16, 1: np.uint8, 2: np.int8}[batch.kv_dtype]
+    kc = np.zeros((smp["nb"], smp["hkv"], 16, batch.head_dim), dt)
     vc = np.zeros_like(kc)
     t0 = time.perf_counter()
     O.kv_append(kc, vc, smp["k"], smp["v"], smp["slots"], batch.kv_dtype, smp["ks"], smp["vs"])
@@ -320,14 +370,25 @@ def _oracle_run(batch, smp):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(batch, nseq):
+def cpu_baseline(batch, nseq, budget_s=15.0):
+    """The oracle on the host cores: append + decode, one (sequence, KV head) unit at a time in order,
+    until `nseq` sequences are done or about `budget_s` seconds of oracle work have been spent."""
     from oracle import oracle as O
-    smp = _oracle_sample(batch, nseq)
-    secs = _oracle_run(batch, smp)
-    return {"value": round(smp["kv_bytes"] / secs / 1e9, 4), "unit": "GB/s", "cores": O.num_threads(),
-            "kind": "oracle",
-            "sample": f"append + decode of the first {len(smp['lens'])} of {batch.num_decode} sequences "
-                      f"({int(smp['lens'].sum())} context tokens), fp64, one run of {secs:.2f} s"}
+    done_bytes, secs, units, tokens = 0, 0.0, 0, 0
+    for s in range(min(nseq, batch.num_decode)):
+        for g in range(batch.num_kv_heads):
+            smp = _oracle_sample(batch, 1, first=s, kv_head=g)
+            secs += _oracle_run(batch, smp)
+            done_bytes += smp["kv_bytes"]
+            units += 1
+            tokens += int(smp["lens"].sum())
+            if secs >= budget_s:
+                break
+        if secs >= budget_s:
+            break
+    return {"value": round(done_bytes / secs / 1e9, 4), "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"append + decode of the first {units} (sequence, KV head) units of {batch.num_decode} x "
+                      f"{batch.num_kv_heads} ({tokens} token-heads), fp64, {secs:.2f} s of oracle time"}
 
 
 def run_reference(args, rank, world):
@@ -339,8 +400,15 @@ def run_reference(args, rank, world):
     smp = _oracle_sample(batch, args.ref_sample_seqs)
     for _ in range(max(0, min(args.warmup, 1))):
         _oracle_run(batch, smp)
+    # each step is the same bounded sample; stop early once the run has used its time budget
     K = max(1, min(args.steps, args.ref_max_steps))
-    secs = sum(_oracle_run(batch, smp) for _ in range(K)) / K
+    times = []
+    for _ in range(K):
+        times.append(_oracle_run(batch, smp))
+        if sum(times) > args.ref_budget_s:
+            break
+    K = len(times)
+    secs = sum(times) / K
     value = smp["kv_bytes"] / secs / 1e9
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
@@ -366,6 +434,7 @@ def main():
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     ap.add_argument("--ref-max-steps", type=int, default=20)
+    ap.add_argument("--ref-budget-s", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 

@@ -20,10 +20,11 @@
  * Common conventions
  *   - Block size is 16 tokens (PA_BLOCK_SIZE).  A KV cache is two device arrays, K and V, each
  *     laid out [num_blocks][num_kv_heads][16][head_dim] ("HND"): one (block, KV head) tile is
- *     16*head_dim contiguous elements.  Elements are bf16 (PA_KV_BF16) or OCP FP8 E4M3
- *     (PA_KV_FP8_E4M3) with one fp32 scale per KV head for K and one for V: value = code * scale.
+ *     16*head_dim contiguous elements.  Elements are bf16 (PA_KV_BF16), OCP FP8 E4M3
+ *     (PA_KV_FP8_E4M3) or signed INT8 (PA_KV_INT8, codes -127..127); the one-byte formats carry one
+ *     fp32 scale per KV head for K and one for V: value = code * scale.
  *   - head_dim is 64 or 128.  num_q_heads must be a multiple of num_kv_heads; query head h uses
- *     KV head h / (num_q_heads / num_kv_heads).  The group size must be 1, 2, 4, 8 or a multiple of 8.
+ *     KV head h / (num_q_heads / num_kv_heads) (any group size).
  *   - bf16 tensors (q, k, v, out) are row-major with the last dimension contiguous.
  *   - A block table is int32 [num_seqs][max_blocks_per_seq]: entry i is the physical block holding
  *     tokens 16*i .. 16*i+15 of that sequence; entries past ceil(context_len/16) are never read.
@@ -59,10 +60,12 @@ typedef int pa_status;
 #define PA_ECUDA (-3)         /* a CUDA launch or query failed */
 #define PA_EDEVICE_OOB (-4)   /* a kernel met a block id / slot / length outside its bounds */
 #define PA_EWORKSPACE (-5)    /* workspace missing or smaller than required */
+#define PA_ENOMEM (-6)        /* block manager: not enough free blocks (nothing was changed) */
 
 #define PA_BLOCK_SIZE 16
 #define PA_KV_BF16 0
 #define PA_KV_FP8_E4M3 1
+#define PA_KV_INT8 2
 
 /*
  * pa_kv_append -- write new tokens' K and V into their slots [Core Concepts §3.2: each new token is
@@ -71,9 +74,12 @@ typedef int pa_status;
  *   k, v             : bf16 [num_tokens][num_kv_heads][head_dim], the new tokens.
  *   slot_mapping     : int64 [num_tokens]; token n goes to block slot/16, offset slot%16.  A negative
  *                      slot means "padding, write nothing".  Slots must be distinct.
- *   kv_dtype         : PA_KV_BF16 (bit copy) or PA_KV_FP8_E4M3: code = E4M3(x / scale[h]), the
- *                      binary32 quotient rounded to nearest even and saturated to +-448.
- *   k_scale, v_scale : fp32 [num_kv_heads] device arrays; read only for FP8, may be NULL for bf16.
+ *   kv_dtype         : PA_KV_BF16 (bit copy), PA_KV_FP8_E4M3: code = E4M3(x / scale[h]), the
+ *                      binary32 quotient rounded to nearest even and saturated to +-448, or
+ *                      PA_KV_INT8: code = clamp(round-half-even(x / scale[h]), -127, 127)
+ *                      [KV Cache to vLLM §2.2: INT8 or FP8 KV at one byte per element].
+ *   k_scale, v_scale : fp32 [num_kv_heads] device arrays; read for the one-byte formats, may be NULL
+ *                      for bf16.
  * num_tokens == 0 launches nothing and returns PA_OK.
  */
 pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *v,
@@ -90,6 +96,21 @@ pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *
  */
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, int num_pairs,
                          int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
+                         pa_stream_t stream);
+
+/*
+ * pa_swap_blocks -- move whole blocks between two pools [vLLM overview, section 三: when GPU memory
+ * runs short KV pages are swapped out to CPU memory, and swapped back in when the request resumes].
+ * For each pair p, block src_dst_pairs[2p] of the source pool (all KV heads, 16 slots, K and V) is
+ * copied into block src_dst_pairs[2p+1] of the destination pool.  Both pools have the cache layout
+ * and the same num_kv_heads, head_dim and kv_dtype; each may live in device memory or in pinned,
+ * mapped host memory (cudaHostAlloc / cudaHostRegister): the kernel reads and writes host memory
+ * directly over the host link.  src_dst_pairs must be device-accessible as well.  Pageable host
+ * memory is rejected with PA_EINVAL.  Destinations must be distinct and must not overlap sources.
+ */
+pa_status pa_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const void *src_k,
+                         const void *src_v, int64_t src_num_blocks, const int32_t *src_dst_pairs,
+                         int num_pairs, int num_kv_heads, int head_dim, int kv_dtype,
                          pa_stream_t stream);
 
 /*
@@ -174,6 +195,49 @@ pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, i
                            int max_blocks_per_seq, const int32_t *context_lens, int num_q_heads,
                            int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
                            int kv_dtype, int max_q_len, int max_context_len, pa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------------------
+ * Host block manager: the control plane that produces block tables, slot mappings and copy-on-write
+ * pairs for the kernels above.  Host memory only; not thread-safe (one manager per scheduler thread).
+ * [Core Concepts §3.2: blocks are taken on demand, a new one when the current block is full;
+ *  vLLM overview, Prefix Sharing: shared pages, copy-on-write on the first write after a fork;
+ *  vLLM overview, Continuous Batching: a finished request's pages return to the pool at once.]
+ * Sequences are named by caller-chosen int64 ids.
+ */
+typedef struct pa_block_manager pa_block_manager;
+
+/* pa_bm_create -- pool of num_blocks physical blocks.  shuffle_seed != 0 hands blocks out in a seeded
+ * random order (a long-running server's scattered placement); 0 hands them out in order.  NULL on
+ * bad arguments or out of host memory. */
+pa_block_manager *pa_bm_create(int64_t num_blocks, uint64_t shuffle_seed);
+void pa_bm_destroy(pa_block_manager *bm);
+/* pa_bm_num_free -- blocks currently free (-1 for a NULL manager). */
+int64_t pa_bm_num_free(const pa_block_manager *bm);
+/* pa_bm_add -- register an empty sequence.  PA_EINVAL if the id exists. */
+pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id);
+/* pa_bm_fork -- child shares every block of parent (reference counts + 1), same length. */
+pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent, int64_t child);
+/*
+ * pa_bm_append -- reserve slots for n_tokens new tokens at the end of seq_id and write them to
+ * slots_out[n_tokens] (slot = block*16 + offset, ready for pa_kv_append).  If the block that receives
+ * the first new token is shared, it is first replaced by a private copy: the (src, dst) pair goes to
+ * cow_pairs_out[2] (run pa_copy_blocks on it before the append) and *num_cow_out = 1, else 0.
+ * PA_ENOMEM if the pool cannot supply the blocks; then nothing changes.
+ */
+pa_status pa_bm_append(pa_block_manager *bm, int64_t seq_id, int32_t n_tokens, int64_t *slots_out,
+                       int32_t *cow_pairs_out, int32_t *num_cow_out);
+/* pa_bm_free -- drop a sequence; blocks no other sequence holds return to the free list. */
+pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id);
+/* pa_bm_length -- tokens written to seq_id (-1 if unknown). */
+int64_t pa_bm_length(const pa_block_manager *bm, int64_t seq_id);
+/* pa_bm_tables -- block tables int32 [n][max_blocks_per_seq] (padded with -1) and lengths int32 [n] of
+ * the given sequences, in host memory.  PA_EINVAL if an id is unknown or a table does not fit. */
+pa_status pa_bm_tables(const pa_block_manager *bm, const int64_t *seq_ids, int32_t n, int32_t *tables_out,
+                       int32_t max_blocks_per_seq, int32_t *lens_out);
+/* pa_bm_stats -- tokens held by the pool (shared blocks counted once), blocks in use, blocks held by
+ * more than one sequence, copy-on-write copies made so far.  Any output pointer may be NULL. */
+pa_status pa_bm_stats(const pa_block_manager *bm, int64_t *tokens_stored, int64_t *blocks_used,
+                      int64_t *blocks_shared, int64_t *cow_copies);
 
 /*
  * pa_get_device_error -- synchronise `stream`, then return PA_EDEVICE_OOB if any kernel of this library

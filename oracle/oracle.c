@@ -99,6 +99,20 @@ uint8_t oracle_e4m3_encode(float x)
 }
 
 /*
+ * INT8 KV element [KV Cache to vLLM §2.2: INT8 and FP8 KV caches store one byte per element]:
+ * symmetric quantisation with one fp32 scale per KV head; code = clamp(round(x / scale), -127, 127),
+ * rounding the binary32 quotient to the nearest integer, ties to even; value = code * scale.
+ */
+int8_t oracle_int8_encode(float x)
+{
+    float r = rintf(x); /* default rounding mode: to nearest, ties to even */
+    if (isnan(x)) return 0;
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/*
  * KV size formula [KV Cache to vLLM §2.1]:
  *   bytes = 2 (K and V) x layers x kv_heads x head_dim x seq_len x batch x bytes/element.
  */
@@ -114,7 +128,8 @@ int64_t oracle_kv_cache_bytes(int64_t layers, int64_t kv_heads, int64_t head_dim
  * Append [Core Concepts §3.2, "PagedAttention 如何工作"]: each token n carries its
  * slot = physical_block * 16 + offset; its K and V rows (all KV heads) are written at
  * cache[slot / 16][h][slot % 16][:].  slot < 0 marks a padding token: nothing written.
- * kv_dtype 0 = bf16 (bit copy), 1 = fp8 E4M3 (code of the binary32 quotient x / scale[h]).
+ * kv_dtype 0 = bf16 (bit copy), 1 = fp8 E4M3 (code of the binary32 quotient x / scale[h]),
+ * 2 = int8 (rounded quotient, see oracle_int8_encode).
  */
 int oracle_kv_append(void *k_cache, void *v_cache, const uint16_t *k, const uint16_t *v,
                      const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
@@ -122,7 +137,7 @@ int oracle_kv_append(void *k_cache, void *v_cache, const uint16_t *k, const uint
                      const float *k_scale, const float *v_scale)
 {
     if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return -1;
-    if (kv_dtype != 0 && kv_dtype != 1) return -1;
+    if (kv_dtype < 0 || kv_dtype > 2) return -1;
     for (int64_t n = 0; n < num_tokens; ++n) {
         int64_t slot = slot_mapping[n];
         if (slot < 0) continue;
@@ -145,8 +160,13 @@ int oracle_kv_append(void *k_cache, void *v_cache, const uint16_t *k, const uint
                     /* binary32 division: C float '/' is the IEEE correctly rounded divide */
                     float qk = bf16_value_f(k[src + d]) / k_scale[h];
                     float qv = bf16_value_f(v[src + d]) / v_scale[h];
-                    ((uint8_t *)k_cache)[dst + d] = oracle_e4m3_encode(qk);
-                    ((uint8_t *)v_cache)[dst + d] = oracle_e4m3_encode(qv);
+                    if (kv_dtype == 1) {
+                        ((uint8_t *)k_cache)[dst + d] = oracle_e4m3_encode(qk);
+                        ((uint8_t *)v_cache)[dst + d] = oracle_e4m3_encode(qv);
+                    } else {
+                        ((int8_t *)k_cache)[dst + d] = oracle_int8_encode(qk);
+                        ((int8_t *)v_cache)[dst + d] = oracle_int8_encode(qv);
+                    }
                 }
             }
         }
@@ -179,6 +199,30 @@ int oracle_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int64
     return 0;
 }
 
+/*
+ * Swap [vLLM overview, section 三 (KV cache eviction): when GPU memory runs short, pages are moved
+ * out to CPU memory, and brought back when needed]: for each (src, dst) pair the whole block of
+ * the source pool (all KV heads, 16 slots, K and V) is copied into block dst of the destination
+ * pool.  The two pools are distinct arrays with the same per-block geometry.
+ */
+int oracle_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const void *src_k, const void *src_v,
+                       int64_t src_num_blocks, const int32_t *pairs, int64_t num_pairs, int num_kv_heads,
+                       int head_dim, int elem_bytes)
+{
+    int64_t block_bytes = (int64_t)num_kv_heads * ORACLE_BLOCK * head_dim * elem_bytes;
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || elem_bytes <= 0) return -1;
+    for (int64_t p = 0; p < num_pairs; ++p) {
+        int32_t s = pairs[2 * p], d = pairs[2 * p + 1];
+        if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) return -4;
+    }
+    for (int64_t p = 0; p < num_pairs; ++p) {
+        int64_t s = pairs[2 * p], d = pairs[2 * p + 1];
+        memcpy((char *)dst_k + d * block_bytes, (const char *)src_k + s * block_bytes, block_bytes);
+        memcpy((char *)dst_v + d * block_bytes, (const char *)src_v + s * block_bytes, block_bytes);
+    }
+    return 0;
+}
+
 /* ---------------------------------------------------------------- attention */
 
 /* value of element d of token t (logical position) of KV head g of one sequence, read
@@ -188,6 +232,7 @@ static double cache_value(const void *cache, int kv_dtype, float scale, int64_t 
 {
     int64_t idx = ((phys * num_kv_heads + g) * ORACLE_BLOCK + (t % ORACLE_BLOCK)) * (int64_t)head_dim + d;
     if (kv_dtype == 0) return bf16_value(((const uint16_t *)cache)[idx]);
+    if (kv_dtype == 2) return (double)((const int8_t *)cache)[idx] * (double)scale;
     return oracle_e4m3_decode(((const uint8_t *)cache)[idx]) * (double)scale;
 }
 

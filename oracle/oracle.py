@@ -35,12 +35,16 @@ def _load():
         lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_int8_encode.restype = ctypes.c_int8
+        lib.oracle_int8_encode.argtypes = [ctypes.c_float]
         lib.oracle_kv_cache_bytes.restype = L
         lib.oracle_kv_cache_bytes.argtypes = [L, L, L, L, L, L]
         lib.oracle_kv_append.restype = I
         lib.oracle_kv_append.argtypes = [P, P, P, P, P, L, I, I, L, I, P, P]
         lib.oracle_copy_blocks.restype = I
         lib.oracle_copy_blocks.argtypes = [P, P, P, L, I, I, L, I]
+        lib.oracle_swap_blocks.restype = I
+        lib.oracle_swap_blocks.argtypes = [P, P, L, P, P, L, P, L, I, I, I]
         lib.oracle_paged_decode.restype = I
         lib.oracle_paged_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, L, D, I, P, P]
         lib.oracle_paged_prefill.restype = I
@@ -91,8 +95,16 @@ def e4m3_encode(x) -> np.ndarray:
     return np.array([lib.oracle_e4m3_encode(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
 
 
+def int8_encode(x) -> np.ndarray:
+    """float32 values -> int8 codes: round to nearest (ties to even), clamp to [-127, 127]."""
+    lib = _load()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([lib.oracle_int8_encode(float(v)) for v in a.ravel()], dtype=np.int8).reshape(a.shape)
+
+
 def kv_append(k_cache, v_cache, k, v, slot_mapping, kv_dtype=0, k_scale=None, v_scale=None):
-    """Scatter token K/V rows into the paged cache in place (see ``oracle_kv_append``)."""
+    """Scatter token K/V rows into the paged cache in place (see ``oracle_kv_append``).
+    kv_dtype 0: uint16 bf16 cache; 1: uint8 E4M3 codes; 2: int8 codes."""
     lib = _load()
     assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
     nb, hkv, bs, d = k_cache.shape
@@ -115,6 +127,18 @@ def copy_blocks(k_cache, v_cache, pairs):
     rc = lib.oracle_copy_blocks(_p(k_cache), _p(v_cache), _p(pr), pr.shape[0], hkv, d, nb,
                                 k_cache.dtype.itemsize)
     _check(rc, "copy_blocks")
+
+
+def swap_blocks(dst_k, dst_v, src_k, src_v, pairs):
+    """Copy whole blocks src (of the source pool) -> dst (of the destination pool), in place."""
+    lib = _load()
+    nbd, hkv, _, d = dst_k.shape
+    nbs = src_k.shape[0]
+    assert src_k.shape[1:] == dst_k.shape[1:] and src_k.dtype == dst_k.dtype
+    pr = _c(pairs, np.int32).reshape(-1, 2)
+    rc = lib.oracle_swap_blocks(_p(dst_k), _p(dst_v), nbd, _p(np.ascontiguousarray(src_k)),
+                                _p(np.ascontiguousarray(src_v)), nbs, _p(pr), pr.shape[0], hkv, d, dst_k.dtype.itemsize)
+    _check(rc, "swap_blocks")
 
 
 def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, kv_dtype=0,

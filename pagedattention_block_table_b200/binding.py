@@ -15,7 +15,7 @@ from typing import Optional
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libpagedattn.so")
+LIB_PATH = os.environ.get("PAGEDATTN_LIB") or os.path.join(HERE, "libpagedattn.so")
 
 PA_OK = 0
 PA_EINVAL = -1
@@ -26,14 +26,18 @@ PA_EWORKSPACE = -5
 PA_BLOCK_SIZE = 16
 PA_KV_BF16 = 0
 PA_KV_FP8_E4M3 = 1
+PA_KV_INT8 = 2
 
 # every entry point include/pagedattn.h declares
 EXPORTED = (
     "pa_kv_append", "pa_copy_blocks", "pa_paged_attention_workspace_size",
     "pa_paged_attention_auto_split", "pa_paged_attention", "pa_paged_prefill",
     "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
-    "pa_paged_attention_noalloc",
+    "pa_paged_attention_noalloc", "pa_swap_blocks",
+    "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
+    "pa_bm_length", "pa_bm_tables", "pa_bm_stats",
 )
+PA_ENOMEM = -6
 
 
 class PagedAttnError(RuntimeError):
@@ -58,6 +62,8 @@ def lib() -> ctypes.CDLL:
         L.pa_kv_append.argtypes = [P, P, P, P, P, I64, I, I, I64, I, P, P, P]
         L.pa_copy_blocks.restype = I
         L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I64, I, P]
+        L.pa_swap_blocks.restype = I
+        L.pa_swap_blocks.argtypes = [P, P, I64, P, P, I64, P, I, I, I, I, P]
         L.pa_paged_attention_workspace_size.restype = SZ
         L.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I]
         L.pa_paged_attention_auto_split.restype = I
@@ -76,6 +82,27 @@ def lib() -> ctypes.CDLL:
         L.pa_kv_cache_bytes.argtypes = [I64] * 6
         L.pa_version.restype = ctypes.c_char_p
         L.pa_version.argtypes = []
+        U64 = ctypes.c_uint64
+        L.pa_bm_create.restype = P
+        L.pa_bm_create.argtypes = [I64, U64]
+        L.pa_bm_destroy.restype = None
+        L.pa_bm_destroy.argtypes = [P]
+        L.pa_bm_num_free.restype = I64
+        L.pa_bm_num_free.argtypes = [P]
+        L.pa_bm_add.restype = I
+        L.pa_bm_add.argtypes = [P, I64]
+        L.pa_bm_fork.restype = I
+        L.pa_bm_fork.argtypes = [P, I64, I64]
+        L.pa_bm_append.restype = I
+        L.pa_bm_append.argtypes = [P, I64, ctypes.c_int32, P, P, P]
+        L.pa_bm_free.restype = I
+        L.pa_bm_free.argtypes = [P, I64]
+        L.pa_bm_length.restype = I64
+        L.pa_bm_length.argtypes = [P, I64]
+        L.pa_bm_tables.restype = I
+        L.pa_bm_tables.argtypes = [P, P, ctypes.c_int32, P, ctypes.c_int32, P]
+        L.pa_bm_stats.restype = I
+        L.pa_bm_stats.argtypes = [P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -109,7 +136,8 @@ def _check(status: int, what: str):
         raise PagedAttnError(status, what)
 
 
-_CACHE_DTYPES = {PA_KV_BF16: (torch.bfloat16,), PA_KV_FP8_E4M3: (torch.uint8, torch.float8_e4m3fn)}
+_CACHE_DTYPES = {PA_KV_BF16: (torch.bfloat16,), PA_KV_FP8_E4M3: (torch.uint8, torch.float8_e4m3fn),
+                 PA_KV_INT8: (torch.int8,)}
 
 
 def _cache_geometry(k_cache: torch.Tensor):
@@ -156,6 +184,25 @@ def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, kv_dtype=PA_KV_BF16, stream=
                               _ptr(pairs, "src_dst_pairs", (torch.int32,)), n, hkv, d, nb, int(kv_dtype),
                               _stream(stream))
     _check(st, "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k, dst_v, src_k, src_v, src_dst_pairs, kv_dtype=PA_KV_BF16, stream=None):
+    """Copy whole blocks between two pools (device cache <-> pinned host pool).  Host tensors must be
+    pinned (``pin_memory()``); the pairs tensor may be on the device or pinned."""
+    nbd, hkv, d = _cache_geometry(dst_k)
+    nbs, hkv2, d2 = _cache_geometry(src_k)
+    if (hkv, d) != (hkv2, d2) or src_k.dtype != dst_k.dtype:
+        raise ValueError("source and destination pools differ in geometry or dtype")
+    for t, n in ((dst_k, "dst_k"), (dst_v, "dst_v"), (src_k, "src_k"), (src_v, "src_v"), (src_dst_pairs, "pairs")):
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError(f"{n} must be a CUDA tensor or pinned host memory")
+    cd = _CACHE_DTYPES[kv_dtype]
+    st = lib().pa_swap_blocks(
+        _ptr(dst_k, "dst_k", cd, cuda=False), _ptr(dst_v, "dst_v", cd, cuda=False), nbd,
+        _ptr(src_k, "src_k", cd, cuda=False), _ptr(src_v, "src_v", cd, cuda=False), nbs,
+        _ptr(src_dst_pairs, "src_dst_pairs", (torch.int32,), cuda=False), int(src_dst_pairs.numel() // 2), hkv, d,
+        int(kv_dtype), _stream(stream))
+    _check(st, "pa_swap_blocks")
 
 
 def pa_paged_attention_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, split_tokens) -> int:
@@ -232,3 +279,68 @@ def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_
 def pa_get_device_error(stream=None) -> int:
     """Synchronise the stream; return PA_EDEVICE_OOB (and clear it) if a kernel flagged a bad index."""
     return int(lib().pa_get_device_error(_stream(stream)))
+
+
+# ------------------------------------------------------------------------------ host block manager
+# Same names as the C entry points; `bm` is the opaque handle pa_bm_create returns.
+
+def pa_bm_create(num_blocks: int, shuffle_seed: int = 0):
+    h = lib().pa_bm_create(int(num_blocks), int(shuffle_seed))
+    if not h:
+        raise PagedAttnError(PA_EINVAL, "pa_bm_create")
+    return h
+
+
+def pa_bm_destroy(bm):
+    lib().pa_bm_destroy(bm)
+
+
+def pa_bm_num_free(bm) -> int:
+    return int(lib().pa_bm_num_free(bm))
+
+
+def pa_bm_add(bm, seq_id: int):
+    _check(lib().pa_bm_add(bm, int(seq_id)), "pa_bm_add")
+
+
+def pa_bm_fork(bm, parent: int, child: int):
+    _check(lib().pa_bm_fork(bm, int(parent), int(child)), "pa_bm_fork")
+
+
+def pa_bm_append(bm, seq_id: int, n_tokens: int):
+    """Reserve slots for n_tokens new tokens.  Returns (slots int64 array, cow pair or None)."""
+    import numpy as np
+    slots = np.zeros(max(1, n_tokens), np.int64)
+    pair = np.zeros(2, np.int32)
+    ncow = ctypes.c_int32(0)
+    st = lib().pa_bm_append(bm, int(seq_id), int(n_tokens), slots.ctypes.data_as(ctypes.c_void_p),
+                            pair.ctypes.data_as(ctypes.c_void_p), ctypes.byref(ncow))
+    _check(st, "pa_bm_append")
+    return slots[:n_tokens], (pair.copy() if ncow.value else None)
+
+
+def pa_bm_free(bm, seq_id: int):
+    _check(lib().pa_bm_free(bm, int(seq_id)), "pa_bm_free")
+
+
+def pa_bm_length(bm, seq_id: int) -> int:
+    return int(lib().pa_bm_length(bm, int(seq_id)))
+
+
+def pa_bm_tables(bm, seq_ids, max_blocks_per_seq: int):
+    """Block tables int32 [n][max_blocks_per_seq] (-1 padded) and lengths int32 [n] of seq_ids."""
+    import numpy as np
+    ids = np.ascontiguousarray(seq_ids, np.int64)
+    tables = np.empty((ids.shape[0], max_blocks_per_seq), np.int32)
+    lens = np.empty(ids.shape[0], np.int32)
+    st = lib().pa_bm_tables(bm, ids.ctypes.data_as(ctypes.c_void_p), ids.shape[0],
+                            tables.ctypes.data_as(ctypes.c_void_p), int(max_blocks_per_seq),
+                            lens.ctypes.data_as(ctypes.c_void_p))
+    _check(st, "pa_bm_tables")
+    return tables, lens
+
+
+def pa_bm_stats(bm) -> dict:
+    v = [ctypes.c_int64(0) for _ in range(4)]
+    _check(lib().pa_bm_stats(bm, *[ctypes.byref(x) for x in v]), "pa_bm_stats")
+    return dict(tokens_stored=v[0].value, blocks_used=v[1].value, blocks_shared=v[2].value, cow_copies=v[3].value)

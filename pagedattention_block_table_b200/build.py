@@ -20,7 +20,7 @@ NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", 
 
 def _sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))
-                  + [os.path.join(ROOT, "include", "pagedattn.h")])
+                  + glob.glob(os.path.join(CSRC, "*.cpp")) + [os.path.join(ROOT, "include", "pagedattn.h")])
 
 
 def source_digest() -> str:
@@ -46,7 +46,10 @@ def build(force: bool = False, out: str = LIB, extra=()) -> str:
         t = os.path.getmtime(out)
         if all(os.path.getmtime(s) <= t for s in _sources()) and not extra:
             return out
-    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", out + ".tmp", os.path.join(CSRC, "api.cu")]
+    # the CUDA side is one translation unit (api.cu includes every kernel header); the host-only
+    # block manager is a separate C++ file
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-o", out + ".tmp", os.path.join(CSRC, "api.cu"),
+           os.path.join(CSRC, "block_manager.cpp")]
     subprocess.run(cmd, check=True)
     os.replace(out + ".tmp", out)
     return out

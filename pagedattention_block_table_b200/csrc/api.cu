@@ -87,6 +87,7 @@ int decode_smem_rt(int kt, int d, int qpb) {
   if (kt == KT && d == D && qpb == Q) return decode_smem<KT, D, Q>();
   PA_SM(0, 64, 1) PA_SM(0, 64, 2) PA_SM(0, 64, 4) PA_SM(0, 128, 1) PA_SM(0, 128, 2) PA_SM(0, 128, 4)
   PA_SM(1, 64, 1) PA_SM(1, 64, 2) PA_SM(1, 64, 4) PA_SM(1, 128, 1) PA_SM(1, 128, 2) PA_SM(1, 128, 4)
+  PA_SM(2, 64, 1) PA_SM(2, 64, 2) PA_SM(2, 64, 4) PA_SM(2, 128, 1) PA_SM(2, 128, 2) PA_SM(2, 128, 4)
 #undef PA_SM
   return 0;
 }
@@ -98,7 +99,7 @@ pa_status launch_decode(const pa::DecodeParams &P, dim3 grid, cudaStream_t st) {
   auto kern = pa::paged_decode_kernel<KT, D, QPB, PA_DEC_NW, S>;
   pa_status s = set_smem(kern, C::SMEM);
   if (s != PA_OK) return s;
-  kern<<<grid, PA_DEC_NW * 32, C::SMEM, st>>>(P);
+  if (pa::launch_pdl(kern, grid, dim3(PA_DEC_NW * 32), C::SMEM, st, P) != cudaSuccess) return launch_status();
   return launch_status();
 }
 
@@ -107,6 +108,7 @@ pa_status dispatch_decode(int kt, int d, int qpb, const pa::DecodeParams &P, dim
   if (kt == KT && d == D && qpb == Q) return launch_decode<KT, D, Q>(P, grid, st);
   PA_DD(0, 64, 1) PA_DD(0, 64, 2) PA_DD(0, 64, 4) PA_DD(0, 128, 1) PA_DD(0, 128, 2) PA_DD(0, 128, 4)
   PA_DD(1, 64, 1) PA_DD(1, 64, 2) PA_DD(1, 64, 4) PA_DD(1, 128, 1) PA_DD(1, 128, 2) PA_DD(1, 128, 4)
+  PA_DD(2, 64, 1) PA_DD(2, 64, 2) PA_DD(2, 64, 4) PA_DD(2, 128, 1) PA_DD(2, 128, 2) PA_DD(2, 128, 4)
 #undef PA_DD
   return PA_EUNSUPPORTED;
 }
@@ -127,6 +129,7 @@ const char *pa_status_string(pa_status s) {
     case PA_ECUDA: return "CUDA error";
     case PA_EDEVICE_OOB: return "device-side out-of-range block id, slot or length";
     case PA_EWORKSPACE: return "workspace missing or too small";
+    case PA_ENOMEM: return "not enough free blocks";
     default: return "unknown status";
   }
 }
@@ -153,12 +156,12 @@ pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *
                        pa_stream_t stream) {
   if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_EINVAL;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
-  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
   if (num_tokens == 0) return PA_OK;
   if (!k_cache || !v_cache || !k || !v || !slot_mapping) return PA_EINVAL;
   if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k) || !aligned16(v) || !aligned16(slot_mapping))
     return PA_EINVAL;
-  if (kv_dtype == PA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return PA_EINVAL;
+  if (kv_dtype != PA_KV_BF16 && (!k_scale || !v_scale)) return PA_EINVAL;
   if (num_blocks > (int64_t(1) << 40)) return PA_EINVAL;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int chunks = head_dim / 8;  // 8 elements per thread
@@ -167,14 +170,14 @@ pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *
   const int64_t want = ceil_div64(total, threads);
   const int grid = static_cast<int>(want < 65536 ? want : 65536);
   if (kv_dtype == PA_KV_BF16) {
-    pa::kv_append_bf16_kernel<<<grid, threads, 0, st>>>(
-        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), static_cast<const uint4 *>(k),
-        static_cast<const uint4 *>(v), slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock);
+    pa::launch_pdl(pa::kv_append_bf16_kernel, dim3(grid), dim3(threads), 0, st, static_cast<uint4 *>(k_cache),
+                   static_cast<uint4 *>(v_cache), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+                   slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock);
   } else {
-    pa::kv_append_fp8_kernel<<<grid, threads, 0, st>>>(
-        static_cast<uint2 *>(k_cache), static_cast<uint2 *>(v_cache), static_cast<const uint4 *>(k),
-        static_cast<const uint4 *>(v), slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock,
-        k_scale, v_scale);
+    auto kern = kv_dtype == PA_KV_FP8_E4M3 ? pa::kv_append_fp8_kernel<1> : pa::kv_append_fp8_kernel<2>;
+    pa::launch_pdl(kern, dim3(grid), dim3(threads), 0, st, static_cast<uint2 *>(k_cache),
+                   static_cast<uint2 *>(v_cache), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+                   slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock, k_scale, v_scale);
   }
   return launch_status();
 }
@@ -183,7 +186,7 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pa
                          int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype, pa_stream_t stream) {
   if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_EINVAL;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
-  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
   if (num_pairs == 0) return PA_OK;
   if (num_pairs > 65535) return PA_EINVAL;
   if (!k_cache || !v_cache || !src_dst_pairs) return PA_EINVAL;
@@ -193,8 +196,52 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pa
   const int threads = 256;
   const int64_t gx = ceil_div64(vecs, threads);
   dim3 grid(static_cast<unsigned>(gx < 64 ? gx : 64), static_cast<unsigned>(num_pairs));
-  pa::copy_blocks_kernel<<<grid, threads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), src_dst_pairs, vecs, num_blocks);
+  pa::launch_pdl(pa::copy_blocks_kernel, grid, dim3(threads), 0, reinterpret_cast<cudaStream_t>(stream),
+                 static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), src_dst_pairs, vecs, num_blocks);
+  return launch_status();
+}
+
+// A pointer the device can dereference: device memory, managed memory, or host memory that is
+// pinned and mapped (its device-side address is returned).  Pageable host memory is rejected.
+static bool device_accessible(const void *p, void **dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+    *dev = const_cast<void *>(p);
+    return true;
+  }
+  if (a.type == cudaMemoryTypeHost && a.devicePointer != nullptr) {
+    *dev = a.devicePointer;
+    return true;
+  }
+  return false;
+}
+
+pa_status pa_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const void *src_k, const void *src_v,
+                         int64_t src_num_blocks, const int32_t *src_dst_pairs, int num_pairs, int num_kv_heads,
+                         int head_dim, int kv_dtype, pa_stream_t stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || dst_num_blocks <= 0 || src_num_blocks <= 0) return PA_EINVAL;
+  if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (num_pairs > 65535) return PA_EINVAL;
+  if (!dst_k || !dst_v || !src_k || !src_v || !src_dst_pairs) return PA_EINVAL;
+  void *dk, *dv, *sk, *sv, *pr;
+  if (!device_accessible(dst_k, &dk) || !device_accessible(dst_v, &dv) || !device_accessible(src_k, &sk) ||
+      !device_accessible(src_v, &sv) || !device_accessible(src_dst_pairs, &pr))
+    return PA_EINVAL;
+  if (!aligned16(dk) || !aligned16(dv) || !aligned16(sk) || !aligned16(sv)) return PA_EINVAL;
+  const int elem = kv_dtype == PA_KV_BF16 ? 2 : 1;
+  const int64_t vecs = (int64_t)num_kv_heads * pa::kBlock * head_dim * elem / 16;
+  const int threads = 256;
+  const int64_t gx = ceil_div64(vecs, threads * 4);
+  dim3 grid(static_cast<unsigned>(gx < 16 ? gx : 16), static_cast<unsigned>(num_pairs));
+  pa::launch_pdl(pa::swap_blocks_kernel, grid, dim3(threads), 0, reinterpret_cast<cudaStream_t>(stream),
+                 static_cast<uint4 *>(dk), static_cast<uint4 *>(dv), dst_num_blocks, static_cast<const uint4 *>(sk),
+                 static_cast<const uint4 *>(sv), src_num_blocks, static_cast<const int32_t *>(pr), vecs);
   return launch_status();
 }
 
@@ -234,14 +281,14 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
     return PA_EINVAL;
   if (num_q_heads % num_kv_heads != 0) return PA_EINVAL;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
-  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3) return PA_EUNSUPPORTED;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
   if (max_context_len < 0 || split_tokens < 0 || split_tokens % pa::kBlock != 0) return PA_EINVAL;
   if (!(scale == scale) || isinf(scale)) return PA_EINVAL;
   if (num_seqs == 0) return PA_OK;
   if (num_seqs > 65535) return PA_EINVAL;
   if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens) return PA_EINVAL;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
-  if (kv_dtype == PA_KV_FP8_E4M3 && (!k_scale || !v_scale)) return PA_EINVAL;
+  if (kv_dtype != PA_KV_BF16 && (!k_scale || !v_scale)) return PA_EINVAL;
   const int group = num_q_heads / num_kv_heads;
   const int qpb = queries_per_cta(group);
   if ((int64_t)num_kv_heads * (group / qpb) > 65535) return PA_EINVAL;
@@ -284,9 +331,9 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
   if (s != PA_OK || max_splits <= 1) return s;
   dim3 rgrid(static_cast<unsigned>((num_q_heads + 3) / 4), static_cast<unsigned>(num_seqs));
   if (head_dim == 128)
-    pa::lse_reduce_kernel<128><<<rgrid, 128, 0, st>>>(P);
+    pa::launch_pdl(pa::lse_reduce_kernel<128>, rgrid, dim3(128), 0, st, P);
   else
-    pa::lse_reduce_kernel<64><<<rgrid, 128, 0, st>>>(P);
+    pa::launch_pdl(pa::lse_reduce_kernel<64>, rgrid, dim3(128), 0, st, P);
   return launch_status();
 }
 

@@ -1,0 +1,202 @@
+// block_manager.cpp -- host-side manager of the paged KV pool (the control plane that feeds the
+// kernels' block tables, slot mappings and copy-on-write pairs).  Plain C++, no device code.
+//
+// Pages followed:
+//   Core Concepts §3.2 ("PagedAttention 如何工作"): blocks are handed out on demand; each decode
+//     step writes the new token at the end of the sequence's current block and takes a new
+//     physical block from the pool when that block is full.  The batch size is bounded by the
+//     number of free blocks, not by a per-request maximum length.
+//   vLLM overview, section 二 "Prefix Sharing": requests with a common prefix share its physical
+//     pages; when a request writes after the shared part, the page it writes into is copied first
+//     (copy-on-write) so the shared page stays unchanged for the others.  Also used for parallel
+//     sampling (a fork shares every page of its parent).
+//   vLLM overview, section "Continuous Batching": finished requests leave the batch and their pages
+//     return to the pool at once.
+//
+// Structure: a free list (FIFO; optionally shuffled once with a seeded generator, so that physical
+// placement is scattered as in a long-running server), a reference count per block, and per
+// sequence its block table and length.  All functions are O(blocks touched).
+#include <stdint.h>
+#include <string.h>
+
+#include <deque>
+#include <new>
+#include <random>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/pagedattn.h"
+
+namespace {
+
+struct Seq {
+  std::vector<int32_t> blocks;  // logical block i -> physical block
+  int64_t len = 0;              // tokens written
+};
+
+}  // namespace
+
+struct pa_block_manager {
+  int64_t num_blocks = 0;
+  std::deque<int32_t> free_list;
+  std::vector<int32_t> refcount;
+  std::unordered_map<int64_t, Seq> seqs;
+  int64_t forks = 0;  // copy-on-write copies handed out so far
+};
+
+namespace {
+
+int32_t take_block(pa_block_manager *bm) {
+  const int32_t b = bm->free_list.front();
+  bm->free_list.pop_front();
+  bm->refcount[b] = 1;
+  return b;
+}
+
+void release_block(pa_block_manager *bm, int32_t b) {
+  if (--bm->refcount[b] == 0) bm->free_list.push_back(b);
+}
+
+}  // namespace
+
+extern "C" {
+
+pa_block_manager *pa_bm_create(int64_t num_blocks, uint64_t shuffle_seed) {
+  if (num_blocks <= 0 || num_blocks > INT32_MAX) return nullptr;
+  pa_block_manager *bm = new (std::nothrow) pa_block_manager();
+  if (!bm) return nullptr;
+  bm->num_blocks = num_blocks;
+  std::vector<int32_t> order(static_cast<size_t>(num_blocks));
+  for (int64_t i = 0; i < num_blocks; ++i) order[i] = static_cast<int32_t>(i);
+  if (shuffle_seed != 0) {
+    std::mt19937_64 rng(shuffle_seed);
+    for (int64_t i = num_blocks - 1; i > 0; --i) {
+      std::uniform_int_distribution<int64_t> pick(0, i);
+      std::swap(order[i], order[pick(rng)]);
+    }
+  }
+  bm->free_list.assign(order.begin(), order.end());
+  bm->refcount.assign(static_cast<size_t>(num_blocks), 0);
+  return bm;
+}
+
+void pa_bm_destroy(pa_block_manager *bm) { delete bm; }
+
+int64_t pa_bm_num_free(const pa_block_manager *bm) { return bm ? static_cast<int64_t>(bm->free_list.size()) : -1; }
+
+pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id) {
+  if (!bm) return PA_EINVAL;
+  if (bm->seqs.count(seq_id)) return PA_EINVAL;
+  bm->seqs.emplace(seq_id, Seq());
+  return PA_OK;
+}
+
+pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent, int64_t child) {
+  if (!bm) return PA_EINVAL;
+  auto it = bm->seqs.find(parent);
+  if (it == bm->seqs.end() || bm->seqs.count(child)) return PA_EINVAL;
+  Seq c = it->second;  // same physical blocks, same length
+  for (int32_t b : c.blocks) ++bm->refcount[b];
+  bm->seqs.emplace(child, std::move(c));
+  return PA_OK;
+}
+
+pa_status pa_bm_append(pa_block_manager *bm, int64_t seq_id, int32_t n_tokens, int64_t *slots_out,
+                       int32_t *cow_pairs_out, int32_t *num_cow_out) {
+  if (!bm || n_tokens < 0 || (n_tokens > 0 && !slots_out) || !num_cow_out) return PA_EINVAL;
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return PA_EINVAL;
+  Seq &s = it->second;
+  *num_cow_out = 0;
+  if (n_tokens == 0) return PA_OK;
+  // blocks this append needs: new blocks past the table, plus one copy if the current last block
+  // is shared and gets written
+  const int64_t first = s.len, last = s.len + n_tokens - 1;
+  const int64_t have = static_cast<int64_t>(s.blocks.size());
+  const int64_t need_blocks = last / PA_BLOCK_SIZE + 1;
+  int64_t needed = need_blocks > have ? need_blocks - have : 0;
+  const int64_t first_blk = first / PA_BLOCK_SIZE;
+  const bool cow = first_blk < have && bm->refcount[s.blocks[first_blk]] > 1;
+  if (cow) {
+    if (!cow_pairs_out) return PA_EINVAL;
+    ++needed;
+  }
+  if (needed > static_cast<int64_t>(bm->free_list.size())) return PA_ENOMEM;  // nothing changed
+  if (cow) {
+    const int32_t src = s.blocks[first_blk];
+    const int32_t dst = take_block(bm);
+    --bm->refcount[src];
+    s.blocks[first_blk] = dst;
+    cow_pairs_out[0] = src;
+    cow_pairs_out[1] = dst;
+    *num_cow_out = 1;
+    ++bm->forks;
+  }
+  while (static_cast<int64_t>(s.blocks.size()) < need_blocks) s.blocks.push_back(take_block(bm));
+  for (int64_t t = first; t <= last; ++t)
+    slots_out[t - first] = static_cast<int64_t>(s.blocks[t / PA_BLOCK_SIZE]) * PA_BLOCK_SIZE + t % PA_BLOCK_SIZE;
+  s.len = last + 1;
+  return PA_OK;
+}
+
+pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
+  if (!bm) return PA_EINVAL;
+  auto it = bm->seqs.find(seq_id);
+  if (it == bm->seqs.end()) return PA_EINVAL;
+  for (int32_t b : it->second.blocks) release_block(bm, b);
+  bm->seqs.erase(it);
+  return PA_OK;
+}
+
+int64_t pa_bm_length(const pa_block_manager *bm, int64_t seq_id) {
+  if (!bm) return -1;
+  auto it = bm->seqs.find(seq_id);
+  return it == bm->seqs.end() ? -1 : it->second.len;
+}
+
+pa_status pa_bm_tables(const pa_block_manager *bm, const int64_t *seq_ids, int32_t n, int32_t *tables_out,
+                       int32_t max_blocks_per_seq, int32_t *lens_out) {
+  if (!bm || n < 0 || (n > 0 && (!seq_ids || !tables_out || !lens_out)) || max_blocks_per_seq <= 0) return PA_EINVAL;
+  for (int32_t i = 0; i < n; ++i) {
+    auto it = bm->seqs.find(seq_ids[i]);
+    if (it == bm->seqs.end()) return PA_EINVAL;
+    if (static_cast<int64_t>(it->second.blocks.size()) > max_blocks_per_seq) return PA_EINVAL;
+  }
+  for (int32_t i = 0; i < n; ++i) {
+    const Seq &s = bm->seqs.find(seq_ids[i])->second;
+    int32_t *row = tables_out + static_cast<int64_t>(i) * max_blocks_per_seq;
+    const size_t nb = s.blocks.size();
+    if (nb) memcpy(row, s.blocks.data(), nb * sizeof(int32_t));
+    for (int32_t k = static_cast<int32_t>(nb); k < max_blocks_per_seq; ++k) row[k] = -1;
+    lens_out[i] = static_cast<int32_t>(s.len);
+  }
+  return PA_OK;
+}
+
+pa_status pa_bm_stats(const pa_block_manager *bm, int64_t *tokens_stored, int64_t *blocks_used,
+                      int64_t *blocks_shared, int64_t *cow_copies) {
+  if (!bm) return PA_EINVAL;
+  int64_t used = 0, shared = 0, toks = 0;
+  for (int32_t rc : bm->refcount) {
+    used += rc > 0;
+    shared += rc > 1;
+  }
+  // tokens held by the pool: per physical block the largest fill any of its holders reached
+  std::vector<int32_t> fill(static_cast<size_t>(bm->num_blocks), 0);
+  for (const auto &kv : bm->seqs) {
+    const Seq &s = kv.second;
+    for (size_t i = 0; i < s.blocks.size(); ++i) {
+      const int64_t f = s.len - static_cast<int64_t>(i) * PA_BLOCK_SIZE;
+      const int32_t fi = static_cast<int32_t>(f > PA_BLOCK_SIZE ? PA_BLOCK_SIZE : (f < 0 ? 0 : f));
+      if (fi > fill[s.blocks[i]]) fill[s.blocks[i]] = fi;
+    }
+  }
+  for (int32_t f : fill) toks += f;
+  if (tokens_stored) *tokens_stored = toks;
+  if (blocks_used) *blocks_used = used;
+  if (blocks_shared) *blocks_shared = shared;
+  if (cow_copies) *cow_copies = bm->forks;
+  return PA_OK;
+}
+
+}  // extern "C"

@@ -56,7 +56,7 @@ struct DecodeCfg {
   static constexpr int LPV = D / 8;                  // lanes per V row in PV (8 elements each)
   static constexpr int RPL = 32 / LPV;               // V rows per PV step
   static constexpr int NU = kBlock / RPL;            // PV steps per block
-  static constexpr int P_BYTES = kBlock * QPB * 4;
+  static constexpr int P_BYTES = kBlock * QPB * 8;    // p as duplicated pairs (p, p)
   static constexpr int A_BYTES = 16;                 // alpha[QPB], padded
   static constexpr int BAR_BYTES = STAGES * 8;
   static constexpr int WARP_BYTES = ((2 * STAGES * TILE + P_BYTES + A_BYTES + BAR_BYTES) + 127) / 128 * 128;
@@ -129,7 +129,10 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     }
   }
   const int n_splits = (L + P.split_tokens - 1) / P.split_tokens;
-  if (split >= (n_splits > 1 ? n_splits : 1)) return;
+  if (split >= (n_splits > 1 ? n_splits : 1)) {
+    griddep_wait();  // keep "this grid done" meaning "the kernel before it done" for the next kernel
+    return;
+  }
   const bool final_out = n_splits <= 1;
   const int t0 = split * P.split_tokens;
   const int t1 = min(L, t0 + P.split_tokens);
@@ -137,8 +140,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   const int blk0 = t0 / kBlock;
 
   uint8_t *wbase = smem + warp * C::WARP_BYTES;
-  float *p_s = reinterpret_cast<float *>(wbase + 2 * STAGES * C::TILE);
-  float *alpha_s = p_s + kBlock * QPB;
+  uint64_t *p_s = reinterpret_cast<uint64_t *>(wbase + 2 * STAGES * C::TILE);
+  float *alpha_s = reinterpret_cast<float *>(p_s + kBlock * QPB);
   uint64_t *bars = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(alpha_s) + C::A_BYTES);
 
   const int nwb = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;  // blocks of this warp
@@ -150,10 +153,10 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 
   // ---- query registers: the dims this lane multiplies in QK, pre-scaled
   const int r = lane / C::LPT, j = lane % C::LPT;
-  float qf[QPB][C::DPL];
+  uint64_t qf2[QPB][C::DPL / 2];  // packed (even, odd) dim pairs, pre-scaled
   {
     float qs = P.qscale;
-    if (KT == 1) qs *= P.k_scale[g];
+    if (KT != 0) qs *= P.k_scale[g];
 #pragma unroll
     for (int qi = 0; qi < QPB; ++qi) {
       const __nv_bfloat16 *qrow = P.q + ((int64_t)b * P.num_q_heads + h0 + qi) * D;
@@ -165,10 +168,8 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
           const uint4 w = *reinterpret_cast<const uint4 *>(qrow + d0 + e8);
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            qf[qi][k * C::CE + e8 + 2 * t] = bf16lo(ww[t]) * qs;
-            qf[qi][k * C::CE + e8 + 2 * t + 1] = bf16hi(ww[t]) * qs;
-          }
+          for (int t = 0; t < 4; ++t)
+            qf2[qi][(k * C::CE + e8) / 2 + t] = f2pack(bf16lo(ww[t]) * qs, bf16hi(ww[t]) * qs);
         }
       }
     }
@@ -191,6 +192,10 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   };
   int tw = load_window(0);
   const uint64_t pol = l2_evict_first_policy();
+  // everything above reads only caller inputs; the cache may still be being written by the
+  // kernel before this one on the stream (the append), so wait for it here
+  griddep_wait();
+  griddep_launch();
   const int64_t head_stride = (int64_t)C::TILE;
   auto issue = [&](int i) {  // warp-uniform call
     if (i >= nwb) return;
@@ -207,11 +212,11 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 
   // ---- running state: this lane's query qsel (m, l); o[q][8 dims] for all queries
   float m_run = -INFINITY, l_run = 0.f;
-  float o[QPB][8];
+  uint64_t o2[QPB][4];  // packed pairs of this lane's 8 output dims, per query
 #pragma unroll
   for (int qi = 0; qi < QPB; ++qi)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) o[qi][e] = 0.f;
+    for (int e = 0; e < 4; ++e) o2[qi][e] = 0ull;
 
   const int c = lane % C::LPV, hv = lane / C::LPV;
   int issued = 0;
@@ -235,9 +240,9 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 #pragma unroll
     for (int pp = 0; pp < C::NP; ++pp) {
       const int t = pp * C::TPP + r;
-      float acc[QPB];
+      uint64_t acc2[QPB];
 #pragma unroll
-      for (int qi = 0; qi < QPB; ++qi) acc[qi] = 0.f;
+      for (int qi = 0; qi < QPB; ++qi) acc2[qi] = 0ull;
 #pragma unroll
       for (int k = 0; k < C::CPL; ++k) {
         const uint4 raw = *reinterpret_cast<const uint4 *>(Kt + t * C::RB + (k * C::LPT + j) * 16);
@@ -245,27 +250,28 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
         if constexpr (KT == 0) {
 #pragma unroll
           for (int t2 = 0; t2 < 4; ++t2) {
-            const float lo = bf16lo(ww[t2]), hi = bf16hi(ww[t2]);
+            const uint64_t kv2 = bf16x2_to_f2(ww[t2]);
 #pragma unroll
-            for (int qi = 0; qi < QPB; ++qi) {
-              acc[qi] = fmaf(qf[qi][k * C::CE + 2 * t2], lo, acc[qi]);
-              acc[qi] = fmaf(qf[qi][k * C::CE + 2 * t2 + 1], hi, acc[qi]);
-            }
+            for (int qi = 0; qi < QPB; ++qi) acc2[qi] = ffma2(qf2[qi][k * C::CE / 2 + t2], kv2, acc2[qi]);
           }
         } else {
 #pragma unroll
           for (int t2 = 0; t2 < 4; ++t2) {
-            const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] & 0xffffu));
-            const float2 bq = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] >> 16));
+            uint64_t a2, b2;
+            bytes4_to_f2<KT>(ww[t2], a2, b2);
 #pragma unroll
             for (int qi = 0; qi < QPB; ++qi) {
-              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 0], a.x, acc[qi]);
-              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 1], a.y, acc[qi]);
-              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 2], bq.x, acc[qi]);
-              acc[qi] = fmaf(qf[qi][k * C::CE + 4 * t2 + 3], bq.y, acc[qi]);
+              acc2[qi] = ffma2(qf2[qi][k * C::CE / 2 + 2 * t2], a2, acc2[qi]);
+              acc2[qi] = ffma2(qf2[qi][k * C::CE / 2 + 2 * t2 + 1], b2, acc2[qi]);
             }
           }
         }
+      }
+      float acc[QPB];
+#pragma unroll
+      for (int qi = 0; qi < QPB; ++qi) {
+        const float2 a = f2unpack(acc2[qi]);
+        acc[qi] = a.x + a.y;
       }
       const float sv = group_reduce_scatter<QPB, C::LPT>(acc, lane);
       sc[pp] = t < nvalid ? sv : -INFINITY;
@@ -284,7 +290,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     for (int pp = 0; pp < C::NP; ++pp) {
       const float pv = exp2f(sc[pp] - m_new);
       ps += pv;
-      p_s[(pp * C::TPP + r) * QPB + qsel] = pv;
+      p_s[(pp * C::TPP + r) * QPB + qsel] = f2pack(pv, pv);
     }
 #pragma unroll
     for (int off = C::LPT; off < 32; off <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
@@ -297,42 +303,34 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 #pragma unroll
     for (int qi = 0; qi < QPB; ++qi) {
       const float a = alpha_s[qi];
+      const uint64_t a2 = f2pack(a, a);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[qi][e] *= a;
+      for (int e = 0; e < 4; ++e) o2[qi][e] = fmul2(o2[qi][e], a2);
     }
 #pragma unroll
     for (int u = 0; u < C::NU; ++u) {
       const int t = u * C::RPL + hv;
       if (t < nvalid) {
-        float v[8];
+        uint64_t v2[4];
         if constexpr (KT == 0) {
           const uint4 raw = *reinterpret_cast<const uint4 *>(Vt + t * C::RB + c * 16);
-          const uint32_t ww[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-          for (int t2 = 0; t2 < 4; ++t2) {
-            v[2 * t2] = bf16lo(ww[t2]);
-            v[2 * t2 + 1] = bf16hi(ww[t2]);
-          }
+          v2[0] = bf16x2_to_f2(raw.x);
+          v2[1] = bf16x2_to_f2(raw.y);
+          v2[2] = bf16x2_to_f2(raw.z);
+          v2[3] = bf16x2_to_f2(raw.w);
         } else {
           const uint2 raw = *reinterpret_cast<const uint2 *>(Vt + t * C::RB + c * 8);
-          const uint32_t ww[2] = {raw.x, raw.y};
-#pragma unroll
-          for (int t2 = 0; t2 < 2; ++t2) {
-            const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] & 0xffffu));
-            const float2 bq = e4m3x2_to_float2(static_cast<uint16_t>(ww[t2] >> 16));
-            v[4 * t2 + 0] = a.x;
-            v[4 * t2 + 1] = a.y;
-            v[4 * t2 + 2] = bq.x;
-            v[4 * t2 + 3] = bq.y;
-          }
+          bytes4_to_f2<KT>(raw.x, v2[0], v2[1]);
+          bytes4_to_f2<KT>(raw.y, v2[2], v2[3]);
         }
-        float pq[QPB];
-        if constexpr (QPB == 4) {
-          const float4 p4 = *reinterpret_cast<const float4 *>(p_s + t * QPB);
-          pq[0] = p4.x;
-          pq[1] = p4.y;
-          pq[2] = p4.z;
-          pq[3] = p4.w;
+        uint64_t pq[QPB];
+        if constexpr (QPB % 2 == 0) {
+#pragma unroll
+          for (int qi = 0; qi < QPB; qi += 2) {
+            const ulonglong2 pp2 = *reinterpret_cast<const ulonglong2 *>(p_s + t * QPB + qi);
+            pq[qi] = pp2.x;
+            pq[qi + 1] = pp2.y;
+          }
         } else {
 #pragma unroll
           for (int qi = 0; qi < QPB; ++qi) pq[qi] = p_s[t * QPB + qi];
@@ -340,7 +338,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 #pragma unroll
         for (int qi = 0; qi < QPB; ++qi)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) o[qi][e] = fmaf(pq[qi], v[e], o[qi][e]);
+          for (int e = 0; e < 4; ++e) o2[qi][e] = ffma2(pq[qi], v2[e], o2[qi][e]);
       }
     }
     __syncwarp();
@@ -355,8 +353,17 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 #pragma unroll
     for (int qi = 0; qi < QPB; ++qi)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) o[qi][e] = 0.f;
+      for (int e = 0; e < 4; ++e) o2[qi][e] = 0ull;
   }
+  float o[QPB][8];
+#pragma unroll
+  for (int qi = 0; qi < QPB; ++qi)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 v = f2unpack(o2[qi][e]);
+      o[qi][2 * e] = v.x;
+      o[qi][2 * e + 1] = v.y;
+    }
 
   // ---- merge the RPL token-parity lane groups, then the warps
 #pragma unroll
@@ -379,7 +386,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   }
   __syncthreads();
 
-  const float vs = KT == 1 ? P.v_scale[g] : 1.f;
+  const float vs = KT != 0 ? P.v_scale[g] : 1.f;
   for (int idx = threadIdx.x; idx < QPB * D; idx += NW * 32) {
     const int qi = idx / D, d = idx % D;
     float M = -INFINITY;
@@ -413,12 +420,15 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 
 // Combine the split partials of every (sequence, query head) whose context spans more than one
 // split: out = sum_p 2^(m_p - M) o_p / sum_p 2^(m_p - M) l_p,  M = max_p m_p.
-// One warp per (sequence, query head); lane owns D/32 dims.
+// One warp per (sequence, query head): lane p holds split p's (m, l) so the max and the weights come
+// from one round of independent loads and shuffles; then every lane sums its D/32 output dims over
+// the splits with independent vector loads.
 template <int D>
 __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
   const int h = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
+  griddep_wait();  // partials come from the decode kernel just before this one
   if (h >= P.num_q_heads) return;
   int L = P.context_lens[b];
   const int lim = min(P.max_blocks_per_seq * kBlock, P.max_context_len);
@@ -426,32 +436,49 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
   const int n = (L + P.split_tokens - 1) / P.split_tokens;
   if (n <= 1) return;  // written directly by the decode kernel
   const int64_t row0 = ((int64_t)b * P.num_q_heads + h) * P.max_splits;
-  float M = -INFINITY;
-  for (int p = 0; p < n; ++p) M = fmaxf(M, P.ws_ml[(row0 + p) * 2]);
   constexpr int DPL = D / 32;
   float acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
   float den = 0.f;
-  for (int p = 0; p < n; ++p) {
-    const float w = M == -INFINITY ? 0.f : exp2f(P.ws_ml[(row0 + p) * 2] - M);
-    den += w * P.ws_ml[(row0 + p) * 2 + 1];
-    const float *op = P.ws_o + (row0 + p) * D + lane * DPL;
-    if constexpr (DPL == 4) {
-      const float4 v = *reinterpret_cast<const float4 *>(op);
-      acc[0] += w * v.x;
-      acc[1] += w * v.y;
-      acc[2] += w * v.z;
-      acc[3] += w * v.w;
-    } else {
+  // global max over all splits first (n may exceed 32)
+  float M = -INFINITY;
+  for (int p = lane; p < n; p += 32) M = fmaxf(M, P.ws_ml[(row0 + p) * 2]);
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] += w * op[e];
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  for (int p0 = 0; p0 < n; p0 += 32) {
+    const int p = p0 + lane;
+    float w = 0.f, lw = 0.f;
+    if (p < n && M != -INFINITY) {
+      w = exp2f(P.ws_ml[(row0 + p) * 2] - M);
+      lw = w * P.ws_ml[(row0 + p) * 2 + 1];
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+    den += lw;
+    const int cnt = min(32, n - p0);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float *op = P.ws_o + (row0 + p0 + k) * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(op);
+        acc[0] = fmaf(wk, v.x, acc[0]);
+        acc[1] = fmaf(wk, v.y, acc[1]);
+        acc[2] = fmaf(wk, v.z, acc[2]);
+        acc[3] = fmaf(wk, v.w, acc[3]);
+      } else {
+        const float2 v = *reinterpret_cast<const float2 *>(op);
+        acc[0] = fmaf(wk, v.x, acc[0]);
+        acc[1] = fmaf(wk, v.y, acc[1]);
+      }
     }
   }
   const float inv = den > 0.f ? 1.f / den : 0.f;
   __nv_bfloat16 *orow = P.out + ((int64_t)b * P.num_q_heads + h) * D + lane * DPL;
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) orow[e] = __float2bfloat16_rn(acc[e] * inv);
+  for (int e = 0; e < DPL; e += 2)
+    *reinterpret_cast<__nv_bfloat162 *>(orow + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
 }
 
 }  // namespace pa

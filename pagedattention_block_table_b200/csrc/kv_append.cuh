@@ -17,6 +17,8 @@ __global__ void kv_append_bf16_kernel(uint4 *__restrict__ k_cache, uint4 *__rest
                                       const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                       const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
                                       int num_kv_heads, int chunks_per_row, int64_t num_slots) {
+  griddep_wait();  // the cache may still be read by the kernel before this one (a decode)
+  griddep_launch();
   const int64_t total = num_tokens * num_kv_heads * chunks_per_row;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -39,7 +41,7 @@ __global__ void kv_append_bf16_kernel(uint4 *__restrict__ k_cache, uint4 *__rest
   }
 }
 
-// FP8 E4M3 variant: one thread = 8 elements.  code = E4M3_rn_satfinite(x / scale[h]), the
+// One-byte variants (FP8 E4M3: KT 1, INT8: KT 2): one thread = 8 elements.  code = E4M3_rn_satfinite(x / scale[h]), the
 // quotient an IEEE round-to-nearest binary32 division.
 __device__ __forceinline__ uint2 quant8(uint4 x, float s) {
   uint32_t w[4] = {x.x, x.y, x.z, x.w};
@@ -59,11 +61,30 @@ __device__ __forceinline__ uint2 quant8(uint4 x, float s) {
   return make_uint2(out[0], out[1]);
 }
 
+// INT8 variant: code = clamp(round-half-even(x / scale[h]), -127, 127), the quotient an IEEE
+// round-to-nearest binary32 division; a NaN quotient stores 0.
+__device__ __forceinline__ uint2 quant8_int8(uint4 x, float s) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t ww = w[e >> 1];
+    const float q = __fdiv_rn((e & 1) ? bf16hi(ww) : bf16lo(ww), s);
+    int c = q == q ? __float2int_rn(q) : 0;
+    c = c > 127 ? 127 : (c < -127 ? -127 : c);
+    out[e >> 2] |= (static_cast<uint32_t>(c) & 0xffu) << (8 * (e & 3));
+  }
+  return make_uint2(out[0], out[1]);
+}
+
+template <int KT>
 __global__ void kv_append_fp8_kernel(uint2 *__restrict__ k_cache, uint2 *__restrict__ v_cache,
                                      const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                      const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
                                      int num_kv_heads, int chunks_per_row, int64_t num_slots,
                                      const float *__restrict__ k_scale, const float *__restrict__ v_scale) {
+  griddep_wait();
+  griddep_launch();
   const int64_t total = num_tokens * num_kv_heads * chunks_per_row;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -79,8 +100,13 @@ __global__ void kv_append_fp8_kernel(uint2 *__restrict__ k_cache, uint2 *__restr
     }
     const int64_t blk = slot / kBlock, off = slot % kBlock;
     const int64_t dst = ((blk * num_kv_heads + h) * kBlock + off) * chunks_per_row + c;
-    k_cache[dst] = quant8(__ldcs(k + i), k_scale[h]);
-    v_cache[dst] = quant8(__ldcs(v + i), v_scale[h]);
+    if constexpr (KT == 1) {
+      k_cache[dst] = quant8(__ldcs(k + i), k_scale[h]);
+      v_cache[dst] = quant8(__ldcs(v + i), v_scale[h]);
+    } else {
+      k_cache[dst] = quant8_int8(__ldcs(k + i), k_scale[h]);
+      v_cache[dst] = quant8_int8(__ldcs(v + i), v_scale[h]);
+    }
   }
 }
 
@@ -88,6 +114,8 @@ __global__ void kv_append_fp8_kernel(uint2 *__restrict__ k_cache, uint2 *__restr
 __global__ void copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                                    const int32_t *__restrict__ pairs, int64_t vecs_per_block,
                                    int64_t num_blocks) {
+  griddep_wait();
+  griddep_launch();
   const int p = blockIdx.y;
   const int32_t src = pairs[2 * p], dst = pairs[2 * p + 1];
   if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
@@ -104,6 +132,48 @@ __global__ void copy_blocks_kernel(uint4 *__restrict__ k_cache, uint4 *__restric
     const uint4 b = vs[i];
     kd[i] = a;
     vd[i] = b;
+  }
+}
+
+// Swap (vLLM overview, section 三: pages move out to CPU memory when GPU memory runs short and come
+// back when needed): copy whole blocks between two pools, typically the device cache and a pinned
+// host pool mapped into the device's address space.  grid.y = pair; every thread keeps several
+// 16-byte loads in flight before storing, since host memory is microseconds away.
+__global__ void swap_blocks_kernel(uint4 *__restrict__ dst_k, uint4 *__restrict__ dst_v, int64_t dst_num_blocks,
+                                   const uint4 *__restrict__ src_k, const uint4 *__restrict__ src_v,
+                                   int64_t src_num_blocks, const int32_t *__restrict__ pairs, int64_t vecs_per_block) {
+  griddep_wait();
+  griddep_launch();
+  const int p = blockIdx.y;
+  const int32_t s = pairs[2 * p], d = pairs[2 * p + 1];
+  if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) flag_error(kErrBlockId);
+    return;
+  }
+  const uint4 *ks = src_k + s * vecs_per_block;
+  const uint4 *vs = src_v + s * vecs_per_block;
+  uint4 *kd = dst_k + d * vecs_per_block;
+  uint4 *vd = dst_v + d * vecs_per_block;
+  constexpr int U = 4;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < vecs_per_block; i0 += U * stride) {
+    uint4 a[U], b[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < vecs_per_block) {
+        a[u] = ks[i];
+        b[u] = vs[i];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < vecs_per_block) {
+        kd[i] = a[u];
+        vd[i] = b[u];
+      }
+    }
   }
 }
 

@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace pa {
 
 constexpr int kBlock = 16;  // tokens per physical block
@@ -61,13 +63,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for phase `parity` of an mbarrier.  Each try_wait already suspends for a
-// hardware-chosen interval; after `kMaxTries` failed tries the wait gives up, flags
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for phase `parity` of an mbarrier.  The waits in this library are for this CTA's own
+// copies and MMAs (microseconds); after kWaitLimitNs of wall time the wait gives up, flags
 // kErrTimeout and returns false so the caller can unwind instead of hanging.
-constexpr uint32_t kMaxTries = 1u << 22;
+constexpr uint64_t kWaitLimitNs = 200ull * 1000 * 1000;
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kMaxTries; ++i)
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) break;
+  }
   flag_error(kErrTimeout);
   return false;
 }
@@ -96,15 +108,85 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Packed pairs of fp32 (sm_100 f32x2 arithmetic: two lanes per instruction).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// bf16x2 word -> packed fp32 pair (element 0 low).
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2pack(bf16lo(w), bf16hi(w)); }
+
 // Two E4M3 codes (low 16 bits of w, element 0 in the low byte) -> two floats (exact).
 __device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t w) {
   __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
   return __half22float2(*reinterpret_cast<__half2 *>(&h));
 }
 
-template <typename T>
-__device__ __forceinline__ T ld_nc(const T *p) {
-  return __ldg(p);
+// Four one-byte KV codes (element 0 in the low byte) -> two packed fp32 pairs (0,1) and (2,3), exact.
+// KT 1: OCP E4M3 through the hardware e4m3x2 -> f16x2 conversion.  KT 2: signed INT8: each byte,
+// biased to unsigned, is placed in the mantissa of 2^23 (byte permute), and 2^23 + 128 is then
+// subtracted (packed), which is exact for every value.
+template <int KT>
+__device__ __forceinline__ void bytes4_to_f2(uint32_t w, uint64_t &p01, uint64_t &p23) {
+  if constexpr (KT == 1) {
+    const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w & 0xffffu));
+    const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w >> 16));
+    p01 = f2pack(a.x, a.y);
+    p23 = f2pack(b.x, b.y);
+  } else {
+    const uint32_t u = w ^ 0x80808080u;
+    const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650));
+    const float f1 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651));
+    const float f2 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7652));
+    const float f3 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7653));
+    const uint64_t bias = f2pack(8388736.f, 8388736.f);  // 2^23 + 128
+    uint64_t d0, d1;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d0) : "l"(f2pack(f0, f1)), "l"(bias));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d1) : "l"(f2pack(f2, f3)), "l"(bias));
+    p01 = d0;
+    p23 = d1;
+  }
+}
+
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may
+// start while the previous kernel on the stream is still running; it must call griddep_wait()
+// before touching anything that kernel writes.  griddep_launch() lets the next kernel start early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch with programmatic stream serialisation (the kernel may begin while its predecessor on the
+// stream finishes; every kernel of this library calls griddep_wait() before touching memory the
+// predecessor may write, and on every exit path).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace pa

@@ -25,6 +25,7 @@ import torch
 
 BLOCK = 16
 E4M3_MAX = 448.0
+INT8_MAX = 127.0
 
 # The five workloads.  Lengths given here are HISTORIES (tokens already cached);
 # every decode sequence then appends one token, so it attends over history + 1.
@@ -73,7 +74,7 @@ class PagedBatch:
     head_dim: int
     num_blocks: int
     scale: float
-    kv_dtype: int                       # 0 = bf16 cache, 1 = fp8 E4M3 cache
+    kv_dtype: int                       # 0 = bf16 cache, 1 = fp8 E4M3 cache, 2 = int8 cache
     num_decode: int
     hist_lens: np.ndarray               # int32 [S] tokens cached before the step
     new_lens: np.ndarray                # int32 [S] tokens appended by the step
@@ -87,7 +88,7 @@ class PagedBatch:
     tok_offsets: np.ndarray             # int64 [S+1] row offsets of each sequence in tok_k/tok_v
     q_decode: torch.Tensor              # bf16 [num_decode][Hq][D]
     q_prefill: torch.Tensor             # bf16 [sum new_lens of chunks][Hq][D]
-    k_scale: Optional[torch.Tensor] = None   # fp32 [Hkv] (fp8 cache only)
+    k_scale: Optional[torch.Tensor] = None   # fp32 [Hkv] (one-byte caches only)
     v_scale: Optional[torch.Tensor] = None
     split_tokens: int = 0
     info: dict = field(default_factory=dict)
@@ -321,12 +322,13 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
     q_dec = randn_bf16((B, hq, D), device, seed, 6)
     q_pre = randn_bf16((int(c_len.sum()), hq, D), device, seed, 7)
 
-    kv_dtype = 1 if spec.get("kv_dtype") == "fp8" else 0
+    kv_dtype = {"fp8": 1, "int8": 2}.get(spec.get("kv_dtype"), 0)
     k_scale = v_scale = None
     if kv_dtype:
-        # one fp32 scale per KV head (and per K/V tensor): absmax of the seeded data / 448
-        k_scale = (tok_k.float().abs().amax(dim=(0, 2)) / E4M3_MAX).to(torch.float32)
-        v_scale = (tok_v.float().abs().amax(dim=(0, 2)) / E4M3_MAX).to(torch.float32)
+        # one fp32 scale per KV head (and per K/V tensor): absmax of the seeded data / largest code
+        top = E4M3_MAX if kv_dtype == 1 else INT8_MAX
+        k_scale = (tok_k.float().abs().amax(dim=(0, 2)) / top).to(torch.float32)
+        v_scale = (tok_v.float().abs().amax(dim=(0, 2)) / top).to(torch.float32)
 
     return PagedBatch(
         name=name, num_q_heads=hq, num_kv_heads=hkv, head_dim=D, num_blocks=num_blocks,

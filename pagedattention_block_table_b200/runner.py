@@ -27,8 +27,8 @@ class DeviceStep:
         self.device = torch.device(device)
         dev = self.device
         nb, hkv, d = batch.num_blocks, batch.num_kv_heads, batch.head_dim
-        self.kv_dtype = B.PA_KV_FP8_E4M3 if batch.kv_dtype else B.PA_KV_BF16
-        cdt = torch.uint8 if batch.kv_dtype else torch.bfloat16
+        self.kv_dtype = batch.kv_dtype
+        cdt = {0: torch.bfloat16, 1: torch.uint8, 2: torch.int8}[batch.kv_dtype]
         alloc = torch.zeros if zero_cache else torch.empty
         self.k_cache = alloc((nb, hkv, 16, d), dtype=cdt, device=dev)
         self.v_cache = alloc((nb, hkv, 16, d), dtype=cdt, device=dev)

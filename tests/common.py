@@ -14,7 +14,7 @@ FP8_MAX = 5e-2       # fp8 cache, vs the oracle on the original bf16 K/V
 def oracle_step(batch: PagedBatch, O, keep_pre_step=False):
     """Fill the history, then run the step (forks, append, decode, prefill) in the oracle."""
     nb, hkv, d = batch.num_blocks, batch.num_kv_heads, batch.head_dim
-    dt = np.uint8 if batch.kv_dtype else np.uint16
+    dt = {0: np.uint16, 1: np.uint8, 2: np.int8}[batch.kv_dtype]
     kc = np.zeros((nb, hkv, 16, d), dt)
     vc = np.zeros((nb, hkv, 16, d), dt)
     tk = bf16_bits(batch.tok_k)
@@ -65,7 +65,7 @@ def oracle_decode_one(batch: PagedBatch, s: int, O, kv_dtype=None):
     tk = bf16_bits(batch.tok_k.index_select(0, rows))
     tv = bf16_bits(batch.tok_v.index_select(0, rows))
     nblk = max(1, (L + 15) // 16)
-    dt = np.uint8 if kv_dtype else np.uint16
+    dt = {0: np.uint16, 1: np.uint8, 2: np.int8}[kv_dtype]
     kc = np.zeros((nblk, batch.num_kv_heads, 16, batch.head_dim), dt)
     vc = np.zeros_like(kc)
     ks = vs = None
@@ -75,3 +75,18 @@ def oracle_decode_one(batch: PagedBatch, s: int, O, kv_dtype=None):
     q = bf16_bits(batch.q_decode[s:s + 1])
     return O.paged_decode(q, kc, vc, np.arange(nblk, dtype=np.int32)[None], np.array([L], np.int32), batch.scale,
                           kv_dtype, ks, vs)[0]
+
+
+def oracle_attend_prefix(batch: PagedBatch, s: int, L: int, q_bits: np.ndarray, O):
+    """Oracle attention of the given query rows (bf16 bits [n][Hq][D]) over the first L tokens of
+    sequence s, from its token rows in a fresh contiguous cache (bf16)."""
+    rows = torch.from_numpy(batch.seq_rows(s)[:L]).to(batch.tok_k.device)
+    tk = bf16_bits(batch.tok_k.index_select(0, rows))
+    tv = bf16_bits(batch.tok_v.index_select(0, rows))
+    nblk = max(1, (L + 15) // 16)
+    kc = np.zeros((nblk, batch.num_kv_heads, 16, batch.head_dim), np.uint16)
+    vc = np.zeros_like(kc)
+    O.kv_append(kc, vc, tk, tv, np.arange(L, dtype=np.int64))
+    n = q_bits.shape[0]
+    tables = np.tile(np.arange(nblk, dtype=np.int32)[None], (n, 1))
+    return O.paged_decode(q_bits, kc, vc, tables, np.full(n, L, np.int32), batch.scale)

@@ -1,0 +1,180 @@
+"""The host block manager (C++, through the C ABI), on the CPU.
+
+Pins: the append rule of the Core Concepts page §3.2 (write at the end of the current block, a
+new block when it is full), copy-on-write of the vLLM overview's Prefix Sharing (a fork shares
+pages; the first write into a shared page goes to a copy; the last holder writes in place), and
+Continuous Batching's release of a finished request's pages.  A randomised run checks the
+manager against a simulated cache: applying its slots and copy pairs to a token-id array, every
+sequence must read back exactly its own tokens through its table.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from pagedattention_block_table_b200 import binding as B
+
+
+@pytest.fixture
+def bm():
+    B.lib()
+    h = B.pa_bm_create(64, 0)
+    yield h
+    B.pa_bm_destroy(h)
+
+
+def test_append_fills_the_current_block_then_takes_a_new_one(bm):
+    B.pa_bm_add(bm, 1)
+    slots, cow = B.pa_bm_append(bm, 1, 17)                 # 16 fill block 0, the 17th opens block 1
+    assert cow is None
+    assert list(slots[:16]) == list(range(16)) and slots[16] == 16
+    slots, _ = B.pa_bm_append(bm, 1, 1)
+    assert slots[0] == 17                                   # end of the current block
+    assert B.pa_bm_length(bm, 1) == 18
+    assert B.pa_bm_num_free(bm) == 62
+
+
+def test_fork_then_write_copies_the_shared_page(bm):
+    B.pa_bm_add(bm, 1)
+    B.pa_bm_append(bm, 1, 20)                               # blocks 0 (full), 1 (4 tokens)
+    B.pa_bm_fork(bm, 1, 2)
+    t1, _ = B.pa_bm_tables(bm, [1], 4)
+    slots, cow = B.pa_bm_append(bm, 2, 1)                   # child writes into shared block 1
+    assert cow is not None and cow[0] == t1[0, 1]
+    t2, l2 = B.pa_bm_tables(bm, [2], 4)
+    assert t2[0, 0] == t1[0, 0]                             # full block stays shared
+    assert t2[0, 1] == cow[1] != t1[0, 1]                   # partial block replaced by its copy
+    assert slots[0] == cow[1] * 16 + 4 and l2[0] == 21
+    s, cow2 = B.pa_bm_append(bm, 1, 1)                      # parent is now the only holder: in place
+    assert cow2 is None and s[0] == t1[0, 1] * 16 + 4
+    st = B.pa_bm_stats(bm)
+    assert st["blocks_shared"] == 1 and st["cow_copies"] == 1
+
+
+def test_free_returns_blocks_only_when_no_holder_is_left(bm):
+    B.pa_bm_add(bm, 1)
+    B.pa_bm_append(bm, 1, 40)                               # 3 blocks
+    B.pa_bm_fork(bm, 1, 2)
+    assert B.pa_bm_num_free(bm) == 61
+    B.pa_bm_free(bm, 1)
+    assert B.pa_bm_num_free(bm) == 61                       # still held by 2
+    B.pa_bm_free(bm, 2)
+    assert B.pa_bm_num_free(bm) == 64
+
+
+def test_exhausted_pool_changes_nothing():
+    h = B.pa_bm_create(4, 0)
+    try:
+        B.pa_bm_add(h, 1)
+        B.pa_bm_append(h, 1, 60)
+        with pytest.raises(B.PagedAttnError) as e:
+            B.pa_bm_append(h, 1, 10)                        # needs a 5th block
+        assert e.value.status == B.PA_ENOMEM
+        assert B.pa_bm_length(h, 1) == 60 and B.pa_bm_num_free(h) == 0
+        B.pa_bm_append(h, 1, 4)                             # still fits in block 3
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_bad_ids_are_rejected(bm):
+    with pytest.raises(B.PagedAttnError):
+        B.pa_bm_append(bm, 99, 1)
+    B.pa_bm_add(bm, 5)
+    with pytest.raises(B.PagedAttnError):
+        B.pa_bm_add(bm, 5)
+    with pytest.raises(B.PagedAttnError):
+        B.pa_bm_fork(bm, 5, 5)
+    assert B.pa_bm_length(bm, 1234) == -1
+
+
+def test_random_operations_read_back_each_sequences_tokens():
+    """Random adds, forks, appends and frees; a simulated cache of token ids written through the
+    manager's slots and copy pairs must read back every live sequence's own token ids."""
+    rng = np.random.default_rng(12)
+    nb = 400
+    h = B.pa_bm_create(nb, 77)
+    cache = np.full(nb * 16, -1, np.int64)       # token id stored in each slot
+    seqs = {}                                    # id -> list of token ids (the truth)
+    next_id, next_tok = 0, 0
+    try:
+        for step in range(3000):
+            op = rng.random()
+            live = list(seqs)
+            if op < 0.15 or not live:
+                B.pa_bm_add(h, next_id)
+                seqs[next_id] = []
+                next_id += 1
+            elif op < 0.25:
+                p = live[rng.integers(len(live))]
+                B.pa_bm_fork(h, p, next_id)
+                seqs[next_id] = list(seqs[p])
+                next_id += 1
+            elif op < 0.35 and len(live) > 3:
+                s = live[rng.integers(len(live))]
+                B.pa_bm_free(h, s)
+                del seqs[s]
+            else:
+                s = live[rng.integers(len(live))]
+                n = int(rng.integers(1, 40))
+                try:
+                    slots, cow = B.pa_bm_append(h, s, n)
+                except B.PagedAttnError as e:
+                    assert e.status == B.PA_ENOMEM
+                    continue
+                if cow is not None:                  # copy the page first, as pa_copy_blocks would
+                    cache[cow[1] * 16:(cow[1] + 1) * 16] = cache[cow[0] * 16:(cow[0] + 1) * 16]
+                toks = list(range(next_tok, next_tok + n))
+                next_tok += n
+                cache[slots] = toks
+                seqs[s].extend(toks)
+            if step % 100 == 0 or step == 2999:
+                ids = list(seqs)
+                if not ids:
+                    continue
+                mbs = max(1, max(math.ceil(len(v) / 16) for v in seqs.values()))
+                tables, lens = B.pa_bm_tables(h, ids, mbs)
+                for i, sid in enumerate(ids):
+                    L = lens[i]
+                    assert L == len(seqs[sid])
+                    t = np.arange(L)
+                    assert np.array_equal(cache[tables[i, t // 16] * 16 + t % 16], np.array(seqs[sid], np.int64))
+                st = B.pa_bm_stats(h)
+                held = set(int(b) for i in range(len(ids)) for b in tables[i] if b >= 0)
+                assert st["blocks_used"] == len(held) == nb - B.pa_bm_num_free(h)
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_paged_vs_reserved_memory_utilisation():
+    """Continuous batching over a synthetic trace: requests with lognormal prompt and output lengths
+    arrive, grow one token per step and leave.  Paged allocation holds only ceil(len/16) blocks per
+    request; a contiguous scheme reserves the maximum length (2048) per request.  The pages report
+    ~50% -> >90% utilisation and >70% waste for reservation (KV Cache to vLLM §2.3, §3.2)."""
+    rng = np.random.default_rng(3)
+    h = B.pa_bm_create(200000, 5)
+    try:
+        live = {}
+        util_paged, util_reserved = [], []
+        rid = 0
+        for step in range(600):
+            for _ in range(rng.poisson(2.0)):
+                prompt = int(min(1500, max(16, rng.lognormal(math.log(300), 0.8))))
+                out = int(min(2048 - prompt, max(8, rng.lognormal(math.log(150), 0.8))))
+                B.pa_bm_add(h, rid)
+                B.pa_bm_append(h, rid, prompt)
+                live[rid] = out
+                rid += 1
+            for r in list(live):
+                B.pa_bm_append(h, r, 1)
+                live[r] -= 1
+                if live[r] == 0:
+                    B.pa_bm_free(h, r)
+                    del live[r]
+            if step >= 100 and live:
+                st = B.pa_bm_stats(h)
+                util_paged.append(st["tokens_stored"] / (16 * st["blocks_used"]))
+                util_reserved.append(st["tokens_stored"] / (2048 * len(live)))
+        assert np.mean(util_paged) > 0.9
+        assert np.mean(util_reserved) < 0.5
+    finally:
+        B.pa_bm_destroy(h)

@@ -98,3 +98,33 @@ def test_out_of_pool_slot_is_flagged_not_written(cuda_lib):
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_EDEVICE_OOB
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK              # cleared
     assert float(kc.float().sum()) == 2 * 64                              # only slot 0 written
+
+
+def test_append_int8_bit_exact(O, cuda_lib):
+    batch = make_batch("mha_fp8_decode", seed=33, overrides=dict(num_seqs=5, num_q_heads=4, num_kv_heads=4,
+                                                               hist=("uniform", 1, 300), kv_dtype="int8"))
+    ref = oracle_step(batch, O)
+    _, _, k, v = _gpu_step_caches(batch, cuda_lib)
+    assert np.array_equal(k, ref["k_cache"]) and np.array_equal(v, ref["v_cache"])
+
+
+def test_int8_quantiser_all_bf16_inputs(O, cuda_lib):
+    """Every finite bf16 value, divided by several scales, quantises to the oracle's INT8 code."""
+    bits = np.arange(0, 1 << 16, dtype=np.uint32)
+    bits = bits[((bits >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    n = (bits.shape[0] + 63) // 64 * 64
+    pad = np.zeros(n, np.uint16)
+    pad[: bits.shape[0]] = bits
+    tok = pad.reshape(-1, 1, 64)
+    T = tok.shape[0]
+    for scale in (1.0, 0.0313, 7.5e-4, 3.0):
+        kc = torch.zeros((T // 16 + 1, 1, 16, 64), dtype=torch.int8, device="cuda")
+        kt = torch.from_numpy(tok.view(np.int16)).view(torch.bfloat16).cuda()
+        s = torch.tensor([scale], dtype=torch.float32, device="cuda")
+        cuda_lib.pa_kv_append(kc, kc.clone(), kt, kt, torch.arange(T, dtype=torch.int64, device="cuda"),
+                              cuda_lib.PA_KV_INT8, s, s)
+        okc = np.zeros(tuple(kc.shape), np.int8)
+        sc = np.array([scale], np.float32)
+        O.kv_append(okc, np.zeros_like(okc), tok, tok, np.arange(T, dtype=np.int64), 2, sc, sc)
+        got = kc.cpu().numpy()
+        assert np.array_equal(got, okc), f"scale {scale}: {(got != okc).sum()} codes differ"

@@ -146,3 +146,23 @@ def test_full_size_sampled(O, cuda_lib, name, split, samples):
         if batch.kv_dtype:
             ref16 = oracle_decode_one(batch, s, O, kv_dtype=0)
             assert_close(got[s], ref16, max_tol=FP8_MAX, mean_tol=None, what=f"{name} seq {s} vs bf16")
+
+
+@pytest.mark.parametrize("d,hq,hkv", [(128, 8, 8), (128, 16, 4), (64, 4, 2)])
+def test_decode_int8_matches_oracle(O, cuda_lib, d, hq, hkv):
+    ov = dict(num_seqs=4, num_q_heads=hq, num_kv_heads=hkv, head_dim=d, hist=("uniform", 1, 700), kv_dtype="int8")
+    batch = make_batch("mha_fp8_decode", seed=49, overrides=ov)
+    got = to_f64(_gpu_decode(batch, 256).out_dec)
+    assert_close(got, oracle_step(batch, O)["decode"], what="int8 vs dequantised")
+    b16 = make_batch("mha_fp8_decode", seed=49, overrides=dict(ov, kv_dtype=None))
+    assert_close(got, oracle_step(b16, O)["decode"], max_tol=FP8_MAX, mean_tol=None, what="int8 vs bf16")
+
+
+def test_kv_head_shards_reproduce_the_unsharded_call(cuda_lib):
+    """Tensor-parallel KV-head shards, run one after the other on one GPU (no rank waits on another),
+    give bit-identical per-head outputs to the unsharded call at the same split."""
+    from pagedattention_block_table_b200 import sharding
+    batch = make_batch("llama3_8b_decode", seed=50, overrides=dict(num_seqs=5, hist=("uniform", 100, 1500)))
+    full = _gpu_decode(batch, 256).out_dec
+    parts = [_gpu_decode(sharding.shard_batch(batch, r, 4), 256).out_dec for r in range(4)]
+    assert torch.equal(torch.cat(parts, dim=1), full)

@@ -1,0 +1,87 @@
+"""GPU parity of the tcgen05 paged prefill (and of the whole mixed step) against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+from pagedattention_block_table_b200.inputs import make_batch, bf16_bits
+from tests.common import assert_close, oracle_attend_prefix, oracle_decode_one, oracle_step, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(batch):
+    from pagedattention_block_table_b200.runner import DeviceStep
+    st = DeviceStep(batch)
+    st.fill_history()
+    st.step()
+    torch.cuda.synchronize()
+    return st
+
+
+def _chunks(**ov):
+    base = dict(num_seqs=1, hist=("fixed", [3]), share_group=0, share_prefix=0, num_q_heads=8, num_kv_heads=2,
+                head_dim=128, prefill_chunks=3, chunk_len=(1, 300), chunk_hist=(1, 400))
+    base.update(ov)
+    return base
+
+
+CASES = {
+    "gqa4_d128": _chunks(),
+    "gqa4_d128_long": _chunks(prefill_chunks=2, chunk_len=(300, 700), chunk_hist=(500, 900)),
+    "mha_d128": _chunks(num_q_heads=4, num_kv_heads=4, chunk_len=(100, 260)),
+    "gqa2_d64": _chunks(head_dim=64, num_q_heads=4, num_kv_heads=2),
+    "tiny_chunks": _chunks(prefill_chunks=5, chunk_len=(1, 17), chunk_hist=(1, 40)),
+}
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_prefill_matches_oracle(O, cuda_lib, case):
+    batch = make_batch("mixed_step", seed=51, overrides=CASES[case])
+    ref = oracle_step(batch, O)
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(st.out_pre), ref["prefill"], what=f"prefill {case}")
+    assert_close(to_f64(st.out_dec), ref["decode"], what=f"decode {case}")
+
+
+def test_prefill_chunk_starting_a_request(O, cuda_lib):
+    """H = 0: row 0 sees only key 0, so its output is exactly V[0]."""
+    batch = make_batch("mixed_step", seed=52, overrides=_chunks(prefill_chunks=1, chunk_len=(200, 200)))
+    st = _run(batch)
+    ref = oracle_step(batch, O)["prefill"]
+    assert_close(to_f64(st.out_pre), ref, what="H=0 chunk")
+    g = batch.num_q_heads // batch.num_kv_heads
+    # appended tokens: the decoding sequence's first, then the chunk's; chunk row 0 is step token 1
+    assert torch.equal(st.out_pre[0], st.v_new[1].repeat_interleave(g, 0))
+
+
+def test_prefill_placement_invariance(cuda_lib):
+    kw = dict(seed=53, overrides=_chunks(prefill_chunks=2, chunk_len=(130, 300), chunk_hist=(17, 300)))
+    a = _run(make_batch("mixed_step", perm_seed=1, **kw)).out_pre
+    b = _run(make_batch("mixed_step", perm_seed=2, **kw)).out_pre
+    assert torch.equal(a, b)
+
+
+def test_mixed_step_full_size_sampled(O, cuda_lib):
+    """The whole mixed step at full size: forks, append, decode of 256 sequences, 4 prefill chunks."""
+    batch = make_batch("mixed_step", device="cuda")
+    assert batch.cow_pairs.shape[0] > 0
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    dec = to_f64(st.out_dec)
+    pre = to_f64(st.out_pre)
+    assert np.all(np.isfinite(dec)) and np.all(np.isfinite(pre))
+    for s in (0, 7, 100, 255):
+        assert_close(dec[s], oracle_decode_one(batch, s, O), what=f"decode seq {s}")
+    cu = batch.cu_q_lens
+    ctx = batch.context_lens
+    for c in range(batch.num_seqs - batch.num_decode):
+        s = batch.num_decode + c
+        C = int(batch.new_lens[s])
+        H = int(ctx[s]) - C
+        for i in sorted({0, 1, 127, 128, C // 2, C - 1}):
+            if i >= C:
+                continue
+            q = bf16_bits(batch.q_prefill[cu[c] + i:cu[c] + i + 1])
+            ref = oracle_attend_prefix(batch, s, H + i + 1, q, O)
+            assert_close(pre[cu[c] + i], ref[0], what=f"chunk {c} row {i}")

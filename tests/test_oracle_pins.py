@@ -291,3 +291,41 @@ def test_fp8_append_codes_follow_quotient_rule(O):
         # relative half-step of a 3-bit mantissa (1/16), or half the smallest subnormal step
         bound = np.maximum(np.abs(x) / 16, 2.0 ** -10 * ks[None, :, None]) * (1 + 1e-6)
         assert np.all(np.abs(deq - x) <= bound)
+
+
+# ----------------------------------------------------------------------------- INT8
+
+def test_int8_encode_points(O):
+    g = _golden("int8_points.json")
+    for p in g["encode"]:
+        assert int(O.int8_encode([p["x"]])[0]) == p["code"], p
+
+
+def test_int8_encode_matches_numpy(O):
+    """numpy's rint rounds half to even; clipped to +-127 it is the symmetric INT8 encoder."""
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.normal(0, 60, 20000), np.arange(-130, 130, 0.5)]).astype(np.float32)
+    ref = np.clip(np.rint(x), -127, 127).astype(np.int8)
+    assert np.array_equal(O.int8_encode(x), ref)
+
+
+def test_int8_append_and_decode_read_back(O):
+    """INT8 append stores round(x/scale); decode of a one-token context returns code * scale exactly."""
+    k = bf16_bits(torch.randn(1, 1, 64).to(torch.bfloat16))
+    v = bf16_bits(torch.randn(1, 1, 64).to(torch.bfloat16))
+    sc = np.array([0.02], np.float32)
+    kc = np.zeros((2, 1, 16, 64), np.int8)
+    vc = np.zeros_like(kc)
+    O.kv_append(kc, vc, k, v, np.array([17], np.int64), 2, sc, sc)
+    xv = _bf16_to_f64(v[0, 0]).astype(np.float32)
+    codes = np.clip(np.rint(xv / np.float32(0.02)), -127, 127)
+    assert np.array_equal(vc[1, 0, 1], codes.astype(np.int8))
+    q = bf16_bits(torch.randn(1, 2, 64).to(torch.bfloat16))
+    # the token sits at slot 17 = block 1, offset 1; a table whose block 0 is physical block 1 and a
+    # context of 2 reads (zero row, token)
+    out = O.paged_decode(q, kc, vc, np.array([[1]], np.int32), np.array([2], np.int32), 0.125, 2, sc, sc)
+    assert np.all(np.isfinite(out))
+    # the two-token result is a convex combination of the two dequantised rows
+    rows = np.stack([vc[1, 0, 0].astype(np.float64), vc[1, 0, 1].astype(np.float64)]) * np.float64(np.float32(0.02))
+    lo, hi = rows.min(axis=0) - 1e-12, rows.max(axis=0) + 1e-12
+    assert np.all((out[0] >= lo) & (out[0] <= hi))
