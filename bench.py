@@ -78,6 +78,20 @@ def bf16_peak():
     return 1590.0, "fallback"
 
 
+def kv_unique_bytes(batch) -> int:
+    """Bytes of the distinct cache slots the decode reads: a prefix block shared by several sequences
+    counts once (it is stored once in HBM; the other readers can be served from L2)."""
+    nd = batch.num_decode
+    e = 1 if batch.kv_dtype else 2
+    slots = []
+    for s in range(nd):
+        L = int(batch.context_lens[s])
+        t = np.arange(L, dtype=np.int64)
+        slots.append(batch.block_tables[s, t // 16].astype(np.int64) * 16 + t % 16)
+    n = np.unique(np.concatenate(slots)).shape[0] if slots else 0
+    return int(n) * 2 * batch.num_kv_heads * batch.head_dim * e
+
+
 def kv_bytes(batch) -> int:
     nd = batch.num_decode
     e = 1 if batch.kv_dtype else 2
@@ -298,12 +312,14 @@ def run_ours(args, rank, world, local_rank):
         "pct_of_peak": round(100 * value / world / peak, 2),
         "seq_steps_per_s": round(world * batch.num_decode / (step_ms * 1e-3), 1),
         "decode_kv_bytes_per_step": kvb,
+        "decode_kv_unique_bytes_per_step": kv_unique_bytes(batch),
         "roofline": {
             "kernel": "pa_paged_attention (paged_decode_kernel + lse_reduce_kernel)",
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "traffic": None if tr is None else tr.get("bytes_per_launch"),
             "algorithmic_bytes": dbytes, "avg_launch_ms": round(dec_ms, 5),
+            "achieved_unique": round((dbytes - kvb + kv_unique_bytes(batch)) / (dec_ms * 1e-3) / 1e9, 2),
         },
         "e2e": {"value": round(agg["bytes"] / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
@@ -421,6 +437,53 @@ def run_reference(args, rank, world):
     }
 
 
+# ----------------------------------------------------------------------------- swap (KV eviction)
+
+def run_swap(args):
+    """Throughput of pa_swap_blocks between the device cache and a pinned host pool, against the
+    host link's own copy bandwidth measured in the same run (a plain pinned <-> device memcpy)."""
+    from pagedattention_block_table_b200 import binding as B
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    nb_dev, nb_host, hkv, d, n = 8192, 4096, 8, 128, 1024
+    g = torch.Generator(device=dev).manual_seed(1)
+    dk = torch.randn((nb_dev, hkv, 16, d), device=dev, generator=g).to(torch.bfloat16)
+    dv = torch.randn((nb_dev, hkv, 16, d), device=dev, generator=g).to(torch.bfloat16)
+    hk = torch.empty((nb_host, hkv, 16, d), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    gc = torch.Generator().manual_seed(2)
+    out_pairs = torch.stack([torch.randperm(nb_dev, generator=gc)[:n], torch.randperm(nb_host, generator=gc)[:n]],
+                            1).int().contiguous().to(dev)
+    in_pairs = out_pairs[:, [1, 0]].contiguous()
+    nbytes = n * 2 * hkv * 16 * d * 2
+
+    def timed(f, k):
+        for _ in range(3):
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        e0.record()
+        for _ in range(k):
+            f()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / k
+
+    K = max(3, min(args.steps, 50))
+    t_out = timed(lambda: B.pa_swap_blocks(hk, hv, dk, dv, out_pairs), K)
+    t_in = timed(lambda: B.pa_swap_blocks(dk, dv, hk, hv, in_pairs), K)
+    big_h = torch.empty(nbytes // 2, dtype=torch.bfloat16).pin_memory()
+    big_d = torch.empty(nbytes // 2, dtype=torch.bfloat16, device=dev)
+    t_d2h = timed(lambda: big_h.copy_(big_d, non_blocking=True), K)
+    t_h2d = timed(lambda: big_d.copy_(big_h, non_blocking=True), K)
+    assert B.pa_get_device_error() == B.PA_OK
+    gbs = lambda t: round(nbytes / (t * 1e-3) / 1e9, 2)
+    return {"metric": "swap_blocks device<->pinned host GB/s", "unit": "GB/s", "blocks": n,
+            "bytes_per_call": nbytes, "swap_out": gbs(t_out), "swap_in": gbs(t_in),
+            "link_memcpy_d2h": gbs(t_d2h), "link_memcpy_h2d": gbs(t_h2d),
+            "frac_out": round(t_d2h / t_out, 3), "frac_in": round(t_h2d / t_in, 3), "steps": K}
+
+
 # ----------------------------------------------------------------------------- main
 
 def main():
@@ -436,7 +499,12 @@ def main():
     ap.add_argument("--ref-max-steps", type=int, default=20)
     ap.add_argument("--ref-budget-s", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", choices=["step", "swap"], default="step",
+                    help="step: the hot-path step (default); swap: KV eviction throughput")
     args = ap.parse_args()
+    if args.mode == "swap":
+        print(json.dumps(run_swap(args)), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -22,36 +22,39 @@ from . import build as _build  # noqa: F401  (relative import when used as a pac
 _lib = None
 
 
+def configure(lib):
+    """Declare the C signatures on a loaded oracle library."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    L = ctypes.c_int64
+    D = ctypes.c_double
+    lib.oracle_e4m3_decode.restype = D
+    lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+    lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.oracle_int8_encode.restype = ctypes.c_int8
+    lib.oracle_int8_encode.argtypes = [ctypes.c_float]
+    lib.oracle_kv_cache_bytes.restype = L
+    lib.oracle_kv_cache_bytes.argtypes = [L, L, L, L, L, L]
+    lib.oracle_kv_append.restype = I
+    lib.oracle_kv_append.argtypes = [P, P, P, P, P, L, I, I, L, I, P, P]
+    lib.oracle_copy_blocks.restype = I
+    lib.oracle_copy_blocks.argtypes = [P, P, P, L, I, I, L, I]
+    lib.oracle_swap_blocks.restype = I
+    lib.oracle_swap_blocks.argtypes = [P, P, L, P, P, L, P, L, I, I, I]
+    lib.oracle_paged_decode.restype = I
+    lib.oracle_paged_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, L, D, I, P, P]
+    lib.oracle_paged_prefill.restype = I
+    lib.oracle_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, L, D, I, P, P]
+    lib.oracle_num_threads.restype = I
+    lib.oracle_num_threads.argtypes = []
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        path = _build.build()
-        lib = ctypes.CDLL(path)
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        L = ctypes.c_int64
-        D = ctypes.c_double
-        lib.oracle_e4m3_decode.restype = D
-        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
-        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
-        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
-        lib.oracle_int8_encode.restype = ctypes.c_int8
-        lib.oracle_int8_encode.argtypes = [ctypes.c_float]
-        lib.oracle_kv_cache_bytes.restype = L
-        lib.oracle_kv_cache_bytes.argtypes = [L, L, L, L, L, L]
-        lib.oracle_kv_append.restype = I
-        lib.oracle_kv_append.argtypes = [P, P, P, P, P, L, I, I, L, I, P, P]
-        lib.oracle_copy_blocks.restype = I
-        lib.oracle_copy_blocks.argtypes = [P, P, P, L, I, I, L, I]
-        lib.oracle_swap_blocks.restype = I
-        lib.oracle_swap_blocks.argtypes = [P, P, L, P, P, L, P, L, I, I, I]
-        lib.oracle_paged_decode.restype = I
-        lib.oracle_paged_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, L, D, I, P, P]
-        lib.oracle_paged_prefill.restype = I
-        lib.oracle_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, L, D, I, P, P]
-        lib.oracle_num_threads.restype = I
-        lib.oracle_num_threads.argtypes = []
-        _lib = lib
+        _lib = configure(ctypes.CDLL(_build.build()))
     return _lib
 
 

@@ -113,11 +113,17 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   using C = DecodeCfg<KT, D, QPB, NW, STAGES>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
+  // grid (heads, sequences, splits): every sequence's first split is scheduled before any second
+  // one, so the CTAs that find their split past a short sequence's end cluster in the last waves
+  const int split = blockIdx.z;
+  const int unit = blockIdx.x;
+  const int b = blockIdx.y;
   const int sub_groups = P.group / QPB;
-  const int g = blockIdx.y / sub_groups;
-  const int h0 = g * P.group + (blockIdx.y % sub_groups) * QPB;  // first query head of this CTA
-  const int b = blockIdx.z;
+  const int g = unit / sub_groups;
+  const int h0 = g * P.group + (unit % sub_groups) * QPB;  // first query head of this CTA
+  // any input may come from the kernel before this one on the stream (launched with PDL)
+  griddep_wait();
+  griddep_launch();
 
   // ---- context length, validated: never read past the table row or the launch bound
   int L = P.context_lens[b];
@@ -129,10 +135,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
     }
   }
   const int n_splits = (L + P.split_tokens - 1) / P.split_tokens;
-  if (split >= (n_splits > 1 ? n_splits : 1)) {
-    griddep_wait();  // keep "this grid done" meaning "the kernel before it done" for the next kernel
-    return;
-  }
+  if (split >= (n_splits > 1 ? n_splits : 1)) return;
   const bool final_out = n_splits <= 1;
   const int t0 = split * P.split_tokens;
   const int t1 = min(L, t0 + P.split_tokens);
@@ -151,29 +154,6 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   }
   __syncwarp();
 
-  // ---- query registers: the dims this lane multiplies in QK, pre-scaled
-  const int r = lane / C::LPT, j = lane % C::LPT;
-  uint64_t qf2[QPB][C::DPL / 2];  // packed (even, odd) dim pairs, pre-scaled
-  {
-    float qs = P.qscale;
-    if (KT != 0) qs *= P.k_scale[g];
-#pragma unroll
-    for (int qi = 0; qi < QPB; ++qi) {
-      const __nv_bfloat16 *qrow = P.q + ((int64_t)b * P.num_q_heads + h0 + qi) * D;
-#pragma unroll
-      for (int k = 0; k < C::CPL; ++k) {
-        const int d0 = (k * C::LPT + j) * C::CE;
-#pragma unroll
-        for (int e8 = 0; e8 < C::CE; e8 += 8) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(qrow + d0 + e8);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t)
-            qf2[qi][(k * C::CE + e8) / 2 + t] = f2pack(bf16lo(ww[t]) * qs, bf16hi(ww[t]) * qs);
-        }
-      }
-    }
-  }
   const int qsel = group_reduce_qsel<QPB, C::LPT>(lane);
 
   // ---- block-table window: lane k holds the entry of this warp's block (win*32 + k)
@@ -192,10 +172,6 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   };
   int tw = load_window(0);
   const uint64_t pol = l2_evict_first_policy();
-  // everything above reads only caller inputs; the cache may still be being written by the
-  // kernel before this one on the stream (the append), so wait for it here
-  griddep_wait();
-  griddep_launch();
   const int64_t head_stride = (int64_t)C::TILE;
   auto issue = [&](int i) {  // warp-uniform call
     if (i >= nwb) return;
@@ -222,6 +198,32 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   int issued = 0;
   for (; issued < STAGES && issued < nwb; ++issued) issue(issued);
   bool ok = true;
+
+  // ---- query registers (loaded while the first tiles are in flight): the dims this lane
+  // multiplies in QK, pre-scaled
+  const int r = lane / C::LPT, j = lane % C::LPT;
+  uint64_t qf2[QPB][C::DPL / 2];  // packed (even, odd) dim pairs, pre-scaled
+  {
+    float qs = P.qscale;
+    if (KT != 0) qs *= P.k_scale[g];
+#pragma unroll
+    for (int qi = 0; qi < QPB; ++qi) {
+      const __nv_bfloat16 *qrow = P.q + ((int64_t)b * P.num_q_heads + h0 + qi) * D;
+#pragma unroll
+      for (int k = 0; k < C::CPL; ++k) {
+        const int d0 = (k * C::LPT + j) * C::CE;
+#pragma unroll
+        for (int e8 = 0; e8 < C::CE; e8 += 8) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(qrow + d0 + e8);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            qf2[qi][(k * C::CE + e8) / 2 + t] = f2pack(bf16lo(ww[t]) * qs, bf16hi(ww[t]) * qs);
+        }
+      }
+    }
+  }
+
   int i = 0;
   for (; i < nwb; ++i) {
     const int s = i % STAGES;
@@ -429,6 +431,7 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   griddep_wait();  // partials come from the decode kernel just before this one
+  griddep_launch();
   if (h >= P.num_q_heads) return;
   int L = P.context_lens[b];
   const int lim = min(P.max_blocks_per_seq * kBlock, P.max_context_len);

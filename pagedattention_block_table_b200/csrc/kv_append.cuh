@@ -17,7 +17,7 @@ __global__ void kv_append_bf16_kernel(uint4 *__restrict__ k_cache, uint4 *__rest
                                       const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                       const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
                                       int num_kv_heads, int chunks_per_row, int64_t num_slots) {
-  griddep_wait();  // the cache may still be read by the kernel before this one (a decode)
+  griddep_wait();  // inputs or the cache may belong to the kernel before this one (PDL launch)
   griddep_launch();
   const int64_t total = num_tokens * num_kv_heads * chunks_per_row;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;

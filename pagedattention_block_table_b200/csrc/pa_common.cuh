@@ -129,6 +129,11 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 // bf16x2 word -> packed fp32 pair (element 0 low).
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2pack(bf16lo(w), bf16hi(w)); }
 
@@ -164,15 +169,15 @@ __device__ __forceinline__ void bytes4_to_f2(uint32_t w, uint64_t &p01, uint64_t
   }
 }
 
-// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may
-// start while the previous kernel on the stream is still running; it must call griddep_wait()
-// before touching anything that kernel writes.  griddep_launch() lets the next kernel start early.
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may be
+// scheduled while the previous kernel on the stream is still running.  Every kernel of this library
+// calls griddep_wait() first, before reading any input (any of them may be that kernel's output), so
+// what PDL buys is the launch latency: the CTAs are resident and start the moment it completes.
+// griddep_launch() lets the next kernel be scheduled early in turn.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Launch with programmatic stream serialisation (the kernel may begin while its predecessor on the
-// stream finishes; every kernel of this library calls griddep_wait() before touching memory the
-// predecessor may write, and on every exit path).
+// Launch with programmatic stream serialisation (see griddep_wait).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                               Args &&...args) {

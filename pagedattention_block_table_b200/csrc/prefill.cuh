@@ -6,19 +6,22 @@
 // of head h attends to positions t <= H_c + i of KV head h / G:
 //     out[i][h] = softmax_t(scale * q[i][h] . K[t]) V[t].
 //
-// Design: one CTA (4 warps, one query row per thread) per (128-row query tile, query head, chunk).
-// Q is staged once into shared memory in the UMMA K-major 128-byte-swizzled layout.  Keys come in
-// tiles of 128 (8 physical blocks): for each block one TMA box of 16 rows x 64 elements per half of
-// head_dim is fetched into the same swizzled layout (tensor map over the cache viewed as
-// [num_blocks*Hkv*16][head_dim]; no multicast), double-buffered.  One thread issues
-//   S = Q K^T   (tcgen05.mma kind::f16, M=128, N=128, K=16 steps, fp32 accumulator in TMEM)
-// each thread reads its row of S from TMEM (tcgen05.ld 32x32b), applies the causal mask and a base-2
-// online softmax, writes P (bf16) into shared memory in the K-major swizzled layout, and one thread
-// issues
-//   O += P V  (V used as an MN-major B operand straight from its TMA layout, fp32 accumulator in TMEM).
-// p is taken relative to a per-row reference max m_ref; only when a tile's max exceeds m_ref by more
-// than 2^8 does the row move m_ref up and rescale its O row in TMEM (tcgen05.ld/st) and its sum l.
-// O and l always share m_ref, so out = O / l is exact whichever m_ref was used; p stays <= 256.
+// Design.  A CTA serves one KV head's query-head group: its rows stack the G query heads of each
+// position (row r = position r / G, head r % G), so every K/V byte fetched serves G heads.  It holds
+// two 128-row query tiles, A and B, that take turns ("ping-pong"): while one warpgroup runs the
+// softmax of its tile, the tensor core computes the other tile's products.
+//   warps 0-3  softmax of tile A, one row per thread = one TMEM lane   warps 4-7  the same for tile B
+//   warp 8     issues every tcgen05.mma (one elected lane)              warp 9     issues the TMA loads
+// Keys come in tiles of 64 (4 physical blocks): one TMA box of 16 rows x 64 elements per block and per
+// 64-element plane of head_dim, into the UMMA 128-byte-swizzled layout, three tiles in flight (tensor
+// map over the cache seen as [num_blocks*Hkv*16][head_dim]; no multicast).  Each query tile has two S
+// buffers in TMEM, so S of key tile j+2 is computed while the softmax still works on tile j.
+// Per key tile j and query tile X:
+//   S_X = Q_X K_j^T  (M=128, N=64, fp32 in TMEM)   ->  softmax warps: base-2 online softmax, P_X (bf16,
+//   K-major swizzled) into shared memory          ->  O_X += P_X V_j  (M=128, N=head_dim, fp32 in TMEM).
+// p is taken relative to a per-row reference max; only when a tile's max exceeds it by more than 2^8
+// does the row move the reference and rescale its O row in TMEM (tcgen05.ld/st) and its sum l.  O and l
+// always share the reference, so out = O / l is exact whichever reference was used.
 #pragma once
 #include "pa_common.cuh"
 
@@ -71,6 +74,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// This thread's TMEM lane, 64 consecutive fp32 columns (one load, one wait).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[64];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
+        "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
+        "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Store 32 fp32 columns of this thread's TMEM lane.
@@ -135,288 +161,355 @@ struct PrefillParams {
   int max_blocks_per_seq;
   int num_q_heads;
   int num_kv_heads;
-  int group;
+  int group;            // Hq / Hkv
+  int hpr;              // query heads stacked per position in a tile (G if 128 % G == 0, else 1)
   int max_context_len;
-  float qscale;  // scale * log2(e)
+  float qscale;         // scale * log2(e)
 };
+
+#ifndef PA_PREFILL_STAGES
+#define PA_PREFILL_STAGES 4
+#endif
 
 template <int D>
 struct PrefillCfg {
-  static constexpr int BM = 128;                  // query rows per CTA (= TMEM lanes = threads)
-  static constexpr int BN = 128;                  // keys per tile (8 blocks of 16)
+  static constexpr int BM = 128;                  // rows per query tile (= TMEM lanes)
+  static constexpr int BN = 64;                   // keys per key tile (4 blocks)
+  static constexpr int STAGES = PA_PREFILL_STAGES;  // K/V tiles in flight: S runs two tiles ahead of PV
   static constexpr int DH = D / 64;               // 64-element (128-byte) planes of a head_dim row
-  static constexpr int PLANE = 128 * 128;         // bytes of one 128-row x 64-element plane
-  static constexpr int Q_BYTES = DH * PLANE;
-  static constexpr int KV_BYTES = DH * PLANE;     // one K or V tile (128 keys)
-  static constexpr int P_BYTES = 2 * PLANE;       // 128 rows x 128 keys
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + 2 * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + 2 * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int SMEM = OFF_BAR + 64 + 1024;  // + slack to align the base to 1024
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t S_COL = 0;
-  static constexpr uint32_t O_COL = 128;
+  static constexpr int Q_PLANE = BM * 128;        // 16 KB
+  static constexpr int KV_PLANE = BN * 128;       // 8 KB
+  static constexpr int Q_BYTES = DH * Q_PLANE;
+  static constexpr int KV_BYTES = DH * KV_PLANE;  // one K or V tile
+  static constexpr int P_BYTES = BM * 128;        // 128 rows x 64 keys bf16
+  static constexpr int OFF_QA = 0;
+  static constexpr int OFF_QB = OFF_QA + Q_BYTES;
+  static constexpr int OFF_K = OFF_QB + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_PA = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_PB = OFF_PA + P_BYTES;
+  static constexpr int OFF_BAR = OFF_PB + P_BYTES;
+  static constexpr int NBAR = 24;
+  static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + slack to align the base to 1024
+  static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns: S of tile X, buffer b at 64*(2X+b); O of tile X at 256 + 128X
+  __host__ __device__ static constexpr uint32_t s_col(int X, int b) { return 64u * (2u * X + b); }
+  __host__ __device__ static constexpr uint32_t o_col(int X) { return 256u + 128u * X; }
+  static constexpr int THREADS = 320;
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+
 };
 
+// mbarrier slots
+// kKvFull/kKvEmpty: per stage; kSFull: per (tile X, buffer b) at kSFull + 2X + b; kOFull, kPFull: per tile
+enum : int {
+  kKvFull = 0,
+  kKvEmpty = kKvFull + PA_PREFILL_STAGES,
+  kSFull = kKvEmpty + PA_PREFILL_STAGES,
+  kOFull = kSFull + 4,
+  kPFull = kOFull + 2,
+  kQReady = kPFull + 2,
+  kDone = kQReady + 1,
+  kNumBars = kDone + 1
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int D>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(320, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                          const PrefillParams P) {
   using C = PrefillCfg<D>;
+  static_assert(kNumBars <= C::NBAR, "barrier slots");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int mt = blockIdx.x, h = blockIdx.y, c = blockIdx.z;
-  const int g = h / P.group;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.z;
+  const int hg0 = blockIdx.y * P.hpr;                 // first query head of this CTA's rows
+  const int g = hg0 / P.group;                        // their KV head
+  const int ppt = C::BM / P.hpr;                      // positions per query tile
+  // any input may come from the kernel before this one on the stream (launched with PDL)
+  griddep_wait();
+  griddep_launch();
 
   const int q0 = P.cu_q_lens[c];
   const int Cn = P.cu_q_lens[c + 1] - q0;
   const int ctx = P.context_lens[c];
   const int H = ctx - Cn;
   if (Cn < 0 || H < 0 || ctx > min(P.max_blocks_per_seq * kBlock, P.max_context_len)) {
-    if (tid == 0 && mt == 0 && h == 0) flag_error(kErrLength);
-    griddep_wait();
+    if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) flag_error(kErrLength);
     return;
   }
-  const int i0 = mt * C::BM;
-  if (i0 >= Cn) {
-    griddep_wait();
-    return;
-  }
-  const int rows = min(C::BM, Cn - i0);
-  const int kv_len = H + i0 + rows;                   // keys visible to some row of this tile
+  const int p0 = blockIdx.x * 2 * ppt;               // first position of tile A
+  if (p0 >= Cn) return;
+  const int p_end = min(Cn, p0 + 2 * ppt);
+  const int kv_len = H + p_end;                       // keys visible to some row of this CTA
   const int ntiles = (kv_len + C::BN - 1) / C::BN;
 
-  uint8_t *sQ = smem + C::OFF_Q;
-  uint8_t *sK = smem + C::OFF_K;
-  uint8_t *sV = smem + C::OFF_V;
-  uint8_t *sP = smem + C::OFF_P;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);  // 0,1: K/V tile stages; 2: S; 3: O
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4);
-
-  if (warp == 0) {
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
+  if (warp == 8) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int b = 0; b < 4; ++b) mbar_init(&bars[b], 1);
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(&bars[kKvFull + i], 1);
+      mbar_init(&bars[kKvEmpty + i], 1);
+    }
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[kSFull + i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars[kOFull + i], 1);
+      mbar_init(&bars[kPFull + i], 128);
+    }
+    mbar_init(&bars[kQReady], 256);
+    mbar_init(&bars[kDone], 1);
     fence_mbar_init();
   }
-
-  // ---- Q rows into shared memory (K-major, 128-byte swizzle: chunk c of row r at c ^ (r % 8))
-  {
-    uint8_t *rowp = sQ + tid * 128;
-    if (tid < rows) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(P.q + ((int64_t)(q0 + i0 + tid) * P.num_q_heads + h) * D);
-#pragma unroll
-      for (int ch = 0; ch < D / 8; ++ch) {
-        const uint4 v = src[ch];
-        *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::PLANE + (((ch & 7) ^ (tid & 7)) << 4)) = v;
-      }
-    } else {
-#pragma unroll
-      for (int ch = 0; ch < D / 8; ++ch)
-        *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::PLANE + (ch & 7) * 16) = make_uint4(0, 0, 0, 0);
-    }
-  }
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int32_t *trow = P.block_tables + (int64_t)c * P.max_blocks_per_seq;
-
-  // K and V of key tile j (blocks 8j .. 8j+7 that hold keys < kv_len) into stage j % 2
-  auto issue_tile = [&](int j) {
-    const int stage = j & 1;
-    const int nb = min(8, (kv_len - j * C::BN + kBlock - 1) / kBlock);
-    mbar_arrive_expect_tx(&bars[stage], nb * 2 * C::DH * (kBlock * 128));
-    for (int bb = 0; bb < nb; ++bb) {
-      int e = __ldg(trow + j * 8 + bb);
-      if (e < 0 || e >= P.num_blocks) {
-        flag_error(kErrBlockId);
-        e = 0;
-      }
-      const int y = (e * P.num_kv_heads + g) * kBlock;
-#pragma unroll
-      for (int hh = 0; hh < C::DH; ++hh) {
-        const int off = stage * C::KV_BYTES + hh * C::PLANE + bb * (kBlock * 128);
-        tma_load_2d(sK + off, &kmap, hh * 64, y, &bars[stage]);
-        tma_load_2d(sV + off, &vmap, hh * 64, y, &bars[stage]);
-      }
-    }
-  };
-  // the cache may still be written by the kernel before this one on the stream (the append)
-  griddep_wait();
-  griddep_launch();
-  int issued = 0;
-  if (tid == 0) {
-    issue_tile(0);
-    if (ntiles > 1) issue_tile(1);
-  }
-  issued = ntiles > 1 ? 2 : 1;
-
-  float m_ref = -INFINITY, l_run = 0.f;
-  const bool row_ok = tid < rows;
-  const int pos = row_ok ? H + i0 + tid : kv_len - 1;   // padding rows behave like the last row
-  const uint32_t lane = static_cast<uint32_t>(warp * 32) << 16;
-  constexpr uint32_t idS = idesc_bf16(128, C::BN, false);
-  constexpr uint32_t idO = idesc_bf16(128, D, true);
-  constexpr float kRescale = 8.f;                       // log2 of the largest p allowed (256)
   bool timeout = false;
-  bool s_inflight = false, o_inflight = false;  // thread 0: committed MMAs not yet seen complete
-  int j = 0;
 
-  for (; j < ntiles; ++j) {
-    const int stage = j & 1;
-    timeout |= !mbar_wait(&bars[stage], (j >> 1) & 1);
-    uint8_t *kt = sK + stage * C::KV_BYTES;
-    uint8_t *vt = sV + stage * C::KV_BYTES;
-    if ((j + 1) * C::BN > kv_len) {
-      // last tile: V rows of keys no row may see are zeroed so that 0 * V stays 0 in the MMA
-      if (j * C::BN + tid >= kv_len) {
+  if (warp < 8) {
+    // ===================================================================== softmax warpgroups
+    const int X = warp >> 2;                          // 0: tile A, 1: tile B
+    const int r = tid & 127;                          // row = TMEM lane
+    const int pos_i = p0 + X * ppt + r / P.hpr;       // position within the chunk
+    const int h = hg0 + r % P.hpr;
+    const bool row_ok = pos_i < Cn;
+    const int pos = row_ok ? H + pos_i : kv_len - 1;  // padding rows behave like the last row
+    uint8_t *sQ = smem + (X ? C::OFF_QB : C::OFF_QA);
+    uint8_t *sP = smem + (X ? C::OFF_PB : C::OFF_PA);
+    // Q row into the K-major 128-byte-swizzled tile (chunk ch of row r at ch ^ (r % 8))
+    {
+      uint8_t *rowp = sQ + r * 128;
+      if (row_ok) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(P.q + ((int64_t)(q0 + pos_i) * P.num_q_heads + h) * D);
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch)
+          *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::Q_PLANE + (((ch & 7) ^ (r & 7)) << 4)) = src[ch];
+      } else {
+#pragma unroll
+        for (int ch = 0; ch < D / 8; ++ch)
+          *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::Q_PLANE + (ch & 7) * 16) = make_uint4(0, 0, 0, 0);
+      }
+      fence_async_smem();
+      mbar_arrive(&bars[kQReady]);
+    }
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t o_addr = tmem + lane_base + C::o_col(X);
+    constexpr float kRescale = 8.f;
+    const float qs = P.qscale;
+    float m_ref = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < ntiles; ++j) {
+      // every wait's outcome is made warp-uniform: the tcgen05.ld/st below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + 2 * X + (j & 1)], (j >> 1) & 1))) { timeout = true; break; }
+      tc_fence_after();
+      float s[C::BN];
+      tmem_ld64(tmem + lane_base + C::s_col(X, j & 1), s);
+      const int kbase = j * C::BN;
+      // scaled row max of this tile; masked keys (past the row's position) become -inf
+      float mt_ = -INFINITY;
+      if (kbase + C::BN - 1 <= pos) {
+        float mx = s[0], mn = s[0];
+#pragma unroll
+        for (int k = 1; k < C::BN; ++k) {
+          mx = fmaxf(mx, s[k]);
+          mn = fminf(mn, s[k]);
+        }
+        mt_ = qs >= 0.f ? mx * qs : mn * qs;
+      } else {
+#pragma unroll
+        for (int k = 0; k < C::BN; ++k)
+          if (kbase + k <= pos) mt_ = fmaxf(mt_, s[k] * qs);
+      }
+      const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
+      // the previous tile's PV must be complete before O is rescaled or P is overwritten
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[kOFull + X], (j - 1) & 1))) { timeout = true; break; }
+      tc_fence_after();
+      const bool bump = mt_ > m_ref + kRescale;
+      if (__any_sync(0xffffffffu, bump)) {
+        const float m_new = bump ? mt_ : m_ref;
+        const float alpha = exp2f(m_ref - m_new);
+        if (j > 0) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            float ov[32];
+            tmem_ld32(o_addr + cc * 32, ov);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ov[k] *= alpha;
+            tmem_st32(o_addr + cc * 32, ov);
+          }
+        }
+        l_run *= alpha;
+        m_ref = m_new;
+      }
+      // last key tile: V rows of keys no row may see are zeroed (tile A's threads, one row each), so
+      // that 0 * (whatever the cache holds past the context) never reaches the MMA
+      if (X == 0 && r < C::BN && (j + 1) * C::BN > kv_len && kbase + r >= kv_len) {
+        uint8_t *vt = smem + C::OFF_V + (j % C::STAGES) * C::KV_BYTES;
 #pragma unroll
         for (int hh = 0; hh < C::DH; ++hh)
 #pragma unroll
           for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4 *>(vt + hh * C::PLANE + tid * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(vt + hh * C::KV_PLANE + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
       }
+      uint64_t ls2 = 0ull;
+      const uint64_t qs2 = f2pack(qs, qs), nm2 = f2pack(-m_ref, -m_ref);
+      uint8_t *prow = sP + r * 128;
+#pragma unroll
+      for (int q8 = 0; q8 < C::BN / 8; ++q8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2) {
+          // x = s * qscale - m_ref for two keys at once; keys past the row's position get p = 0
+          float2 x = f2unpack(ffma2(f2pack(s[q8 * 8 + 2 * k2], s[q8 * 8 + 2 * k2 + 1]), qs2, nm2));
+          if (diag) {
+            const int t = kbase + q8 * 8 + 2 * k2;
+            if (t > pos) x.x = -INFINITY;
+            if (t + 1 > pos) x.y = -INFINITY;
+          }
+          const float a = ex2(x.x);
+          const float b = ex2(x.y);
+          ls2 = f2add(ls2, f2pack(a, b));
+          pk[k2] = pack_bf16x2(a, b);
+        }
+        *reinterpret_cast<uint4 *>(prow + ((q8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      const float2 lsv = f2unpack(ls2);
+      const float ls = lsv.x + lsv.y;
+      l_run += ls;
       fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars[kPFull + X]);
     }
-    tc_fence_before();
-    if (__syncthreads_or(timeout)) break;
-    if (tid == 0) {
+    // ---- epilogue: out = O / l once the last PV is done
+    if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + X], (ntiles - 1) & 1))) {
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * C::PLANE + (kk & 3) * 32;
-        mma_bf16(tmem + C::S_COL, sw128_desc(smem_u32(sQ) + koff, 16, 1024), sw128_desc(smem_u32(kt) + koff, 16, 1024),
-                 idS, kk > 0);
-      }
-      mma_commit(&bars[2]);
-      s_inflight = true;
-    }
-    {
-      const bool ok = mbar_wait(&bars[2], j & 1);
-      timeout |= !ok;
-      if (ok) s_inflight = false;
-    }
-    tc_fence_after();
-
-    // -- row max of this tile (masked)
-    const int kbase = j * C::BN;
-    float mt_ = -INFINITY;
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      uint4 *dst = reinterpret_cast<uint4 *>(P.out + ((int64_t)(q0 + (row_ok ? pos_i : 0)) * P.num_q_heads + h) * D);
 #pragma unroll 1
-    for (int cc = 0; cc < C::BN / 32; ++cc) {
-      float s[32];
-      tmem_ld32(tmem + lane + C::S_COL + cc * 32, s);
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float ov[32];
+        tmem_ld32(o_addr + cc * 32, ov);
+        if (row_ok) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        const float x = (kbase + cc * 32 + k <= pos) ? s[k] * P.qscale : -INFINITY;
-        mt_ = fmaxf(mt_, x);
-      }
-    }
-    // -- move the reference max (and rescale this row of O and l) only when p would exceed 2^8
-    const bool bump = mt_ > m_ref + kRescale;
-    if (__any_sync(0xffffffffu, bump)) {
-      const float m_new = bump ? mt_ : m_ref;
-      const float alpha = exp2f(m_ref - m_new);          // 0 when m_ref is still -inf
-      if (j > 0) {
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          float ov[32];
-          tmem_ld32(tmem + lane + C::O_COL + cc * 32, ov);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) ov[k] *= alpha;
-          tmem_st32(tmem + lane + C::O_COL + cc * 32, ov);
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[cc * 4 + q4] = make_uint4(pack_bf16x2(ov[8 * q4] * inv, ov[8 * q4 + 1] * inv),
+                                          pack_bf16x2(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv),
+                                          pack_bf16x2(ov[8 * q4 + 4] * inv, ov[8 * q4 + 5] * inv),
+                                          pack_bf16x2(ov[8 * q4 + 6] * inv, ov[8 * q4 + 7] * inv));
         }
       }
-      l_run *= alpha;
-      m_ref = m_new;
     }
-    // -- p = 2^(s - m_ref) into the P tile (bf16, K-major swizzled), row sum
-    float ls = 0.f;
-    uint8_t *prow = sP + tid * 128;
-#pragma unroll 1
-    for (int cc = 0; cc < C::BN / 32; ++cc) {
-      float s[32];
-      tmem_ld32(tmem + lane + C::S_COL + cc * 32, s);
-      uint32_t pk[16];
+  } else if (warp == 8) {
+    // ===================================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(128, C::BN, false);
+      constexpr uint32_t idO = idesc_bf16(128, D, true);
+      const uint32_t qa = smem_u32(smem + C::OFF_QA), qb = smem_u32(smem + C::OFF_QB);
+      const uint32_t pa = smem_u32(smem + C::OFF_PA), pb = smem_u32(smem + C::OFF_PB);
+      const uint32_t kb0 = smem_u32(smem + C::OFF_K), vb0 = smem_u32(smem + C::OFF_V);
+      auto issue_s = [&](int X, int j) {
+        const uint32_t qx = X ? qb : qa;
+        const uint32_t kt = kb0 + (j % C::STAGES) * C::KV_BYTES;
 #pragma unroll
-      for (int k = 0; k < 32; k += 2) {
-        const int t = kbase + cc * 32 + k;
-        const float p0 = (t <= pos) ? exp2f(s[k] * P.qscale - m_ref) : 0.f;
-        const float p1 = (t + 1 <= pos) ? exp2f(s[k + 1] * P.qscale - m_ref) : 0.f;
-        ls += p0 + p1;
-        pk[k / 2] = pack_bf16x2(p0, p1);
-      }
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk & 3) * 32;
+          mma_bf16(tmem + C::s_col(X, j & 1), sw128_desc(qx + (kk >> 2) * C::Q_PLANE + ko, 16, 1024),
+                   sw128_desc(kt + (kk >> 2) * C::KV_PLANE + ko, 16, 1024), idS, kk > 0);
+        }
+        mma_commit(&bars[kSFull + 2 * X + (j & 1)]);
+      };
+      auto issue_o = [&](int X, int j) {
+        const uint32_t px = X ? pb : pa;
+        const uint32_t vt = vb0 + (j % C::STAGES) * C::KV_BYTES;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int kb = cc * 32 + q4 * 8;              // first key of this 16-byte chunk
-        const int ch = (kb & 63) >> 3;
-        *reinterpret_cast<uint4 *>(prow + (kb >> 6) * C::PLANE + ((ch ^ (tid & 7)) << 4)) =
-            make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
+        for (int kk = 0; kk < C::BN / 16; ++kk)
+          mma_bf16(tmem + C::o_col(X), sw128_desc(px + kk * 32, 16, 1024),
+                   sw128_desc(vt + kk * (16 * 128), C::KV_PLANE, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars[kOFull + X]);
+      };
+      auto kv_ready = [&](int j) {
+        const bool r = mbar_wait(&bars[kKvFull + (j % C::STAGES)], (j / C::STAGES) & 1);
+        tc_fence_after();
+        return r;
+      };
+      // S runs up to two key tiles ahead of PV (two S buffers per query tile)
+      bool ok = mbar_wait(&bars[kQReady], 0) && kv_ready(0);
+      if (ok) {
+        issue_s(0, 0);
+        issue_s(1, 0);
       }
-    }
-    l_run += ls;
-    fence_async_smem();
-    tc_fence_before();
-    if (__syncthreads_or(timeout)) break;
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < C::BN / 16; ++kk) {
-        const uint32_t aoff = (kk >> 2) * C::PLANE + (kk & 3) * 32;
-        mma_bf16(tmem + C::O_COL, sw128_desc(smem_u32(sP) + aoff, 16, 1024),
-                 sw128_desc(smem_u32(vt) + kk * (16 * 128), C::PLANE, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+      if (ok && ntiles > 1 && (ok = kv_ready(1))) {
+        issue_s(0, 1);
+        issue_s(1, 1);
       }
-      mma_commit(&bars[3]);
-      o_inflight = true;
-    }
-    {
-      const bool ok = mbar_wait(&bars[3], j & 1);
-      timeout |= !ok;
-      if (ok) o_inflight = false;
-    }
-    tc_fence_after();
-    if (j + 2 < ntiles) {
-      if (tid == 0) issue_tile(j + 2);  // both MMAs reading this stage are complete
-      issued = j + 3;
-    }
-  }
-
-  if (j < ntiles) {
-    // a wait gave up (error word already set): let this CTA's outstanding copies and MMAs land
-    // (bounded), then release TMEM and leave without writing
-    if (tid == 0) {
-      for (int k = j; k < issued; ++k) (void)mbar_wait(&bars[k & 1], (k >> 1) & 1);
-      if (s_inflight) (void)mbar_wait(&bars[2], j & 1);
-      if (o_inflight) (void)mbar_wait(&bars[3], j & 1);
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (!(ok = mbar_wait(&bars[kPFull + 0], j & 1))) break;
+        tc_fence_after();
+        issue_o(0, j);
+        const bool more = j + 2 < ntiles;
+        if (more) {
+          if (!(ok = kv_ready(j + 2))) break;
+          issue_s(0, j + 2);   // into the buffer softmax A has just finished reading
+        }
+        if (!(ok = mbar_wait(&bars[kPFull + 1], j & 1))) break;
+        tc_fence_after();
+        issue_o(1, j);
+        mma_commit(&bars[kKvEmpty + (j % C::STAGES)]);   // every product reading tile j issued
+        if (more) issue_s(1, j + 2);
+      }
+      mma_commit(&bars[kDone]);                    // fires once every MMA issued above has completed
+      if (!ok) timeout = true;
     }
   } else {
-    // out = O / l, read back from TMEM in 32-column pieces (every thread takes part in the loads)
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    uint4 *dst = reinterpret_cast<uint4 *>(P.out + ((int64_t)(q0 + i0 + (row_ok ? tid : 0)) * P.num_q_heads + h) * D);
-#pragma unroll 1
-    for (int cc = 0; cc < D / 32; ++cc) {
-      float ov[32];
-      tmem_ld32(tmem + lane + C::O_COL + cc * 32, ov);
-      if (row_ok) {
+    // ===================================================================== TMA producer
+    if (lane == 0) {
+      const int32_t *trow = P.block_tables + (int64_t)c * P.max_blocks_per_seq;
+      int j = 0;
+      for (; j < ntiles; ++j) {
+        const int st = j % C::STAGES;
+        if (j >= C::STAGES && !mbar_wait(&bars[kKvEmpty + st], ((j - C::STAGES) / C::STAGES) & 1)) {
+          timeout = true;
+          break;
+        }
+        const int nb = min(C::BN / kBlock, (kv_len - j * C::BN + kBlock - 1) / kBlock);
+        mbar_arrive_expect_tx(&bars[kKvFull + st], nb * 2 * C::DH * (kBlock * 128));
+        for (int bb = 0; bb < nb; ++bb) {
+          int e = __ldg(trow + j * (C::BN / kBlock) + bb);
+          if (e < 0 || e >= P.num_blocks) {
+            flag_error(kErrBlockId);
+            e = 0;
+          }
+          const int y = (e * P.num_kv_heads + g) * kBlock;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          dst[cc * 4 + q4] = make_uint4(pack_bf16x2(ov[8 * q4] * inv, ov[8 * q4 + 1] * inv),
-                                        pack_bf16x2(ov[8 * q4 + 2] * inv, ov[8 * q4 + 3] * inv),
-                                        pack_bf16x2(ov[8 * q4 + 4] * inv, ov[8 * q4 + 5] * inv),
-                                        pack_bf16x2(ov[8 * q4 + 6] * inv, ov[8 * q4 + 7] * inv));
+          for (int hh = 0; hh < C::DH; ++hh) {
+            const int off = st * C::KV_BYTES + hh * C::KV_PLANE + bb * (kBlock * 128);
+            tma_load_2d(smem + C::OFF_K + off, &kmap, hh * 64, y, &bars[kKvFull + st]);
+            tma_load_2d(smem + C::OFF_V + off, &vmap, hh * 64, y, &bars[kKvFull + st]);
+          }
+        }
       }
+      // before leaving, the last (at most two) tiles this thread issued must have landed (a no-op when
+      // the MMA warp consumed them; bounded when a wait elsewhere gave up)
+      for (int k = max(0, j - C::STAGES); k < j; ++k)
+        (void)mbar_wait(&bars[kKvFull + (k % C::STAGES)], (k / C::STAGES) & 1);
     }
   }
+  // ---- teardown: every MMA has completed before TMEM is released (bounded waits throughout; on a
+  // timeout the error word is set and the CTA leaves without its output)
+  if (warp == 8 && lane == 0) (void)mbar_wait(&bars[kDone], 0);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
@@ -464,8 +557,9 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
   if (cudaFuncSetAttribute(paged_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return -3;
-  dim3 grid((max_q_len + C::BM - 1) / C::BM, P.num_q_heads, num_chunks);
-  return launch_pdl(paged_prefill_kernel<D>, grid, dim3(128), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;
+  const int ppt = C::BM / P.hpr;
+  dim3 grid((max_q_len + 2 * ppt - 1) / (2 * ppt), P.num_q_heads / P.hpr, num_chunks);
+  return launch_pdl(paged_prefill_kernel<D>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;
 }
 
 inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
@@ -485,6 +579,7 @@ inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, in
   P.num_q_heads = num_q_heads;
   P.num_kv_heads = num_kv_heads;
   P.group = num_q_heads / num_kv_heads;
+  P.hpr = (P.group <= 128 && 128 % P.group == 0) ? P.group : 1;
   P.max_context_len = max_context_len;
   P.qscale = scale * 1.4426950408889634f;
   return head_dim == 128 ? launch_prefill_d<128>(P, k_cache, v_cache, num_chunks, max_q_len, st)

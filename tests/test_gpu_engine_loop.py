@@ -1,0 +1,120 @@
+"""Several continuous-batching iterations driven by the native block manager, on the GPU.
+
+Per iteration, as the pages describe an engine step (vLLM overview, "Continuous Batching" and
+"Prefix Sharing"; Core Concepts §3.2):
+- requests join (their prompt is appended and attended by the causal prefill);
+- running requests decode one token each (append at the end of the current block, new block when
+  full, copy-on-write when the block is shared after a fork);
+- a request forks for parallel sampling;
+- a finished request leaves and its blocks are reused.
+Every attention output is checked against the oracle, computed from each request's own token history
+in a fresh contiguous cache.
+"""
+import numpy as np
+import pytest
+import torch
+
+from pagedattention_block_table_b200.inputs import bf16_bits
+from tests.common import assert_close, to_f64
+
+pytestmark = pytest.mark.gpu
+
+HQ, HKV, D = 8, 2, 128
+SCALE = D ** -0.5
+
+
+def _oracle_rows(O, k_rows, v_rows, q_rows, lens):
+    """Attention of q_rows[i] over the first lens[i] tokens of (k_rows, v_rows), contiguous cache."""
+    L = k_rows.shape[0]
+    nblk = (L + 15) // 16
+    kc = np.zeros((nblk, HKV, 16, D), np.uint16)
+    vc = np.zeros_like(kc)
+    O.kv_append(kc, vc, k_rows, v_rows, np.arange(L, dtype=np.int64))
+    n = q_rows.shape[0]
+    tables = np.tile(np.arange(nblk, dtype=np.int32)[None], (n, 1))
+    return O.paged_decode(q_rows, kc, vc, tables, np.asarray(lens, np.int32), SCALE)
+
+
+def test_block_manager_drives_append_prefill_decode(O, cuda_lib):
+    B = cuda_lib
+    g = torch.Generator(device="cuda").manual_seed(7)
+    nb = 256
+    kc = torch.zeros((nb, HKV, 16, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    bm = B.pa_bm_create(nb, 99)
+    hist = {}                                   # request id -> (K rows, V rows) on the device
+
+    def new_tokens(n):
+        return (torch.randn((n, HKV, D), generator=g, device="cuda").to(torch.bfloat16),
+                torch.randn((n, HKV, D), generator=g, device="cuda").to(torch.bfloat16))
+
+    def append(rid, k, v):
+        slots, cow = B.pa_bm_append(bm, rid, k.shape[0])
+        if cow is not None:
+            B.pa_copy_blocks(kc, vc, torch.from_numpy(cow.reshape(1, 2)).cuda())
+        B.pa_kv_append(kc, vc, k, v, torch.from_numpy(slots).cuda())
+        hk, hv = hist.get(rid, (k[:0], v[:0]))
+        hist[rid] = (torch.cat([hk, k]), torch.cat([hv, v]))
+        return cow
+
+    def prefill(rids, chunks):
+        """Causal prefill of the chunks just appended to requests `rids`."""
+        lens = [B.pa_bm_length(bm, r) for r in rids]
+        mbs = max((L + 15) // 16 for L in lens)
+        tables, tl = B.pa_bm_tables(bm, rids, mbs)
+        cu = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+        q = torch.randn((int(cu[-1]), HQ, D), generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty_like(q)
+        B.pa_paged_prefill(out, q, torch.from_numpy(cu).cuda(), kc, vc, torch.from_numpy(tables).cuda(),
+                           torch.from_numpy(tl).cuda(), SCALE, max(chunks), max(lens))
+        torch.cuda.synchronize()
+        got = to_f64(out)
+        for i, r in enumerate(rids):
+            C, L = chunks[i], lens[i]
+            k, v = hist[r]
+            qb = bf16_bits(q[cu[i]:cu[i + 1]])
+            ref = _oracle_rows(O, bf16_bits(k), bf16_bits(v), qb, [L - C + j + 1 for j in range(C)])
+            assert_close(got[cu[i]:cu[i + 1]], ref, what=f"prefill of request {r}")
+
+    def decode(rids):
+        lens = [B.pa_bm_length(bm, r) for r in rids]
+        mbs = max((L + 15) // 16 for L in lens)
+        tables, tl = B.pa_bm_tables(bm, rids, mbs)
+        q = torch.randn((len(rids), HQ, D), generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty_like(q)
+        ws = torch.empty(B.pa_paged_attention_workspace_size(len(rids), HQ, D, max(lens), 64) // 4 + 4,
+                         device="cuda")
+        B.pa_paged_attention(out, q, kc, vc, torch.from_numpy(tables).cuda(), torch.from_numpy(tl).cuda(), SCALE,
+                             max(lens), split_tokens=64, workspace=ws)
+        torch.cuda.synchronize()
+        got = to_f64(out)
+        for i, r in enumerate(rids):
+            k, v = hist[r]
+            ref = _oracle_rows(O, bf16_bits(k), bf16_bits(v), bf16_bits(q[i:i + 1]), [lens[i]])
+            assert_close(got[i], ref[0], what=f"decode of request {r}")
+
+    try:
+        # iteration 1: two requests join with prompts of 37 and 100 tokens
+        for rid, n in ((1, 37), (2, 100)):
+            B.pa_bm_add(bm, rid)
+            append(rid, *new_tokens(n))
+        prefill([1, 2], [37, 100])
+        cows = 0
+        for it in range(6):
+            if it == 2:                          # request 1 forks (parallel sampling): shares every page
+                B.pa_bm_fork(bm, 1, 3)
+                hist[3] = hist[1]
+            if it == 4:                          # request 2 finishes and leaves; request 4 joins
+                B.pa_bm_free(bm, 2)
+                del hist[2]
+                B.pa_bm_add(bm, 4)
+                append(4, *new_tokens(50))
+                prefill([4], [50])
+            running = sorted(hist)
+            for r in running:
+                cows += append(r, *new_tokens(1)) is not None
+            decode(running)
+        assert cows >= 1, "the fork must have triggered copy-on-write"
+        assert B.pa_get_device_error() == B.PA_OK
+    finally:
+        B.pa_bm_destroy(bm)

@@ -31,6 +31,9 @@ CASES = {
     "mha_d128": _chunks(num_q_heads=4, num_kv_heads=4, chunk_len=(100, 260)),
     "gqa2_d64": _chunks(head_dim=64, num_q_heads=4, num_kv_heads=2),
     "tiny_chunks": _chunks(prefill_chunks=5, chunk_len=(1, 17), chunk_hist=(1, 40)),
+    "gqa8_d128": _chunks(num_q_heads=16, num_kv_heads=2, chunk_len=(20, 150)),
+    "gqa3_d128": _chunks(num_q_heads=6, num_kv_heads=2, chunk_len=(60, 200)),
+    "gqa16_d64": _chunks(num_q_heads=16, num_kv_heads=1, head_dim=64, chunk_len=(5, 90)),
 }
 
 

@@ -85,8 +85,9 @@ def test_e4m3_encode_matches_torch_cast(O):
     (the quotients an FP8 append forms), plus all code midpoints (ties)."""
     bits = np.arange(0, 0x7F80, 7, dtype=np.uint32)
     xs = [(bits << 16).view(np.float32)]
-    for s in (0.0123, 0.5, 1.0 / 448 * 3.7):
-        xs.append((xs[0] / np.float32(s)).astype(np.float32))
+    with np.errstate(over="ignore"):
+        for s in (0.0123, 0.5, 1.0 / 448 * 3.7):
+            xs.append((xs[0] / np.float32(s)).astype(np.float32))
     vals = O.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
     mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
     x = np.concatenate(xs + [mids, -mids])
