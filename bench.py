@@ -55,7 +55,7 @@ def decode_bytes(batch) -> int:
     e = 1 if batch.kv_dtype else 2
     kv = int(ctx.sum()) * 2 * batch.num_kv_heads * batch.head_dim * e
     qo = 2 * nd * batch.num_q_heads * batch.head_dim * 2
-    tables = int(((ctx + 15) // 16).sum()) * 4 + 4 * nd
+    tables = int(((ctx + batch.block_size - 1) // batch.block_size).sum()) * 4 + 4 * nd
     return kv + qo + tables
 
 
@@ -87,7 +87,8 @@ def kv_unique_bytes(batch) -> int:
     for s in range(nd):
         L = int(batch.context_lens[s])
         t = np.arange(L, dtype=np.int64)
-        slots.append(batch.block_tables[s, t // 16].astype(np.int64) * 16 + t % 16)
+        bs = batch.block_size
+        slots.append(batch.block_tables[s, t // bs].astype(np.int64) * bs + t % bs)
     n = np.unique(np.concatenate(slots)).shape[0] if slots else 0
     return int(n) * 2 * batch.num_kv_heads * batch.head_dim * e
 
@@ -302,7 +303,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             "workload": args.workload,
             "num_seqs": batch.num_decode, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
-            "head_dim": batch.head_dim, "block_size": 16, "num_blocks": batch.num_blocks,
+            "head_dim": batch.head_dim, "block_size": batch.block_size, "num_blocks": batch.num_blocks,
             "context_tokens": int(batch.context_lens[:batch.num_decode].sum()),
             "prefill_chunks": int(batch.num_seqs - batch.num_decode), "cow_pairs": int(batch.cow_pairs.shape[0]),
             "split_tokens": st.split_tokens,

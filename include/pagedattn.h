@@ -18,16 +18,17 @@
  *                      query heads share one KV head).
  *
  * Common conventions
- *   - Block size is 16 tokens (PA_BLOCK_SIZE).  A KV cache is two device arrays, K and V, each
- *     laid out [num_blocks][num_kv_heads][16][head_dim] ("HND"): one (block, KV head) tile is
- *     16*head_dim contiguous elements.  Elements are bf16 (PA_KV_BF16), OCP FP8 E4M3
+ *   - Block size bs is 16 (PA_BLOCK_SIZE) or 32 tokens [Core Concepts §3.2: "usually 16 or 32"], passed
+ *     as `block_size`.  A KV cache is two device arrays, K and V, each laid out
+ *     [num_blocks][num_kv_heads][bs][head_dim] ("HND"): one (block, KV head) tile is bs*head_dim
+ *     contiguous elements.  Elements are bf16 (PA_KV_BF16), OCP FP8 E4M3
  *     (PA_KV_FP8_E4M3) or signed INT8 (PA_KV_INT8, codes -127..127); the one-byte formats carry one
  *     fp32 scale per KV head for K and one for V: value = code * scale.
  *   - head_dim is 64 or 128.  num_q_heads must be a multiple of num_kv_heads; query head h uses
  *     KV head h / (num_q_heads / num_kv_heads) (any group size).
  *   - bf16 tensors (q, k, v, out) are row-major with the last dimension contiguous.
  *   - A block table is int32 [num_seqs][max_blocks_per_seq]: entry i is the physical block holding
- *     tokens 16*i .. 16*i+15 of that sequence; entries past ceil(context_len/16) are never read.
+ *     tokens bs*i .. bs*i+bs-1 of that sequence; entries past ceil(context_len/bs) are never read.
  *   - All pointers are DEVICE pointers unless stated; all buffers are owned by the caller; the
  *     library never allocates device memory.  Every call is asynchronous on `stream` (0 = the
  *     legacy default stream) and returns after launching.
@@ -62,7 +63,7 @@ typedef int pa_status;
 #define PA_EWORKSPACE (-5)    /* workspace missing or smaller than required */
 #define PA_ENOMEM (-6)        /* block manager: not enough free blocks (nothing was changed) */
 
-#define PA_BLOCK_SIZE 16
+#define PA_BLOCK_SIZE 16      /* the default block size; 32 is also supported */
 #define PA_KV_BF16 0
 #define PA_KV_FP8_E4M3 1
 #define PA_KV_INT8 2
@@ -72,7 +73,7 @@ typedef int pa_status;
  * written at the end of its sequence's current block; prefill writes all prompt tokens].
  *   k_cache, v_cache : the cache (see conventions), written in place.
  *   k, v             : bf16 [num_tokens][num_kv_heads][head_dim], the new tokens.
- *   slot_mapping     : int64 [num_tokens]; token n goes to block slot/16, offset slot%16.  A negative
+ *   slot_mapping     : int64 [num_tokens]; token n goes to block slot/bs, offset slot%bs.  A negative
  *                      slot means "padding, write nothing".  Slots must be distinct.
  *   kv_dtype         : PA_KV_BF16 (bit copy), PA_KV_FP8_E4M3: code = E4M3(x / scale[h]), the
  *                      binary32 quotient rounded to nearest even and saturated to +-448, or
@@ -84,33 +85,33 @@ typedef int pa_status;
  */
 pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *v,
                        const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
-                       int head_dim, int64_t num_blocks, int kv_dtype, const float *k_scale,
-                       const float *v_scale, pa_stream_t stream);
+                       int head_dim, int64_t num_blocks, int block_size, int kv_dtype,
+                       const float *k_scale, const float *v_scale, pa_stream_t stream);
 
 /*
  * pa_copy_blocks -- copy-on-write fork [vLLM overview, Prefix Sharing: after divergence the new token
  * is written into a copied page; the shared page stays unchanged].  For each pair p the whole physical
- * block src_dst_pairs[2p] (all KV heads, 16 slots, K and V) is copied to block src_dst_pairs[2p+1].
+ * block src_dst_pairs[2p] (all KV heads, bs slots, K and V) is copied to block src_dst_pairs[2p+1].
  *   src_dst_pairs : int32 [num_pairs][2] on the device.  Preconditions: destinations are distinct and
  *                   no destination is also a source in the same call (copies run concurrently).
  */
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, int num_pairs,
-                         int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype,
-                         pa_stream_t stream);
+                         int num_kv_heads, int head_dim, int64_t num_blocks, int block_size,
+                         int kv_dtype, pa_stream_t stream);
 
 /*
  * pa_swap_blocks -- move whole blocks between two pools [vLLM overview, section 三: when GPU memory
  * runs short KV pages are swapped out to CPU memory, and swapped back in when the request resumes].
- * For each pair p, block src_dst_pairs[2p] of the source pool (all KV heads, 16 slots, K and V) is
+ * For each pair p, block src_dst_pairs[2p] of the source pool (all KV heads, bs slots, K and V) is
  * copied into block src_dst_pairs[2p+1] of the destination pool.  Both pools have the cache layout
- * and the same num_kv_heads, head_dim and kv_dtype; each may live in device memory or in pinned,
+ * and the same num_kv_heads, head_dim, block_size and kv_dtype; each may live in device memory or in pinned,
  * mapped host memory (cudaHostAlloc / cudaHostRegister): the kernel reads and writes host memory
  * directly over the host link.  src_dst_pairs must be device-accessible as well.  Pageable host
  * memory is rejected with PA_EINVAL.  Destinations must be distinct and must not overlap sources.
  */
 pa_status pa_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const void *src_k,
                          const void *src_v, int64_t src_num_blocks, const int32_t *src_dst_pairs,
-                         int num_pairs, int num_kv_heads, int head_dim, int kv_dtype,
+                         int num_pairs, int num_kv_heads, int head_dim, int block_size, int kv_dtype,
                          pa_stream_t stream);
 
 /*
@@ -131,7 +132,7 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
  * non-contiguous K/V through the block table; KV Cache to vLLM §1.2: the new token's query attends
  * over all cached keys and takes the weighted sum of values; §2.2 GQA].  For every sequence b and
  * query head h:  out[b][h] = softmax_t(scale * q[b][h] . K_b[t]) . V_b[t]  over t < context_lens[b],
- * K_b[t] = k_cache[block_tables[b][t/16]][h/G][t%16].  context_lens counts the newest token (append
+ * K_b[t] = k_cache[block_tables[b][t/bs]][h/G][t%bs].  context_lens counts the newest token (append
  * first, then attend).  A context length of 0 gives a zero row.
  *   out          : bf16 [num_seqs][num_q_heads][head_dim]
  *   q            : bf16 [num_seqs][num_q_heads][head_dim]
@@ -146,8 +147,8 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
 pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *block_tables, int max_blocks_per_seq,
                              const int32_t *context_lens, int num_seqs, int num_q_heads,
-                             int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
-                             int kv_dtype, const float *k_scale, const float *v_scale,
+                             int num_kv_heads, int head_dim, int64_t num_blocks, int block_size,
+                             float scale, int kv_dtype, const float *k_scale, const float *v_scale,
                              int max_context_len, int split_tokens, void *workspace,
                              size_t workspace_bytes, pa_stream_t stream);
 
@@ -157,7 +158,8 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
  * themselves: a plugin inside a serving engine that has already reserved the GPU's memory for its
  * own KV pool and forbids further allocations, or a latency-critical loop that must not take the
  * device-wide synchronisation a cudaMalloc/cudaFree implies.  Arguments and results are those of
- * pa_paged_attention without `workspace`; the caller still passes every input and output buffer.
+ * pa_paged_attention without `workspace`, for 16-token blocks; the caller still passes every input and
+ * output buffer.
  *
  * Instead of a caller workspace, the split-K partials go to one library-owned scratch array of
  * PA_NOALLOC_SCRATCH_BYTES (a file-scope __device__ array: every GPU that loads the library holds
@@ -193,8 +195,9 @@ pa_status pa_paged_attention_noalloc(void *out, const void *q, const void *k_cac
 pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks,
                            const void *k_cache, const void *v_cache, const int32_t *block_tables,
                            int max_blocks_per_seq, const int32_t *context_lens, int num_q_heads,
-                           int num_kv_heads, int head_dim, int64_t num_blocks, float scale,
-                           int kv_dtype, int max_q_len, int max_context_len, pa_stream_t stream);
+                           int num_kv_heads, int head_dim, int64_t num_blocks, int block_size,
+                           float scale, int kv_dtype, int max_q_len, int max_context_len,
+                           pa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------------
  * Host block manager: the control plane that produces block tables, slot mappings and copy-on-write
@@ -219,7 +222,7 @@ pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id);
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent, int64_t child);
 /*
  * pa_bm_append -- reserve slots for n_tokens new tokens at the end of seq_id and write them to
- * slots_out[n_tokens] (slot = block*16 + offset, ready for pa_kv_append).  If the block that receives
+ * slots_out[n_tokens] (slot = block*16 + offset, ready for pa_kv_append with 16-token blocks).  If the block that receives
  * the first new token is shared, it is first replaced by a private copy: the (src, dst) pair goes to
  * cow_pairs_out[2] (run pa_copy_blocks on it before the append) and *num_cow_out = 1, else 0.
  * PA_ENOMEM if the pool cannot supply the blocks; then nothing changes.

@@ -20,7 +20,8 @@
  *                    §2.1 (KV size formula), §2.2 (1-byte KV storage, GQA head sharing).
  *
  * Conventions (the pages fix none of these; the readings are listed with the design notes):
- *   - block size 16 tokens; cache layout [num_blocks][num_kv_heads][16][head_dim];
+ *   - block size bs = 16 or 32 tokens (Core Concepts §3.2: "usually 16 or 32");
+ *     cache layout [num_blocks][num_kv_heads][bs][head_dim];
  *   - bf16 values are passed as their 16-bit patterns (uint16_t), fp8 as E4M3 bytes;
  *   - query head h uses KV head floor(h / (Hq / Hkv)) (contiguous GQA groups);
  *   - all attention arithmetic is fp64 on the exact values of the inputs.
@@ -33,7 +34,6 @@
 #include <stdlib.h>
 #include <string.h>
 
-#define ORACLE_BLOCK 16
 
 /* ---------------------------------------------------------------- value formats */
 
@@ -126,32 +126,32 @@ int64_t oracle_kv_cache_bytes(int64_t layers, int64_t kv_heads, int64_t head_dim
 
 /*
  * Append [Core Concepts §3.2, "PagedAttention 如何工作"]: each token n carries its
- * slot = physical_block * 16 + offset; its K and V rows (all KV heads) are written at
- * cache[slot / 16][h][slot % 16][:].  slot < 0 marks a padding token: nothing written.
+ * slot = physical_block * bs + offset; its K and V rows (all KV heads) are written at
+ * cache[slot / bs][h][slot % bs][:].  slot < 0 marks a padding token: nothing written.
  * kv_dtype 0 = bf16 (bit copy), 1 = fp8 E4M3 (code of the binary32 quotient x / scale[h]),
  * 2 = int8 (rounded quotient, see oracle_int8_encode).
  */
 int oracle_kv_append(void *k_cache, void *v_cache, const uint16_t *k, const uint16_t *v,
                      const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads,
-                     int head_dim, int64_t num_blocks, int kv_dtype,
+                     int head_dim, int64_t num_blocks, int bs, int kv_dtype,
                      const float *k_scale, const float *v_scale)
 {
-    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0) return -1;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || bs <= 0) return -1;
     if (kv_dtype < 0 || kv_dtype > 2) return -1;
     for (int64_t n = 0; n < num_tokens; ++n) {
         int64_t slot = slot_mapping[n];
         if (slot < 0) continue;
-        if (slot >= num_blocks * ORACLE_BLOCK) return -4;
+        if (slot >= num_blocks * bs) return -4;
     }
     for (int64_t n = 0; n < num_tokens; ++n) {
         int64_t slot = slot_mapping[n];
         int64_t blk, off;
         if (slot < 0) continue;
-        blk = slot / ORACLE_BLOCK;
-        off = slot % ORACLE_BLOCK;
+        blk = slot / bs;
+        off = slot % bs;
         for (int h = 0; h < num_kv_heads; ++h) {
             int64_t src = (n * num_kv_heads + h) * (int64_t)head_dim;
-            int64_t dst = ((blk * num_kv_heads + h) * ORACLE_BLOCK + off) * (int64_t)head_dim;
+            int64_t dst = ((blk * num_kv_heads + h) * bs + off) * (int64_t)head_dim;
             for (int d = 0; d < head_dim; ++d) {
                 if (kv_dtype == 0) {
                     ((uint16_t *)k_cache)[dst + d] = k[src + d];
@@ -183,9 +183,9 @@ int oracle_kv_append(void *k_cache, void *v_cache, const uint16_t *k, const uint
  * Pairs are applied in order.
  */
 int oracle_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int64_t num_pairs,
-                       int num_kv_heads, int head_dim, int64_t num_blocks, int elem_bytes)
+                       int num_kv_heads, int head_dim, int64_t num_blocks, int bs, int elem_bytes)
 {
-    int64_t block_bytes = (int64_t)num_kv_heads * ORACLE_BLOCK * head_dim * elem_bytes;
+    int64_t block_bytes = (int64_t)num_kv_heads * bs * head_dim * elem_bytes;
     if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || elem_bytes <= 0) return -1;
     for (int64_t p = 0; p < num_pairs; ++p) {
         int32_t s = pairs[2 * p], d = pairs[2 * p + 1];
@@ -207,9 +207,9 @@ int oracle_copy_blocks(void *k_cache, void *v_cache, const int32_t *pairs, int64
  */
 int oracle_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const void *src_k, const void *src_v,
                        int64_t src_num_blocks, const int32_t *pairs, int64_t num_pairs, int num_kv_heads,
-                       int head_dim, int elem_bytes)
+                       int head_dim, int bs, int elem_bytes)
 {
-    int64_t block_bytes = (int64_t)num_kv_heads * ORACLE_BLOCK * head_dim * elem_bytes;
+    int64_t block_bytes = (int64_t)num_kv_heads * bs * head_dim * elem_bytes;
     if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || elem_bytes <= 0) return -1;
     for (int64_t p = 0; p < num_pairs; ++p) {
         int32_t s = pairs[2 * p], d = pairs[2 * p + 1];
@@ -226,11 +226,11 @@ int oracle_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const v
 /* ---------------------------------------------------------------- attention */
 
 /* value of element d of token t (logical position) of KV head g of one sequence, read
- * through that sequence's block table: physical block = table[t / 16], slot t % 16. */
-static double cache_value(const void *cache, int kv_dtype, float scale, int64_t phys,
+ * through that sequence's block table: physical block = table[t / bs], slot t % bs. */
+static double cache_value(const void *cache, int kv_dtype, float scale, int64_t phys, int bs,
                           int num_kv_heads, int g, int64_t t, int head_dim, int d)
 {
-    int64_t idx = ((phys * num_kv_heads + g) * ORACLE_BLOCK + (t % ORACLE_BLOCK)) * (int64_t)head_dim + d;
+    int64_t idx = ((phys * num_kv_heads + g) * bs + (t % bs)) * (int64_t)head_dim + d;
     if (kv_dtype == 0) return bf16_value(((const uint16_t *)cache)[idx]);
     if (kv_dtype == 2) return (double)((const int8_t *)cache)[idx] * (double)scale;
     return oracle_e4m3_decode(((const uint8_t *)cache)[idx]) * (double)scale;
@@ -245,18 +245,18 @@ static double cache_value(const void *cache, int kv_dtype, float scale, int64_t 
  */
 static int attend_one(double *out, const uint16_t *q, const void *k_cache, const void *v_cache,
                       int kv_dtype, float ks, float vs, const int32_t *table, int64_t n_keys,
-                      int num_kv_heads, int g, int head_dim, int64_t num_blocks, double scale,
+                      int num_kv_heads, int g, int head_dim, int64_t num_blocks, int bs, double scale,
                       double *K, double *V, double *s)
 {
     double mx, sum;
     for (int d = 0; d < head_dim; ++d) out[d] = 0.0;
     if (n_keys == 0) return 0;
     for (int64_t t = 0; t < n_keys; ++t) {
-        int64_t phys = table[t / ORACLE_BLOCK];
+        int64_t phys = table[t / bs];
         if (phys < 0 || phys >= num_blocks) return -4;
         for (int d = 0; d < head_dim; ++d) {
-            K[t * head_dim + d] = cache_value(k_cache, kv_dtype, ks, phys, num_kv_heads, g, t, head_dim, d);
-            V[t * head_dim + d] = cache_value(v_cache, kv_dtype, vs, phys, num_kv_heads, g, t, head_dim, d);
+            K[t * head_dim + d] = cache_value(k_cache, kv_dtype, ks, phys, bs, num_kv_heads, g, t, head_dim, d);
+            V[t * head_dim + d] = cache_value(v_cache, kv_dtype, vs, phys, bs, num_kv_heads, g, t, head_dim, d);
         }
     }
     for (int64_t t = 0; t < n_keys; ++t) {
@@ -284,7 +284,7 @@ static int attend_one(double *out, const uint16_t *q, const void *k_cache, const
 int oracle_paged_decode(double *out, const uint16_t *q, const void *k_cache, const void *v_cache,
                         const int32_t *block_tables, int max_blocks_per_seq,
                         const int32_t *context_lens, int num_seqs, int num_q_heads,
-                        int num_kv_heads, int head_dim, int64_t num_blocks, double scale,
+                        int num_kv_heads, int head_dim, int64_t num_blocks, int bs, double scale,
                         int kv_dtype, const float *k_scale, const float *v_scale)
 {
     int64_t max_len = 0;
@@ -293,7 +293,7 @@ int oracle_paged_decode(double *out, const uint16_t *q, const void *k_cache, con
     if (num_q_heads % num_kv_heads != 0) return -1;
     for (int b = 0; b < num_seqs; ++b) {
         if (context_lens[b] < 0) return -1;
-        if ((context_lens[b] + ORACLE_BLOCK - 1) / ORACLE_BLOCK > max_blocks_per_seq) return -1;
+        if ((context_lens[b] + bs - 1) / bs > max_blocks_per_seq) return -1;
         if (context_lens[b] > max_len) max_len = context_lens[b];
     }
 #pragma omp parallel reduction(min : status)
@@ -308,7 +308,7 @@ int oracle_paged_decode(double *out, const uint16_t *q, const void *k_cache, con
             float ks = kv_dtype ? k_scale[g] : 1.0f, vs = kv_dtype ? v_scale[g] : 1.0f;
             int r = attend_one(out + bh * head_dim, q + bh * head_dim, k_cache, v_cache, kv_dtype,
                                ks, vs, block_tables + (int64_t)b * max_blocks_per_seq,
-                               context_lens[b], num_kv_heads, g, head_dim, num_blocks, scale,
+                               context_lens[b], num_kv_heads, g, head_dim, num_blocks, bs, scale,
                                K, V, s);
             if (r < status) status = r;
         }
@@ -330,7 +330,7 @@ int oracle_paged_decode(double *out, const uint16_t *q, const void *k_cache, con
 int oracle_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q_lens, int num_chunks,
                          const void *k_cache, const void *v_cache, const int32_t *block_tables,
                          int max_blocks_per_seq, const int32_t *context_lens, int num_q_heads,
-                         int num_kv_heads, int head_dim, int64_t num_blocks, double scale,
+                         int num_kv_heads, int head_dim, int64_t num_blocks, int bs, double scale,
                          int kv_dtype, const float *k_scale, const float *v_scale)
 {
     int64_t max_len = 0, total_q;
@@ -340,7 +340,7 @@ int oracle_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q_len
     for (int c = 0; c < num_chunks; ++c) {
         int32_t C = cu_q_lens[c + 1] - cu_q_lens[c];
         if (C < 0 || context_lens[c] < C) return -1;
-        if ((context_lens[c] + ORACLE_BLOCK - 1) / ORACLE_BLOCK > max_blocks_per_seq) return -1;
+        if ((context_lens[c] + bs - 1) / bs > max_blocks_per_seq) return -1;
         if (context_lens[c] > max_len) max_len = context_lens[c];
     }
     total_q = num_chunks > 0 ? cu_q_lens[num_chunks] : 0;
@@ -363,7 +363,7 @@ int oracle_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q_len
             hist = context_lens[c] - (cu_q_lens[c + 1] - cu_q_lens[c]);
             r = attend_one(out + ih * head_dim, q + ih * head_dim, k_cache, v_cache, kv_dtype, ks, vs,
                            block_tables + (int64_t)c * max_blocks_per_seq, hist + i + 1,
-                           num_kv_heads, g, head_dim, num_blocks, scale, K, V, s);
+                           num_kv_heads, g, head_dim, num_blocks, bs, scale, K, V, s);
             if (r < status) status = r;
         }
         free(K);

@@ -37,15 +37,15 @@ def configure(lib):
     lib.oracle_kv_cache_bytes.restype = L
     lib.oracle_kv_cache_bytes.argtypes = [L, L, L, L, L, L]
     lib.oracle_kv_append.restype = I
-    lib.oracle_kv_append.argtypes = [P, P, P, P, P, L, I, I, L, I, P, P]
+    lib.oracle_kv_append.argtypes = [P, P, P, P, P, L, I, I, L, I, I, P, P]
     lib.oracle_copy_blocks.restype = I
-    lib.oracle_copy_blocks.argtypes = [P, P, P, L, I, I, L, I]
+    lib.oracle_copy_blocks.argtypes = [P, P, P, L, I, I, L, I, I]
     lib.oracle_swap_blocks.restype = I
-    lib.oracle_swap_blocks.argtypes = [P, P, L, P, P, L, P, L, I, I, I]
+    lib.oracle_swap_blocks.argtypes = [P, P, L, P, P, L, P, L, I, I, I, I]
     lib.oracle_paged_decode.restype = I
-    lib.oracle_paged_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, L, D, I, P, P]
+    lib.oracle_paged_decode.argtypes = [P, P, P, P, P, I, P, I, I, I, I, L, I, D, I, P, P]
     lib.oracle_paged_prefill.restype = I
-    lib.oracle_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, L, D, I, P, P]
+    lib.oracle_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, L, I, D, I, P, P]
     lib.oracle_num_threads.restype = I
     lib.oracle_num_threads.argtypes = []
     return lib
@@ -111,14 +111,13 @@ def kv_append(k_cache, v_cache, k, v, slot_mapping, kv_dtype=0, k_scale=None, v_
     lib = _load()
     assert k_cache.flags.c_contiguous and v_cache.flags.c_contiguous
     nb, hkv, bs, d = k_cache.shape
-    assert bs == 16
     k = _c(k, np.uint16)
     v = _c(v, np.uint16)
     sm = _c(slot_mapping, np.int64)
     ks = None if k_scale is None else _c(k_scale, np.float32)
     vs = None if v_scale is None else _c(v_scale, np.float32)
     rc = lib.oracle_kv_append(_p(k_cache), _p(v_cache), _p(k), _p(v), _p(sm), sm.shape[0], hkv, d,
-                              nb, kv_dtype, _p(ks), _p(vs))
+                              nb, bs, kv_dtype, _p(ks), _p(vs))
     _check(rc, "kv_append")
 
 
@@ -127,7 +126,7 @@ def copy_blocks(k_cache, v_cache, pairs):
     lib = _load()
     nb, hkv, bs, d = k_cache.shape
     pr = _c(pairs, np.int32).reshape(-1, 2)
-    rc = lib.oracle_copy_blocks(_p(k_cache), _p(v_cache), _p(pr), pr.shape[0], hkv, d, nb,
+    rc = lib.oracle_copy_blocks(_p(k_cache), _p(v_cache), _p(pr), pr.shape[0], hkv, d, nb, bs,
                                 k_cache.dtype.itemsize)
     _check(rc, "copy_blocks")
 
@@ -135,12 +134,13 @@ def copy_blocks(k_cache, v_cache, pairs):
 def swap_blocks(dst_k, dst_v, src_k, src_v, pairs):
     """Copy whole blocks src (of the source pool) -> dst (of the destination pool), in place."""
     lib = _load()
-    nbd, hkv, _, d = dst_k.shape
+    nbd, hkv, bs, d = dst_k.shape
     nbs = src_k.shape[0]
     assert src_k.shape[1:] == dst_k.shape[1:] and src_k.dtype == dst_k.dtype
     pr = _c(pairs, np.int32).reshape(-1, 2)
     rc = lib.oracle_swap_blocks(_p(dst_k), _p(dst_v), nbd, _p(np.ascontiguousarray(src_k)),
-                                _p(np.ascontiguousarray(src_v)), nbs, _p(pr), pr.shape[0], hkv, d, dst_k.dtype.itemsize)
+                                _p(np.ascontiguousarray(src_v)), nbs, _p(pr), pr.shape[0], hkv, d, bs,
+                                dst_k.dtype.itemsize)
     _check(rc, "swap_blocks")
 
 
@@ -150,7 +150,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, kv_dtyp
     lib = _load()
     q = _c(q, np.uint16)
     b, hq, d = q.shape
-    nb, hkv, _, d2 = k_cache.shape
+    nb, hkv, bs, d2 = k_cache.shape
     assert d == d2
     bt = _c(block_tables, np.int32)
     cl = _c(context_lens, np.int32)
@@ -158,7 +158,7 @@ def paged_decode(q, k_cache, v_cache, block_tables, context_lens, scale, kv_dtyp
     ks = None if k_scale is None else _c(k_scale, np.float32)
     vs = None if v_scale is None else _c(v_scale, np.float32)
     rc = lib.oracle_paged_decode(_p(out), _p(q), _p(k_cache), _p(v_cache), _p(bt), bt.shape[1],
-                                 _p(cl), b, hq, hkv, d, nb, float(scale), kv_dtype, _p(ks), _p(vs))
+                                 _p(cl), b, hq, hkv, d, nb, bs, float(scale), kv_dtype, _p(ks), _p(vs))
     _check(rc, "paged_decode")
     return out
 
@@ -169,7 +169,7 @@ def paged_prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, sc
     lib = _load()
     q = _c(q, np.uint16)
     tq, hq, d = q.shape
-    nb, hkv, _, _ = k_cache.shape
+    nb, hkv, bs, _ = k_cache.shape
     cu = _c(cu_q_lens, np.int32)
     bt = _c(block_tables, np.int32)
     cl = _c(context_lens, np.int32)
@@ -178,7 +178,7 @@ def paged_prefill(q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, sc
     ks = None if k_scale is None else _c(k_scale, np.float32)
     vs = None if v_scale is None else _c(v_scale, np.float32)
     rc = lib.oracle_paged_prefill(_p(out), _p(q), _p(cu), cu.shape[0] - 1, _p(k_cache), _p(v_cache),
-                                  _p(bt), bt.shape[1], _p(cl), hq, hkv, d, nb, float(scale), kv_dtype,
+                                  _p(bt), bt.shape[1], _p(cl), hq, hkv, d, nb, bs, float(scale), kv_dtype,
                                   _p(ks), _p(vs))
     _check(rc, "paged_prefill")
     return out

@@ -59,21 +59,21 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I, I64, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
         L.pa_kv_append.restype = I
-        L.pa_kv_append.argtypes = [P, P, P, P, P, I64, I, I, I64, I, P, P, P]
+        L.pa_kv_append.argtypes = [P, P, P, P, P, I64, I, I, I64, I, I, P, P, P]
         L.pa_copy_blocks.restype = I
-        L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I64, I, P]
+        L.pa_copy_blocks.argtypes = [P, P, P, I, I, I, I64, I, I, P]
         L.pa_swap_blocks.restype = I
-        L.pa_swap_blocks.argtypes = [P, P, I64, P, P, I64, P, I, I, I, I, P]
+        L.pa_swap_blocks.argtypes = [P, P, I64, P, P, I64, P, I, I, I, I, I, P]
         L.pa_paged_attention_workspace_size.restype = SZ
         L.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I]
         L.pa_paged_attention_auto_split.restype = I
         L.pa_paged_attention_auto_split.argtypes = [I, I, I, I, I, I]
         L.pa_paged_attention.restype = I
-        L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P, SZ, P]
+        L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, I, F, I, P, P, I, I, P, SZ, P]
         L.pa_paged_attention_noalloc.restype = I
         L.pa_paged_attention_noalloc.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P]
         L.pa_paged_prefill.restype = I
-        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, F, I, I, I, P]
+        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, I, F, I, I, I, P]
         L.pa_get_device_error.restype = I
         L.pa_get_device_error.argtypes = [P]
         L.pa_status_string.restype = ctypes.c_char_p
@@ -141,10 +141,11 @@ _CACHE_DTYPES = {PA_KV_BF16: (torch.bfloat16,), PA_KV_FP8_E4M3: (torch.uint8, to
 
 
 def _cache_geometry(k_cache: torch.Tensor):
-    if k_cache.dim() != 4 or k_cache.shape[2] != PA_BLOCK_SIZE:
-        raise ValueError("cache must be [num_blocks][num_kv_heads][16][head_dim]")
-    nb, hkv, _, d = k_cache.shape
-    return int(nb), int(hkv), int(d)
+    """(num_blocks, num_kv_heads, head_dim, block_size) of a [num_blocks][Hkv][16 or 32][D] cache."""
+    if k_cache.dim() != 4 or k_cache.shape[2] not in (16, 32):
+        raise ValueError("cache must be [num_blocks][num_kv_heads][block_size 16 or 32][head_dim]")
+    nb, hkv, bs, d = k_cache.shape
+    return int(nb), int(hkv), int(d), int(bs)
 
 
 # ------------------------------------------------------------------------------ entry points
@@ -163,25 +164,25 @@ def pa_kv_cache_bytes(layers, kv_heads, head_dim, seq_len, batch, elem_bytes) ->
 
 def pa_kv_append(k_cache, v_cache, k, v, slot_mapping, kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None,
                  stream=None):
-    nb, hkv, d = _cache_geometry(k_cache)
+    nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     if k.shape != (slot_mapping.shape[0], hkv, d) or v.shape != k.shape:
         raise ValueError("k/v must be [num_tokens][num_kv_heads][head_dim]")
     st = lib().pa_kv_append(
         _ptr(k_cache, "k_cache", cd), _ptr(v_cache, "v_cache", cd), _ptr(k, "k", (torch.bfloat16,)),
         _ptr(v, "v", (torch.bfloat16,)), _ptr(slot_mapping, "slot_mapping", (torch.int64,)),
-        int(slot_mapping.shape[0]), hkv, d, nb, int(kv_dtype),
+        int(slot_mapping.shape[0]), hkv, d, nb, bs, int(kv_dtype),
         _ptr(k_scale, "k_scale", (torch.float32,)), _ptr(v_scale, "v_scale", (torch.float32,)), _stream(stream))
     _check(st, "pa_kv_append")
 
 
 def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, kv_dtype=PA_KV_BF16, stream=None):
-    nb, hkv, d = _cache_geometry(k_cache)
+    nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     pairs = src_dst_pairs
     n = int(pairs.numel() // 2)
     st = lib().pa_copy_blocks(_ptr(k_cache, "k_cache", cd), _ptr(v_cache, "v_cache", cd),
-                              _ptr(pairs, "src_dst_pairs", (torch.int32,)), n, hkv, d, nb, int(kv_dtype),
+                              _ptr(pairs, "src_dst_pairs", (torch.int32,)), n, hkv, d, nb, bs, int(kv_dtype),
                               _stream(stream))
     _check(st, "pa_copy_blocks")
 
@@ -189,9 +190,9 @@ def pa_copy_blocks(k_cache, v_cache, src_dst_pairs, kv_dtype=PA_KV_BF16, stream=
 def pa_swap_blocks(dst_k, dst_v, src_k, src_v, src_dst_pairs, kv_dtype=PA_KV_BF16, stream=None):
     """Copy whole blocks between two pools (device cache <-> pinned host pool).  Host tensors must be
     pinned (``pin_memory()``); the pairs tensor may be on the device or pinned."""
-    nbd, hkv, d = _cache_geometry(dst_k)
-    nbs, hkv2, d2 = _cache_geometry(src_k)
-    if (hkv, d) != (hkv2, d2) or src_k.dtype != dst_k.dtype:
+    nbd, hkv, d, bs = _cache_geometry(dst_k)
+    nbs, hkv2, d2, bs2 = _cache_geometry(src_k)
+    if (hkv, d, bs) != (hkv2, d2, bs2) or src_k.dtype != dst_k.dtype:
         raise ValueError("source and destination pools differ in geometry or dtype")
     for t, n in ((dst_k, "dst_k"), (dst_v, "dst_v"), (src_k, "src_k"), (src_v, "src_v"), (src_dst_pairs, "pairs")):
         if not t.is_cuda and not t.is_pinned():
@@ -201,7 +202,7 @@ def pa_swap_blocks(dst_k, dst_v, src_k, src_v, src_dst_pairs, kv_dtype=PA_KV_BF1
         _ptr(dst_k, "dst_k", cd, cuda=False), _ptr(dst_v, "dst_v", cd, cuda=False), nbd,
         _ptr(src_k, "src_k", cd, cuda=False), _ptr(src_v, "src_v", cd, cuda=False), nbs,
         _ptr(src_dst_pairs, "src_dst_pairs", (torch.int32,), cuda=False), int(src_dst_pairs.numel() // 2), hkv, d,
-        int(kv_dtype), _stream(stream))
+        bs, int(kv_dtype), _stream(stream))
     _check(st, "pa_swap_blocks")
 
 
@@ -219,7 +220,7 @@ def pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim,
 def pa_paged_attention(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                        kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, split_tokens=0, workspace=None,
                        stream=None):
-    nb, hkv, d = _cache_geometry(k_cache)
+    nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     b, hq, dq = q.shape
     if dq != d or out.shape != q.shape:
@@ -230,7 +231,7 @@ def pa_paged_attention(out, q, k_cache, v_cache, block_tables, context_lens, sca
     st = lib().pa_paged_attention(
         _ptr(out, "out", (torch.bfloat16,)), _ptr(q, "q", (torch.bfloat16,)), _ptr(k_cache, "k_cache", cd),
         _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
-        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), b, hq, hkv, d, nb,
+        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), b, hq, hkv, d, nb, bs,
         float(scale), int(kv_dtype), _ptr(k_scale, "k_scale", (torch.float32,)),
         _ptr(v_scale, "v_scale", (torch.float32,)), int(max_context_len), int(split_tokens),
         _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
@@ -241,7 +242,9 @@ def pa_paged_attention_noalloc(out, q, k_cache, v_cache, block_tables, context_l
                                kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, split_tokens=0, stream=None):
     """pa_paged_attention without a workspace argument, for callers that cannot allocate device memory:
     the split partials go to the library's static per-device scratch (shared by every call)."""
-    nb, hkv, d = _cache_geometry(k_cache)
+    nb, hkv, d, bs = _cache_geometry(k_cache)
+    if bs != PA_BLOCK_SIZE:
+        raise ValueError("pa_paged_attention_noalloc takes 16-token blocks")
     cd = _CACHE_DTYPES[kv_dtype]
     b, hq, dq = q.shape
     if dq != d or out.shape != q.shape:
@@ -259,7 +262,7 @@ def pa_paged_attention_noalloc(out, q, k_cache, v_cache, block_tables, context_l
 
 def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, max_q_len,
                      max_context_len, kv_dtype=PA_KV_BF16, stream=None):
-    nb, hkv, d = _cache_geometry(k_cache)
+    nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     tq, hq, dq = q.shape
     n = int(cu_q_lens.shape[0]) - 1
@@ -271,7 +274,7 @@ def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_
         _ptr(out, "out", (torch.bfloat16,)), _ptr(q, "q", (torch.bfloat16,)),
         _ptr(cu_q_lens, "cu_q_lens", (torch.int32,)), n, _ptr(k_cache, "k_cache", cd),
         _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
-        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), hq, hkv, d, nb,
+        int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), hq, hkv, d, nb, bs,
         float(scale), int(kv_dtype), int(max_q_len), int(max_context_len), _stream(stream))
     _check(st, "pa_paged_prefill")
 

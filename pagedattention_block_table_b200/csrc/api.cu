@@ -150,11 +150,14 @@ pa_status pa_get_device_error(pa_stream_t stream) {
   return PA_EDEVICE_OOB;
 }
 
+static bool block_size_ok(int bs) { return bs == 16 || bs == 32; }
+
 pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *v,
                        const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
-                       int64_t num_blocks, int kv_dtype, const float *k_scale, const float *v_scale,
-                       pa_stream_t stream) {
+                       int64_t num_blocks, int block_size, int kv_dtype, const float *k_scale,
+                       const float *v_scale, pa_stream_t stream) {
   if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_EINVAL;
+  if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
   if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
   if (num_tokens == 0) return PA_OK;
@@ -172,19 +175,22 @@ pa_status pa_kv_append(void *k_cache, void *v_cache, const void *k, const void *
   if (kv_dtype == PA_KV_BF16) {
     pa::launch_pdl(pa::kv_append_bf16_kernel, dim3(grid), dim3(threads), 0, st, static_cast<uint4 *>(k_cache),
                    static_cast<uint4 *>(v_cache), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-                   slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock);
+                   slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * block_size, block_size);
   } else {
     auto kern = kv_dtype == PA_KV_FP8_E4M3 ? pa::kv_append_fp8_kernel<1> : pa::kv_append_fp8_kernel<2>;
     pa::launch_pdl(kern, dim3(grid), dim3(threads), 0, st, static_cast<uint2 *>(k_cache),
                    static_cast<uint2 *>(v_cache), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-                   slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * pa::kBlock, k_scale, v_scale);
+                   slot_mapping, num_tokens, num_kv_heads, chunks, num_blocks * block_size, block_size, k_scale,
+                   v_scale);
   }
   return launch_status();
 }
 
 pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pairs, int num_pairs,
-                         int num_kv_heads, int head_dim, int64_t num_blocks, int kv_dtype, pa_stream_t stream) {
+                         int num_kv_heads, int head_dim, int64_t num_blocks, int block_size, int kv_dtype,
+                         pa_stream_t stream) {
   if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0) return PA_EINVAL;
+  if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
   if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
   if (num_pairs == 0) return PA_OK;
@@ -192,7 +198,7 @@ pa_status pa_copy_blocks(void *k_cache, void *v_cache, const int32_t *src_dst_pa
   if (!k_cache || !v_cache || !src_dst_pairs) return PA_EINVAL;
   if (!aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
   const int elem = kv_dtype == PA_KV_BF16 ? 2 : 1;
-  const int64_t vecs = (int64_t)num_kv_heads * pa::kBlock * head_dim * elem / 16;
+  const int64_t vecs = (int64_t)num_kv_heads * block_size * head_dim * elem / 16;
   const int threads = 256;
   const int64_t gx = ceil_div64(vecs, threads);
   dim3 grid(static_cast<unsigned>(gx < 64 ? gx : 64), static_cast<unsigned>(num_pairs));
@@ -222,8 +228,9 @@ static bool device_accessible(const void *p, void **dev) {
 
 pa_status pa_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const void *src_k, const void *src_v,
                          int64_t src_num_blocks, const int32_t *src_dst_pairs, int num_pairs, int num_kv_heads,
-                         int head_dim, int kv_dtype, pa_stream_t stream) {
+                         int head_dim, int block_size, int kv_dtype, pa_stream_t stream) {
   if (num_pairs < 0 || num_kv_heads <= 0 || dst_num_blocks <= 0 || src_num_blocks <= 0) return PA_EINVAL;
+  if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
   if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
   if (num_pairs == 0) return PA_OK;
@@ -235,7 +242,7 @@ pa_status pa_swap_blocks(void *dst_k, void *dst_v, int64_t dst_num_blocks, const
     return PA_EINVAL;
   if (!aligned16(dk) || !aligned16(dv) || !aligned16(sk) || !aligned16(sv)) return PA_EINVAL;
   const int elem = kv_dtype == PA_KV_BF16 ? 2 : 1;
-  const int64_t vecs = (int64_t)num_kv_heads * pa::kBlock * head_dim * elem / 16;
+  const int64_t vecs = (int64_t)num_kv_heads * block_size * head_dim * elem / 16;
   const int threads = 256;
   const int64_t gx = ceil_div64(vecs, threads * 4);
   dim3 grid(static_cast<unsigned>(gx < 16 ? gx : 16), static_cast<unsigned>(num_pairs));
@@ -278,11 +285,13 @@ size_t pa_paged_attention_workspace_size(int num_seqs, int num_q_heads, int head
 pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, const void *v_cache,
                              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                              int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int64_t num_blocks,
-                             float scale, int kv_dtype, const float *k_scale, const float *v_scale,
+                             int block_size, float scale, int kv_dtype, const float *k_scale, const float *v_scale,
                              int max_context_len, int split_tokens, void *workspace, size_t workspace_bytes,
                              pa_stream_t stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
     return PA_EINVAL;
+  if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
+  if (num_blocks * num_kv_heads * (block_size / pa::kBlock) >= (int64_t(1) << 31)) return PA_EINVAL;
   if (num_q_heads % num_kv_heads != 0) return PA_EINVAL;
   if (head_dim != 64 && head_dim != 128) return PA_EUNSUPPORTED;
   if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return PA_EUNSUPPORTED;
@@ -313,6 +322,7 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
   P.k_scale = k_scale;
   P.v_scale = v_scale;
   P.num_blocks = num_blocks;
+  P.block_size = block_size;
   P.max_blocks_per_seq = max_blocks_per_seq;
   P.num_q_heads = num_q_heads;
   P.num_kv_heads = num_kv_heads;
@@ -344,10 +354,11 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
 pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
                            const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                            const int32_t *context_lens, int num_q_heads, int num_kv_heads, int head_dim,
-                           int64_t num_blocks, float scale, int kv_dtype, int max_q_len, int max_context_len,
-                           pa_stream_t stream) {
+                           int64_t num_blocks, int block_size, float scale, int kv_dtype, int max_q_len,
+                           int max_context_len, pa_stream_t stream) {
   if (num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
     return PA_EINVAL;
+  if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
   if (num_q_heads % num_kv_heads != 0) return PA_EINVAL;
   if (head_dim != 128 && head_dim != 64) return PA_EUNSUPPORTED;
   if (kv_dtype != PA_KV_BF16) return PA_EUNSUPPORTED;
@@ -357,8 +368,8 @@ pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, i
   if (!out || !q || !cu_q_lens || !k_cache || !v_cache || !block_tables || !context_lens) return PA_EINVAL;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
   return pa::launch_prefill(out, q, cu_q_lens, num_chunks, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                            context_lens, num_q_heads, num_kv_heads, head_dim, num_blocks, scale, max_q_len,
-                            max_context_len, reinterpret_cast<cudaStream_t>(stream));
+                            context_lens, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
+                            max_q_len, max_context_len, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -417,6 +428,6 @@ extern "C" pa_status pa_paged_attention_noalloc(void *out, const void *q, const 
     if (ws == nullptr) return PA_ECUDA;
   }
   return pa_paged_attention(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
-                            num_q_heads, num_kv_heads, head_dim, num_blocks, scale, kv_dtype, k_scale, v_scale,
-                            max_context_len, S, ws, ws ? cap : 0, stream);
+                            num_q_heads, num_kv_heads, head_dim, num_blocks, PA_BLOCK_SIZE, scale, kv_dtype, k_scale,
+                            v_scale, max_context_len, S, ws, ws ? cap : 0, stream);
 }

@@ -32,6 +32,7 @@ struct DecodeParams {
   float *ws_o;   // [B][Hq][max_splits][D] partial outputs (unnormalised)
   float *ws_ml;  // [B][Hq][max_splits][2]  partial (max in log2 units, sum)
   int64_t num_blocks;
+  int block_size;       // 16 or 32 tokens per physical block
   int max_blocks_per_seq;
   int num_q_heads;
   int num_kv_heads;
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
   // ---- context length, validated: never read past the table row or the launch bound
   int L = P.context_lens[b];
   {
-    const int lim = min(P.max_blocks_per_seq * kBlock, P.max_context_len);
+    const int lim = min(P.max_blocks_per_seq * P.block_size, P.max_context_len);
     if (L < 0 || L > lim) {
       if (threadIdx.x == 0 && split == 0) flag_error(kErrLength);
       L = L < 0 ? 0 : lim;
@@ -156,30 +157,34 @@ __global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParam
 
   const int qsel = group_reduce_qsel<QPB, C::LPT>(lane);
 
-  // ---- block-table window: lane k holds the entry of this warp's block (win*32 + k)
+  // ---- block-table window: lane k holds the 16-token tile index (in the flat array of 16-row tiles
+  // [num_blocks][Hkv][block_size/16]) of this warp's unit win*32 + k; a unit is 16 tokens, so a
+  // 32-token block is read as two units
   const int32_t *trow = P.block_tables + (int64_t)b * P.max_blocks_per_seq;
+  const int upb = P.block_size / kBlock;   // units per block: 1 or 2
   auto load_window = [&](int win) -> int {
     const int i = win * 32 + lane;
-    int e = 0;
+    int tile = 0;
     if (i < nwb) {
-      e = __ldg(trow + blk0 + warp + NW * i);
+      const int u = blk0 + warp + NW * i;   // unit index within the sequence
+      int e = __ldg(trow + u / upb);
       if (e < 0 || e >= P.num_blocks) {
         flag_error(kErrBlockId);
         e = 0;
       }
+      tile = (e * P.num_kv_heads + g) * upb + u % upb;
     }
-    return e;
+    return tile;
   };
   int tw = load_window(0);
   const uint64_t pol = l2_evict_first_policy();
-  const int64_t head_stride = (int64_t)C::TILE;
   auto issue = [&](int i) {  // warp-uniform call
     if (i >= nwb) return;
     if ((i & 31) == 0 && i > 0) tw = load_window(i >> 5);
-    const int e = __shfl_sync(0xffffffffu, tw, i & 31);
+    const int tile = __shfl_sync(0xffffffffu, tw, i & 31);
     if (lane == 0) {
       const int s = i % STAGES;
-      const int64_t off = ((int64_t)e * P.num_kv_heads + g) * head_stride;
+      const int64_t off = (int64_t)tile * C::TILE;
       mbar_arrive_expect_tx(&bars[s], 2 * C::TILE);
       bulk_g2s(wbase + s * C::TILE, P.k_cache + off, C::TILE, &bars[s], pol);
       bulk_g2s(wbase + (STAGES + s) * C::TILE, P.v_cache + off, C::TILE, &bars[s], pol);
@@ -434,7 +439,7 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
   griddep_launch();
   if (h >= P.num_q_heads) return;
   int L = P.context_lens[b];
-  const int lim = min(P.max_blocks_per_seq * kBlock, P.max_context_len);
+  const int lim = min(P.max_blocks_per_seq * P.block_size, P.max_context_len);
   L = L < 0 ? 0 : (L > lim ? lim : L);
   const int n = (L + P.split_tokens - 1) / P.split_tokens;
   if (n <= 1) return;  // written directly by the decode kernel

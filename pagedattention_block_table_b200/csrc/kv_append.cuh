@@ -12,11 +12,11 @@
 namespace pa {
 
 // One thread = one 16-byte chunk (8 bf16) of one token's row for one KV head, K and V.
-// Row n*Hkv + h of k/v goes to cache[slot/16][h][slot%16][:].
+// Row n*Hkv + h of k/v goes to cache[slot/bs][h][slot%bs][:] (bs = block size, 16 or 32).
 __global__ void kv_append_bf16_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
                                       const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                       const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
-                                      int num_kv_heads, int chunks_per_row, int64_t num_slots) {
+                                      int num_kv_heads, int chunks_per_row, int64_t num_slots, int bs) {
   griddep_wait();  // inputs or the cache may belong to the kernel before this one (PDL launch)
   griddep_launch();
   const int64_t total = num_tokens * num_kv_heads * chunks_per_row;
@@ -32,8 +32,8 @@ __global__ void kv_append_bf16_kernel(uint4 *__restrict__ k_cache, uint4 *__rest
       flag_error(kErrSlot);
       continue;
     }
-    const int64_t blk = slot / kBlock, off = slot % kBlock;
-    const int64_t dst = ((blk * num_kv_heads + h) * kBlock + off) * chunks_per_row + c;
+    const int64_t blk = slot / bs, off = slot % bs;
+    const int64_t dst = ((blk * num_kv_heads + h) * bs + off) * chunks_per_row + c;
     const uint4 kv = __ldcs(k + i);  // streamed: read once
     const uint4 vv = __ldcs(v + i);
     k_cache[dst] = kv;
@@ -81,7 +81,7 @@ template <int KT>
 __global__ void kv_append_fp8_kernel(uint2 *__restrict__ k_cache, uint2 *__restrict__ v_cache,
                                      const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                      const int64_t *__restrict__ slot_mapping, int64_t num_tokens,
-                                     int num_kv_heads, int chunks_per_row, int64_t num_slots,
+                                     int num_kv_heads, int chunks_per_row, int64_t num_slots, int bs,
                                      const float *__restrict__ k_scale, const float *__restrict__ v_scale) {
   griddep_wait();
   griddep_launch();
@@ -98,8 +98,8 @@ __global__ void kv_append_fp8_kernel(uint2 *__restrict__ k_cache, uint2 *__restr
       flag_error(kErrSlot);
       continue;
     }
-    const int64_t blk = slot / kBlock, off = slot % kBlock;
-    const int64_t dst = ((blk * num_kv_heads + h) * kBlock + off) * chunks_per_row + c;
+    const int64_t blk = slot / bs, off = slot % bs;
+    const int64_t dst = ((blk * num_kv_heads + h) * bs + off) * chunks_per_row + c;
     if constexpr (KT == 1) {
       k_cache[dst] = quant8(__ldcs(k + i), k_scale[h]);
       v_cache[dst] = quant8(__ldcs(v + i), v_scale[h]);

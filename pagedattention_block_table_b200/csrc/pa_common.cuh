@@ -13,7 +13,9 @@
 
 namespace pa {
 
-constexpr int kBlock = 16;  // tokens per physical block
+// Kernels walk the cache in units of 16 tokens (one 16-row run of a (block, KV head) tile); a
+// physical block holds 16 or 32 tokens, i.e. one or two units.
+constexpr int kBlock = 16;
 
 // Bit set in the per-device error word when a kernel meets an out-of-range value.
 enum : unsigned {

@@ -158,6 +158,7 @@ struct PrefillParams {
   const int32_t *block_tables;
   const int32_t *context_lens;
   int64_t num_blocks;
+  int block_size;       // 16 or 32 tokens per physical block
   int max_blocks_per_seq;
   int num_q_heads;
   int num_kv_heads;
@@ -220,6 +221,33 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x for a packed pair on the FMA pipe (to take load off the MUFU unit): x = n + f with n = rint(x)
+// (add/subtract 1.5*2^23) and f in [-0.5, 0.5]; 2^f by a cubic fitted here to minimise the relative
+// error on that interval (max 7.5e-5, below the bf16 resolution P is rounded to); 2^n is added to the
+// exponent field.  Arguments below -125 give 0 (as the flush-to-zero ex2 does for results in the
+// denormal range); -inf gives 0.
+__device__ __forceinline__ uint64_t ex2_poly2(float xa, float xb) {
+  const float x0 = fmaxf(xa, -125.f), x1 = fmaxf(xb, -125.f);
+  const uint64_t shifter = f2pack(12582912.f, 12582912.f), xx = f2pack(x0, x1);
+  uint64_t t, n2, f2;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xx), "l"(shifter));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n2) : "l"(t), "l"(shifter));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f2) : "l"(xx), "l"(n2));
+  uint64_t p = f2pack(0.05517394095659256f, 0.05517394095659256f);
+  p = ffma2(p, f2, f2pack(0.24261131882667542f, 0.24261131882667542f));
+  p = ffma2(p, f2, f2pack(0.6932605504989624f, 0.6932605504989624f));
+  p = ffma2(p, f2, f2pack(0.9999280571937561f, 0.9999280571937561f));
+  const float2 tv = f2unpack(t), pv = f2unpack(p);
+  const float a = x0 > -125.f ? __int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)) : 0.f;
+  const float b = x1 > -125.f ? __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)) : 0.f;
+  return f2pack(a, b);
+}
+
+// One 8-key chunk in PA_PREFILL_POLY_EVERY takes its exponentials from ex2_poly2 (0 = none).
+#ifndef PA_PREFILL_POLY_EVERY
+#define PA_PREFILL_POLY_EVERY 0
+#endif
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -241,7 +269,7 @@ __global__ void __launch_bounds__(320, 1)
   const int Cn = P.cu_q_lens[c + 1] - q0;
   const int ctx = P.context_lens[c];
   const int H = ctx - Cn;
-  if (Cn < 0 || H < 0 || ctx > min(P.max_blocks_per_seq * kBlock, P.max_context_len)) {
+  if (Cn < 0 || H < 0 || ctx > min(P.max_blocks_per_seq * P.block_size, P.max_context_len)) {
     if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) flag_error(kErrLength);
     return;
   }
@@ -318,17 +346,39 @@ __global__ void __launch_bounds__(320, 1)
       // scaled row max of this tile; masked keys (past the row's position) become -inf
       float mt_ = -INFINITY;
       if (kbase + C::BN - 1 <= pos) {
-        float mx = s[0], mn = s[0];
+        // max of s * qscale: the max of s for a positive scale, the min for a negative one; eight
+        // independent partial results so the reduction is not one long dependent chain
+        float e[8];
 #pragma unroll
-        for (int k = 1; k < C::BN; ++k) {
-          mx = fmaxf(mx, s[k]);
-          mn = fminf(mn, s[k]);
+        for (int k = 0; k < 8; ++k) e[k] = s[k];
+        if (qs >= 0.f) {
+#pragma unroll
+          for (int k = 8; k < C::BN; ++k) e[k & 7] = fmaxf(e[k & 7], s[k]);
+#pragma unroll
+          for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+            for (int k = 0; k < w; ++k) e[k] = fmaxf(e[k], e[k + w]);
+        } else {
+#pragma unroll
+          for (int k = 8; k < C::BN; ++k) e[k & 7] = fminf(e[k & 7], s[k]);
+#pragma unroll
+          for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+            for (int k = 0; k < w; ++k) e[k] = fminf(e[k], e[k + w]);
         }
-        mt_ = qs >= 0.f ? mx * qs : mn * qs;
+        mt_ = e[0] * qs;
       } else {
+        float e[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) e[k] = -INFINITY;
 #pragma unroll
         for (int k = 0; k < C::BN; ++k)
-          if (kbase + k <= pos) mt_ = fmaxf(mt_, s[k] * qs);
+          if (kbase + k <= pos) e[k & 7] = fmaxf(e[k & 7], s[k] * qs);
+#pragma unroll
+        for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+          for (int k = 0; k < w; ++k) e[k] = fmaxf(e[k], e[k + w]);
+        mt_ = e[0];
       }
       const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
       // the previous tile's PV must be complete before O is rescaled or P is overwritten
@@ -361,7 +411,7 @@ __global__ void __launch_bounds__(320, 1)
           for (int ch = 0; ch < 8; ++ch)
             *reinterpret_cast<uint4 *>(vt + hh * C::KV_PLANE + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
       }
-      uint64_t ls2 = 0ull;
+      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};   // independent partial row sums
       const uint64_t qs2 = f2pack(qs, qs), nm2 = f2pack(-m_ref, -m_ref);
       uint8_t *prow = sP + r * 128;
 #pragma unroll
@@ -376,14 +426,26 @@ __global__ void __launch_bounds__(320, 1)
             if (t > pos) x.x = -INFINITY;
             if (t + 1 > pos) x.y = -INFINITY;
           }
+#if PA_PREFILL_POLY_EVERY > 0
+          float a, b;
+          if (q8 % PA_PREFILL_POLY_EVERY == PA_PREFILL_POLY_EVERY - 1) {
+            const float2 e = f2unpack(ex2_poly2(x.x, x.y));
+            a = e.x;
+            b = e.y;
+          } else {
+            a = ex2(x.x);
+            b = ex2(x.y);
+          }
+#else
           const float a = ex2(x.x);
           const float b = ex2(x.y);
-          ls2 = f2add(ls2, f2pack(a, b));
+#endif
+          ls2[k2] = f2add(ls2[k2], f2pack(a, b));
           pk[k2] = pack_bf16x2(a, b);
         }
         *reinterpret_cast<uint4 *>(prow + ((q8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      const float2 lsv = f2unpack(ls2);
+      const float2 lsv = f2unpack(f2add(f2add(ls2[0], ls2[1]), f2add(ls2[2], ls2[3])));
       const float ls = lsv.x + lsv.y;
       l_run += ls;
       fence_async_smem();
@@ -483,13 +545,15 @@ __global__ void __launch_bounds__(320, 1)
         }
         const int nb = min(C::BN / kBlock, (kv_len - j * C::BN + kBlock - 1) / kBlock);
         mbar_arrive_expect_tx(&bars[kKvFull + st], nb * 2 * C::DH * (kBlock * 128));
+        const int upb = P.block_size / kBlock;   // 16-row units per physical block
         for (int bb = 0; bb < nb; ++bb) {
-          int e = __ldg(trow + j * (C::BN / kBlock) + bb);
+          const int u = j * (C::BN / kBlock) + bb;   // 16-token unit of the sequence
+          int e = __ldg(trow + u / upb);
           if (e < 0 || e >= P.num_blocks) {
             flag_error(kErrBlockId);
             e = 0;
           }
-          const int y = (e * P.num_kv_heads + g) * kBlock;
+          const int y = ((e * P.num_kv_heads + g) * upb + u % upb) * kBlock;
 #pragma unroll
           for (int hh = 0; hh < C::DH; ++hh) {
             const int off = st * C::KV_BYTES + hh * C::KV_PLANE + bb * (kBlock * 128);
@@ -552,7 +616,7 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
                      cudaStream_t st) {
   using C = PrefillCfg<D>;
   CUtensorMap km, vm;
-  const int64_t rows = P.num_blocks * P.num_kv_heads * kBlock;
+  const int64_t rows = P.num_blocks * P.num_kv_heads * P.block_size;
   if (!make_cache_map(&km, k_cache, rows, D) || !make_cache_map(&vm, v_cache, rows, D)) return -3;
   if (cudaFuncSetAttribute(paged_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
@@ -565,9 +629,10 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
 inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
                           const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                           const int32_t *context_lens, int num_q_heads, int num_kv_heads, int head_dim,
-                          int64_t num_blocks, float scale, int max_q_len, int max_context_len, cudaStream_t st) {
+                          int64_t num_blocks, int block_size, float scale, int max_q_len, int max_context_len,
+                          cudaStream_t st) {
   if (num_chunks > 65535 || num_q_heads > 65535) return -1;
-  if (num_blocks * num_kv_heads * kBlock >= (int64_t(1) << 31)) return -2;
+  if (num_blocks * num_kv_heads * block_size >= (int64_t(1) << 31)) return -2;
   PrefillParams P;
   P.out = static_cast<__nv_bfloat16 *>(out);
   P.q = static_cast<const __nv_bfloat16 *>(q);
@@ -575,6 +640,7 @@ inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, in
   P.block_tables = block_tables;
   P.context_lens = context_lens;
   P.num_blocks = num_blocks;
+  P.block_size = block_size;
   P.max_blocks_per_seq = max_blocks_per_seq;
   P.num_q_heads = num_q_heads;
   P.num_kv_heads = num_kv_heads;

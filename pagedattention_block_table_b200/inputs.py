@@ -7,12 +7,12 @@ in the physical pool, the slot of every token, and -- for the prefix-sharing ste
 which blocks are shared and which copy-on-write pairs a fork needs.  It holds none
 of the method's arithmetic: no attention, no quantisation, no copying of caches.
 
-Cache layout used throughout: ``[num_blocks][num_kv_heads][16][head_dim]``; a
-token at logical position ``t`` of a sequence lives in physical block
-``block_table[t // 16]`` at offset ``t % 16``, so its slot is
-``block_table[t // 16] * 16 + t % 16`` (Core Concepts page, section 3.2: the block
-table maps logical blocks to physical blocks; vLLM overview page, section 二: pages
-of 16 tokens).
+Cache layout used throughout: ``[num_blocks][num_kv_heads][bs][head_dim]`` with block size
+bs = 16 (default) or 32; a token at logical position ``t`` of a sequence lives in physical
+block ``block_table[t // bs]`` at offset ``t % bs``, so its slot is
+``block_table[t // bs] * bs + t % bs`` (Core Concepts page, section 3.2: the block table
+maps logical blocks to physical blocks, blocks of 16 or 32 tokens; vLLM overview page,
+section 二: pages of 16 tokens).
 """
 from __future__ import annotations
 
@@ -75,6 +75,7 @@ class PagedBatch:
     num_blocks: int
     scale: float
     kv_dtype: int                       # 0 = bf16 cache, 1 = fp8 E4M3 cache, 2 = int8 cache
+    block_size: int                     # tokens per physical block (16 or 32)
     num_decode: int
     hist_lens: np.ndarray               # int32 [S] tokens cached before the step
     new_lens: np.ndarray                # int32 [S] tokens appended by the step
@@ -170,8 +171,8 @@ class _Pool:
         return out
 
 
-def _nblk(n) -> int:
-    return (int(n) + BLOCK - 1) // BLOCK
+def _nblk(n, bs=BLOCK) -> int:
+    return (int(n) + bs - 1) // bs
 
 
 # ---------------------------------------------------------------------- builder
@@ -191,6 +192,9 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
     rng = np.random.default_rng([seed, 0])
     prng = None if perm_seed == -1 else np.random.default_rng([seed if perm_seed is None else perm_seed, 1])
 
+    bs = int(spec.get("block_size", BLOCK))
+    if bs not in (16, 32):
+        raise ValueError("block_size must be 16 or 32")
     B = int(spec["num_seqs"])
     hq, hkv, D = int(spec["num_q_heads"]), int(spec["num_kv_heads"]), int(spec["head_dim"])
     hist_dec = _draw_hist(spec["hist"], B, rng)
@@ -226,12 +230,12 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
     group_blocks_needed = []
     for gi in range(n_groups):
         mem = range(gi * group, min(B, (gi + 1) * group))
-        group_blocks_needed.append(max(_nblk(shared_cover[s]) for s in mem))
+        group_blocks_needed.append(max(_nblk(shared_cover[s], bs) for s in mem))
     for s in range(S):
         # private blocks: logical blocks not covered by the shared prefix, plus one spare
         # for a copy-on-write fork of the last shared block
-        nb_total = _nblk(ctx[s])
-        nb_shared = _nblk(shared_cover[s])
+        nb_total = _nblk(ctx[s], bs)
+        nb_shared = _nblk(shared_cover[s], bs)
         need_private.append(nb_total - nb_shared + (1 if nb_shared else 0))
     need = sum(group_blocks_needed) + sum(need_private)
     num_blocks = int(spec.get("num_blocks") or math.ceil(1.25 * need))
@@ -239,18 +243,18 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
         raise ValueError("pool smaller than the workload needs")
     pool = _Pool(num_blocks, prng)
 
-    mbs = max(_nblk(c) for c in ctx) if S else 1
+    mbs = max(_nblk(c, bs) for c in ctx) if S else 1
     tables = np.full((S, mbs), -1, np.int32)
     group_blocks = [pool.take(n) for n in group_blocks_needed]
     refcount: Dict[int, int] = {}
     for s in range(S):
-        nb_shared = _nblk(shared_cover[s])
+        nb_shared = _nblk(shared_cover[s], bs)
         if nb_shared:
             gb = group_blocks[s // group]
             tables[s, :nb_shared] = gb[:nb_shared]
             for b in gb[:nb_shared]:
                 refcount[int(b)] = refcount.get(int(b), 0) + 1
-        nb_hist = _nblk(hist[s])
+        nb_hist = _nblk(hist[s], bs)
         if nb_hist > nb_shared:
             tables[s, nb_shared:nb_hist] = pool.take(nb_hist - nb_shared)
     shared_blocks = np.array(sorted(b for b, c in refcount.items() if c > 1), np.int32)
@@ -259,7 +263,7 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
     pairs: List[List[int]] = []
     for s in range(S):
         for t in range(int(hist[s]), int(ctx[s])):
-            lb = t // BLOCK
+            lb = t // bs
             if tables[s, lb] < 0:
                 tables[s, lb] = pool.take(1)[0]
                 refcount[int(tables[s, lb])] = 1
@@ -305,8 +309,8 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
         pre_tables[pre_tables == dst] = src
     for s in range(S):
         t = np.arange(int(hist[s]), dtype=np.int64)
-        phys = pre_tables[s, t // BLOCK].astype(np.int64)
-        slots = phys * BLOCK + t % BLOCK
+        phys = pre_tables[s, t // bs].astype(np.int64)
+        slots = phys * bs + t % bs
         if shared_cover[s]:
             # shared-prefix tokens are written once, by the first member that covers them
             keep = np.array([int(x) not in written for x in slots], dtype=bool)
@@ -316,7 +320,7 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
     step_slots = []
     for s in range(S):
         t = np.arange(int(hist[s]), int(ctx[s]), dtype=np.int64)
-        step_slots.append(tables[s, t // BLOCK].astype(np.int64) * BLOCK + t % BLOCK)
+        step_slots.append(tables[s, t // bs].astype(np.int64) * bs + t % bs)
     step_slots = np.concatenate(step_slots) if step_slots else np.zeros(0, np.int64)
 
     q_dec = randn_bf16((B, hq, D), device, seed, 6)
@@ -332,7 +336,7 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
 
     return PagedBatch(
         name=name, num_q_heads=hq, num_kv_heads=hkv, head_dim=D, num_blocks=num_blocks,
-        scale=1.0 / math.sqrt(D), kv_dtype=kv_dtype, num_decode=B,
+        scale=1.0 / math.sqrt(D), kv_dtype=kv_dtype, block_size=bs, num_decode=B,
         hist_lens=hist, new_lens=new, block_tables=tables, setup_slots=setup_slots,
         step_slots=step_slots, cow_pairs=cow_pairs, shared_blocks=shared_blocks,
         tok_k=tok_k, tok_v=tok_v, tok_offsets=offsets, q_decode=q_dec, q_prefill=q_pre,

@@ -30,8 +30,9 @@ class DeviceStep:
         self.kv_dtype = batch.kv_dtype
         cdt = {0: torch.bfloat16, 1: torch.uint8, 2: torch.int8}[batch.kv_dtype]
         alloc = torch.zeros if zero_cache else torch.empty
-        self.k_cache = alloc((nb, hkv, 16, d), dtype=cdt, device=dev)
-        self.v_cache = alloc((nb, hkv, 16, d), dtype=cdt, device=dev)
+        bs = batch.block_size
+        self.k_cache = alloc((nb, hkv, bs, d), dtype=cdt, device=dev)
+        self.v_cache = alloc((nb, hkv, bs, d), dtype=cdt, device=dev)
         self.k_scale = None if batch.k_scale is None else batch.k_scale.to(dev, torch.float32).contiguous()
         self.v_scale = None if batch.v_scale is None else batch.v_scale.to(dev, torch.float32).contiguous()
 

@@ -15,8 +15,8 @@ def oracle_step(batch: PagedBatch, O, keep_pre_step=False):
     """Fill the history, then run the step (forks, append, decode, prefill) in the oracle."""
     nb, hkv, d = batch.num_blocks, batch.num_kv_heads, batch.head_dim
     dt = {0: np.uint16, 1: np.uint8, 2: np.int8}[batch.kv_dtype]
-    kc = np.zeros((nb, hkv, 16, d), dt)
-    vc = np.zeros((nb, hkv, 16, d), dt)
+    kc = np.zeros((nb, hkv, batch.block_size, d), dt)
+    vc = np.zeros((nb, hkv, batch.block_size, d), dt)
     tk = bf16_bits(batch.tok_k)
     tv = bf16_bits(batch.tok_v)
     ks = None if batch.k_scale is None else batch.k_scale.cpu().numpy()

@@ -63,13 +63,13 @@ def test_workspace_size(L):
 
 
 def _raw_attention(L, **kw):
-    args = dict(out=16, q=16, k=16, v=16, bt=16, mbs=4, cl=16, ns=2, hq=8, hkv=2, d=128, nb=10, scale=0.1,
+    args = dict(out=16, q=16, k=16, v=16, bt=16, mbs=4, cl=16, ns=2, hq=8, hkv=2, d=128, nb=10, bs=16, scale=0.1,
                 dt=0, ks=None, vs=None, maxl=64, split=0, ws=None, wsb=0)
     args.update(kw)
     P = ctypes.c_void_p
     return L.pa_paged_attention(P(args["out"]), P(args["q"]), P(args["k"]), P(args["v"]), P(args["bt"]), args["mbs"],
                                 P(args["cl"]), args["ns"], args["hq"], args["hkv"], args["d"], args["nb"],
-                                args["scale"], args["dt"], P(args["ks"]) if args["ks"] else None,
+                                args["bs"], args["scale"], args["dt"], P(args["ks"]) if args["ks"] else None,
                                 P(args["vs"]) if args["vs"] else None, args["maxl"], args["split"],
                                 P(args["ws"]) if args["ws"] else None, args["wsb"], None)
 
@@ -85,6 +85,7 @@ def _raw_attention(L, **kw):
     (dict(maxl=4096, split=512), B.PA_EWORKSPACE),  # needs a workspace, none given
     (dict(nb=0), B.PA_EINVAL),
     (dict(scale=float("nan")), B.PA_EINVAL),
+    (dict(bs=8), B.PA_EUNSUPPORTED),           # block size other than 16 / 32
 ])
 def test_attention_rejects_bad_arguments_before_launch(L, bad, status):
     assert _raw_attention(L, **bad) == status
@@ -93,14 +94,15 @@ def test_attention_rejects_bad_arguments_before_launch(L, bad, status):
 def test_empty_batch_is_a_no_op(L):
     assert _raw_attention(L, ns=0, q=0, out=0) == B.PA_OK
     P = ctypes.c_void_p
-    assert L.pa_kv_append(None, None, None, None, None, 0, 8, 128, 10, 0, None, None, None) == B.PA_OK
-    assert L.pa_copy_blocks(None, None, None, 0, 8, 128, 10, 0, None) == B.PA_OK
-    assert L.pa_kv_append(P(16), P(16), P(16), P(16), P(16), 4, 8, 96, 10, 0, None, None, None) == B.PA_EUNSUPPORTED
-    assert L.pa_kv_append(P(16), P(16), P(16), P(16), None, 4, 8, 128, 10, 0, None, None, None) == B.PA_EINVAL
+    assert L.pa_kv_append(None, None, None, None, None, 0, 8, 128, 10, 16, 0, None, None, None) == B.PA_OK
+    assert L.pa_copy_blocks(None, None, None, 0, 8, 128, 10, 16, 0, None) == B.PA_OK
+    assert L.pa_kv_append(P(16), P(16), P(16), P(16), P(16), 4, 8, 96, 10, 16, 0, None, None, None) == B.PA_EUNSUPPORTED
+    assert L.pa_kv_append(P(16), P(16), P(16), P(16), None, 4, 8, 128, 10, 16, 0, None, None, None) == B.PA_EINVAL
+    assert L.pa_kv_append(P(16), P(16), P(16), P(16), P(16), 4, 8, 128, 10, 24, 0, None, None, None) == B.PA_EUNSUPPORTED
 
 
 def test_prefill_rejects_fp8_and_bad_heads(L):
     P = ctypes.c_void_p
     f = L.pa_paged_prefill
-    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 0.1, 1, 16, 64, None) == B.PA_EUNSUPPORTED
-    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 0.1, 0, 16, 64, None) == B.PA_EINVAL
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 1, 16, 64, None) == B.PA_EUNSUPPORTED
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 16, 0.1, 0, 16, 64, None) == B.PA_EINVAL

@@ -31,9 +31,9 @@ def _gpu_step_caches(batch, cuda_lib):
     return k_pre, v_pre, _cache_np(st.k_cache), _cache_np(st.v_cache)
 
 
-@pytest.mark.parametrize("head_dim", [64, 128])
-def test_append_and_fork_bf16_bit_exact(O, cuda_lib, head_dim):
-    batch = make_batch("mixed_step", seed=31, overrides=dict(SMALL_MIXED, head_dim=head_dim))
+@pytest.mark.parametrize("head_dim,bs", [(64, 16), (128, 16), (128, 32)])
+def test_append_and_fork_bf16_bit_exact(O, cuda_lib, head_dim, bs):
+    batch = make_batch("mixed_step", seed=31, overrides=dict(SMALL_MIXED, head_dim=head_dim, block_size=bs))
     assert batch.cow_pairs.shape[0] > 0
     ref = oracle_step(batch, O, keep_pre_step=True)
     k_pre, v_pre, k, v = _gpu_step_caches(batch, cuda_lib)
@@ -100,9 +100,11 @@ def test_out_of_pool_slot_is_flagged_not_written(cuda_lib):
     assert float(kc.float().sum()) == 2 * 64                              # only slot 0 written
 
 
-def test_append_int8_bit_exact(O, cuda_lib):
+@pytest.mark.parametrize("bs", [16, 32])
+def test_append_int8_bit_exact(O, cuda_lib, bs):
     batch = make_batch("mha_fp8_decode", seed=33, overrides=dict(num_seqs=5, num_q_heads=4, num_kv_heads=4,
-                                                               hist=("uniform", 1, 300), kv_dtype="int8"))
+                                                               hist=("uniform", 1, 300), kv_dtype="int8",
+                                                               block_size=bs))
     ref = oracle_step(batch, O)
     _, _, k, v = _gpu_step_caches(batch, cuda_lib)
     assert np.array_equal(k, ref["k_cache"]) and np.array_equal(v, ref["v_cache"])

@@ -29,6 +29,10 @@ SMALL = {
     "mha_d64": ("tiny_decode", dict(num_seqs=3, num_q_heads=3, num_kv_heads=3, hist=("uniform", 200, 600),
                                     num_blocks=None)),
     "gqa3_d128": ("llama3_8b_decode", dict(num_seqs=2, num_q_heads=6, num_kv_heads=2, hist=("uniform", 40, 300))),
+    # 32-token blocks (Core Concepts §3.2: blocks of 16 or 32 tokens)
+    "gqa4_d128_bs32": ("llama3_8b_decode", dict(num_seqs=5, hist=("fixed", [0, 31, 32, 700, 1500]), block_size=32)),
+    "gqa2_d64_bs32": ("tiny_decode", dict(num_seqs=4, num_q_heads=4, num_kv_heads=2, hist=("uniform", 1, 400),
+                                          num_blocks=None, block_size=32)),
 }
 
 
@@ -43,18 +47,19 @@ def test_decode_bf16_matches_oracle(O, cuda_lib, case, split):
     assert_close(to_f64(st.out_dec), ref, what=f"{case} split={split}")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d,bs", [(64, 16), (128, 16), (128, 32)])
 @pytest.mark.parametrize("split", [None, 128])
-def test_decode_fp8_matches_oracle(O, cuda_lib, d, split):
+def test_decode_fp8_matches_oracle(O, cuda_lib, d, bs, split):
     batch = make_batch("mha_fp8_decode", seed=42, overrides=dict(num_seqs=4, num_q_heads=8, num_kv_heads=8,
-                                                               head_dim=d, hist=("uniform", 1, 700)))
+                                                               head_dim=d, hist=("uniform", 1, 700), block_size=bs))
     st = _gpu_decode(batch, split)
     got = to_f64(st.out_dec)
     # against the oracle on the dequantised cache: kernel arithmetic only
     assert_close(got, oracle_step(batch, O)["decode"], what="fp8 vs dequantised")
     # against the oracle on the original bf16 K/V: includes the quantisation error
     b16 = make_batch("mha_fp8_decode", seed=42, overrides=dict(num_seqs=4, num_q_heads=8, num_kv_heads=8,
-                                                             head_dim=d, hist=("uniform", 1, 700), kv_dtype=None))
+                                                             head_dim=d, hist=("uniform", 1, 700), kv_dtype=None,
+                                                             block_size=bs))
     assert_close(got, oracle_step(b16, O)["decode"], max_tol=FP8_MAX, mean_tol=None, what="fp8 vs bf16")
 
 

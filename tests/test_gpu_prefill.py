@@ -34,6 +34,7 @@ CASES = {
     "gqa8_d128": _chunks(num_q_heads=16, num_kv_heads=2, chunk_len=(20, 150)),
     "gqa3_d128": _chunks(num_q_heads=6, num_kv_heads=2, chunk_len=(60, 200)),
     "gqa16_d64": _chunks(num_q_heads=16, num_kv_heads=1, head_dim=64, chunk_len=(5, 90)),
+    "gqa4_d128_bs32": _chunks(block_size=32, chunk_len=(40, 300), chunk_hist=(1, 300)),
 }
 
 

@@ -14,8 +14,9 @@ def _np(t):
     return bf16_bits(t) if t.dtype == torch.bfloat16 else t.numpy().copy()
 
 
-@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.uint8, 128), (torch.bfloat16, 64)])
-def test_swap_out_and_in_bit_exact(O, cuda_lib, dtype, d):
+@pytest.mark.parametrize("dtype,d,bs", [(torch.bfloat16, 128, 16), (torch.uint8, 128, 16), (torch.bfloat16, 64, 16),
+                                        (torch.bfloat16, 128, 32)])
+def test_swap_out_and_in_bit_exact(O, cuda_lib, dtype, d, bs):
     B = cuda_lib
     g = torch.Generator().manual_seed(9)
     nb_dev, nb_host, hkv = 40, 24, 8
@@ -23,8 +24,8 @@ def test_swap_out_and_in_bit_exact(O, cuda_lib, dtype, d):
 
     def rnd(n):
         if dtype == torch.bfloat16:
-            return torch.randn((n, hkv, 16, d), generator=g).to(dtype)
-        return torch.randint(0, 256, (n, hkv, 16, d), generator=g, dtype=torch.uint8)
+            return torch.randn((n, hkv, bs, d), generator=g).to(dtype)
+        return torch.randint(0, 256, (n, hkv, bs, d), generator=g, dtype=torch.uint8)
 
     dk, dv = rnd(nb_dev).cuda(), rnd(nb_dev).cuda()
     hk, hv = rnd(nb_host).pin_memory(), rnd(nb_host).pin_memory()
@@ -55,7 +56,7 @@ def test_swap_rejects_pageable_host_memory(cuda_lib):
     pairs = torch.tensor([[0, 1]], dtype=torch.int32, device="cuda")
     P = ctypes.c_void_p
     st = B.lib().pa_swap_blocks(P(hk.data_ptr()), P(hk.data_ptr()), 4, P(dk.data_ptr()), P(dk.data_ptr()), 4,
-                                P(pairs.data_ptr()), 1, 2, 64, 0, None)
+                                P(pairs.data_ptr()), 1, 2, 64, 16, 0, None)
     assert st == B.PA_EINVAL
 
 

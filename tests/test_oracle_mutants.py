@@ -17,10 +17,10 @@ MUTANTS = {
     "scale dropped": ("s[t] = scale * acc;", "s[t] = acc;"),
     "GQA map modulo": ("int g = h / (num_q_heads / num_kv_heads);\n            float ks",
                        "int g = h % num_kv_heads;\n            float ks"),
-    "block/offset swapped": ("int64_t phys = table[t / ORACLE_BLOCK];", "int64_t phys = table[t % ORACLE_BLOCK];"),
-    "slot offset by one": ("off = slot % ORACLE_BLOCK;", "off = (slot + 1) % ORACLE_BLOCK;"),
-    "head/slot transposed": ("int64_t idx = ((phys * num_kv_heads + g) * ORACLE_BLOCK + (t % ORACLE_BLOCK)) * (int64_t)head_dim + d;",
-                             "int64_t idx = ((phys * ORACLE_BLOCK + (t % ORACLE_BLOCK)) * num_kv_heads + g) * (int64_t)head_dim + d;"),
+    "block/offset swapped": ("int64_t phys = table[t / bs];", "int64_t phys = table[t % bs];"),
+    "slot offset by one": ("off = slot % bs;", "off = (slot + 1) % bs;"),
+    "head/slot transposed": ("int64_t idx = ((phys * num_kv_heads + g) * bs + (t % bs)) * (int64_t)head_dim + d;",
+                             "int64_t idx = ((phys * bs + (t % bs)) * num_kv_heads + g) * (int64_t)head_dim + d;"),
     "causal off by one": ("hist + i + 1,", "hist + i,"),
     "softmax not normalised": ("double p = s[t] / sum;", "double p = s[t];"),
     "max not subtracted in sum": ("s[t] = exp(s[t] - mx); sum += s[t];", "s[t] = exp(s[t] - mx); sum += exp(s[t]);"),
@@ -38,10 +38,10 @@ PIN_TESTS = [
     (pins.test_e4m3_decode_spec_points, {}),
     (pins.test_e4m3_encode_spec_points, {}),
     (pins.test_e4m3_encode_matches_torch_cast, {}),
-    (pins.test_decode_matches_sdpa_on_unpaged_kv, dict(hq=8, hkv=2, d=64)),
+    (pins.test_decode_matches_sdpa_on_unpaged_kv, dict(hq=8, hkv=2, d=64, bs=16)),
     (pins.test_prefill_matches_sdpa_with_causal_offset, {}),
     (pins.test_context_of_one_returns_v, {}),
-    (pins.test_tables_read_back_each_sequences_tokens, {}),
+    (pins.test_tables_read_back_each_sequences_tokens, dict(bs=16)),
     (pins.test_copy_on_write_copies_and_keeps_parent, {}),
     (pins.test_int8_encode_points, {}),
     (pins.test_int8_encode_matches_numpy, {}),

@@ -122,11 +122,11 @@ def _sdpa_decode_reference(batch):
     return np.stack(outs)
 
 
-@pytest.mark.parametrize("hq,hkv,d", [(8, 2, 64), (4, 1, 128), (6, 6, 64)])
-def test_decode_matches_sdpa_on_unpaged_kv(O, hq, hkv, d):
+@pytest.mark.parametrize("hq,hkv,d,bs", [(8, 2, 64, 16), (4, 1, 128, 16), (6, 6, 64, 16), (8, 2, 64, 32)])
+def test_decode_matches_sdpa_on_unpaged_kv(O, hq, hkv, d, bs):
     batch = make_batch("tiny_decode", seed=7, overrides=dict(num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
                                                           num_seqs=5, hist=("fixed", [0, 15, 16, 47, 130]),
-                                                          num_blocks=40))
+                                                          num_blocks=40, block_size=bs))
     res = oracle_step(batch, O)
     ref = _sdpa_decode_reference(batch)
     np.testing.assert_allclose(res["decode"], ref, rtol=0, atol=1e-12)
@@ -207,22 +207,25 @@ def test_physical_placement_does_not_change_results(O):
     assert np.array_equal(a["decode"], b["decode"]) and np.array_equal(a["decode"], c["decode"])
 
 
-def test_tables_read_back_each_sequences_tokens(O):
+@pytest.mark.parametrize("bs", [16, 32])
+def test_tables_read_back_each_sequences_tokens(O, bs):
     """After set-up, forks and append, each sequence read through its table is exactly its tokens."""
     batch = make_batch("mixed_step", seed=5, overrides=dict(
         num_seqs=24, hist=("lognormal", 40.0, 1.0, 1, 200), share_group=8, share_prefix=64,
-        prefill_chunks=2, chunk_len=(3, 40), chunk_hist=(1, 60), num_q_heads=4, num_kv_heads=2, head_dim=64))
+        prefill_chunks=2, chunk_len=(3, 40), chunk_hist=(1, 60), num_q_heads=4, num_kv_heads=2, head_dim=64,
+        block_size=bs))
     assert batch.cow_pairs.shape[0] > 0, "workload must exercise copy-on-write"
     res = oracle_step(batch, O, keep_pre_step=True)
     kc, vc = res["k_cache"], res["v_cache"]
     tk, tv = bf16_bits(batch.tok_k), bf16_bits(batch.tok_v)
     ctx = batch.context_lens
+    B = batch.block_size
     for s in range(batch.num_seqs):
         t = np.arange(ctx[s])
-        phys = batch.block_tables[s, t // 16]
+        phys = batch.block_tables[s, t // B]
         assert np.all(phys >= 0)
-        got_k = kc[phys, :, t % 16]
-        got_v = vc[phys, :, t % 16]
+        got_k = kc[phys, :, t % B]
+        got_v = vc[phys, :, t % B]
         rows = batch.seq_rows(s)[: ctx[s]]
         assert np.array_equal(got_k, tk[rows]) and np.array_equal(got_v, tv[rows]), s
 
