@@ -218,8 +218,15 @@ def run_ours(args, rank, world, local_rank):
     d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     p1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     with ClockSampler(local_rank) as clk:
+        # the step value: K steps back to back, no event between the kernels (an event record between
+        # two launches ends the programmatic overlap of the second with the first)
         torch.cuda.synchronize(dev)
         ev0.record(stream)
+        for i in range(K):
+            st.step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        # the same K steps again with events around each attention call: the kernels' own durations
         for i in range(K):
             st.fork()
             st.append()
@@ -228,7 +235,6 @@ def run_ours(args, rank, world, local_rank):
             d1[i].record(stream)
             st.prefill()
             p1[i].record(stream)
-        ev1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -238,33 +244,14 @@ def run_ours(args, rank, world, local_rank):
     if B.pa_get_device_error() != B.PA_OK:
         raise RuntimeError("device error flagged during the timed region")
 
-    # end to end: inputs from pinned host memory, result back to the host, every step
-    host = {
-        "q": st.q_dec.cpu().pin_memory(), "k": st.k_new.cpu().pin_memory(), "v": st.v_new.cpu().pin_memory(),
-        "slots": st.step_slots.cpu().pin_memory(), "tables": st.dec_tables.cpu().pin_memory(),
-        "lens": st.dec_lens.cpu().pin_memory(),
-    }
-    if st.max_q:
-        host["qp"] = st.q_pre.cpu().pin_memory()
-    dst = {"q": st.q_dec, "k": st.k_new, "v": st.v_new, "slots": st.step_slots, "tables": st.dec_tables,
-           "lens": st.dec_lens, "qp": st.q_pre}
-    out_host = torch.empty_like(st.out_dec, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-    if st.max_q:
-        out_pre_host = torch.empty_like(st.out_pre, device="cpu").pin_memory()
-        d2h += out_pre_host.numel() * out_pre_host.element_size()
-
-    def e2e_step():
-        for k, t in host.items():
-            dst[k].copy_(t, non_blocking=True)
-        st.step()
-        out_host.copy_(st.out_dec, non_blocking=True)
-        if st.max_q:
-            out_pre_host.copy_(st.out_pre, non_blocking=True)
-
+    # end to end through the public API: every step copies its inputs in from pinned host memory and
+    # its outputs back out; a copy stream overlaps those copies with the neighbouring steps' compute
+    from pagedattention_block_table_b200.runner import HostPipeline
+    pipe = HostPipeline(st)
+    h2d, d2h = pipe.h2d_bytes, pipe.d2h_bytes
     for _ in range(max(3, args.warmup)):
-        e2e_step()
+        pipe.step()
+    pipe.finish()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
@@ -273,7 +260,8 @@ def run_ours(args, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(K2):
-        e2e_step()
+        pipe.step()
+    pipe.finish()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / K2

@@ -12,18 +12,27 @@
 // softmax of its tile, the tensor core computes the other tile's products.
 //   warps 0-3  softmax of tile A, one row per thread = one TMEM lane   warps 4-7  the same for tile B
 //   warp 8     issues every tcgen05.mma (one elected lane)              warp 9     issues the TMA loads
-// Keys come in tiles of 64 (4 physical blocks): one TMA box of 16 rows x 64 elements per block and per
-// 64-element plane of head_dim, into the UMMA 128-byte-swizzled layout, three tiles in flight (tensor
-// map over the cache seen as [num_blocks*Hkv*16][head_dim]; no multicast).  Each query tile has two S
-// buffers in TMEM, so S of key tile j+2 is computed while the softmax still works on tile j.
+// Keys come in tiles of 128 (8 units of 16 tokens).  K and V tiles take turns in one ring of shared
+// memory slots (K0, V0, K1, V1, ...), filled by TMA with one 16-row x 64-element box per unit and per
+// 64-element plane of head_dim, in the UMMA 128-byte-swizzled layout (tensor map over the cache seen
+// as [num_blocks*Hkv*block_size][head_dim]; no multicast).
+// TMEM (512 columns): S_A, S_B (128 columns each), O_A, O_B (head_dim columns each).
 // Per key tile j and query tile X:
-//   S_X = Q_X K_j^T  (M=128, N=64, fp32 in TMEM)   ->  softmax warps: base-2 online softmax, P_X (bf16,
-//   K-major swizzled) into shared memory          ->  O_X += P_X V_j  (M=128, N=head_dim, fp32 in TMEM).
-// p is taken relative to a per-row reference max; only when a tile's max exceeds it by more than 2^8
-// does the row move the reference and rescale its O row in TMEM (tcgen05.ld/st) and its sum l.  O and l
-// always share the reference, so out = O / l is exact whichever reference was used.
+//   S_X = Q_X K_j^T        M=128, N=128, both operands in shared memory, fp32 into TMEM
+//   softmax warps          read S_X, base-2 online softmax, write P_X (bf16 pairs) back into the first
+//                          64 columns of S_X with tcgen05.st
+//   O_X += P_X V_j         A operand (P) read from TMEM, V from shared memory, fp32 accumulator in TMEM
+// The tensor core runs O_A(j), S_A(j+1), O_B(j), S_B(j+1), ... in issue order, so S_X(j+1) overwrites
+// the columns P_X(j) occupies only after O_X(j) has read them.  p is taken relative to a per-row
+// reference max; only when a tile's max exceeds it by more than 2^8 does the row move the reference
+// and rescale its O row in TMEM (tcgen05.ld/st) and its sum l.  O and l always share the reference,
+// so out = O / l is exact whichever reference was used.
 #pragma once
 #include "pa_common.cuh"
+
+#ifndef PA_PREFILL_SPLIT_REGS
+#define PA_PREFILL_SPLIT_REGS 0
+#endif
 
 namespace pa {
 
@@ -59,32 +68,39 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
                : "memory");
 }
 
-// This thread's TMEM lane, 32 consecutive fp32 columns starting at taddr's column.
+// This thread's TMEM lane, 32 consecutive fp32 columns starting at taddr's column.  The load and its
+// wait are one asm statement, so no use of the registers can be scheduled before the wait.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      : "r"(taddr)
+      : "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// This thread's TMEM lane, 64 consecutive fp32 columns (one load, one wait).
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[64];
+// 128 consecutive 32-bit columns of this thread's TMEM lane (two loads, one wait, one asm statement).
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
       "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
       "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
-      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%128];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+      "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95, "
+      "%96, %97, %98, %99, %100, %101, %102, %103, %104, %105, %106, %107, %108, %109, %110, %111, "
+      "%112, %113, %114, %115, %116, %117, %118, %119, %120, %121, %122, %123, %124, %125, %126, %127}, [%129];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
         "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
@@ -92,11 +108,18 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
         "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]),
         "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]),
         "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
-        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63]),
+        "=r"(r[64]), "=r"(r[65]), "=r"(r[66]), "=r"(r[67]), "=r"(r[68]), "=r"(r[69]), "=r"(r[70]), "=r"(r[71]),
+        "=r"(r[72]), "=r"(r[73]), "=r"(r[74]), "=r"(r[75]), "=r"(r[76]), "=r"(r[77]), "=r"(r[78]), "=r"(r[79]),
+        "=r"(r[80]), "=r"(r[81]), "=r"(r[82]), "=r"(r[83]), "=r"(r[84]), "=r"(r[85]), "=r"(r[86]), "=r"(r[87]),
+        "=r"(r[88]), "=r"(r[89]), "=r"(r[90]), "=r"(r[91]), "=r"(r[92]), "=r"(r[93]), "=r"(r[94]), "=r"(r[95]),
+        "=r"(r[96]), "=r"(r[97]), "=r"(r[98]), "=r"(r[99]), "=r"(r[100]), "=r"(r[101]), "=r"(r[102]),
+        "=r"(r[103]), "=r"(r[104]), "=r"(r[105]), "=r"(r[106]), "=r"(r[107]), "=r"(r[108]), "=r"(r[109]),
+        "=r"(r[110]), "=r"(r[111]), "=r"(r[112]), "=r"(r[113]), "=r"(r[114]), "=r"(r[115]), "=r"(r[116]),
+        "=r"(r[117]), "=r"(r[118]), "=r"(r[119]), "=r"(r[120]), "=r"(r[121]), "=r"(r[122]), "=r"(r[123]),
+        "=r"(r[124]), "=r"(r[125]), "=r"(r[126]), "=r"(r[127])
+      : "r"(taddr), "r"(taddr + 64)
+      : "memory");
 }
 
 // Store 32 fp32 columns of this thread's TMEM lane.
@@ -116,6 +139,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: A (M rows = TMEM lanes, K packed two bf16 per column) from
+// tensor memory, bf16 inputs, fp32 accumulate; issued by one thread.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Store 32 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st32u_nowait(uint32_t taddr, const uint32_t *v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
+      "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
+      "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 2-D tiled TMA load global -> shared, completing on `bar`.  x is the innermost coordinate.
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
@@ -168,48 +217,47 @@ struct PrefillParams {
   float qscale;         // scale * log2(e)
 };
 
-#ifndef PA_PREFILL_STAGES
-#define PA_PREFILL_STAGES 4
-#endif
-
 template <int D>
 struct PrefillCfg {
   static constexpr int BM = 128;                  // rows per query tile (= TMEM lanes)
-  static constexpr int BN = 64;                   // keys per key tile (4 blocks)
-  static constexpr int STAGES = PA_PREFILL_STAGES;  // K/V tiles in flight: S runs two tiles ahead of PV
+  static constexpr int BN = 128;                  // keys per key tile (8 units of 16 tokens)
   static constexpr int DH = D / 64;               // 64-element (128-byte) planes of a head_dim row
   static constexpr int Q_PLANE = BM * 128;        // 16 KB
-  static constexpr int KV_PLANE = BN * 128;       // 8 KB
   static constexpr int Q_BYTES = DH * Q_PLANE;
-  static constexpr int KV_BYTES = DH * KV_PLANE;  // one K or V tile
-  static constexpr int P_BYTES = BM * 128;        // 128 rows x 64 keys bf16
+  static constexpr int KV_PLANE = BN * 128;       // 16 KB
+  static constexpr int SLOT_BYTES = DH * KV_PLANE;  // one K or V tile
+  static constexpr int NSLOT = D == 128 ? 5 : 8;  // ring of K/V tiles (K and V alternate)
   static constexpr int OFF_QA = 0;
   static constexpr int OFF_QB = OFF_QA + Q_BYTES;
-  static constexpr int OFF_K = OFF_QB + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_PA = OFF_V + STAGES * KV_BYTES;
-  static constexpr int OFF_PB = OFF_PA + P_BYTES;
-  static constexpr int OFF_BAR = OFF_PB + P_BYTES;
-  static constexpr int NBAR = 24;
+  static constexpr int OFF_KV = OFF_QB + Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NSLOT * SLOT_BYTES;
+  static constexpr int NBAR = 32;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + slack to align the base to 1024
   static constexpr uint32_t TMEM_COLS = 512;
-  // TMEM columns: S of tile X, buffer b at 64*(2X+b); O of tile X at 256 + 128X
-  __host__ __device__ static constexpr uint32_t s_col(int X, int b) { return 64u * (2u * X + b); }
-  __host__ __device__ static constexpr uint32_t o_col(int X) { return 256u + 128u * X; }
+  // TMEM columns: S of tile X at 128X (P_X in its first 64 columns); O of tile X at 256 + D*X
+  __host__ __device__ static constexpr uint32_t s_col(int X) { return 128u * X; }
+  __host__ __device__ static constexpr uint32_t o_col(int X) { return 256u + static_cast<uint32_t>(D) * X; }
+#if PA_PREFILL_SPLIT_REGS
+  // three warpgroups: softmax A, softmax B, and one holding the MMA and TMA warps (plus two idle warps)
+  // that hands registers to the softmax warpgroups with setmaxnreg
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_LAUNCH = 168;         // 65536 / 384, rounded down to a multiple of 8
+  static constexpr int REGS_SOFTMAX = 216;
+  static constexpr int REGS_PRODUCER = 64;
+  static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_PRODUCER <= THREADS * REGS_LAUNCH, "register split");
+#else
   static constexpr int THREADS = 320;
+#endif
   static_assert(D == 64 || D == 128, "head_dim");
   static_assert(SMEM <= 227 * 1024, "shared memory");
-
 };
 
-// mbarrier slots
-// kKvFull/kKvEmpty: per stage; kSFull: per (tile X, buffer b) at kSFull + 2X + b; kOFull, kPFull: per tile
+// mbarrier slots: kFull/kEmpty per ring slot; kSFull, kPFull per query tile
 enum : int {
-  kKvFull = 0,
-  kKvEmpty = kKvFull + PA_PREFILL_STAGES,
-  kSFull = kKvEmpty + PA_PREFILL_STAGES,
-  kOFull = kSFull + 4,
-  kPFull = kOFull + 2,
+  kFull = 0,
+  kEmpty = kFull + 8,
+  kSFull = kEmpty + 8,
+  kPFull = kSFull + 2,
   kQReady = kPFull + 2,
   kDone = kQReady + 1,
   kNumBars = kDone + 1
@@ -221,39 +269,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x for a packed pair on the FMA pipe (to take load off the MUFU unit): x = n + f with n = rint(x)
-// (add/subtract 1.5*2^23) and f in [-0.5, 0.5]; 2^f by a cubic fitted here to minimise the relative
-// error on that interval (max 7.5e-5, below the bf16 resolution P is rounded to); 2^n is added to the
-// exponent field.  Arguments below -125 give 0 (as the flush-to-zero ex2 does for results in the
-// denormal range); -inf gives 0.
-__device__ __forceinline__ uint64_t ex2_poly2(float xa, float xb) {
-  const float x0 = fmaxf(xa, -125.f), x1 = fmaxf(xb, -125.f);
-  const uint64_t shifter = f2pack(12582912.f, 12582912.f), xx = f2pack(x0, x1);
-  uint64_t t, n2, f2;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xx), "l"(shifter));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(n2) : "l"(t), "l"(shifter));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f2) : "l"(xx), "l"(n2));
-  uint64_t p = f2pack(0.05517394095659256f, 0.05517394095659256f);
-  p = ffma2(p, f2, f2pack(0.24261131882667542f, 0.24261131882667542f));
-  p = ffma2(p, f2, f2pack(0.6932605504989624f, 0.6932605504989624f));
-  p = ffma2(p, f2, f2pack(0.9999280571937561f, 0.9999280571937561f));
-  const float2 tv = f2unpack(t), pv = f2unpack(p);
-  const float a = x0 > -125.f ? __int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)) : 0.f;
-  const float b = x1 > -125.f ? __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)) : 0.f;
-  return f2pack(a, b);
-}
-
-// One 8-key chunk in PA_PREFILL_POLY_EVERY takes its exponentials from ex2_poly2 (0 = none).
-#ifndef PA_PREFILL_POLY_EVERY
-#define PA_PREFILL_POLY_EVERY 0
-#endif
-
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                          const PrefillParams P) {
   using C = PrefillCfg<D>;
-  static_assert(kNumBars <= C::NBAR, "barrier slots");
+  static_assert(kNumBars <= C::NBAR && C::NSLOT <= 8, "barrier slots");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -278,6 +299,8 @@ __global__ void __launch_bounds__(320, 1)
   const int p_end = min(Cn, p0 + 2 * ppt);
   const int kv_len = H + p_end;                       // keys visible to some row of this CTA
   const int ntiles = (kv_len + C::BN - 1) / C::BN;
+  // 16-key steps of the last tile that hold a visible key (the PV product stops there)
+  const int last_k16 = (kv_len - (ntiles - 1) * C::BN + 15) / 16;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
@@ -286,13 +309,12 @@ __global__ void __launch_bounds__(320, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < C::STAGES; ++i) {
-      mbar_init(&bars[kKvFull + i], 1);
-      mbar_init(&bars[kKvEmpty + i], 1);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(&bars[kFull + i], 1);
+      mbar_init(&bars[kEmpty + i], 1);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[kSFull + i], 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&bars[kOFull + i], 1);
+      mbar_init(&bars[kSFull + i], 1);
       mbar_init(&bars[kPFull + i], 128);
     }
     mbar_init(&bars[kQReady], 256);
@@ -304,9 +326,14 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   bool timeout = false;
+  // ring item i (K of tile i/2 when i is even, V when odd) sits in slot i % NSLOT; its use count is i / NSLOT
+  auto slot_of = [&](int i) { return smem + C::OFF_KV + (i % C::NSLOT) * C::SLOT_BYTES; };
 
   if (warp < 8) {
     // ===================================================================== softmax warpgroups
+#if PA_PREFILL_SPLIT_REGS
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+#endif
     const int X = warp >> 2;                          // 0: tile A, 1: tile B
     const int r = tid & 127;                          // row = TMEM lane
     const int pos_i = p0 + X * ppt + r / P.hpr;       // position within the chunk
@@ -314,7 +341,6 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_ok = pos_i < Cn;
     const int pos = row_ok ? H + pos_i : kv_len - 1;  // padding rows behave like the last row
     uint8_t *sQ = smem + (X ? C::OFF_QB : C::OFF_QA);
-    uint8_t *sP = smem + (X ? C::OFF_PB : C::OFF_PA);
     // Q row into the K-major 128-byte-swizzled tile (chunk ch of row r at ch ^ (r % 8))
     {
       uint8_t *rowp = sQ + r * 128;
@@ -332,128 +358,113 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(&bars[kQReady]);
     }
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_addr = tmem + lane_base + C::s_col(X);
     const uint32_t o_addr = tmem + lane_base + C::o_col(X);
     constexpr float kRescale = 8.f;
     const float qs = P.qscale;
     float m_ref = -INFINITY, l_run = 0.f;
     for (int j = 0; j < ntiles; ++j) {
-      // every wait's outcome is made warp-uniform: the tcgen05.ld/st below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + 2 * X + (j & 1)], (j >> 1) & 1))) { timeout = true; break; }
+      // every wait's outcome is made warp-uniform: the tcgen05.ld/st below are warp-collective.
+      // S_X(j) complete also means O_X(j-1) complete (issued before it, tracked by the same commit).
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + X], j & 1))) { timeout = true; break; }
       tc_fence_after();
-      float s[C::BN];
-      tmem_ld64(tmem + lane_base + C::s_col(X, j & 1), s);
+      uint32_t sr[C::BN];
+      tmem_ld128(s_addr, sr);
       const int kbase = j * C::BN;
-      // scaled row max of this tile; masked keys (past the row's position) become -inf
+      const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
+      // scaled row max of this tile; masked keys (past the row's position) do not take part
       float mt_ = -INFINITY;
-      if (kbase + C::BN - 1 <= pos) {
-        // max of s * qscale: the max of s for a positive scale, the min for a negative one; eight
-        // independent partial results so the reduction is not one long dependent chain
-        float e[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) e[k] = s[k];
+      if (!diag) {
+        // max of s * qscale: the max of s for a positive scale, the min for a negative one
+        float e0 = __uint_as_float(sr[0]), e1 = __uint_as_float(sr[1]), e2 = __uint_as_float(sr[2]),
+              e3 = __uint_as_float(sr[3]);
         if (qs >= 0.f) {
 #pragma unroll
-          for (int k = 8; k < C::BN; ++k) e[k & 7] = fmaxf(e[k & 7], s[k]);
-#pragma unroll
-          for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-            for (int k = 0; k < w; ++k) e[k] = fmaxf(e[k], e[k + w]);
+          for (int k = 4; k < C::BN; k += 4) {
+            e0 = fmaxf(e0, __uint_as_float(sr[k]));
+            e1 = fmaxf(e1, __uint_as_float(sr[k + 1]));
+            e2 = fmaxf(e2, __uint_as_float(sr[k + 2]));
+            e3 = fmaxf(e3, __uint_as_float(sr[k + 3]));
+          }
+          mt_ = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3)) * qs;
         } else {
 #pragma unroll
-          for (int k = 8; k < C::BN; ++k) e[k & 7] = fminf(e[k & 7], s[k]);
-#pragma unroll
-          for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-            for (int k = 0; k < w; ++k) e[k] = fminf(e[k], e[k + w]);
+          for (int k = 4; k < C::BN; k += 4) {
+            e0 = fminf(e0, __uint_as_float(sr[k]));
+            e1 = fminf(e1, __uint_as_float(sr[k + 1]));
+            e2 = fminf(e2, __uint_as_float(sr[k + 2]));
+            e3 = fminf(e3, __uint_as_float(sr[k + 3]));
+          }
+          mt_ = fminf(fminf(e0, e1), fminf(e2, e3)) * qs;
         }
-        mt_ = e[0] * qs;
       } else {
-        float e[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) e[k] = -INFINITY;
 #pragma unroll
         for (int k = 0; k < C::BN; ++k)
-          if (kbase + k <= pos) e[k & 7] = fmaxf(e[k & 7], s[k] * qs);
-#pragma unroll
-        for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-          for (int k = 0; k < w; ++k) e[k] = fmaxf(e[k], e[k + w]);
-        mt_ = e[0];
+          if (kbase + k <= pos) mt_ = fmaxf(mt_, __uint_as_float(sr[k]) * qs);
       }
-      const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
-      // the previous tile's PV must be complete before O is rescaled or P is overwritten
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars[kOFull + X], (j - 1) & 1))) { timeout = true; break; }
-      tc_fence_after();
+      // move the reference when the tile's max exceeds it by more than 2^8 (O and l follow below)
       const bool bump = mt_ > m_ref + kRescale;
-      if (__any_sync(0xffffffffu, bump)) {
-        const float m_new = bump ? mt_ : m_ref;
-        const float alpha = exp2f(m_ref - m_new);
-        if (j > 0) {
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            float ov[32];
-            tmem_ld32(o_addr + cc * 32, ov);
+      const bool any_bump = __any_sync(0xffffffffu, bump);
+      float alpha = 1.f;
+      if (bump) {
+        alpha = exp2f(m_ref - mt_);
+        m_ref = mt_;
+      }
+      // last key tile: V rows of keys no row may see, up to the last 16-key step the PV product reads,
+      // are zeroed (tile A's threads, one row each) once the V tile has landed, so that 0 * (whatever
+      // the cache holds past the context) never reaches the MMA
+      if (X == 0 && j == ntiles - 1 && kbase + r >= kv_len && r < last_k16 * 16) {
+        const int it = 2 * j + 1;
+        if (mbar_wait(&bars[kFull + it % C::NSLOT], (it / C::NSLOT) & 1)) {
+          uint8_t *vt = slot_of(it);
 #pragma unroll
-            for (int k = 0; k < 32; ++k) ov[k] *= alpha;
-            tmem_st32(o_addr + cc * 32, ov);
-          }
+          for (int hh = 0; hh < C::DH; ++hh)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4 *>(vt + hh * C::KV_PLANE + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
+          fence_async_smem();
         }
-        l_run *= alpha;
-        m_ref = m_new;
       }
-      // last key tile: V rows of keys no row may see are zeroed (tile A's threads, one row each), so
-      // that 0 * (whatever the cache holds past the context) never reaches the MMA
-      if (X == 0 && r < C::BN && (j + 1) * C::BN > kv_len && kbase + r >= kv_len) {
-        uint8_t *vt = smem + C::OFF_V + (j % C::STAGES) * C::KV_BYTES;
-#pragma unroll
-        for (int hh = 0; hh < C::DH; ++hh)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch)
-            *reinterpret_cast<uint4 *>(vt + hh * C::KV_PLANE + r * 128 + ch * 16) = make_uint4(0, 0, 0, 0);
-      }
-      uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};   // independent partial row sums
+      uint64_t ls2 = 0ull;
       const uint64_t qs2 = f2pack(qs, qs), nm2 = f2pack(-m_ref, -m_ref);
-      uint8_t *prow = sP + r * 128;
 #pragma unroll
-      for (int q8 = 0; q8 < C::BN / 8; ++q8) {
-        uint32_t pk[4];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int k2 = 0; k2 < 4; ++k2) {
+        for (int k2 = 0; k2 < 32; ++k2) {
+          const int k = half * 64 + 2 * k2;
           // x = s * qscale - m_ref for two keys at once; keys past the row's position get p = 0
-          float2 x = f2unpack(ffma2(f2pack(s[q8 * 8 + 2 * k2], s[q8 * 8 + 2 * k2 + 1]), qs2, nm2));
+          float2 x = f2unpack(ffma2(f2pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), qs2, nm2));
           if (diag) {
-            const int t = kbase + q8 * 8 + 2 * k2;
-            if (t > pos) x.x = -INFINITY;
-            if (t + 1 > pos) x.y = -INFINITY;
+            if (kbase + k > pos) x.x = -INFINITY;
+            if (kbase + k + 1 > pos) x.y = -INFINITY;
           }
-#if PA_PREFILL_POLY_EVERY > 0
-          float a, b;
-          if (q8 % PA_PREFILL_POLY_EVERY == PA_PREFILL_POLY_EVERY - 1) {
-            const float2 e = f2unpack(ex2_poly2(x.x, x.y));
-            a = e.x;
-            b = e.y;
-          } else {
-            a = ex2(x.x);
-            b = ex2(x.y);
-          }
-#else
           const float a = ex2(x.x);
           const float b = ex2(x.y);
-#endif
-          ls2[k2] = f2add(ls2[k2], f2pack(a, b));
+          ls2 = f2add(ls2, f2pack(a, b));
           pk[k2] = pack_bf16x2(a, b);
         }
-        *reinterpret_cast<uint4 *>(prow + ((q8 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st32u_nowait(s_addr + half * 32, pk);
       }
-      const float2 lsv = f2unpack(f2add(f2add(ls2[0], ls2[1]), f2add(ls2[2], ls2[3])));
-      const float ls = lsv.x + lsv.y;
-      l_run += ls;
-      fence_async_smem();
+      const float2 lsv = f2unpack(ls2);
+      l_run = l_run * alpha + (lsv.x + lsv.y);
+      if (any_bump && j > 0) {
+        // rescale this row's O to the new reference (O_X(j-1) is complete; O_X(j) waits for P_X(j))
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] *= alpha;
+          tmem_st32(o_addr + cc * 32, ov);
+        }
+      }
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[kPFull + X]);
     }
     // ---- epilogue: out = O / l once the last PV is done
-    if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kOFull + X], (ntiles - 1) & 1))) {
+    if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0))) {
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       uint4 *dst = reinterpret_cast<uint4 *>(P.out + ((int64_t)(q0 + (row_ok ? pos_i : 0)) * P.num_q_heads + h) * D);
@@ -471,102 +482,125 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  } else if (warp == 8) {
+  } else {
+#if PA_PREFILL_SPLIT_REGS
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_PRODUCER));
+#endif
+  if (warp == 8) {
     // ===================================================================== MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(128, C::BN, false);
       constexpr uint32_t idO = idesc_bf16(128, D, true);
       const uint32_t qa = smem_u32(smem + C::OFF_QA), qb = smem_u32(smem + C::OFF_QB);
-      const uint32_t pa = smem_u32(smem + C::OFF_PA), pb = smem_u32(smem + C::OFF_PB);
-      const uint32_t kb0 = smem_u32(smem + C::OFF_K), vb0 = smem_u32(smem + C::OFF_V);
-      auto issue_s = [&](int X, int j) {
-        const uint32_t qx = X ? qb : qa;
-        const uint32_t kt = kb0 + (j % C::STAGES) * C::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk & 3) * 32;
-          mma_bf16(tmem + C::s_col(X, j & 1), sw128_desc(qx + (kk >> 2) * C::Q_PLANE + ko, 16, 1024),
-                   sw128_desc(kt + (kk >> 2) * C::KV_PLANE + ko, 16, 1024), idS, kk > 0);
-        }
-        mma_commit(&bars[kSFull + 2 * X + (j & 1)]);
-      };
-      auto issue_o = [&](int X, int j) {
-        const uint32_t px = X ? pb : pa;
-        const uint32_t vt = vb0 + (j % C::STAGES) * C::KV_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < C::BN / 16; ++kk)
-          mma_bf16(tmem + C::o_col(X), sw128_desc(px + kk * 32, 16, 1024),
-                   sw128_desc(vt + kk * (16 * 128), C::KV_PLANE, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars[kOFull + X]);
-      };
-      auto kv_ready = [&](int j) {
-        const bool r = mbar_wait(&bars[kKvFull + (j % C::STAGES)], (j / C::STAGES) & 1);
+      auto ready = [&](int i) {
+        const bool r = mbar_wait(&bars[kFull + i % C::NSLOT], (i / C::NSLOT) & 1);
         tc_fence_after();
         return r;
       };
-      // S runs up to two key tiles ahead of PV (two S buffers per query tile)
-      bool ok = mbar_wait(&bars[kQReady], 0) && kv_ready(0);
+      auto release = [&](int i) { mma_commit(&bars[kEmpty + i % C::NSLOT]); };
+      auto issue_s = [&](int X, int j) {
+        const uint32_t qx = X ? qb : qa;
+        const uint32_t kt = smem_u32(slot_of(2 * j));
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk & 3) * 32;
+          mma_bf16(tmem + C::s_col(X), sw128_desc(qx + (kk >> 2) * C::Q_PLANE + ko, 16, 1024),
+                   sw128_desc(kt + (kk >> 2) * C::KV_PLANE + ko, 16, 1024), idS, kk > 0);
+        }
+        mma_commit(&bars[kSFull + X]);
+      };
+      auto issue_o = [&](int X, int j) {
+        const uint32_t vt = smem_u32(slot_of(2 * j + 1));
+        const int nk = j == ntiles - 1 ? last_k16 : C::BN / 16;
+        for (int kk = 0; kk < nk; ++kk)
+          mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
+                      sw128_desc(vt + kk * (16 * 128), C::KV_PLANE, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&bars[kQReady], 0) && ready(0);
       if (ok) {
         issue_s(0, 0);
         issue_s(1, 0);
-      }
-      if (ok && ntiles > 1 && (ok = kv_ready(1))) {
-        issue_s(0, 1);
-        issue_s(1, 1);
+        release(0);
       }
       for (int j = 0; ok && j < ntiles; ++j) {
-        if (!(ok = mbar_wait(&bars[kPFull + 0], j & 1))) break;
+        const bool more = j + 1 < ntiles;
+        if (!(ok = ready(2 * j + 1))) break;                       // V_j
+        if (!(ok = mbar_wait(&bars[kPFull + 0], j & 1))) break;    // P_A(j) in TMEM
         tc_fence_after();
         issue_o(0, j);
-        const bool more = j + 2 < ntiles;
         if (more) {
-          if (!(ok = kv_ready(j + 2))) break;
-          issue_s(0, j + 2);   // into the buffer softmax A has just finished reading
+          if (!(ok = ready(2 * j + 2))) break;                     // K_{j+1}
+          issue_s(0, j + 1);                                       // after O_A(j) has read P_A(j)
         }
-        if (!(ok = mbar_wait(&bars[kPFull + 1], j & 1))) break;
+        if (!(ok = mbar_wait(&bars[kPFull + 1], j & 1))) break;    // P_B(j)
         tc_fence_after();
         issue_o(1, j);
-        mma_commit(&bars[kKvEmpty + (j % C::STAGES)]);   // every product reading tile j issued
-        if (more) issue_s(1, j + 2);
+        release(2 * j + 1);                                        // V_j read by both PV products
+        if (more) {
+          issue_s(1, j + 1);
+          release(2 * j + 2);                                      // K_{j+1} read by both QK products
+        }
       }
       mma_commit(&bars[kDone]);                    // fires once every MMA issued above has completed
       if (!ok) timeout = true;
     }
-  } else {
+  } else if (warp == 9) {
     // ===================================================================== TMA producer
     if (lane == 0) {
       const int32_t *trow = P.block_tables + (int64_t)c * P.max_blocks_per_seq;
-      int j = 0;
-      for (; j < ntiles; ++j) {
-        const int st = j % C::STAGES;
-        if (j >= C::STAGES && !mbar_wait(&bars[kKvEmpty + st], ((j - C::STAGES) / C::STAGES) & 1)) {
-          timeout = true;
-          break;
-        }
-        const int nb = min(C::BN / kBlock, (kv_len - j * C::BN + kBlock - 1) / kBlock);
-        mbar_arrive_expect_tx(&bars[kKvFull + st], nb * 2 * C::DH * (kBlock * 128));
-        const int upb = P.block_size / kBlock;   // 16-row units per physical block
-        for (int bb = 0; bb < nb; ++bb) {
-          const int u = j * (C::BN / kBlock) + bb;   // 16-token unit of the sequence
-          int e = __ldg(trow + u / upb);
-          if (e < 0 || e >= P.num_blocks) {
-            flag_error(kErrBlockId);
-            e = 0;
-          }
-          const int y = ((e * P.num_kv_heads + g) * upb + u % upb) * kBlock;
+      const int ush = P.block_size == 32 ? 1 : 0;   // log2(16-row units per physical block)
+      constexpr int UPT = C::BN / kBlock;             // units per key tile
+      // cache-row index of each unit of key tile j: the table entries of a tile are loaded together,
+      // one tile ahead of the copies that use them
+      auto rows_of = [&](int j, int (&y)[UPT]) {
 #pragma unroll
-          for (int hh = 0; hh < C::DH; ++hh) {
-            const int off = st * C::KV_BYTES + hh * C::KV_PLANE + bb * (kBlock * 128);
-            tma_load_2d(smem + C::OFF_K + off, &kmap, hh * 64, y, &bars[kKvFull + st]);
-            tma_load_2d(smem + C::OFF_V + off, &vmap, hh * 64, y, &bars[kKvFull + st]);
+        for (int bb = 0; bb < UPT; ++bb) {
+          const int u = j * UPT + bb;
+          int e = 0;
+          if (u * kBlock < kv_len) {
+            e = __ldg(trow + (u >> ush));
+            if (e < 0 || e >= P.num_blocks) {
+              flag_error(kErrBlockId);
+              e = 0;
+            }
+          }
+          y[bb] = (((e * P.num_kv_heads + g) << ush) + (u & ((1 << ush) - 1))) * kBlock;
+        }
+      };
+      int ycur[UPT], ynext[UPT];
+      rows_of(0, ycur);
+      int i = 0;
+      for (int j = 0; j < ntiles; ++j) {
+        if (j + 1 < ntiles) rows_of(j + 1, ynext);
+        const int nu = min(UPT, (kv_len - j * C::BN + kBlock - 1) / kBlock);
+        for (int v = 0; v < 2; ++v, ++i) {
+          const int slot = i % C::NSLOT;
+          if (i >= C::NSLOT && !mbar_wait(&bars[kEmpty + slot], ((i / C::NSLOT) - 1) & 1)) {
+            timeout = true;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars[kFull + slot], nu * C::DH * (kBlock * 128));
+          const CUtensorMap *map = v ? &vmap : &kmap;
+          uint8_t *dst = slot_of(i);
+#pragma unroll
+          for (int bb = 0; bb < UPT; ++bb) {
+            if (bb < nu) {
+#pragma unroll
+              for (int hh = 0; hh < C::DH; ++hh)
+                tma_load_2d(dst + hh * C::KV_PLANE + bb * (kBlock * 128), map, hh * 64, ycur[bb], &bars[kFull + slot]);
+            }
           }
         }
+        if (timeout) break;
+#pragma unroll
+        for (int bb = 0; bb < UPT; ++bb) ycur[bb] = ynext[bb];
       }
-      // before leaving, the last (at most two) tiles this thread issued must have landed (a no-op when
-      // the MMA warp consumed them; bounded when a wait elsewhere gave up)
-      for (int k = max(0, j - C::STAGES); k < j; ++k)
-        (void)mbar_wait(&bars[kKvFull + (k % C::STAGES)], (k / C::STAGES) & 1);
+      // before leaving, the last tiles this thread issued must have landed (a no-op when the MMA warp
+      // consumed them; bounded when a wait elsewhere gave up)
+      for (int k = max(0, i - C::NSLOT); k < i; ++k)
+        (void)mbar_wait(&bars[kFull + (k % C::NSLOT)], (k / C::NSLOT) & 1);
     }
+  }
   }
   // ---- teardown: every MMA has completed before TMEM is released (bounded waits throughout; on a
   // timeout the error word is set and the CTA leaves without its output)
@@ -621,6 +655,14 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
   if (cudaFuncSetAttribute(paged_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return -3;
+#if PA_PREFILL_SPLIT_REGS
+  // setmaxnreg.inc waits until the block's launch allocation can cover the new split: never launch a
+  // build whose register count per thread would not
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, paged_prefill_kernel<D>) != cudaSuccess ||
+      fa.numRegs * C::THREADS < 2 * 128 * C::REGS_SOFTMAX + 128 * C::REGS_PRODUCER)
+    return -3;
+#endif
   const int ppt = C::BM / P.hpr;
   dim3 grid((max_q_len + 2 * ppt - 1) / (2 * ppt), P.num_q_heads / P.hpr, num_chunks);
   return launch_pdl(paged_prefill_kernel<D>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;

@@ -106,3 +106,72 @@ class DeviceStep:
         self.append(stream)
         self.decode(stream)
         self.prefill(stream)
+
+
+
+class HostPipeline:
+    """Serving steps fed from host memory, double-buffered: while the device computes step i, a copy
+    stream brings step i+1's inputs (queries, new K/V, slots, tables, lengths) in from pinned host
+    buffers and takes step i-1's outputs back out.  Every step still moves all of its own inputs and
+    outputs across the host link; the copies only overlap the computation instead of preceding it.
+    """
+
+    IN_KEYS = ("q_dec", "k_new", "v_new", "step_slots", "dec_tables", "dec_lens", "q_pre")
+
+    def __init__(self, st: DeviceStep):
+        self.st = st
+        dev = st.device
+        self.host_in = {k: getattr(st, k).detach().cpu().pin_memory() for k in self.IN_KEYS}
+        self.slots_in = [{k: torch.empty_like(getattr(st, k)) for k in self.IN_KEYS} for _ in range(2)]
+        self.slots_out = [(torch.empty_like(st.out_dec), torch.empty_like(st.out_pre)) for _ in range(2)]
+        self.host_out = [(torch.empty_like(st.out_dec, device="cpu").pin_memory(),
+                          torch.empty_like(st.out_pre, device="cpu").pin_memory()) for _ in range(2)]
+        self.copy = torch.cuda.Stream(device=dev)
+        self.comp = torch.cuda.current_stream(dev)
+        self.h2d_done = [torch.cuda.Event() for _ in range(2)]
+        self.comp_done = [torch.cuda.Event() for _ in range(2)]
+        self.d2h_done = [torch.cuda.Event() for _ in range(2)]
+        self.i = 0
+
+    @property
+    def h2d_bytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in self.host_in.values())
+
+    @property
+    def d2h_bytes(self) -> int:
+        a, b = self.host_out[0]
+        return a.numel() * a.element_size() + b.numel() * b.element_size()
+
+    def _load(self, slot: int):
+        with torch.cuda.stream(self.copy):
+            if self.i >= 2:
+                self.copy.wait_event(self.comp_done[slot])      # slot's previous step has read its inputs
+            for k, t in self.host_in.items():
+                self.slots_in[slot][k].copy_(t, non_blocking=True)
+            self.h2d_done[slot].record(self.copy)
+
+    def step(self):
+        """Run one step on the inputs already in flight, and start the next step's input copies."""
+        s = self.i % 2
+        if self.i == 0:
+            self._load(0)
+        st = self.st
+        self.comp.wait_event(self.h2d_done[s])
+        if self.i >= 2:
+            self.comp.wait_event(self.d2h_done[s])              # output slot free again
+        for k, t in self.slots_in[s].items():
+            setattr(st, k, t)
+        st.out_dec, st.out_pre = self.slots_out[s]
+        st.step(self.comp)
+        self.comp_done[s].record(self.comp)
+        self.i += 1
+        self._load(self.i % 2)
+        with torch.cuda.stream(self.copy):
+            self.copy.wait_event(self.comp_done[s])
+            self.host_out[s][0].copy_(self.slots_out[s][0], non_blocking=True)
+            self.host_out[s][1].copy_(self.slots_out[s][1], non_blocking=True)
+            self.d2h_done[s].record(self.copy)
+
+    def finish(self):
+        """Wait for the last outputs to reach the host."""
+        torch.cuda.current_stream(self.st.device).wait_stream(self.copy)

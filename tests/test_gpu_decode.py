@@ -171,3 +171,25 @@ def test_kv_head_shards_reproduce_the_unsharded_call(cuda_lib):
     full = _gpu_decode(batch, 256).out_dec
     parts = [_gpu_decode(sharding.shard_batch(batch, r, 4), 256).out_dec for r in range(4)]
     assert torch.equal(torch.cat(parts, dim=1), full)
+
+
+def test_host_pipeline_delivers_the_step_outputs(cuda_lib):
+    """The double-buffered host-fed pipeline (inputs copied in and outputs copied out every step,
+    overlapped with compute) returns the same outputs to the host as a plain device step."""
+    from pagedattention_block_table_b200.runner import DeviceStep, HostPipeline
+    # no shared prefixes: a repeated step is then idempotent (with forks, re-copying a page that its
+    # last holder already appended into would change the copy)
+    batch = make_batch("mixed_step", seed=53, overrides=dict(
+        num_seqs=6, hist=("uniform", 20, 300), share_group=0, share_prefix=0, prefill_chunks=2,
+        chunk_len=(30, 150), chunk_hist=(1, 100), num_q_heads=8, num_kv_heads=2))
+    ref = _gpu_decode(batch, 64)
+    st = DeviceStep(batch, split_tokens=64)
+    st.fill_history()
+    pipe = HostPipeline(st)
+    for _ in range(5):
+        pipe.step()
+    pipe.finish()
+    torch.cuda.synchronize()
+    for s in range(2):
+        assert torch.equal(pipe.host_out[s][0], ref.out_dec.cpu())
+        assert torch.equal(pipe.host_out[s][1], ref.out_pre.cpu())

@@ -89,3 +89,24 @@ def test_mixed_step_full_size_sampled(O, cuda_lib):
             q = bf16_bits(batch.q_prefill[cu[c] + i:cu[c] + i + 1])
             ref = oracle_attend_prefix(batch, s, H + i + 1, q, O)
             assert_close(pre[cu[c] + i], ref[0], what=f"chunk {c} row {i}")
+
+
+@pytest.mark.parametrize("scale", [2.5, -2.5])
+def test_prefill_large_and_negative_scale(O, cuda_lib, scale):
+    """Scores with a standard deviation of ~40 in log2 units: the running max of a row climbs by more
+    than 2^8 several times along the history, so the kernel moves its reference and rescales O in TMEM.
+    A negative scale turns the tile max into the min of the raw scores."""
+    batch = make_batch("mixed_step", seed=54, overrides=_chunks(prefill_chunks=2, chunk_len=(200, 400),
+                                                                chunk_hist=(600, 1200)))
+    batch.scale = scale
+    ref = oracle_step(batch, O)
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    # Near one-hot rows make out ~ one V row (|v| up to ~4.5), so the bf16 roundings are not averaged
+    # away: P rounded to bf16 (relative 2^-9 per weight, weights summing to 1) moves out by at most
+    # 2^-9 max|v|, and the bf16 output by half an ulp, 2^-9 |out|.
+    vmax = float(batch.tok_v.float().abs().max())
+    for name in ("prefill", "decode"):
+        got = to_f64(st.out_pre if name == "prefill" else st.out_dec)
+        bound = 2.0 ** -9 * (vmax + float(np.abs(ref[name]).max())) + 1e-3
+        assert_close(got, ref[name], max_tol=bound, mean_tol=bound / 4, what=f"{name}, scale {scale}")
