@@ -190,6 +190,8 @@ pa_status pa_paged_attention_noalloc(void *out, const void *q, const void *k_cac
  *   cu_q_lens    : int32 [num_chunks + 1] on the device, non-decreasing, cu_q_lens[0] = 0
  *   block_tables : int32 [num_chunks][max_blocks_per_seq];  context_lens : int32 [num_chunks]
  *   max_q_len    : host-side upper bound of C_c;  max_context_len : upper bound of context_lens.
+ * A chunk whose C_c exceeds max_q_len, or whose context exceeds max_context_len or its table row,
+ * sets the device error word (PA_EDEVICE_OOB from pa_get_device_error) and its rows are not written.
  * bf16 caches only (kv_dtype must be PA_KV_BF16).  Runs on the tcgen05 tensor cores.
  */
 pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks,

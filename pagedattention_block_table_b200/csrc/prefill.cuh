@@ -31,7 +31,7 @@
 #include "pa_common.cuh"
 
 #ifndef PA_PREFILL_SPLIT_REGS
-#define PA_PREFILL_SPLIT_REGS 0
+#define PA_PREFILL_SPLIT_REGS 1
 #endif
 
 namespace pa {
@@ -214,8 +214,11 @@ struct PrefillParams {
   int group;            // Hq / Hkv
   int hpr;              // query heads stacked per position in a tile (G if 128 % G == 0, else 1)
   int max_context_len;
+  int num_chunks;
   float qscale;         // scale * log2(e)
 };
+
+constexpr int kOrderedChunks = 64;   // chunks the prefill grid orders by context length
 
 template <int D>
 struct PrefillCfg {
@@ -263,6 +266,18 @@ enum : int {
   kNumBars = kDone + 1
 };
 
+// Three-input max / min (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -278,14 +293,32 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.z;
-  const int hg0 = blockIdx.y * P.hpr;                 // first query head of this CTA's rows
+  const int hg0 = blockIdx.x * P.hpr;                 // first query head of this CTA's rows
   const int g = hg0 / P.group;                        // their KV head
   const int ppt = C::BM / P.hpr;                      // positions per query tile
   // any input may come from the kernel before this one on the stream (launched with PDL)
   griddep_wait();
   griddep_launch();
 
+  // Longest work first (CTAs are dispatched in index order): chunk rank blockIdx.z serves the chunk
+  // with the rank-th longest context (ties by index), and within a chunk blockIdx.y counts query
+  // tiles down from the last one, which sees the most keys.  Up to kOrderedChunks chunks; beyond
+  // that, blockIdx.z is the chunk.
+  int c = blockIdx.z;
+  if (P.num_chunks <= kOrderedChunks) {
+    int *s_chunk = reinterpret_cast<int *>(smem + C::OFF_BAR + C::NBAR * 8 + 8);
+    if (tid < P.num_chunks) {
+      const int mine = P.context_lens[tid];
+      int rank = 0;
+      for (int k = 0; k < P.num_chunks; ++k) {
+        const int other = P.context_lens[k];
+        rank += (other > mine || (other == mine && k < tid)) ? 1 : 0;
+      }
+      if (rank == static_cast<int>(blockIdx.z)) *s_chunk = tid;
+    }
+    __syncthreads();
+    c = *s_chunk;
+  }
   const int q0 = P.cu_q_lens[c];
   const int Cn = P.cu_q_lens[c + 1] - q0;
   const int ctx = P.context_lens[c];
@@ -294,8 +327,13 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) flag_error(kErrLength);
     return;
   }
-  const int p0 = blockIdx.x * 2 * ppt;               // first position of tile A
-  if (p0 >= Cn) return;
+  const int nx = (Cn + 2 * ppt - 1) / (2 * ppt);      // CTAs (pairs of query tiles) of this chunk
+  if (nx > static_cast<int>(gridDim.y)) {             // chunk longer than the max_q_len launched for
+    if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) flag_error(kErrLength);
+    return;
+  }
+  if (static_cast<int>(blockIdx.y) >= nx) return;
+  const int p0 = (nx - 1 - static_cast<int>(blockIdx.y)) * 2 * ppt;   // first position of tile A
   const int p_end = min(Cn, p0 + 2 * ppt);
   const int kv_len = H + p_end;                       // keys visible to some row of this CTA
   const int ntiles = (kv_len + C::BN - 1) / C::BN;
@@ -376,26 +414,30 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       float mt_ = -INFINITY;
       if (!diag) {
         // max of s * qscale: the max of s for a positive scale, the min for a negative one
-        float e0 = __uint_as_float(sr[0]), e1 = __uint_as_float(sr[1]), e2 = __uint_as_float(sr[2]),
-              e3 = __uint_as_float(sr[3]);
+        // (three-input max/min: two new keys per instruction, four independent chains)
+        const float s0 = __uint_as_float(sr[0]), s1 = __uint_as_float(sr[1]), s2 = __uint_as_float(sr[2]),
+                    s3 = __uint_as_float(sr[3]), s4 = __uint_as_float(sr[4]), s5 = __uint_as_float(sr[5]),
+                    s6 = __uint_as_float(sr[6]), s7 = __uint_as_float(sr[7]);
         if (qs >= 0.f) {
+          float e0 = fmaxf(s0, s1), e1 = fmaxf(s2, s3), e2 = fmaxf(s4, s5), e3 = fmaxf(s6, s7);
 #pragma unroll
-          for (int k = 4; k < C::BN; k += 4) {
-            e0 = fmaxf(e0, __uint_as_float(sr[k]));
-            e1 = fmaxf(e1, __uint_as_float(sr[k + 1]));
-            e2 = fmaxf(e2, __uint_as_float(sr[k + 2]));
-            e3 = fmaxf(e3, __uint_as_float(sr[k + 3]));
+          for (int k = 8; k < C::BN; k += 8) {
+            e0 = fmax3(e0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+            e1 = fmax3(e1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
+            e2 = fmax3(e2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
+            e3 = fmax3(e3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
           }
-          mt_ = fmaxf(fmaxf(e0, e1), fmaxf(e2, e3)) * qs;
+          mt_ = fmax3(fmaxf(e0, e1), e2, e3) * qs;
         } else {
+          float e0 = fminf(s0, s1), e1 = fminf(s2, s3), e2 = fminf(s4, s5), e3 = fminf(s6, s7);
 #pragma unroll
-          for (int k = 4; k < C::BN; k += 4) {
-            e0 = fminf(e0, __uint_as_float(sr[k]));
-            e1 = fminf(e1, __uint_as_float(sr[k + 1]));
-            e2 = fminf(e2, __uint_as_float(sr[k + 2]));
-            e3 = fminf(e3, __uint_as_float(sr[k + 3]));
+          for (int k = 8; k < C::BN; k += 8) {
+            e0 = fmin3(e0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+            e1 = fmin3(e1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
+            e2 = fmin3(e2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
+            e3 = fmin3(e3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
           }
-          mt_ = fminf(fminf(e0, e1), fminf(e2, e3)) * qs;
+          mt_ = fmin3(fminf(e0, e1), e2, e3) * qs;
         }
       } else {
 #pragma unroll
@@ -545,60 +587,60 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       if (!ok) timeout = true;
     }
   } else if (warp == 9) {
-    // ===================================================================== TMA producer
-    if (lane == 0) {
+    // ===================================================================== TMA producer (whole warp)
+    // One copy per lane: a key tile is UPT units x DH planes for K and as many for V (32 copies at
+    // head_dim 128), so lane l copies plane l % DH of unit (l / DH) % UPT of K (first half of the
+    // warp) or V (second half).  Each lane loads its unit's block-table entry two tiles ahead.
+    {
       const int32_t *trow = P.block_tables + (int64_t)c * P.max_blocks_per_seq;
       const int ush = P.block_size == 32 ? 1 : 0;   // log2(16-row units per physical block)
       constexpr int UPT = C::BN / kBlock;             // units per key tile
-      // cache-row index of each unit of key tile j: the table entries of a tile are loaded together,
-      // one tile ahead of the copies that use them
-      auto rows_of = [&](int j, int (&y)[UPT]) {
-#pragma unroll
-        for (int bb = 0; bb < UPT; ++bb) {
-          const int u = j * UPT + bb;
-          int e = 0;
-          if (u * kBlock < kv_len) {
-            e = __ldg(trow + (u >> ush));
-            if (e < 0 || e >= P.num_blocks) {
-              flag_error(kErrBlockId);
-              e = 0;
-            }
+      constexpr int PER = UPT * C::DH;                // copies per K or V tile
+      static_assert(2 * PER <= 32, "one copy per lane");
+      const int w_lane = lane / PER;                  // 0: K, 1: V, 2+: idle
+      const int bb = (lane / C::DH) % UPT;            // unit of the tile
+      const int hh = lane % C::DH;                    // 64-element plane
+      auto row_of = [&](int j) {                      // cache row of this lane's unit of key tile j
+        const int u = j * UPT + bb;
+        int e = 0;
+        if (w_lane < 2 && j < ntiles && u * kBlock < kv_len) {
+          e = __ldg(trow + (u >> ush));
+          if (e < 0 || e >= P.num_blocks) {
+            flag_error(kErrBlockId);
+            e = 0;
           }
-          y[bb] = (((e * P.num_kv_heads + g) << ush) + (u & ((1 << ush) - 1))) * kBlock;
         }
+        return (((e * P.num_kv_heads + g) << ush) + (u & ((1 << ush) - 1))) * kBlock;
       };
-      int ycur[UPT], ynext[UPT];
-      rows_of(0, ycur);
-      int i = 0;
-      for (int j = 0; j < ntiles; ++j) {
-        if (j + 1 < ntiles) rows_of(j + 1, ynext);
+      int y0 = row_of(0), y1 = row_of(1);
+      int issued = 0;                                 // ring items whose copies are in flight
+      for (int j = 0; j < ntiles && !timeout; ++j) {
+        const int y2 = row_of(j + 2);
         const int nu = min(UPT, (kv_len - j * C::BN + kBlock - 1) / kBlock);
-        for (int v = 0; v < 2; ++v, ++i) {
-          const int slot = i % C::NSLOT;
-          if (i >= C::NSLOT && !mbar_wait(&bars[kEmpty + slot], ((i / C::NSLOT) - 1) & 1)) {
+        for (int w = 0; w < 2; ++w) {                 // K, then V of tile j
+          const int it = 2 * j + w, slot = it % C::NSLOT;
+          int ok = 1;
+          if (lane == 0) {
+            if (it >= C::NSLOT) ok = mbar_wait(&bars[kEmpty + slot], ((it / C::NSLOT) - 1) & 1);
+            if (ok) mbar_arrive_expect_tx(&bars[kFull + slot], nu * C::DH * (kBlock * 128));
+          }
+          if (!__shfl_sync(0xffffffffu, ok, 0)) {
             timeout = true;
             break;
           }
-          mbar_arrive_expect_tx(&bars[kFull + slot], nu * C::DH * (kBlock * 128));
-          const CUtensorMap *map = v ? &vmap : &kmap;
-          uint8_t *dst = slot_of(i);
-#pragma unroll
-          for (int bb = 0; bb < UPT; ++bb) {
-            if (bb < nu) {
-#pragma unroll
-              for (int hh = 0; hh < C::DH; ++hh)
-                tma_load_2d(dst + hh * C::KV_PLANE + bb * (kBlock * 128), map, hh * 64, ycur[bb], &bars[kFull + slot]);
-            }
-          }
+          if (w_lane == w && bb < nu)
+            tma_load_2d(slot_of(it) + hh * C::KV_PLANE + bb * (kBlock * 128), w ? &vmap : &kmap, hh * 64, y0,
+                        &bars[kFull + slot]);
+          issued = it + 1;
         }
-        if (timeout) break;
-#pragma unroll
-        for (int bb = 0; bb < UPT; ++bb) ycur[bb] = ynext[bb];
+        y0 = y1;
+        y1 = y2;
       }
-      // before leaving, the last tiles this thread issued must have landed (a no-op when the MMA warp
+      // before leaving, the last tiles this warp issued must have landed (a no-op when the MMA warp
       // consumed them; bounded when a wait elsewhere gave up)
-      for (int k = max(0, i - C::NSLOT); k < i; ++k)
-        (void)mbar_wait(&bars[kFull + (k % C::NSLOT)], (k / C::NSLOT) & 1);
+      if (lane == 0)
+        for (int k = max(0, issued - C::NSLOT); k < issued; ++k)
+          (void)mbar_wait(&bars[kFull + (k % C::NSLOT)], (k / C::NSLOT) & 1);
     }
   }
   }
@@ -664,7 +706,9 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
     return -3;
 #endif
   const int ppt = C::BM / P.hpr;
-  dim3 grid((max_q_len + 2 * ppt - 1) / (2 * ppt), P.num_q_heads / P.hpr, num_chunks);
+  const int tiles = (max_q_len + 2 * ppt - 1) / (2 * ppt);
+  if (tiles > 65535) return -1;
+  dim3 grid(P.num_q_heads / P.hpr, tiles, num_chunks);
   return launch_pdl(paged_prefill_kernel<D>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;
 }
 
@@ -689,6 +733,7 @@ inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, in
   P.group = num_q_heads / num_kv_heads;
   P.hpr = (P.group <= 128 && 128 % P.group == 0) ? P.group : 1;
   P.max_context_len = max_context_len;
+  P.num_chunks = num_chunks;
   P.qscale = scale * 1.4426950408889634f;
   return head_dim == 128 ? launch_prefill_d<128>(P, k_cache, v_cache, num_chunks, max_q_len, st)
                          : launch_prefill_d<64>(P, k_cache, v_cache, num_chunks, max_q_len, st);

@@ -110,3 +110,18 @@ def test_prefill_large_and_negative_scale(O, cuda_lib, scale):
         got = to_f64(st.out_pre if name == "prefill" else st.out_dec)
         bound = 2.0 ** -9 * (vmax + float(np.abs(ref[name]).max())) + 1e-3
         assert_close(got, ref[name], max_tol=bound, mean_tol=bound / 4, what=f"{name}, scale {scale}")
+
+
+def test_prefill_chunk_longer_than_max_q_is_flagged(cuda_lib):
+    """A chunk longer than the max_q_len the call was given is reported, not silently cut short."""
+    from pagedattention_block_table_b200.runner import DeviceStep
+    batch = make_batch("mixed_step", seed=55, overrides=_chunks(prefill_chunks=2, chunk_len=(300, 300)))
+    st = DeviceStep(batch)
+    st.fill_history()
+    st.append()
+    torch.cuda.synchronize()
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    cuda_lib.pa_paged_prefill(st.out_pre, st.q_pre, st.cu_q, st.k_cache, st.v_cache, st.pre_tables, st.pre_lens,
+                              batch.scale, 100, st.pre_max_len)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_EDEVICE_OOB
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK          # reading the word clears it
