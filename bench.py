@@ -188,6 +188,17 @@ def combine_over_ranks(times_ms: dict, bytes_per_step: int, world: int, device) 
 
 # ----------------------------------------------------------------------------- our arm
 
+def workload_config(name, batch) -> dict:
+    """The workload's identifying sizes (the same keys on both arms)."""
+    return {
+        "workload": name,
+        "num_seqs": batch.num_decode, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
+        "head_dim": batch.head_dim, "block_size": batch.block_size, "num_blocks": batch.num_blocks,
+        "context_tokens": int(batch.context_lens[:batch.num_decode].sum()),
+        "prefill_chunks": int(batch.num_seqs - batch.num_decode), "cow_pairs": int(batch.cow_pairs.shape[0]),
+    }
+
+
 def run_ours(args, rank, world, local_rank):
     from pagedattention_block_table_b200 import binding as B
     from pagedattention_block_table_b200.inputs import make_batch
@@ -289,16 +300,13 @@ def run_ours(args, rank, world, local_rank):
                   2: "int8 KV, bf16 q/out, fp32 accumulate"}[batch.kv_dtype],
         "data": "synthetic",
         "config": {
-            "workload": args.workload,
-            "num_seqs": batch.num_decode, "num_q_heads": batch.num_q_heads, "num_kv_heads": batch.num_kv_heads,
-            "head_dim": batch.head_dim, "block_size": batch.block_size, "num_blocks": batch.num_blocks,
-            "context_tokens": int(batch.context_lens[:batch.num_decode].sum()),
-            "prefill_chunks": int(batch.num_seqs - batch.num_decode), "cow_pairs": int(batch.cow_pairs.shape[0]),
+            **workload_config(args.workload, batch),
             "split_tokens": st.split_tokens,
             "l2": "inputs larger than L2: KV pool %.2f GB vs 126 MB" % (2 * st.k_cache.numel() * st.k_cache.element_size() / 1e9),
             "parallelism": f"replicas x{world}",
         },
         "pct_of_peak": round(100 * value / world / peak, 2),
+        "pct_of_spec_8000_gbs": round(100 * value / world / 8000.0, 2),   # B200 HBM3e datasheet figure
         "seq_steps_per_s": round(world * batch.num_decode / (step_ms * 1e-3), 1),
         "decode_kv_bytes_per_step": kvb,
         "decode_kv_unique_bytes_per_step": kv_unique_bytes(batch),
@@ -419,7 +427,7 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(secs * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "sample_seqs": len(smp["lens"])},
+        "config": {**workload_config(args.workload, batch), "sample_seqs": len(smp["lens"])},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
                          "sample": f"append + decode of {len(smp['lens'])} of {batch.num_decode} sequences per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
