@@ -141,6 +141,12 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
  *   split_tokens : tokens per split-K partition (a multiple of 16); 0 = pa_paged_attention_auto_split.
  *                  When a sequence spans several splits each writes a partial (max, sum, unnormalised
  *                  output) to the workspace and a log-sum-exp reduce combines them.
+ *   host_context_lens : optional host copy of context_lens (int32 [num_seqs]), or NULL.  When given,
+ *                  the (sequence, split) work items are launched longest first (a counting sort on
+ *                  the host), so the launch ends on short items instead of idling on a long one.
+ *                  Every split up to max_context_len is launched whatever these values are: they
+ *                  decide only the order, never the result.  Up to 4000 (sequence, split) pairs;
+ *                  beyond that the natural order is used.
  *   workspace    : device scratch of at least pa_paged_attention_workspace_size(...) bytes, or NULL
  *                  when that is 0.  Its contents need no initialisation and are clobbered.
  */
@@ -149,7 +155,8 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
                              const int32_t *context_lens, int num_seqs, int num_q_heads,
                              int num_kv_heads, int head_dim, int64_t num_blocks, int block_size,
                              float scale, int kv_dtype, const float *k_scale, const float *v_scale,
-                             int max_context_len, int split_tokens, void *workspace,
+                             int max_context_len, int split_tokens,
+                             const int32_t *host_context_lens, void *workspace,
                              size_t workspace_bytes, pa_stream_t stream);
 
 /*

@@ -69,7 +69,7 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_attention_auto_split.restype = I
         L.pa_paged_attention_auto_split.argtypes = [I, I, I, I, I, I]
         L.pa_paged_attention.restype = I
-        L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, I, F, I, P, P, I, I, P, SZ, P]
+        L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, I, F, I, P, P, I, I, P, P, SZ, P]
         L.pa_paged_attention_noalloc.restype = I
         L.pa_paged_attention_noalloc.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P]
         L.pa_paged_prefill.restype = I
@@ -217,9 +217,25 @@ def pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                                    max_context_len, kv_dtype))
 
 
+def _host_i32(a, n):
+    """Host pointer of an int32 array of n elements (numpy or CPU tensor), or None."""
+    if a is None:
+        return None
+    if isinstance(a, torch.Tensor):
+        if a.device.type != "cpu" or a.dtype != torch.int32 or not a.is_contiguous() or a.numel() != n:
+            raise ValueError("host_context_lens must be a contiguous int32 CPU tensor of num_seqs elements")
+        return a.data_ptr()
+    import numpy as np
+    if not isinstance(a, np.ndarray) or a.dtype != np.int32 or not a.flags["C_CONTIGUOUS"] or a.size != n:
+        raise ValueError("host_context_lens must be a contiguous int32 array of num_seqs elements")
+    return a.ctypes.data
+
+
 def pa_paged_attention(out, q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                        kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, split_tokens=0, workspace=None,
-                       stream=None):
+                       stream=None, host_context_lens=None):
+    """host_context_lens: optional host copy of context_lens (int32 numpy array or CPU tensor); it only
+    orders the launch's work items longest first."""
     nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     b, hq, dq = q.shape
@@ -234,7 +250,7 @@ def pa_paged_attention(out, q, k_cache, v_cache, block_tables, context_lens, sca
         int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), b, hq, hkv, d, nb, bs,
         float(scale), int(kv_dtype), _ptr(k_scale, "k_scale", (torch.float32,)),
         _ptr(v_scale, "v_scale", (torch.float32,)), int(max_context_len), int(split_tokens),
-        _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
+        _host_i32(host_context_lens, b), _ptr(workspace, "workspace"), ws_bytes, _stream(stream))
     _check(st, "pa_paged_attention")
 
 

@@ -6,6 +6,7 @@
 #include <stdio.h>
 
 #include <atomic>
+#include <vector>
 
 #include "../../include/pagedattn.h"
 #include "decode.cuh"
@@ -92,20 +93,62 @@ int decode_smem_rt(int kt, int d, int qpb) {
   return 0;
 }
 
-template <int KT, int D, int QPB>
-pa_status launch_decode(const pa::DecodeParams &P, dim3 grid, cudaStream_t st) {
+template <int KT, int D, int QPB, bool ORDERED>
+pa_status launch_decode_as(const pa::DecodeParams &P, const pa::WorkOrder<ORDERED> &W, dim3 grid, cudaStream_t st) {
   constexpr int S = stages_for<KT, D, QPB>();
   using C = pa::DecodeCfg<KT, D, QPB, PA_DEC_NW, S>;
-  auto kern = pa::paged_decode_kernel<KT, D, QPB, PA_DEC_NW, S>;
+  auto kern = pa::paged_decode_kernel<KT, D, QPB, PA_DEC_NW, S, ORDERED>;
   pa_status s = set_smem(kern, C::SMEM);
   if (s != PA_OK) return s;
-  if (pa::launch_pdl(kern, grid, dim3(PA_DEC_NW * 32), C::SMEM, st, P) != cudaSuccess) return launch_status();
+  if (pa::launch_pdl(kern, grid, dim3(PA_DEC_NW * 32), C::SMEM, st, P, W) != cudaSuccess) return launch_status();
   return launch_status();
 }
 
-pa_status dispatch_decode(int kt, int d, int qpb, const pa::DecodeParams &P, dim3 grid, cudaStream_t st) {
+// order: null for the natural order over grid (units, sequences, splits); else the longest-first list
+// of (sequence, split) pairs with grid (units, its length)
+template <int KT, int D, int QPB>
+pa_status launch_decode(const pa::DecodeParams &P, const pa::WorkOrder<true> *order, int n_order, dim3 grid,
+                        cudaStream_t st) {
+  if (order) return launch_decode_as<KT, D, QPB, true>(P, *order, dim3(grid.x, n_order, 1), st);
+  return launch_decode_as<KT, D, QPB, false>(P, pa::WorkOrder<false>{}, grid, st);
+}
+
+// Longest-first list of every (sequence, split) pair of a launch, from the host's copy of the context
+// lengths: a counting sort on the tokens each pair holds (min(S, L - z*S), clamped to [0, S]), stable
+// in (split, sequence).  Every pair z < max_splits is listed whatever the host lengths say, so the
+// result never depends on them, only the order does.  Returns the number of pairs, or 0 (natural
+// order) when they do not fit the kernel-parameter list or all lengths are equal.
+int build_work_order(const int32_t *host_lens, int num_seqs, int S, int max_context_len, int max_splits,
+                     int32_t *item) {
+  const int64_t n = (int64_t)num_seqs * max_splits;
+  if (n <= 1 || n > pa::kOrderedItems || S <= 0) return 0;
+  bool uniform = true;   // equal lengths: the sorted list is the natural order, so launch without one
+  for (int b = 1; b < num_seqs && uniform; ++b) uniform = host_lens[b] == host_lens[0];
+  if (uniform) return 0;
+  std::vector<int> count(S + 2, 0);
+  auto tokens = [&](int b, int z) {
+    int L = host_lens[b];
+    L = L < 0 ? 0 : (L > max_context_len ? max_context_len : L);
+    const int64_t t = (int64_t)L - (int64_t)z * S;
+    return static_cast<int>(t < 0 ? 0 : (t > S ? S : t));
+  };
+  for (int z = 0; z < max_splits; ++z)
+    for (int b = 0; b < num_seqs; ++b) ++count[S - tokens(b, z)];   // bucket 0 holds the longest
+  int run = 0;
+  for (int k = 0; k <= S; ++k) {
+    const int c = count[k];
+    count[k] = run;
+    run += c;
+  }
+  for (int z = 0; z < max_splits; ++z)
+    for (int b = 0; b < num_seqs; ++b) item[count[S - tokens(b, z)]++] = (z << 16) | b;
+  return static_cast<int>(n);
+}
+
+pa_status dispatch_decode(int kt, int d, int qpb, const pa::DecodeParams &P, const pa::WorkOrder<true> *order,
+                          int n_order, dim3 grid, cudaStream_t st) {
 #define PA_DD(KT, D, Q) \
-  if (kt == KT && d == D && qpb == Q) return launch_decode<KT, D, Q>(P, grid, st);
+  if (kt == KT && d == D && qpb == Q) return launch_decode<KT, D, Q>(P, order, n_order, grid, st);
   PA_DD(0, 64, 1) PA_DD(0, 64, 2) PA_DD(0, 64, 4) PA_DD(0, 128, 1) PA_DD(0, 128, 2) PA_DD(0, 128, 4)
   PA_DD(1, 64, 1) PA_DD(1, 64, 2) PA_DD(1, 64, 4) PA_DD(1, 128, 1) PA_DD(1, 128, 2) PA_DD(1, 128, 4)
   PA_DD(2, 64, 1) PA_DD(2, 64, 2) PA_DD(2, 64, 4) PA_DD(2, 128, 1) PA_DD(2, 128, 2) PA_DD(2, 128, 4)
@@ -286,8 +329,8 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
                              const int32_t *block_tables, int max_blocks_per_seq, const int32_t *context_lens,
                              int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int64_t num_blocks,
                              int block_size, float scale, int kv_dtype, const float *k_scale, const float *v_scale,
-                             int max_context_len, int split_tokens, void *workspace, size_t workspace_bytes,
-                             pa_stream_t stream) {
+                             int max_context_len, int split_tokens, const int32_t *host_context_lens,
+                             void *workspace, size_t workspace_bytes, pa_stream_t stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
     return PA_EINVAL;
   if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
@@ -341,7 +384,12 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   dim3 grid(static_cast<unsigned>(num_kv_heads * (group / qpb)), static_cast<unsigned>(num_seqs),
             static_cast<unsigned>(max_splits));
-  pa_status s = dispatch_decode(kv_dtype, head_dim, qpb, P, grid, st);
+  // longest-first order of the (sequence, split) pairs when the caller also has the lengths on the host
+  static thread_local pa::WorkOrder<true> order;
+  const int n_order = host_context_lens ? build_work_order(host_context_lens, num_seqs, S, max_context_len,
+                                                           static_cast<int>(max_splits), order.item)
+                                        : 0;
+  pa_status s = dispatch_decode(kv_dtype, head_dim, qpb, P, n_order ? &order : nullptr, n_order, grid, st);
   if (s != PA_OK || max_splits <= 1) return s;
   dim3 rgrid(static_cast<unsigned>((num_q_heads + 3) / 4), static_cast<unsigned>(num_seqs));
   if (head_dim == 128)
@@ -429,5 +477,5 @@ extern "C" pa_status pa_paged_attention_noalloc(void *out, const void *q, const 
   }
   return pa_paged_attention(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                             num_q_heads, num_kv_heads, head_dim, num_blocks, PA_BLOCK_SIZE, scale, kv_dtype, k_scale,
-                            v_scale, max_context_len, S, ws, ws ? cap : 0, stream);
+                            v_scale, max_context_len, S, nullptr, ws, ws ? cap : 0, stream);
 }

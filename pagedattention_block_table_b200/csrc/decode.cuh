@@ -109,16 +109,28 @@ __device__ __forceinline__ int group_reduce_qsel(int lane) {
   return qb;
 }
 
-template <int KT, int D, int QPB, int NW, int STAGES>
-__global__ void __launch_bounds__(NW * 32) paged_decode_kernel(const DecodeParams P) {
+// Work order of an ordered launch: row y of the grid (units, count) serves the (sequence, split) pair
+// item[y] = split << 16 | sequence.  The host lists every pair, longest first, so the launch ends on
+// the short ones; CTAs are dispatched in index order.  Passed as a kernel parameter (read from the
+// constant bank, no extra memory round trip before a CTA can start).
+constexpr int kOrderedItems = 4000;
+template <bool ORDERED>
+struct WorkOrder {
+  int32_t item[ORDERED ? kOrderedItems : 1];   // a natural-order launch carries no list
+};
+
+template <int KT, int D, int QPB, int NW, int STAGES, bool ORDERED>
+__global__ void __launch_bounds__(NW * 32)
+    paged_decode_kernel(const DecodeParams P, const __grid_constant__ WorkOrder<ORDERED> W) {
   using C = DecodeCfg<KT, D, QPB, NW, STAGES>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // grid (heads, sequences, splits): every sequence's first split is scheduled before any second
-  // one, so the CTAs that find their split past a short sequence's end cluster in the last waves
-  const int split = blockIdx.z;
+  // natural order, grid (units, sequences, splits): every sequence's first split is scheduled before
+  // any second one, so the CTAs that find their split past a short sequence's end cluster in the last
+  // waves.  Ordered launch, grid (units, count): see WorkOrder.
+  const int split = ORDERED ? (W.item[blockIdx.y] >> 16) : static_cast<int>(blockIdx.z);
   const int unit = blockIdx.x;
-  const int b = blockIdx.y;
+  const int b = ORDERED ? (W.item[blockIdx.y] & 0xffff) : static_cast<int>(blockIdx.y);
   const int sub_groups = P.group / QPB;
   const int g = unit / sub_groups;
   const int h0 = g * P.group + (unit % sub_groups) * QPB;  // first query head of this CTA

@@ -39,7 +39,8 @@ class DeviceStep:
         nd = batch.num_decode
         ctx = batch.context_lens
         self.dec_tables = torch.from_numpy(batch.decode_tables).to(dev)
-        self.dec_lens = torch.from_numpy(np.ascontiguousarray(ctx[:nd])).to(dev)
+        self.dec_lens_host = np.ascontiguousarray(ctx[:nd], dtype=np.int32)   # orders the decode launch
+        self.dec_lens = torch.from_numpy(self.dec_lens_host).to(dev)
         self.dec_max_len = int(ctx[:nd].max()) if nd else 0
         self.pre_tables = torch.from_numpy(batch.prefill_tables).to(dev)
         self.pre_lens = torch.from_numpy(np.ascontiguousarray(ctx[nd:])).to(dev)
@@ -92,7 +93,8 @@ class DeviceStep:
             return
         B.pa_paged_attention(self.out_dec, self.q_dec, self.k_cache, self.v_cache, self.dec_tables, self.dec_lens,
                              self.batch.scale, self.dec_max_len, self.kv_dtype, self.k_scale, self.v_scale,
-                             self.split_tokens if split_tokens is None else split_tokens, self.workspace, stream)
+                             self.split_tokens if split_tokens is None else split_tokens, self.workspace, stream,
+                             host_context_lens=self.dec_lens_host)
 
     def prefill(self, stream=None):
         if self.max_q == 0:

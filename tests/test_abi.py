@@ -70,7 +70,7 @@ def _raw_attention(L, **kw):
     return L.pa_paged_attention(P(args["out"]), P(args["q"]), P(args["k"]), P(args["v"]), P(args["bt"]), args["mbs"],
                                 P(args["cl"]), args["ns"], args["hq"], args["hkv"], args["d"], args["nb"],
                                 args["bs"], args["scale"], args["dt"], P(args["ks"]) if args["ks"] else None,
-                                P(args["vs"]) if args["vs"] else None, args["maxl"], args["split"],
+                                P(args["vs"]) if args["vs"] else None, args["maxl"], args["split"], None,
                                 P(args["ws"]) if args["ws"] else None, args["wsb"], None)
 
 

@@ -193,3 +193,32 @@ def test_host_pipeline_delivers_the_step_outputs(cuda_lib):
     for s in range(2):
         assert torch.equal(pipe.host_out[s][0], ref.out_dec.cpu())
         assert torch.equal(pipe.host_out[s][1], ref.out_pre.cpu())
+
+
+@pytest.mark.parametrize("split", [64, 256])
+def test_longest_first_order_changes_nothing_but_the_order(O, cuda_lib, split):
+    """The host copy of the context lengths only orders the launch (longest (sequence, split) first):
+    natural order, the true lengths and deliberately wrong ones all give bit-identical outputs, and
+    they match the oracle."""
+    from pagedattention_block_table_b200 import binding as B
+    batch = make_batch("llama3_8b_decode", seed=61, overrides=dict(num_seqs=9, hist=("uniform", 0, 1500)))
+    st = _gpu_decode(batch, split)
+    ref = oracle_step(batch, O)["decode"]
+    outs = {}
+    true_lens = st.dec_lens_host
+    for name, host in (("natural", None), ("true", true_lens), ("reversed", np.ascontiguousarray(true_lens[::-1])),
+                       ("zeros", np.zeros_like(true_lens)), ("huge", np.full_like(true_lens, 1 << 30)),
+                       ("cpu tensor", torch.from_numpy(true_lens.copy()))):
+        out = torch.full_like(st.out_dec, float("nan"))
+        B.pa_paged_attention(out, st.q_dec, st.k_cache, st.v_cache, st.dec_tables, st.dec_lens, batch.scale,
+                             st.dec_max_len, split_tokens=split, workspace=st.workspace, host_context_lens=host)
+        torch.cuda.synchronize()
+        outs[name] = out
+    assert B.pa_get_device_error() == B.PA_OK
+    for name, out in outs.items():
+        assert torch.equal(out, outs["natural"]), name
+    assert_close(to_f64(outs["true"]), ref, what=f"ordered launch, split {split}")
+    with pytest.raises(ValueError):
+        B.pa_paged_attention(st.out_dec, st.q_dec, st.k_cache, st.v_cache, st.dec_tables, st.dec_lens, batch.scale,
+                             st.dec_max_len, split_tokens=split, workspace=st.workspace,
+                             host_context_lens=true_lens[:-1])
