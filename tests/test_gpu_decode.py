@@ -222,3 +222,20 @@ def test_longest_first_order_changes_nothing_but_the_order(O, cuda_lib, split):
         B.pa_paged_attention(st.out_dec, st.q_dec, st.k_cache, st.v_cache, st.dec_tables, st.dec_lens, batch.scale,
                              st.dec_max_len, split_tokens=split, workspace=st.workspace,
                              host_context_lens=true_lens[:-1])
+
+
+def test_many_splits_and_a_reused_workspace(O, cuda_lib):
+    """79 and 313 splits of one sequence (the reduce kernel loops over more than 32 partials per lane
+    group), a second call on the same workspace, and sampled rows against the oracle."""
+    from pagedattention_block_table_b200 import binding as B
+    batch = make_batch("llama3_8b_decode", seed=62, overrides=dict(num_seqs=3, hist=("fixed", [20000, 7000, 300])))
+    for split in (256, 64):
+        st = _gpu_decode(batch, split)
+        first = st.out_dec.clone()
+        st.decode()
+        torch.cuda.synchronize()
+        assert torch.equal(st.out_dec, first), f"second call on the same workspace, split {split}"
+        got = to_f64(st.out_dec)
+        for s in range(3):
+            assert_close(got[s], oracle_decode_one(batch, s, O), what=f"seq {s}, split {split}")
+    assert B.pa_get_device_error() == B.PA_OK
