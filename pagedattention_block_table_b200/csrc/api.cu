@@ -306,13 +306,12 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 8) per_sm = 8;
   const int64_t slots = (int64_t)device_sm_count() * per_sm;
-  // Splits of at most 1024 tokens, shortened (powers of two, down to 256) until there are ~4 waves
-  // of work units.  Measured on B200 (pa_paged_attention GB/s by split length): Llama-3-8B decode
-  // batch 512: 5414, 1024: 5373, 2048: 4674, none: 4136; long context (8 x 32768) 512: 5462,
-  // 1024: 5720, 2048: 5520; mixed step 512: 5518, 1024: 5871, 8192: 4663; FP8 MHA 1024: 4774,
-  // 2048: 4768, 8192: 4424.
+  // Splits of at most 2048 tokens, shortened (powers of two, down to 256) until there are ~4 waves
+  // of work units.  Measured on B200 (pa_paged_attention GB/s by split length, longest-first launch
+  // order): Llama-3-8B decode batch 512: 5182, 1024: 5461, 2048: 5018 (the wave rule picks 1024);
+  // mixed step 512: 5264, 1024: 5807, 2048: 6035; FP8 MHA 512: 4544, 1024: 4736, 2048: 4839.
   int64_t S = 256;
-  while (S < max_context_len && S < 1024) S *= 2;
+  while (S < max_context_len && S < 2048) S *= 2;
   while (S > 256 && units * ceil_div64(max_context_len, S) < 4 * slots) S /= 2;
   return static_cast<int>(S);
 }
