@@ -228,13 +228,36 @@ def run_ours(args, rank, world, local_rank):
     d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     p1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    # The step value replays the K steps from CUDA graphs of G steps each, so that the Python launch path
+    # (ctypes marshalling, the GIL shared with the clock sampler) cannot leave gaps between kernels.  The
+    # graph holds the same launches as st.step(), with their programmatic (PDL) dependencies.
+    G = next(g for g in (10, 8, 5, 4, 2, 1) if K % g == 0) if not args.no_graph else 0
+    graph = None
+    if G:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev)):
+                for _ in range(G):
+                    st.step()
+            torch.cuda.synchronize(dev)
+            for _ in range(2):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+        except RuntimeError as e:            # capture refused: time stream launches instead, and say so
+            print(f"bench: CUDA graph capture failed ({e}); timing stream launches", file=sys.stderr)
+            graph, G = None, 0
+            torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clk:
         # the step value: K steps back to back, no event between the kernels (an event record between
         # two launches ends the programmatic overlap of the second with the first)
         torch.cuda.synchronize(dev)
         ev0.record(stream)
-        for i in range(K):
-            st.step()
+        if graph is not None:
+            for _ in range(K // G):
+                graph.replay()
+        else:
+            for i in range(K):
+                st.step()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
         # the same K steps again with events around each attention call: the kernels' own durations
@@ -302,6 +325,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {
             **workload_config(args.workload, batch),
             "split_tokens": st.split_tokens,
+            "launch": f"CUDA graph of {G} steps, replayed" if G else "stream launches",
             "l2": "inputs larger than L2: KV pool %.2f GB vs 126 MB" % (2 * st.k_cache.numel() * st.k_cache.element_size() / 1e9),
             "parallelism": f"replicas x{world}",
         },
@@ -491,6 +515,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--split", type=int, default=0, help="split_tokens (0 = library default)")
+    ap.add_argument("--no-graph", action="store_true", help="time the steps as stream launches, not graph replays")
     ap.add_argument("--cpu-sample-seqs", type=int, default=16)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     ap.add_argument("--ref-max-steps", type=int, default=20)
