@@ -442,6 +442,8 @@ __global__ void __launch_bounds__(NW * 32)
 // One warp per (sequence, query head): lane p holds split p's (m, l) so the max and the weights come
 // from one round of independent loads and shuffles; then every lane sums its D/32 output dims over
 // the splits with independent vector loads.
+constexpr int kReduceFast = 8;   // splits up to which the reduce issues all its loads at once
+
 template <int D>
 __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
   const int h = blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -461,36 +463,72 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeParams P) {
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
   float den = 0.f;
-  // global max over all splits first (n may exceed 32)
-  float M = -INFINITY;
-  for (int p = lane; p < n; p += 32) M = fmaxf(M, P.ws_ml[(row0 + p) * 2]);
+  if (n <= kReduceFast) {
+    // up to kReduceFast splits: every load is issued before any result is used (one memory round trip)
+    const float m_l = lane < n ? P.ws_ml[(row0 + lane) * 2] : -INFINITY;
+    const float l_l = lane < n ? P.ws_ml[(row0 + lane) * 2 + 1] : 0.f;
+    float ov[kReduceFast][DPL];
 #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  for (int p0 = 0; p0 < n; p0 += 32) {
-    const int p = p0 + lane;
-    float w = 0.f, lw = 0.f;
-    if (p < n && M != -INFINITY) {
-      w = exp2f(P.ws_ml[(row0 + p) * 2] - M);
-      lw = w * P.ws_ml[(row0 + p) * 2 + 1];
+    for (int k = 0; k < kReduceFast; ++k) {
+      if (k < n) {
+        const float *op = P.ws_o + (row0 + k) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(op);
+          ov[k][0] = v.x; ov[k][1] = v.y; ov[k][2] = v.z; ov[k][3] = v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(op);
+          ov[k][0] = v.x; ov[k][1] = v.y;
+        }
+      }
     }
+    float M = m_l;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float w = (lane < n && M != -INFINITY) ? exp2f(m_l - M) : 0.f;
+    float lw = w * l_l;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
-    den += lw;
-    const int cnt = min(32, n - p0);
-#pragma unroll 4
-    for (int k = 0; k < cnt; ++k) {
+    den = lw;
+#pragma unroll
+    for (int k = 0; k < kReduceFast; ++k) {
       const float wk = __shfl_sync(0xffffffffu, w, k);
-      const float *op = P.ws_o + (row0 + p0 + k) * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(op);
-        acc[0] = fmaf(wk, v.x, acc[0]);
-        acc[1] = fmaf(wk, v.y, acc[1]);
-        acc[2] = fmaf(wk, v.z, acc[2]);
-        acc[3] = fmaf(wk, v.w, acc[3]);
-      } else {
-        const float2 v = *reinterpret_cast<const float2 *>(op);
-        acc[0] = fmaf(wk, v.x, acc[0]);
-        acc[1] = fmaf(wk, v.y, acc[1]);
+      if (k < n) {
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wk, ov[k][e], acc[e]);
+      }
+    }
+  } else {
+    // global max over all splits first (n may exceed 32)
+    float M = -INFINITY;
+    for (int p = lane; p < n; p += 32) M = fmaxf(M, P.ws_ml[(row0 + p) * 2]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    for (int p0 = 0; p0 < n; p0 += 32) {
+      const int p = p0 + lane;
+      float w = 0.f, lw = 0.f;
+      if (p < n && M != -INFINITY) {
+        w = exp2f(P.ws_ml[(row0 + p) * 2] - M);
+        lw = w * P.ws_ml[(row0 + p) * 2 + 1];
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, off);
+      den += lw;
+      const int cnt = min(32, n - p0);
+#pragma unroll 4
+      for (int k = 0; k < cnt; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, w, k);
+        const float *op = P.ws_o + (row0 + p0 + k) * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 v = *reinterpret_cast<const float4 *>(op);
+          acc[0] = fmaf(wk, v.x, acc[0]);
+          acc[1] = fmaf(wk, v.y, acc[1]);
+          acc[2] = fmaf(wk, v.z, acc[2]);
+          acc[3] = fmaf(wk, v.w, acc[3]);
+        } else {
+          const float2 v = *reinterpret_cast<const float2 *>(op);
+          acc[0] = fmaf(wk, v.x, acc[0]);
+          acc[1] = fmaf(wk, v.y, acc[1]);
+        }
       }
     }
   }
