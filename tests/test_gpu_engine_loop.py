@@ -118,3 +118,29 @@ def test_block_manager_drives_append_prefill_decode(O, cuda_lib):
         assert B.pa_get_device_error() == B.PA_OK
     finally:
         B.pa_bm_destroy(bm)
+
+
+def test_cuda_graph_replay_matches_eager(cuda_lib):
+    """A serving step captured in a CUDA graph (the library's launches keep their programmatic
+    dependencies inside the graph) and replayed gives bit-identical outputs to the eager step.
+    The step is the mixed one without forks, so that repeating it is idempotent."""
+    from pagedattention_block_table_b200.inputs import make_batch
+    from pagedattention_block_table_b200.runner import DeviceStep
+    small = dict(num_seqs=6, hist=("uniform", 100, 2500), share_group=0, share_prefix=0, num_q_heads=8,
+                 num_kv_heads=2, head_dim=128, prefill_chunks=2, chunk_len=(40, 300), chunk_hist=(1, 600))
+    st = DeviceStep(make_batch("mixed_step", seed=81, overrides=small), split_tokens=256)
+    st.fill_history()
+    st.step()
+    torch.cuda.synchronize()
+    eager_dec, eager_pre = st.out_dec.clone(), st.out_pre.clone()
+    st.out_dec.zero_()
+    st.out_pre.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=torch.cuda.Stream()):
+        st.step()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert torch.equal(st.out_dec, eager_dec)
+    assert torch.equal(st.out_pre, eager_pre)
