@@ -258,6 +258,15 @@ pa_status pa_bm_stats(const pa_block_manager *bm, int64_t *tokens_stored, int64_
  */
 pa_status pa_get_device_error(pa_stream_t stream);
 
+/*
+ * pa_selftest_bounded_wait -- launch one thread on `stream` that waits on an mbarrier nothing ever
+ * completes.  Every wait in this library's kernels is bounded: after 0.2 s the wait gives up, sets the
+ * device error word (read by pa_get_device_error as PA_EDEVICE_OOB) and the kernel returns, so the
+ * context stays usable.  This call exists to show that on a device (the tests use it); it launches
+ * nothing else and touches no caller memory.
+ */
+pa_status pa_selftest_bounded_wait(pa_stream_t stream);
+
 /* pa_status_string -- static text for a status code. */
 const char *pa_status_string(pa_status status);
 

@@ -35,7 +35,7 @@ EXPORTED = (
     "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
     "pa_paged_attention_noalloc", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
-    "pa_bm_length", "pa_bm_tables", "pa_bm_stats",
+    "pa_bm_length", "pa_bm_tables", "pa_bm_stats", "pa_selftest_bounded_wait",
 )
 PA_ENOMEM = -6
 
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, I, F, I, I, I, P]
         L.pa_get_device_error.restype = I
         L.pa_get_device_error.argtypes = [P]
+        L.pa_selftest_bounded_wait.restype = I
+        L.pa_selftest_bounded_wait.argtypes = [P]
         L.pa_status_string.restype = ctypes.c_char_p
         L.pa_status_string.argtypes = [I]
         L.pa_kv_cache_bytes.restype = I64
@@ -293,6 +295,11 @@ def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_
         int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), hq, hkv, d, nb, bs,
         float(scale), int(kv_dtype), int(max_q_len), int(max_context_len), _stream(stream))
     _check(st, "pa_paged_prefill")
+
+
+def pa_selftest_bounded_wait(stream=None):
+    """Launch the library's never-completing bounded wait (it gives up after 0.2 s and sets the error word)."""
+    _check(lib().pa_selftest_bounded_wait(_stream(stream)), "pa_selftest_bounded_wait")
 
 
 def pa_get_device_error(stream=None) -> int:

@@ -183,6 +183,11 @@ int64_t pa_kv_cache_bytes(int64_t layers, int64_t kv_heads, int64_t head_dim, in
   return 2 * layers * kv_heads * head_dim * seq_len * batch * elem_bytes;
 }
 
+pa_status pa_selftest_bounded_wait(pa_stream_t stream) {
+  pa::bounded_wait_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>();
+  return launch_status();
+}
+
 pa_status pa_get_device_error(pa_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return launch_status();
   unsigned v = 0;

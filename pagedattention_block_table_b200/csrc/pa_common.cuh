@@ -86,6 +86,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   return false;
 }
 
+// One thread waits on a barrier that nothing will ever complete: the bounded wait above must give up,
+// flag kErrTimeout and return (pa_selftest_bounded_wait).
+__global__ void bounded_wait_selftest_kernel() {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  (void)mbar_wait(&bar, 0);
+}
+
 // ----------------------------------------------------------------------------- bulk copies
 // L2 policy: streamed once, evict first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
