@@ -236,7 +236,8 @@ def run_ours(args, rank, world, local_rank):
     if G:
         try:
             graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev)):
+            # thread_local: the capture rules apply to this thread only, not to NCCL's helper threads
+            with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev), capture_error_mode="thread_local"):
                 for _ in range(G):
                     st.step()
             torch.cuda.synchronize(dev)
