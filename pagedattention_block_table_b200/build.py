@@ -24,10 +24,11 @@ def _sources():
 
 
 def source_digest() -> str:
-    """sha256 of the library's sources: identifies which kernels a profile was taken on."""
+    """sha256 of the CUDA sources (the kernels and their launch code, csrc/*.cu and *.cuh): identifies
+    which kernels a profile was taken on.  Host-only C++ (the block manager) does not enter it."""
     import hashlib
     h = hashlib.sha256()
-    for src in _sources():
+    for src in sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
         with open(src, "rb") as f:
             h.update(os.path.basename(src).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
