@@ -227,6 +227,20 @@ void pa_bm_destroy(pa_block_manager *bm);
 int64_t pa_bm_num_free(const pa_block_manager *bm);
 /* pa_bm_add -- register an empty sequence.  PA_EINVAL if the id exists. */
 pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id);
+/*
+ * pa_bm_add_prompt -- register a new sequence with a prompt of n_tokens token ids, sharing the blocks of
+ * any earlier prompt that starts alike [vLLM overview, Prefix Sharing].  The prompt's full 16-token
+ * blocks form a prefix tree keyed by (previous block, token ids); the longest chain of blocks that
+ * exactly match a live node is shared (reference counts + 1), and *reused_out is its length in tokens
+ * (a multiple of 16).  The remaining n_tokens - *reused_out tokens get slots in new blocks, written to
+ * slots_out[0 ..] in order: only those need their K/V appended; the shared ones are already in the
+ * cache.  The prompt's own full blocks join the tree.  A node lives while some sequence holds its block.
+ * PA_EINVAL if the id exists; PA_ENOMEM (nothing changed) if the pool is short.
+ */
+pa_status pa_bm_add_prompt(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens, int64_t n_tokens,
+                           int64_t *slots_out, int64_t *reused_out);
+/* pa_bm_prefix_stats -- blocks currently in the prefix tree, and prompt tokens served from it so far. */
+pa_status pa_bm_prefix_stats(const pa_block_manager *bm, int64_t *cached_blocks, int64_t *tokens_reused);
 /* pa_bm_fork -- child shares every block of parent (reference counts + 1), same length. */
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent, int64_t child);
 /*

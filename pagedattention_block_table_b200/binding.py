@@ -35,7 +35,8 @@ EXPORTED = (
     "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
     "pa_paged_attention_noalloc", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
-    "pa_bm_length", "pa_bm_tables", "pa_bm_stats", "pa_selftest_bounded_wait",
+    "pa_bm_length", "pa_bm_tables", "pa_bm_stats", "pa_selftest_bounded_wait", "pa_bm_add_prompt",
+    "pa_bm_prefix_stats",
 )
 PA_ENOMEM = -6
 
@@ -105,6 +106,10 @@ def lib() -> ctypes.CDLL:
         L.pa_bm_tables.argtypes = [P, P, ctypes.c_int32, P, ctypes.c_int32, P]
         L.pa_bm_stats.restype = I
         L.pa_bm_stats.argtypes = [P, P, P, P, P]
+        L.pa_bm_add_prompt.restype = I
+        L.pa_bm_add_prompt.argtypes = [P, I64, P, I64, P, P]
+        L.pa_bm_prefix_stats.restype = I
+        L.pa_bm_prefix_stats.argtypes = [P, P, P]
         _lib = L
     return _lib
 
@@ -327,6 +332,25 @@ def pa_bm_num_free(bm) -> int:
 
 def pa_bm_add(bm, seq_id: int):
     _check(lib().pa_bm_add(bm, int(seq_id)), "pa_bm_add")
+
+
+def pa_bm_add_prompt(bm, seq_id: int, tokens):
+    """Register a sequence with a prompt of token ids, sharing the blocks of earlier prompts that start
+    alike.  Returns (slots int64 array of the tokens not shared, number of shared tokens)."""
+    import numpy as np
+    toks = np.ascontiguousarray(tokens, np.int32)
+    slots = np.zeros(max(1, toks.shape[0]), np.int64)
+    reused = ctypes.c_int64(0)
+    st = lib().pa_bm_add_prompt(bm, int(seq_id), toks.ctypes.data_as(ctypes.c_void_p), int(toks.shape[0]),
+                                slots.ctypes.data_as(ctypes.c_void_p), ctypes.byref(reused))
+    _check(st, "pa_bm_add_prompt")
+    return slots[:toks.shape[0] - reused.value], int(reused.value)
+
+
+def pa_bm_prefix_stats(bm) -> dict:
+    v = [ctypes.c_int64(0) for _ in range(2)]
+    _check(lib().pa_bm_prefix_stats(bm, *[ctypes.byref(x) for x in v]), "pa_bm_prefix_stats")
+    return dict(cached_blocks=v[0].value, tokens_reused=v[1].value)
 
 
 def pa_bm_fork(bm, parent: int, child: int):

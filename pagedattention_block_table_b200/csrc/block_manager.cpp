@@ -16,6 +16,13 @@
 // Structure: a free list (FIFO; optionally shuffled once with a seeded generator, so that physical
 // placement is scattered as in a long-running server), a reference count per block, and per
 // sequence its block table and length.  All functions are O(blocks touched).
+//
+// Prefix tree (vLLM overview, "Prefix Sharing": requests whose prompts start alike share the pages of
+// the common part).  Every full block a prompt fills is a node keyed by (parent node, its 16 token ids);
+// a new prompt walks the tree block by block and shares every node it matches exactly, so only its
+// remaining tokens need K/V written.  Nodes are looked up through a hash of the whole prefix and then
+// compared exactly (parent block and token ids), so a hash collision can never share a wrong block.  A
+// node lives while some sequence holds its block; when the block returns to the pool the node goes.
 #include <stdint.h>
 #include <string.h>
 
@@ -34,6 +41,28 @@ struct Seq {
   int64_t len = 0;              // tokens written
 };
 
+// A full prompt block in the prefix tree.
+struct PrefixNode {
+  bool live = false;
+  int32_t parent = -1;            // block of the previous 16 tokens (-1: the prompt's first block)
+  uint64_t key = 0;               // hash of the whole prefix up to and including this block
+  int32_t tokens[PA_BLOCK_SIZE];  // the block's token ids, compared exactly on every match
+};
+
+uint64_t prefix_key(uint64_t parent_key, const int32_t *tokens) {
+  // FNV-1a over the parent's key and the 16 token ids, then a splitmix64 finaliser
+  uint64_t h = 1469598103934665603ull ^ parent_key;
+  for (int i = 0; i < PA_BLOCK_SIZE; ++i) {
+    h ^= static_cast<uint32_t>(tokens[i]);
+    h *= 1099511628211ull;
+  }
+  h ^= h >> 30;
+  h *= 0xbf58476d1ce4e5b9ull;
+  h ^= h >> 27;
+  h *= 0x94d049bb133111ebull;
+  return h ^ (h >> 31);
+}
+
 }  // namespace
 
 struct pa_block_manager {
@@ -42,9 +71,35 @@ struct pa_block_manager {
   std::vector<int32_t> refcount;
   std::unordered_map<int64_t, Seq> seqs;
   int64_t forks = 0;  // copy-on-write copies handed out so far
+  // prefix tree: key -> blocks whose prefix hashes to it (exact match decides), node per block
+  std::unordered_multimap<uint64_t, int32_t> prefix_index;
+  std::vector<PrefixNode> nodes;
+  int64_t prefix_tokens_reused = 0;
 };
 
 namespace {
+
+// the live node for (parent block, 16 tokens), or -1
+int32_t prefix_find(const pa_block_manager *bm, int32_t parent, uint64_t key, const int32_t *tokens) {
+  auto range = bm->prefix_index.equal_range(key);
+  for (auto it = range.first; it != range.second; ++it) {
+    const PrefixNode &nd = bm->nodes[it->second];
+    if (nd.live && nd.parent == parent && memcmp(nd.tokens, tokens, sizeof nd.tokens) == 0) return it->second;
+  }
+  return -1;
+}
+
+void prefix_forget(pa_block_manager *bm, int32_t b) {
+  PrefixNode &nd = bm->nodes[b];
+  if (!nd.live) return;
+  auto range = bm->prefix_index.equal_range(nd.key);
+  for (auto it = range.first; it != range.second; ++it)
+    if (it->second == b) {
+      bm->prefix_index.erase(it);
+      break;
+    }
+  nd.live = false;
+}
 
 int32_t take_block(pa_block_manager *bm) {
   const int32_t b = bm->free_list.front();
@@ -54,7 +109,10 @@ int32_t take_block(pa_block_manager *bm) {
 }
 
 void release_block(pa_block_manager *bm, int32_t b) {
-  if (--bm->refcount[b] == 0) bm->free_list.push_back(b);
+  if (--bm->refcount[b] == 0) {
+    prefix_forget(bm, b);   // its contents may be overwritten from now on
+    bm->free_list.push_back(b);
+  }
 }
 
 }  // namespace
@@ -77,6 +135,7 @@ pa_block_manager *pa_bm_create(int64_t num_blocks, uint64_t shuffle_seed) {
   }
   bm->free_list.assign(order.begin(), order.end());
   bm->refcount.assign(static_cast<size_t>(num_blocks), 0);
+  bm->nodes.resize(static_cast<size_t>(num_blocks));
   return bm;
 }
 
@@ -88,6 +147,62 @@ pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id) {
   if (!bm) return PA_EINVAL;
   if (bm->seqs.count(seq_id)) return PA_EINVAL;
   bm->seqs.emplace(seq_id, Seq());
+  return PA_OK;
+}
+
+pa_status pa_bm_add_prompt(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens, int64_t n_tokens,
+                           int64_t *slots_out, int64_t *reused_out) {
+  if (!bm || n_tokens < 0 || (n_tokens > 0 && (!tokens || !slots_out)) || !reused_out) return PA_EINVAL;
+  if (bm->seqs.count(seq_id)) return PA_EINVAL;
+  // walk the tree over the prompt's full blocks
+  const int64_t full = n_tokens / PA_BLOCK_SIZE;
+  std::vector<int32_t> shared;
+  std::vector<uint64_t> keys;
+  int32_t parent = -1;
+  uint64_t key = 0;
+  for (int64_t i = 0; i < full; ++i) {
+    key = prefix_key(key, tokens + i * PA_BLOCK_SIZE);
+    keys.push_back(key);
+    if (static_cast<int64_t>(shared.size()) == i) {
+      const int32_t b = prefix_find(bm, parent, key, tokens + i * PA_BLOCK_SIZE);
+      if (b >= 0) {
+        shared.push_back(b);
+        parent = b;
+      }
+    }
+  }
+  const int64_t reused = static_cast<int64_t>(shared.size()) * PA_BLOCK_SIZE;
+  const int64_t need = (n_tokens + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE - static_cast<int64_t>(shared.size());
+  if (need > static_cast<int64_t>(bm->free_list.size())) return PA_ENOMEM;  // nothing changed
+  Seq s;
+  for (int32_t b : shared) {
+    ++bm->refcount[b];
+    s.blocks.push_back(b);
+  }
+  for (int64_t i = 0; i < need; ++i) s.blocks.push_back(take_block(bm));
+  // the prompt's own full blocks become nodes that later prompts can share
+  for (int64_t i = static_cast<int64_t>(shared.size()); i < full; ++i) {
+    const int32_t b = s.blocks[i];
+    PrefixNode &nd = bm->nodes[b];
+    nd.live = true;
+    nd.parent = i > 0 ? s.blocks[i - 1] : -1;
+    nd.key = keys[i];
+    memcpy(nd.tokens, tokens + i * PA_BLOCK_SIZE, sizeof nd.tokens);
+    bm->prefix_index.emplace(nd.key, b);
+  }
+  for (int64_t t = reused; t < n_tokens; ++t)
+    slots_out[t - reused] = static_cast<int64_t>(s.blocks[t / PA_BLOCK_SIZE]) * PA_BLOCK_SIZE + t % PA_BLOCK_SIZE;
+  s.len = n_tokens;
+  bm->seqs.emplace(seq_id, std::move(s));
+  bm->prefix_tokens_reused += reused;
+  *reused_out = reused;
+  return PA_OK;
+}
+
+pa_status pa_bm_prefix_stats(const pa_block_manager *bm, int64_t *cached_blocks, int64_t *tokens_reused) {
+  if (!bm) return PA_EINVAL;
+  if (cached_blocks) *cached_blocks = static_cast<int64_t>(bm->prefix_index.size());
+  if (tokens_reused) *tokens_reused = bm->prefix_tokens_reused;
   return PA_OK;
 }
 

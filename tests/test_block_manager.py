@@ -178,3 +178,132 @@ def test_paged_vs_reserved_memory_utilisation():
         assert np.mean(util_reserved) < 0.5
     finally:
         B.pa_bm_destroy(h)
+
+
+# ----------------------------------------------------------------------------- prefix tree
+
+def _read_back(h, cache, ids, mbs):
+    tables, lens = B.pa_bm_tables(h, ids, mbs)
+    return [cache[tables[i, np.arange(lens[i]) // 16] * 16 + np.arange(lens[i]) % 16] for i in range(len(ids))]
+
+
+def test_prompts_that_start_alike_share_their_full_blocks():
+    """vLLM overview, Prefix Sharing: a second prompt with the same first 40 tokens shares the two full
+    blocks (32 tokens) of the first; only its other tokens get new slots, and every sequence reads back
+    exactly its own prompt through its table."""
+    h = B.pa_bm_create(64, 3)
+    try:
+        rng = np.random.default_rng(1)
+        common = rng.integers(0, 32000, 40)
+        p1 = np.concatenate([common, rng.integers(0, 32000, 9)])
+        p2 = np.concatenate([common, rng.integers(0, 32000, 30)])
+        cache = np.full(64 * 16, -1, np.int64)
+        s1, r1 = B.pa_bm_add_prompt(h, 1, p1)
+        assert r1 == 0 and len(s1) == len(p1)
+        cache[s1] = p1
+        free_before = B.pa_bm_num_free(h)
+        s2, r2 = B.pa_bm_add_prompt(h, 2, p2)
+        assert r2 == 32 and len(s2) == len(p2) - 32
+        cache[s2] = p2[32:]
+        assert free_before - B.pa_bm_num_free(h) == -(-(len(p2) - 32) // 16)   # only the unshared blocks
+        t, _ = B.pa_bm_tables(h, [1, 2], 8)
+        assert list(t[0, :2]) == list(t[1, :2]) and t[0, 2] != t[1, 2]        # block 2 holds 40 != 40 tokens
+        got1, got2 = _read_back(h, cache, [1, 2], 8)
+        assert np.array_equal(got1, p1) and np.array_equal(got2, p2)
+        st = B.pa_bm_prefix_stats(h)
+        assert st["tokens_reused"] == 32 and st["cached_blocks"] == 3 + 2      # full blocks of p1 and p2's own
+        assert B.pa_bm_stats(h)["blocks_shared"] == 2
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_prefix_nodes_live_while_a_holder_does():
+    h = B.pa_bm_create(32, 0)
+    try:
+        p = np.arange(48, dtype=np.int32)                          # three full blocks
+        B.pa_bm_add_prompt(h, 1, p)
+        B.pa_bm_add_prompt(h, 2, p[:40])                           # shares two, owns one partial block
+        B.pa_bm_free(h, 1)                                         # 2 still holds the first two blocks
+        _, r = B.pa_bm_add_prompt(h, 3, p)
+        assert r == 32                                             # block 3 of p went back to the pool
+        B.pa_bm_free(h, 2)
+        B.pa_bm_free(h, 3)
+        assert B.pa_bm_num_free(h) == 32 and B.pa_bm_prefix_stats(h)["cached_blocks"] == 0
+        _, r = B.pa_bm_add_prompt(h, 4, p)                         # nothing held: nothing to share
+        assert r == 0
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_prefix_sharing_stops_at_the_first_block_that_differs():
+    h = B.pa_bm_create(32, 0)
+    try:
+        p = np.arange(64, dtype=np.int32)
+        q = p.copy()
+        q[20] = -7                                                 # second block differs
+        B.pa_bm_add_prompt(h, 1, p)
+        _, r = B.pa_bm_add_prompt(h, 2, q)
+        assert r == 16
+        r3 = B.pa_bm_add_prompt(h, 3, p[16:])[1]                   # same tokens, other position: no match
+        assert r3 == 0
+        B.pa_bm_append(h, 2, 5)                                    # the shared block is full: no copy
+        assert B.pa_bm_stats(h)["cow_copies"] == 0
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_prompt_that_does_not_fit_changes_nothing():
+    h = B.pa_bm_create(4, 0)
+    try:
+        B.pa_bm_add_prompt(h, 1, np.arange(48, dtype=np.int32))       # 3 blocks
+        with pytest.raises(B.PagedAttnError) as e:
+            B.pa_bm_add_prompt(h, 2, np.arange(100, 140, dtype=np.int32))   # 3 more blocks, 1 free
+        assert e.value.status == B.PA_ENOMEM
+        assert B.pa_bm_num_free(h) == 1 and B.pa_bm_length(h, 2) == -1
+        _, r = B.pa_bm_add_prompt(h, 2, np.arange(60, dtype=np.int32))      # shares 3 blocks, needs 1
+        assert r == 48 and B.pa_bm_num_free(h) == 0
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_random_prompts_with_shared_system_prefixes():
+    """Prompts built from a few 'system' prefixes plus random tails, with decode appends and frees in
+    between: every live sequence reads back exactly its tokens, and sharing saves blocks."""
+    rng = np.random.default_rng(5)
+    h = B.pa_bm_create(2000, 9)
+    try:
+        systems = [rng.integers(0, 32000, int(rng.integers(20, 200))) for _ in range(4)]
+        cache = np.full(2000 * 16, -1, np.int64)
+        seqs, nid, reused_total, tok = {}, 0, 0, 10 ** 6
+        for step in range(400):
+            if rng.random() < 0.5 or len(seqs) < 3:
+                p = np.concatenate([systems[rng.integers(4)], rng.integers(0, 32000, int(rng.integers(0, 60)))])
+                try:
+                    slots, r = B.pa_bm_add_prompt(h, nid, p)
+                except B.PagedAttnError:
+                    continue
+                cache[slots] = p[r:]
+                seqs[nid] = list(p)
+                reused_total += r
+                nid += 1
+            elif rng.random() < 0.6:
+                s = list(seqs)[rng.integers(len(seqs))]
+                slots, cow = B.pa_bm_append(h, s, 3)
+                if cow is not None:
+                    cache[cow[1] * 16:(cow[1] + 1) * 16] = cache[cow[0] * 16:(cow[0] + 1) * 16]
+                cache[slots] = np.arange(tok, tok + 3)
+                seqs[s] += list(range(tok, tok + 3))
+                tok += 3
+            else:
+                s = list(seqs)[rng.integers(len(seqs))]
+                B.pa_bm_free(h, s)
+                del seqs[s]
+            ids = list(seqs)
+            mbs = max(1, max(-(-len(v) // 16) for v in seqs.values()))
+            for sid, got in zip(ids, _read_back(h, cache, ids, mbs)):
+                assert np.array_equal(got, np.array(seqs[sid], np.int64))
+        assert reused_total > 0 and B.pa_bm_prefix_stats(h)["tokens_reused"] == reused_total
+        st = B.pa_bm_stats(h)
+        assert st["blocks_used"] < sum(-(-len(v) // 16) for v in seqs.values())   # sharing saved blocks
+    finally:
+        B.pa_bm_destroy(h)
