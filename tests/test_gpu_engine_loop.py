@@ -144,3 +144,44 @@ def test_cuda_graph_replay_matches_eager(cuda_lib):
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
     assert torch.equal(st.out_dec, eager_dec)
     assert torch.equal(st.out_pre, eager_pre)
+
+
+def test_prefix_tree_shared_blocks_feed_the_kernels(O, cuda_lib):
+    """Two prompts with a common 40-token start: the second shares the first's two full blocks through
+    the block manager's prefix tree, appends K/V only for its own tokens, and its causal prefill over
+    the whole prompt (read through the shared blocks) matches the oracle on its own contiguous K/V."""
+    B = cuda_lib
+    g = torch.Generator(device="cuda").manual_seed(11)
+    nb = 64
+    kc = torch.zeros((nb, HKV, 16, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    rnd = lambda n: torch.randn((n, HKV, D), generator=g, device="cuda").to(torch.bfloat16)
+    common_k, common_v = rnd(40), rnd(40)        # K/V of the common start (same tokens, same positions)
+    rng = np.random.default_rng(2)
+    common = rng.integers(0, 32000, 40)
+    p1 = np.concatenate([common, rng.integers(0, 32000, 25)])
+    p2 = np.concatenate([common, rng.integers(0, 32000, 57)])
+    k1 = torch.cat([common_k, rnd(25)])
+    v1 = torch.cat([common_v, rnd(25)])
+    k2 = torch.cat([common_k, rnd(57)])
+    v2 = torch.cat([common_v, rnd(57)])
+    bm = B.pa_bm_create(nb, 4)
+    try:
+        s1, r1 = B.pa_bm_add_prompt(bm, 1, p1)
+        B.pa_kv_append(kc, vc, k1, v1, torch.from_numpy(s1).cuda())
+        s2, r2 = B.pa_bm_add_prompt(bm, 2, p2)
+        assert r1 == 0 and r2 == 32
+        B.pa_kv_append(kc, vc, k2[r2:].contiguous(), v2[r2:].contiguous(), torch.from_numpy(s2).cuda())
+        n = len(p2)
+        tables, tl = B.pa_bm_tables(bm, [2], (n + 15) // 16)
+        q = torch.randn((n, HQ, D), generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty_like(q)
+        cu = torch.tensor([0, n], dtype=torch.int32, device="cuda")
+        B.pa_paged_prefill(out, q, cu, kc, vc, torch.from_numpy(tables).cuda(), torch.from_numpy(tl).cuda(),
+                           SCALE, n, n)
+        torch.cuda.synchronize()
+        assert B.pa_get_device_error() == B.PA_OK
+        ref = _oracle_rows(O, bf16_bits(k2), bf16_bits(v2), bf16_bits(q), [i + 1 for i in range(n)])
+        assert_close(to_f64(out), ref, what="prefill over prefix-shared blocks")
+    finally:
+        B.pa_bm_destroy(bm)
