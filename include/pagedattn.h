@@ -223,7 +223,8 @@ typedef struct pa_block_manager pa_block_manager;
  * bad arguments or out of host memory. */
 pa_block_manager *pa_bm_create(int64_t num_blocks, uint64_t shuffle_seed);
 void pa_bm_destroy(pa_block_manager *bm);
-/* pa_bm_num_free -- blocks currently free (-1 for a NULL manager). */
+/* pa_bm_num_free -- blocks available for new contents: free ones and, with prefix caching, cached
+ * evictable ones (-1 for a NULL manager). */
 int64_t pa_bm_num_free(const pa_block_manager *bm);
 /* pa_bm_add -- register an empty sequence.  PA_EINVAL if the id exists. */
 pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id);
@@ -239,6 +240,14 @@ pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id);
  */
 pa_status pa_bm_add_prompt(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens, int64_t n_tokens,
                            int64_t *slots_out, int64_t *reused_out);
+/*
+ * pa_bm_set_prefix_caching -- keep_freed != 0: a prompt block whose last holder leaves stays in the
+ * prefix tree as a cached, evictable block (counted by pa_bm_num_free), so that a later prompt that
+ * starts alike can take it back without recomputing its K/V.  Allocation uses free blocks first, then
+ * evicts the least recently freed cached block that no other cached block builds on.  keep_freed == 0
+ * (the default) drops the cache at once: cached blocks become free.
+ */
+pa_status pa_bm_set_prefix_caching(pa_block_manager *bm, int keep_freed);
 /* pa_bm_prefix_stats -- blocks currently in the prefix tree, and prompt tokens served from it so far. */
 pa_status pa_bm_prefix_stats(const pa_block_manager *bm, int64_t *cached_blocks, int64_t *tokens_reused);
 /* pa_bm_fork -- child shares every block of parent (reference counts + 1), same length. */

@@ -36,7 +36,7 @@ EXPORTED = (
     "pa_paged_attention_noalloc", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
     "pa_bm_length", "pa_bm_tables", "pa_bm_stats", "pa_selftest_bounded_wait", "pa_bm_add_prompt",
-    "pa_bm_prefix_stats",
+    "pa_bm_prefix_stats", "pa_bm_set_prefix_caching",
 )
 PA_ENOMEM = -6
 
@@ -110,6 +110,8 @@ def lib() -> ctypes.CDLL:
         L.pa_bm_add_prompt.argtypes = [P, I64, P, I64, P, P]
         L.pa_bm_prefix_stats.restype = I
         L.pa_bm_prefix_stats.argtypes = [P, P, P]
+        L.pa_bm_set_prefix_caching.restype = I
+        L.pa_bm_set_prefix_caching.argtypes = [P, I]
         _lib = L
     return _lib
 
@@ -345,6 +347,10 @@ def pa_bm_add_prompt(bm, seq_id: int, tokens):
                                 slots.ctypes.data_as(ctypes.c_void_p), ctypes.byref(reused))
     _check(st, "pa_bm_add_prompt")
     return slots[:toks.shape[0] - reused.value], int(reused.value)
+
+
+def pa_bm_set_prefix_caching(bm, keep_freed: bool):
+    _check(lib().pa_bm_set_prefix_caching(bm, 1 if keep_freed else 0), "pa_bm_set_prefix_caching")
 
 
 def pa_bm_prefix_stats(bm) -> dict:

@@ -21,12 +21,18 @@
 // the common part).  Every full block a prompt fills is a node keyed by (parent node, its 16 token ids);
 // a new prompt walks the tree block by block and shares every node it matches exactly, so only its
 // remaining tokens need K/V written.  Nodes are looked up through a hash of the whole prefix and then
-// compared exactly (parent block and token ids), so a hash collision can never share a wrong block.  A
-// node lives while some sequence holds its block; when the block returns to the pool the node goes.
+// compared exactly (parent block and token ids), so a hash collision can never share a wrong block.  By
+// default a node lives while some sequence holds its block.  With prefix caching on
+// (pa_bm_set_prefix_caching), a prompt block whose last holder leaves stays in the tree on an LRU list
+// of evictable blocks; a later prompt can revive it, and allocation takes truly free blocks first, then
+// evicts the least recently freed cached block that no other cached node builds on.  So a cached node's
+// parent is never reused under it.
 #include <stdint.h>
 #include <string.h>
 
 #include <deque>
+#include <iterator>
+#include <list>
 #include <new>
 #include <random>
 #include <unordered_map>
@@ -74,7 +80,13 @@ struct pa_block_manager {
   // prefix tree: key -> blocks whose prefix hashes to it (exact match decides), node per block
   std::unordered_multimap<uint64_t, int32_t> prefix_index;
   std::vector<PrefixNode> nodes;
+  std::vector<int32_t> children;  // live nodes whose parent is this block
   int64_t prefix_tokens_reused = 0;
+  // prefix caching: blocks with a live node and no holder, least recently freed first
+  bool keep_freed = false;
+  std::list<int32_t> evictable;
+  std::vector<std::list<int32_t>::iterator> ev_pos;
+  std::vector<char> in_ev;
 };
 
 namespace {
@@ -92,6 +104,7 @@ int32_t prefix_find(const pa_block_manager *bm, int32_t parent, uint64_t key, co
 void prefix_forget(pa_block_manager *bm, int32_t b) {
   PrefixNode &nd = bm->nodes[b];
   if (!nd.live) return;
+  if (nd.parent >= 0) --bm->children[nd.parent];
   auto range = bm->prefix_index.equal_range(nd.key);
   for (auto it = range.first; it != range.second; ++it)
     if (it->second == b) {
@@ -101,17 +114,44 @@ void prefix_forget(pa_block_manager *bm, int32_t b) {
   nd.live = false;
 }
 
+int64_t available(const pa_block_manager *bm) {
+  return static_cast<int64_t>(bm->free_list.size() + bm->evictable.size());
+}
+
+void unlist_evictable(pa_block_manager *bm, int32_t b) {
+  bm->evictable.erase(bm->ev_pos[b]);
+  bm->in_ev[b] = 0;
+}
+
+// A block for new contents (the caller has checked available() first): a free one, else the least
+// recently freed cached block on which no other cached node builds (one exists whenever the list is
+// not empty: children of an evictable block have no holder either, and chains end).
 int32_t take_block(pa_block_manager *bm) {
-  const int32_t b = bm->free_list.front();
-  bm->free_list.pop_front();
+  int32_t b;
+  if (!bm->free_list.empty()) {
+    b = bm->free_list.front();
+    bm->free_list.pop_front();
+  } else {
+    auto it = bm->evictable.begin();
+    while (bm->children[*it] != 0) ++it;
+    b = *it;
+    unlist_evictable(bm, b);
+    prefix_forget(bm, b);   // its contents are about to be overwritten
+  }
   bm->refcount[b] = 1;
   return b;
 }
 
 void release_block(pa_block_manager *bm, int32_t b) {
   if (--bm->refcount[b] == 0) {
-    prefix_forget(bm, b);   // its contents may be overwritten from now on
-    bm->free_list.push_back(b);
+    if (bm->keep_freed && bm->nodes[b].live) {
+      bm->evictable.push_back(b);
+      bm->ev_pos[b] = std::prev(bm->evictable.end());
+      bm->in_ev[b] = 1;
+    } else {
+      prefix_forget(bm, b);   // its contents may be overwritten from now on
+      bm->free_list.push_back(b);
+    }
   }
 }
 
@@ -136,12 +176,28 @@ pa_block_manager *pa_bm_create(int64_t num_blocks, uint64_t shuffle_seed) {
   bm->free_list.assign(order.begin(), order.end());
   bm->refcount.assign(static_cast<size_t>(num_blocks), 0);
   bm->nodes.resize(static_cast<size_t>(num_blocks));
+  bm->children.assign(static_cast<size_t>(num_blocks), 0);
+  bm->ev_pos.resize(static_cast<size_t>(num_blocks));
+  bm->in_ev.assign(static_cast<size_t>(num_blocks), 0);
   return bm;
 }
 
 void pa_bm_destroy(pa_block_manager *bm) { delete bm; }
 
-int64_t pa_bm_num_free(const pa_block_manager *bm) { return bm ? static_cast<int64_t>(bm->free_list.size()) : -1; }
+int64_t pa_bm_num_free(const pa_block_manager *bm) { return bm ? available(bm) : -1; }
+
+pa_status pa_bm_set_prefix_caching(pa_block_manager *bm, int keep_freed) {
+  if (!bm) return PA_EINVAL;
+  bm->keep_freed = keep_freed != 0;
+  if (!bm->keep_freed)
+    while (!bm->evictable.empty()) {   // drop the cache: every cached block becomes free
+      const int32_t b = bm->evictable.front();
+      unlist_evictable(bm, b);
+      prefix_forget(bm, b);
+      bm->free_list.push_back(b);
+    }
+  return PA_OK;
+}
 
 pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id) {
   if (!bm) return PA_EINVAL;
@@ -173,9 +229,12 @@ pa_status pa_bm_add_prompt(pa_block_manager *bm, int64_t seq_id, const int32_t *
   }
   const int64_t reused = static_cast<int64_t>(shared.size()) * PA_BLOCK_SIZE;
   const int64_t need = (n_tokens + PA_BLOCK_SIZE - 1) / PA_BLOCK_SIZE - static_cast<int64_t>(shared.size());
-  if (need > static_cast<int64_t>(bm->free_list.size())) return PA_ENOMEM;  // nothing changed
+  int64_t revived = 0;   // cached blocks this prompt takes back off the evictable list
+  for (int32_t b : shared) revived += bm->in_ev[b];
+  if (need > available(bm) - revived) return PA_ENOMEM;  // nothing changed
   Seq s;
   for (int32_t b : shared) {
+    if (bm->in_ev[b]) unlist_evictable(bm, b);
     ++bm->refcount[b];
     s.blocks.push_back(b);
   }
@@ -189,6 +248,7 @@ pa_status pa_bm_add_prompt(pa_block_manager *bm, int64_t seq_id, const int32_t *
     nd.key = keys[i];
     memcpy(nd.tokens, tokens + i * PA_BLOCK_SIZE, sizeof nd.tokens);
     bm->prefix_index.emplace(nd.key, b);
+    if (nd.parent >= 0) ++bm->children[nd.parent];
   }
   for (int64_t t = reused; t < n_tokens; ++t)
     slots_out[t - reused] = static_cast<int64_t>(s.blocks[t / PA_BLOCK_SIZE]) * PA_BLOCK_SIZE + t % PA_BLOCK_SIZE;
@@ -236,7 +296,7 @@ pa_status pa_bm_append(pa_block_manager *bm, int64_t seq_id, int32_t n_tokens, i
     if (!cow_pairs_out) return PA_EINVAL;
     ++needed;
   }
-  if (needed > static_cast<int64_t>(bm->free_list.size())) return PA_ENOMEM;  // nothing changed
+  if (needed > available(bm)) return PA_ENOMEM;  // nothing changed
   if (cow) {
     const int32_t src = s.blocks[first_blk];
     const int32_t dst = take_block(bm);
@@ -258,7 +318,9 @@ pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id) {
   if (!bm) return PA_EINVAL;
   auto it = bm->seqs.find(seq_id);
   if (it == bm->seqs.end()) return PA_EINVAL;
-  for (int32_t b : it->second.blocks) release_block(bm, b);
+  // last block first: a prompt's deeper blocks reach the evictable list before their parents
+  const std::vector<int32_t> &blocks = it->second.blocks;
+  for (size_t i = blocks.size(); i-- > 0;) release_block(bm, blocks[i]);
   bm->seqs.erase(it);
   return PA_OK;
 }

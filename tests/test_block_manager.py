@@ -307,3 +307,95 @@ def test_random_prompts_with_shared_system_prefixes():
         assert st["blocks_used"] < sum(-(-len(v) // 16) for v in seqs.values())   # sharing saved blocks
     finally:
         B.pa_bm_destroy(h)
+
+
+# ----------------------------------------------------------------------------- prefix caching
+
+def test_prefix_caching_keeps_freed_prompt_blocks_for_later_prompts():
+    h = B.pa_bm_create(16, 0)
+    try:
+        B.pa_bm_set_prefix_caching(h, True)
+        p = np.arange(53, dtype=np.int32)                          # 3 full blocks + 5 tokens
+        B.pa_bm_add_prompt(h, 1, p)
+        B.pa_bm_free(h, 1)
+        assert B.pa_bm_num_free(h) == 16                           # cached blocks count as available
+        assert B.pa_bm_prefix_stats(h)["cached_blocks"] == 3
+        slots, r = B.pa_bm_add_prompt(h, 2, p)
+        assert r == 48 and len(slots) == 5                         # only the partial block is new
+        assert B.pa_bm_num_free(h) == 16 - 4
+        B.pa_bm_set_prefix_caching(h, False)                       # held blocks stay, nothing cached
+        B.pa_bm_free(h, 2)
+        assert B.pa_bm_prefix_stats(h)["cached_blocks"] == 0 and B.pa_bm_num_free(h) == 16
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_prefix_cache_evicts_least_recently_freed_leaves_first():
+    h = B.pa_bm_create(7, 0)
+    try:
+        B.pa_bm_set_prefix_caching(h, True)
+        a = np.arange(48, dtype=np.int32)                          # three full blocks A0 <- A1 <- A2
+        B.pa_bm_add_prompt(h, 1, a)
+        B.pa_bm_free(h, 1)                                         # all three cached, four free
+        B.pa_bm_add_prompt(h, 2, np.arange(1000, 1080, dtype=np.int32))   # 5 blocks: 4 free + 1 evicted
+        assert B.pa_bm_num_free(h) == 2 and B.pa_bm_prefix_stats(h)["cached_blocks"] == 5 + 2
+        _, r = B.pa_bm_add_prompt(h, 3, a[:32])                    # the leaf A2 went; A0 and A1 revive
+        assert r == 32 and B.pa_bm_num_free(h) == 0
+        with pytest.raises(B.PagedAttnError) as e:                 # 1 block needed, none available
+            B.pa_bm_add_prompt(h, 4, np.arange(2000, 2016, dtype=np.int32))
+        assert e.value.status == B.PA_ENOMEM
+        B.pa_bm_free(h, 3)                                         # A0, A1 cached again
+        _, r = B.pa_bm_add_prompt(h, 5, np.arange(3000, 3032, dtype=np.int32))  # evicts A1 (leaf), then A0
+        assert r == 0 and B.pa_bm_prefix_stats(h)["cached_blocks"] == 5 + 2
+    finally:
+        B.pa_bm_destroy(h)
+
+
+def test_random_prompts_with_prefix_caching_and_eviction():
+    """Same as the random system-prompt test, with caching on and a pool small enough to evict: every
+    live sequence reads back exactly its tokens (a revived block still holds the K/V it was given, an
+    evicted one is never shared again)."""
+    rng = np.random.default_rng(6)
+    h = B.pa_bm_create(120, 2)
+    try:
+        B.pa_bm_set_prefix_caching(h, True)
+        systems = [rng.integers(0, 32000, int(rng.integers(20, 120))) for _ in range(5)]
+        cache = np.full(120 * 16, -1, np.int64)
+        seqs, nid, tok = {}, 0, 10 ** 6
+        for step in range(600):
+            r_ = rng.random()
+            if r_ < 0.45 or len(seqs) < 2:
+                p = np.concatenate([systems[rng.integers(5)], rng.integers(0, 32000, int(rng.integers(0, 40)))])
+                try:
+                    slots, r = B.pa_bm_add_prompt(h, nid, p)
+                except B.PagedAttnError as e:
+                    assert e.status == B.PA_ENOMEM
+                    continue
+                assert np.array_equal(_read_back(h, cache, [nid], -(-len(p) // 16))[0][:r], p[:r])
+                cache[slots] = p[r:]
+                seqs[nid] = list(p)
+                nid += 1
+            elif r_ < 0.7:
+                s = list(seqs)[rng.integers(len(seqs))]
+                try:
+                    slots, cow = B.pa_bm_append(h, s, 2)
+                except B.PagedAttnError as e:
+                    assert e.status == B.PA_ENOMEM
+                    continue
+                if cow is not None:
+                    cache[cow[1] * 16:(cow[1] + 1) * 16] = cache[cow[0] * 16:(cow[0] + 1) * 16]
+                cache[slots] = [tok, tok + 1]
+                seqs[s] += [tok, tok + 1]
+                tok += 2
+            else:
+                s = list(seqs)[rng.integers(len(seqs))]
+                B.pa_bm_free(h, s)
+                del seqs[s]
+            if seqs:
+                ids = list(seqs)
+                mbs = max(1, max(-(-len(v) // 16) for v in seqs.values()))
+                for sid, got in zip(ids, _read_back(h, cache, ids, mbs)):
+                    assert np.array_equal(got, np.array(seqs[sid], np.int64))
+        assert B.pa_bm_prefix_stats(h)["tokens_reused"] > 0
+    finally:
+        B.pa_bm_destroy(h)
