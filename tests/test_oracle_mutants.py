@@ -6,6 +6,7 @@ import os
 import subprocess
 import tempfile
 
+import numpy as np
 import pytest
 
 from oracle import oracle as O
@@ -31,6 +32,16 @@ MUTANTS = {
     "copy forgets V": ("        memmove((char *)v_cache + d * block_bytes, (char *)v_cache + s * block_bytes, block_bytes);\n", ""),
     "INT8 truncates": ("float r = rintf(x);", "float r = truncf(x);"),
     "INT8 range -128": ("if (r < -127.0f) r = -127.0f;", "if (r < -128.0f) r = -128.0f;"),
+    "FP8 dequant drops the scale": ("return oracle_e4m3_decode(((const uint8_t *)cache)[idx]) * (double)scale;",
+                                    "return oracle_e4m3_decode(((const uint8_t *)cache)[idx]);"),
+    "INT8 dequant drops the scale": ("return (double)((const int8_t *)cache)[idx] * (double)scale;",
+                                     "return (double)((const int8_t *)cache)[idx];"),
+    "decode V uses k_scale": ("vs = kv_dtype ? v_scale[g] : 1.0f;\n            int r = attend_one",
+                              "vs = kv_dtype ? k_scale[g] : 1.0f;\n            int r = attend_one"),
+    "prefill V uses k_scale": ("vs = kv_dtype ? v_scale[g] : 1.0f;\n            int r;",
+                               "vs = kv_dtype ? k_scale[g] : 1.0f;\n            int r;"),
+    "swap copies K into V": ("memcpy((char *)dst_v + d * block_bytes, (const char *)src_v + s * block_bytes",
+                             "memcpy((char *)dst_v + d * block_bytes, (const char *)src_k + s * block_bytes"),
 }
 
 PIN_TESTS = [
@@ -45,6 +56,11 @@ PIN_TESTS = [
     (pins.test_copy_on_write_copies_and_keeps_parent, {}),
     (pins.test_int8_encode_points, {}),
     (pins.test_int8_encode_matches_numpy, {}),
+    (pins.test_one_byte_decode_matches_sdpa_on_dequantised_kv, dict(kv_dtype=1, bs=16)),
+    (pins.test_one_byte_decode_matches_sdpa_on_dequantised_kv, dict(kv_dtype=2, bs=32)),
+    (pins.test_one_byte_prefill_matches_sdpa_on_dequantised_kv, dict(kv_dtype=1)),
+    (pins.test_one_byte_prefill_matches_sdpa_on_dequantised_kv, dict(kv_dtype=2)),
+    (pins.test_swap_reads_back_each_moved_block, dict(dtype=np.uint16, bs=16)),
 ]
 
 

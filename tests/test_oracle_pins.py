@@ -333,3 +333,102 @@ def test_int8_append_and_decode_read_back(O):
     rows = np.stack([vc[1, 0, 0].astype(np.float64), vc[1, 0, 1].astype(np.float64)]) * np.float64(np.float32(0.02))
     lo, hi = rows.min(axis=0) - 1e-12, rows.max(axis=0) + 1e-12
     assert np.all((out[0] >= lo) & (out[0] <= hi))
+
+
+# ----------------------------------------------------------------------------- one-byte caches: dequantisation
+
+def _dequant_reference(codes, kv_dtype, scale):
+    """Values of one-byte cache codes [..][Hkv][bs][D] with one scale per KV head, from the library
+    routines: torch's float8_e4m3fn reinterpretation (FP8) or the integer itself (INT8), times the scale."""
+    c = torch.from_numpy(np.ascontiguousarray(codes))
+    v = c.view(torch.float8_e4m3fn).to(torch.float64) if kv_dtype == 1 else c.to(torch.float64)
+    return v * torch.from_numpy(np.asarray(scale, np.float32)).to(torch.float64)[None, :, None, None]
+
+
+def _one_byte_case(kv_dtype, bs, seed):
+    """A shuffled pool of random one-byte codes (no NaN codes), two KV heads with four different scales."""
+    rng = np.random.default_rng(seed)
+    nb, hkv, d = 24, 2, 64
+    if kv_dtype == 1:
+        codes = rng.integers(0, 256, size=(2, nb, hkv, bs, d)).astype(np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0x3C                 # the NaN codes never come out of the encoder
+    else:
+        codes = rng.integers(-127, 128, size=(2, nb, hkv, bs, d)).astype(np.int8)
+    k_scale = np.array([0.013, 0.041], np.float32)             # every scale different: K vs V and per head
+    v_scale = np.array([0.37, 0.0029], np.float32)
+    return codes[0], codes[1], k_scale, v_scale, rng
+
+
+def _gather(pool, table, L, bs):
+    """Rows 0..L-1 of one sequence, [Hkv][L][D], read from a [NB][Hkv][bs][D] tensor through its table."""
+    t = torch.arange(L)
+    return pool[torch.from_numpy(table.astype(np.int64))[t // bs], :, t % bs].permute(1, 0, 2)
+
+
+@pytest.mark.parametrize("kv_dtype", [1, 2])
+@pytest.mark.parametrize("bs", [16, 32])
+def test_one_byte_decode_matches_sdpa_on_dequantised_kv(O, kv_dtype, bs):
+    """Decode over an FP8 / INT8 cache equals torch fp64 SDPA on code * scale, with K and V dequantised by
+    their own per-head scales (KV Cache to vLLM §2.2: one byte per element with a scale)."""
+    kc, vc, ks, vs, rng = _one_byte_case(kv_dtype, bs, 31 + kv_dtype)
+    hq, hkv, d = 6, 2, 64
+    kf, vf = _dequant_reference(kc, kv_dtype, ks), _dequant_reference(vc, kv_dtype, vs)
+    lens = np.array([1, 29, bs * 3, 150], np.int32)
+    mbs = (int(lens.max()) + bs - 1) // bs
+    tables = np.stack([rng.permutation(kc.shape[0])[:mbs] for _ in lens]).astype(np.int32)
+    q = bf16_bits(torch.randn(len(lens), hq, d, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16))
+    got = O.paged_decode(q, kc, vc, tables, lens, 0.125, kv_dtype, ks, vs)
+    qf = torch.from_numpy(_bf16_to_f64(q))
+    for b, L in enumerate(lens):
+        k = _gather(kf, tables[b], int(L), bs).repeat_interleave(hq // hkv, 0)
+        v = _gather(vf, tables[b], int(L), bs).repeat_interleave(hq // hkv, 0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qf[b][None, :, None, :], k[None], v[None], scale=0.125)
+        np.testing.assert_allclose(got[b], ref[0, :, 0].numpy(), atol=1e-12, rtol=1e-12)
+
+
+@pytest.mark.parametrize("kv_dtype", [1, 2])
+def test_one_byte_prefill_matches_sdpa_on_dequantised_kv(O, kv_dtype):
+    """Causal chunks over an FP8 / INT8 cache equal torch fp64 SDPA (causal offset mask) on code * scale."""
+    bs = 16
+    kc, vc, ks, vs, rng = _one_byte_case(kv_dtype, bs, 41 + kv_dtype)
+    hq, hkv, d = 4, 2, 64
+    kf, vf = _dequant_reference(kc, kv_dtype, ks), _dequant_reference(vc, kv_dtype, vs)
+    C = np.array([7, 19], np.int32)
+    ctx = np.array([7, 60], np.int32)                          # chunk 0 starts a request, chunk 1 has H = 41
+    cu = np.concatenate([[0], np.cumsum(C)]).astype(np.int32)
+    mbs = (int(ctx.max()) + bs - 1) // bs
+    tables = np.stack([rng.permutation(kc.shape[0])[:mbs] for _ in C]).astype(np.int32)
+    q = bf16_bits(torch.randn(int(cu[-1]), hq, d, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16))
+    got = O.paged_prefill(q, cu, kc, vc, tables, ctx, 0.1, kv_dtype, ks, vs)
+    qf = torch.from_numpy(_bf16_to_f64(q))
+    for c in range(len(C)):
+        L, H = int(ctx[c]), int(ctx[c] - C[c])
+        k = _gather(kf, tables[c], L, bs).repeat_interleave(hq // hkv, 0)
+        v = _gather(vf, tables[c], L, bs).repeat_interleave(hq // hkv, 0)
+        mask = torch.arange(L)[None, :] <= (H + torch.arange(int(C[c])))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qf[cu[c]:cu[c + 1]].permute(1, 0, 2)[None], k[None],
+                                                               v[None], attn_mask=mask, scale=0.1)
+        np.testing.assert_allclose(got[cu[c]:cu[c + 1]], ref[0].permute(1, 0, 2).numpy(), atol=1e-12, rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- swap
+
+@pytest.mark.parametrize("dtype,bs", [(np.uint16, 16), (np.uint8, 32)])
+def test_swap_reads_back_each_moved_block(O, dtype, bs):
+    """After a swap (vLLM overview, section 三: KV pages move to CPU memory and back), block dst of the
+    destination pool equals block src of the source pool, for K and for V separately; every other
+    destination block and the whole source pool are unchanged."""
+    rng = np.random.default_rng(17)
+    hkv, d, nsrc, ndst = 2, 64, 30, 20
+    hi = np.iinfo(dtype).max
+    src_k, src_v = (rng.integers(0, hi, size=(nsrc, hkv, bs, d)).astype(dtype) for _ in range(2))
+    dst_k, dst_v = (rng.integers(0, hi, size=(ndst, hkv, bs, d)).astype(dtype) for _ in range(2))
+    pairs = np.stack([rng.permutation(nsrc)[:9], rng.permutation(ndst)[:9]], 1).astype(np.int32)
+    before = [a.copy() for a in (src_k, src_v, dst_k, dst_v)]
+    O.swap_blocks(dst_k, dst_v, src_k, src_v, pairs)
+    assert np.array_equal(src_k, before[0]) and np.array_equal(src_v, before[1])
+    for s, t in pairs:
+        assert np.array_equal(dst_k[t], before[0][s]) and np.array_equal(dst_v[t], before[1][s])
+    untouched = np.setdiff1d(np.arange(ndst), pairs[:, 1])
+    assert np.array_equal(dst_k[untouched], before[2][untouched])
+    assert np.array_equal(dst_v[untouched], before[3][untouched])
