@@ -218,11 +218,13 @@ pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, i
  */
 typedef struct pa_block_manager pa_block_manager;
 
-/* pa_bm_create -- pool of num_blocks physical blocks.  shuffle_seed != 0 hands blocks out in a seeded
- * random order (a long-running server's scattered placement); 0 hands them out in order.  NULL on
- * bad arguments or out of host memory. */
-pa_block_manager *pa_bm_create(int64_t num_blocks, uint64_t shuffle_seed);
+/* pa_bm_create -- pool of num_blocks physical blocks of block_size tokens (16 or 32).  shuffle_seed != 0
+ * hands blocks out in a seeded random order (a long-running server's scattered placement); 0 hands them
+ * out in order.  NULL on bad arguments or out of host memory. */
+pa_block_manager *pa_bm_create(int64_t num_blocks, int block_size, uint64_t shuffle_seed);
 void pa_bm_destroy(pa_block_manager *bm);
+/* pa_bm_block_size -- tokens per block of the manager (-1 for a NULL manager). */
+int pa_bm_block_size(const pa_block_manager *bm);
 /* pa_bm_num_free -- blocks available for new contents: free ones and, with prefix caching, cached
  * evictable ones (-1 for a NULL manager). */
 int64_t pa_bm_num_free(const pa_block_manager *bm);
@@ -230,31 +232,43 @@ int64_t pa_bm_num_free(const pa_block_manager *bm);
 pa_status pa_bm_add(pa_block_manager *bm, int64_t seq_id);
 /*
  * pa_bm_add_prompt -- register a new sequence with a prompt of n_tokens token ids, sharing the blocks of
- * any earlier prompt that starts alike [vLLM overview, Prefix Sharing].  The prompt's full 16-token
- * blocks form a prefix tree keyed by (previous block, token ids); the longest chain of blocks that
- * exactly match a live node is shared (reference counts + 1), and *reused_out is its length in tokens
- * (a multiple of 16).  The remaining n_tokens - *reused_out tokens get slots in new blocks, written to
- * slots_out[0 ..] in order: only those need their K/V appended; the shared ones are already in the
- * cache.  The prompt's own full blocks join the tree.  A node lives while some sequence holds its block.
+ * any earlier prompt that starts alike [vLLM overview, Prefix Sharing].  Full prompt blocks whose K/V
+ * have been committed (pa_bm_commit) form a prefix tree keyed by (previous block, token ids); the
+ * longest chain of blocks that exactly match a node is shared (reference counts + 1), and *reused_out
+ * is its length in tokens (a multiple of the block size).  The block holding the prompt's last token is
+ * never shared, so at least one token stays new: its query is what the next token depends on.  The
+ * remaining n_tokens - *reused_out tokens get slots in new blocks, written to slots_out[0 ..] in order:
+ * only those need their K/V appended; the shared ones are already in the cache.  The prompt's own full
+ * blocks join the tree when pa_bm_commit reports them written, never before.  A node lives while some
+ * sequence holds its block (or, with prefix caching on, until it is evicted).
  * PA_EINVAL if the id exists; PA_ENOMEM (nothing changed) if the pool is short.
  */
 pa_status pa_bm_add_prompt(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens, int64_t n_tokens,
                            int64_t *slots_out, int64_t *reused_out);
 /*
- * pa_bm_set_prefix_caching -- keep_freed != 0: a prompt block whose last holder leaves stays in the
- * prefix tree as a cached, evictable block (counted by pa_bm_num_free), so that a later prompt that
- * starts alike can take it back without recomputing its K/V.  Allocation uses free blocks first, then
- * evicts the least recently freed cached block that no other cached block builds on.  keep_freed == 0
+ * pa_bm_commit -- report that the K/V of the first tokens_written tokens of seq_id are in the cache (for
+ * a prompt prefilled in chunks: call it after each chunk's append).  Every full prompt block within them
+ * joins the prefix tree and can be shared by later prompts from then on.  A sequence freed before its
+ * blocks are committed leaves nothing in the tree.  PA_EINVAL if the id is unknown or tokens_written is
+ * negative or beyond the tokens reserved for it.
+ */
+pa_status pa_bm_commit(pa_block_manager *bm, int64_t seq_id, int64_t tokens_written);
+/*
+ * pa_bm_set_prefix_caching -- keep_freed != 0: a committed prompt block whose last holder leaves stays
+ * in the prefix tree as a cached, evictable block (counted by pa_bm_num_free), so that a later prompt
+ * that starts alike can take it back without recomputing its K/V.  Allocation uses free blocks first,
+ * then evicts the least recently freed cached block that no other node builds on.  keep_freed == 0
  * (the default) drops the cache at once: cached blocks become free.
  */
 pa_status pa_bm_set_prefix_caching(pa_block_manager *bm, int keep_freed);
 /* pa_bm_prefix_stats -- blocks currently in the prefix tree, and prompt tokens served from it so far. */
 pa_status pa_bm_prefix_stats(const pa_block_manager *bm, int64_t *cached_blocks, int64_t *tokens_reused);
-/* pa_bm_fork -- child shares every block of parent (reference counts + 1), same length. */
+/* pa_bm_fork -- child shares every block of parent (reference counts + 1), same length.  Prompt blocks
+ * still waiting for pa_bm_commit are committed through the parent only. */
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent, int64_t child);
 /*
  * pa_bm_append -- reserve slots for n_tokens new tokens at the end of seq_id and write them to
- * slots_out[n_tokens] (slot = block*16 + offset, ready for pa_kv_append with 16-token blocks).  If the block that receives
+ * slots_out[n_tokens] (slot = block*block_size + offset, ready for pa_kv_append).  If the block that receives
  * the first new token is shared, it is first replaced by a private copy: the (src, dst) pair goes to
  * cow_pairs_out[2] (run pa_copy_blocks on it before the append) and *num_cow_out = 1, else 0.
  * PA_ENOMEM if the pool cannot supply the blocks; then nothing changes.
@@ -263,7 +277,7 @@ pa_status pa_bm_append(pa_block_manager *bm, int64_t seq_id, int32_t n_tokens, i
                        int32_t *cow_pairs_out, int32_t *num_cow_out);
 /* pa_bm_free -- drop a sequence; blocks no other sequence holds return to the free list. */
 pa_status pa_bm_free(pa_block_manager *bm, int64_t seq_id);
-/* pa_bm_length -- tokens written to seq_id (-1 if unknown). */
+/* pa_bm_length -- tokens reserved for seq_id, i.e. slots handed out (-1 if unknown). */
 int64_t pa_bm_length(const pa_block_manager *bm, int64_t seq_id);
 /* pa_bm_tables -- block tables int32 [n][max_blocks_per_seq] (padded with -1) and lengths int32 [n] of
  * the given sequences, in host memory.  PA_EINVAL if an id is unknown or a table does not fit. */

@@ -36,7 +36,7 @@ EXPORTED = (
     "pa_paged_attention_noalloc", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
     "pa_bm_length", "pa_bm_tables", "pa_bm_stats", "pa_selftest_bounded_wait", "pa_bm_add_prompt",
-    "pa_bm_prefix_stats", "pa_bm_set_prefix_caching",
+    "pa_bm_prefix_stats", "pa_bm_set_prefix_caching", "pa_bm_commit", "pa_bm_block_size",
 )
 PA_ENOMEM = -6
 
@@ -87,7 +87,11 @@ def lib() -> ctypes.CDLL:
         L.pa_version.argtypes = []
         U64 = ctypes.c_uint64
         L.pa_bm_create.restype = P
-        L.pa_bm_create.argtypes = [I64, U64]
+        L.pa_bm_create.argtypes = [I64, I, U64]
+        L.pa_bm_block_size.restype = I
+        L.pa_bm_block_size.argtypes = [P]
+        L.pa_bm_commit.restype = I
+        L.pa_bm_commit.argtypes = [P, I64, I64]
         L.pa_bm_destroy.restype = None
         L.pa_bm_destroy.argtypes = [P]
         L.pa_bm_num_free.restype = I64
@@ -317,11 +321,21 @@ def pa_get_device_error(stream=None) -> int:
 # ------------------------------------------------------------------------------ host block manager
 # Same names as the C entry points; `bm` is the opaque handle pa_bm_create returns.
 
-def pa_bm_create(num_blocks: int, shuffle_seed: int = 0):
-    h = lib().pa_bm_create(int(num_blocks), int(shuffle_seed))
+def pa_bm_create(num_blocks: int, block_size: int = PA_BLOCK_SIZE, shuffle_seed: int = 0):
+    h = lib().pa_bm_create(int(num_blocks), int(block_size), int(shuffle_seed))
     if not h:
         raise PagedAttnError(PA_EINVAL, "pa_bm_create")
     return h
+
+
+def pa_bm_block_size(bm) -> int:
+    return int(lib().pa_bm_block_size(bm))
+
+
+def pa_bm_commit(bm, seq_id: int, tokens_written: int):
+    """Report the K/V of the first tokens_written tokens of seq_id written: its full prompt blocks within
+    them join the prefix tree."""
+    _check(lib().pa_bm_commit(bm, int(seq_id), int(tokens_written)), "pa_bm_commit")
 
 
 def pa_bm_destroy(bm):

@@ -35,13 +35,14 @@ def _oracle_rows(O, k_rows, v_rows, q_rows, lens):
     return O.paged_decode(q_rows, kc, vc, tables, np.asarray(lens, np.int32), SCALE)
 
 
-def test_block_manager_drives_append_prefill_decode(O, cuda_lib):
+@pytest.mark.parametrize("bs", [16, 32])
+def test_block_manager_drives_append_prefill_decode(O, cuda_lib, bs):
     B = cuda_lib
     g = torch.Generator(device="cuda").manual_seed(7)
-    nb = 256
-    kc = torch.zeros((nb, HKV, 16, D), dtype=torch.bfloat16, device="cuda")
+    nb = 256 * 16 // bs
+    kc = torch.zeros((nb, HKV, bs, D), dtype=torch.bfloat16, device="cuda")
     vc = torch.zeros_like(kc)
-    bm = B.pa_bm_create(nb, 99)
+    bm = B.pa_bm_create(nb, bs, 99)
     hist = {}                                   # request id -> (K rows, V rows) on the device
 
     def new_tokens(n):
@@ -60,7 +61,7 @@ def test_block_manager_drives_append_prefill_decode(O, cuda_lib):
     def prefill(rids, chunks):
         """Causal prefill of the chunks just appended to requests `rids`."""
         lens = [B.pa_bm_length(bm, r) for r in rids]
-        mbs = max((L + 15) // 16 for L in lens)
+        mbs = max((L + bs - 1) // bs for L in lens)
         tables, tl = B.pa_bm_tables(bm, rids, mbs)
         cu = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
         q = torch.randn((int(cu[-1]), HQ, D), generator=g, device="cuda").to(torch.bfloat16)
@@ -78,7 +79,7 @@ def test_block_manager_drives_append_prefill_decode(O, cuda_lib):
 
     def decode(rids):
         lens = [B.pa_bm_length(bm, r) for r in rids]
-        mbs = max((L + 15) // 16 for L in lens)
+        mbs = max((L + bs - 1) // bs for L in lens)
         tables, tl = B.pa_bm_tables(bm, rids, mbs)
         q = torch.randn((len(rids), HQ, D), generator=g, device="cuda").to(torch.bfloat16)
         out = torch.empty_like(q)
@@ -148,8 +149,12 @@ def test_cuda_graph_replay_matches_eager(cuda_lib):
 
 def test_prefix_tree_shared_blocks_feed_the_kernels(O, cuda_lib):
     """Two prompts with a common 40-token start: the second shares the first's two full blocks through
-    the block manager's prefix tree, appends K/V only for its own tokens, and its causal prefill over
-    the whole prompt (read through the shared blocks) matches the oracle on its own contiguous K/V."""
+    the block manager's prefix tree (once the first has committed them), appends K/V only for its own
+    tokens, and
+    - its causal prefill over the whole prompt (read through the shared blocks), and
+    - the prefill of only its new rows as one chunk whose history is the shared part (H = reused, the
+      flow a serving engine runs)
+    match the oracle on its own contiguous K/V."""
     B = cuda_lib
     g = torch.Generator(device="cuda").manual_seed(11)
     nb = 64
@@ -165,23 +170,33 @@ def test_prefix_tree_shared_blocks_feed_the_kernels(O, cuda_lib):
     v1 = torch.cat([common_v, rnd(25)])
     k2 = torch.cat([common_k, rnd(57)])
     v2 = torch.cat([common_v, rnd(57)])
-    bm = B.pa_bm_create(nb, 4)
+    bm = B.pa_bm_create(nb, 16, 4)
     try:
         s1, r1 = B.pa_bm_add_prompt(bm, 1, p1)
         B.pa_kv_append(kc, vc, k1, v1, torch.from_numpy(s1).cuda())
+        B.pa_bm_commit(bm, 1, len(p1))
         s2, r2 = B.pa_bm_add_prompt(bm, 2, p2)
         assert r1 == 0 and r2 == 32
         B.pa_kv_append(kc, vc, k2[r2:].contiguous(), v2[r2:].contiguous(), torch.from_numpy(s2).cuda())
+        B.pa_bm_commit(bm, 2, len(p2))
         n = len(p2)
         tables, tl = B.pa_bm_tables(bm, [2], (n + 15) // 16)
         q = torch.randn((n, HQ, D), generator=g, device="cuda").to(torch.bfloat16)
+        ref = _oracle_rows(O, bf16_bits(k2), bf16_bits(v2), bf16_bits(q), [i + 1 for i in range(n)])
+        # the whole prompt as one chunk (H = 0)
         out = torch.empty_like(q)
         cu = torch.tensor([0, n], dtype=torch.int32, device="cuda")
         B.pa_paged_prefill(out, q, cu, kc, vc, torch.from_numpy(tables).cuda(), torch.from_numpy(tl).cuda(),
                            SCALE, n, n)
+        # only the new rows r2 .. n-1, as one chunk over the shared history (H = r2)
+        qn = q[r2:].contiguous()
+        outn = torch.empty_like(qn)
+        cun = torch.tensor([0, n - r2], dtype=torch.int32, device="cuda")
+        B.pa_paged_prefill(outn, qn, cun, kc, vc, torch.from_numpy(tables).cuda(), torch.from_numpy(tl).cuda(),
+                           SCALE, n - r2, n)
         torch.cuda.synchronize()
         assert B.pa_get_device_error() == B.PA_OK
-        ref = _oracle_rows(O, bf16_bits(k2), bf16_bits(v2), bf16_bits(q), [i + 1 for i in range(n)])
         assert_close(to_f64(out), ref, what="prefill over prefix-shared blocks")
+        assert_close(to_f64(outn), ref[r2:], what="new rows over the shared history")
     finally:
         B.pa_bm_destroy(bm)
