@@ -73,28 +73,36 @@ double oracle_e4m3_decode(uint8_t code)
     return sign ? -v : v;
 }
 
+/* values of the 127 non-negative finite E4M3 codes 0x00 .. 0x7E, which ascend with the code */
+static double e4m3_pos_value[127];
+
+__attribute__((constructor)) static void e4m3_table_init(void)
+{
+    for (int c = 0; c < 127; ++c) e4m3_pos_value[c] = oracle_e4m3_decode((uint8_t)c);
+}
+
 /*
- * E4M3 encode of a binary32 value: round to nearest, ties to the code with an even
- * mantissa, saturating to +-448 (the largest finite magnitude).  Done by brute force
- * over the 127 non-negative finite codes, so it follows the definition rather than a
- * bit trick.  NaN maps to the NaN code 0x7F (sign kept).
+ * E4M3 encode of a binary32 value: round to nearest, ties to the code with an even mantissa,
+ * saturating to +-448 (the largest finite magnitude).  |x| is bracketed between two consecutive
+ * non-negative codes by bisection over their ascending values, then the nearer one is taken (on a tie
+ * the even one: consecutive codes differ in the last mantissa bit).  NaN maps to the NaN code 0x7F
+ * (sign kept).
  */
 uint8_t oracle_e4m3_encode(float x)
 {
     uint8_t sign = signbit(x) ? 0x80 : 0x00;
     double a = fabs((double)x);
-    int best = 0;
-    double best_err;
+    int lo = 0, hi = 126, best;
+    double below, above;
     if (isnan(x)) return (uint8_t)(sign | 0x7F);
     if (a >= 448.0) return (uint8_t)(sign | 0x7E); /* satfinite */
-    best_err = a; /* code 0 = +0 */
-    for (int c = 1; c < 0x7F; ++c) {
-        double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
-        if (err < best_err || (err == best_err && (c & 1) == 0 && (best & 1) == 1)) {
-            best = c;
-            best_err = err;
-        }
+    while (hi - lo > 1) { /* invariant: value[lo] <= a < value[hi] */
+        int mid = (lo + hi) / 2;
+        if (e4m3_pos_value[mid] <= a) lo = mid; else hi = mid;
     }
+    below = a - e4m3_pos_value[lo];
+    above = e4m3_pos_value[hi] - a;
+    best = (above < below || (above == below && (hi & 1) == 0)) ? hi : lo;
     return (uint8_t)(sign | best);
 }
 
@@ -143,13 +151,15 @@ int oracle_kv_append(void *k_cache, void *v_cache, const uint16_t *k, const uint
         if (slot < 0) continue;
         if (slot >= num_blocks * bs) return -4;
     }
-    for (int64_t n = 0; n < num_tokens; ++n) {
-        int64_t slot = slot_mapping[n];
-        int64_t blk, off;
-        if (slot < 0) continue;
-        blk = slot / bs;
-        off = slot % bs;
-        for (int h = 0; h < num_kv_heads; ++h) {
+    /* KV heads are disjoint parts of the cache: one thread per head, tokens in order within it */
+#pragma omp parallel for schedule(static)
+    for (int h = 0; h < num_kv_heads; ++h) {
+        for (int64_t n = 0; n < num_tokens; ++n) {
+            int64_t slot = slot_mapping[n];
+            int64_t blk, off;
+            if (slot < 0) continue;
+            blk = slot / bs;
+            off = slot % bs;
             int64_t src = (n * num_kv_heads + h) * (int64_t)head_dim;
             int64_t dst = ((blk * num_kv_heads + h) * bs + off) * (int64_t)head_dim;
             for (int d = 0; d < head_dim; ++d) {
@@ -237,20 +247,13 @@ static double cache_value(const void *cache, int kv_dtype, float scale, int64_t 
 }
 
 /*
- * Attention of one query vector over the first n_keys tokens of one sequence's paged
- * K/V (one KV head): the blocks are first gathered into contiguous [n_keys][D] arrays
- * (the block table "stitches the pages back together", vLLM overview, section 二), then
- *   s_t = scale * sum_d q_d K_td,  p = softmax(s),  o_d = sum_t p_t V_td
- * [KV Cache to vLLM §1.2; Core Concepts §3.1].  n_keys == 0 gives o = 0.
+ * Gather the first n_keys tokens of one sequence's paged K/V (one KV head) into contiguous [n_keys][D]
+ * arrays: the block table "stitches the pages back together" (vLLM overview, section 二).
  */
-static int attend_one(double *out, const uint16_t *q, const void *k_cache, const void *v_cache,
-                      int kv_dtype, float ks, float vs, const int32_t *table, int64_t n_keys,
-                      int num_kv_heads, int g, int head_dim, int64_t num_blocks, int bs, double scale,
-                      double *K, double *V, double *s)
+static int gather_kv(double *K, double *V, const void *k_cache, const void *v_cache, int kv_dtype, float ks,
+                     float vs, const int32_t *table, int64_t n_keys, int num_kv_heads, int g, int head_dim,
+                     int64_t num_blocks, int bs)
 {
-    double mx, sum;
-    for (int d = 0; d < head_dim; ++d) out[d] = 0.0;
-    if (n_keys == 0) return 0;
     for (int64_t t = 0; t < n_keys; ++t) {
         int64_t phys = table[t / bs];
         if (phys < 0 || phys >= num_blocks) return -4;
@@ -259,6 +262,21 @@ static int attend_one(double *out, const uint16_t *q, const void *k_cache, const
             V[t * head_dim + d] = cache_value(v_cache, kv_dtype, vs, phys, bs, num_kv_heads, g, t, head_dim, d);
         }
     }
+    return 0;
+}
+
+/*
+ * Attention of one query vector over the first n_keys rows of gathered K/V
+ * [KV Cache to vLLM §1.2; Core Concepts §3.1]:
+ *   s_t = scale * sum_d q_d K_td,  p = softmax(s),  o_d = sum_t p_t V_td.
+ * n_keys == 0 gives o = 0.
+ */
+static void attend_gathered(double *out, const uint16_t *q, const double *K, const double *V, int64_t n_keys,
+                            int head_dim, double scale, double *s)
+{
+    double mx, sum;
+    for (int d = 0; d < head_dim; ++d) out[d] = 0.0;
+    if (n_keys == 0) return;
     for (int64_t t = 0; t < n_keys; ++t) {
         double acc = 0.0;
         for (int d = 0; d < head_dim; ++d) acc += bf16_value(q[d]) * K[t * head_dim + d];
@@ -272,7 +290,6 @@ static int attend_one(double *out, const uint16_t *q, const void *k_cache, const
         double p = s[t] / sum;
         for (int d = 0; d < head_dim; ++d) out[d] += p * V[t * head_dim + d];
     }
-    return 0;
 }
 
 /*
@@ -306,11 +323,12 @@ int oracle_paged_decode(double *out, const uint16_t *q, const void *k_cache, con
             int b = (int)(bh / num_q_heads), h = (int)(bh % num_q_heads);
             int g = h / (num_q_heads / num_kv_heads);
             float ks = kv_dtype ? k_scale[g] : 1.0f, vs = kv_dtype ? v_scale[g] : 1.0f;
-            int r = attend_one(out + bh * head_dim, q + bh * head_dim, k_cache, v_cache, kv_dtype,
-                               ks, vs, block_tables + (int64_t)b * max_blocks_per_seq,
-                               context_lens[b], num_kv_heads, g, head_dim, num_blocks, bs, scale,
-                               K, V, s);
+            int r = gather_kv(K, V, k_cache, v_cache, kv_dtype, ks, vs,
+                              block_tables + (int64_t)b * max_blocks_per_seq, context_lens[b],
+                              num_kv_heads, g, head_dim, num_blocks, bs);
             if (r < status) status = r;
+            if (r == 0)
+                attend_gathered(out + bh * head_dim, q + bh * head_dim, K, V, context_lens[b], head_dim, scale, s);
         }
         free(K);
         free(V);
@@ -333,7 +351,7 @@ int oracle_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q_len
                          int num_kv_heads, int head_dim, int64_t num_blocks, int bs, double scale,
                          int kv_dtype, const float *k_scale, const float *v_scale)
 {
-    int64_t max_len = 0, total_q;
+    int64_t max_len = 0;
     int status = 0;
     if (num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0) return -1;
     if (num_q_heads % num_kv_heads != 0) return -1;
@@ -343,28 +361,29 @@ int oracle_paged_prefill(double *out, const uint16_t *q, const int32_t *cu_q_len
         if ((context_lens[c] + bs - 1) / bs > max_blocks_per_seq) return -1;
         if (context_lens[c] > max_len) max_len = context_lens[c];
     }
-    total_q = num_chunks > 0 ? cu_q_lens[num_chunks] : 0;
 #pragma omp parallel reduction(min : status)
     {
         double *K = (double *)malloc(sizeof(double) * (size_t)(max_len + 1) * head_dim);
         double *V = (double *)malloc(sizeof(double) * (size_t)(max_len + 1) * head_dim);
         double *s = (double *)malloc(sizeof(double) * (size_t)(max_len + 1));
+        /* per (chunk, query head): the chunk's context is gathered once; row i then attends over its
+         * first hist + i + 1 keys */
 #pragma omp for schedule(dynamic)
-        for (int64_t ih = 0; ih < total_q * num_q_heads; ++ih) {
-            int64_t row = ih / num_q_heads;
-            int h = (int)(ih % num_q_heads);
+        for (int64_t ch = 0; ch < (int64_t)num_chunks * num_q_heads; ++ch) {
+            int c = (int)(ch / num_q_heads), h = (int)(ch % num_q_heads);
             int g = h / (num_q_heads / num_kv_heads);
-            int c = 0;
-            int64_t hist, i;
             float ks = kv_dtype ? k_scale[g] : 1.0f, vs = kv_dtype ? v_scale[g] : 1.0f;
-            int r;
-            while (cu_q_lens[c + 1] <= row) ++c;
-            i = row - cu_q_lens[c];
-            hist = context_lens[c] - (cu_q_lens[c + 1] - cu_q_lens[c]);
-            r = attend_one(out + ih * head_dim, q + ih * head_dim, k_cache, v_cache, kv_dtype, ks, vs,
-                           block_tables + (int64_t)c * max_blocks_per_seq, hist + i + 1,
-                           num_kv_heads, g, head_dim, num_blocks, bs, scale, K, V, s);
+            int64_t C = cu_q_lens[c + 1] - cu_q_lens[c];
+            int64_t hist = context_lens[c] - C;
+            int r = gather_kv(K, V, k_cache, v_cache, kv_dtype, ks, vs,
+                              block_tables + (int64_t)c * max_blocks_per_seq, context_lens[c],
+                              num_kv_heads, g, head_dim, num_blocks, bs);
             if (r < status) status = r;
+            for (int64_t i = 0; r == 0 && i < C; ++i) {
+                int64_t ih = (cu_q_lens[c] + i) * num_q_heads + h;
+                attend_gathered(out + ih * head_dim, q + ih * head_dim, K, V,
+                                hist + i + 1, head_dim, scale, s);
+            }
         }
         free(K);
         free(V);

@@ -26,7 +26,7 @@ MUTANTS = {
     "softmax not normalised": ("double p = s[t] / sum;", "double p = s[t];"),
     "max not subtracted in sum": ("s[t] = exp(s[t] - mx); sum += s[t];", "s[t] = exp(s[t] - mx); sum += exp(s[t]);"),
     "E4M3 bias 6": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 6);"),
-    "E4M3 ties to odd": ("(c & 1) == 0 && (best & 1) == 1", "(c & 1) == 1 && (best & 1) == 0"),
+    "E4M3 ties to odd": ("(above == below && (hi & 1) == 0)", "(above == below && (hi & 1) == 1)"),
     "E4M3 no saturation": ("if (a >= 448.0) return (uint8_t)(sign | 0x7E);", "if (a >= 480.0) return (uint8_t)(sign | 0x7F);"),
     "KV bytes without K+V factor": ("return 2 * layers * kv_heads", "return layers * kv_heads"),
     "copy forgets V": ("        memmove((char *)v_cache + d * block_bytes, (char *)v_cache + s * block_bytes, block_bytes);\n", ""),
@@ -36,10 +36,10 @@ MUTANTS = {
                                     "return oracle_e4m3_decode(((const uint8_t *)cache)[idx]);"),
     "INT8 dequant drops the scale": ("return (double)((const int8_t *)cache)[idx] * (double)scale;",
                                      "return (double)((const int8_t *)cache)[idx];"),
-    "decode V uses k_scale": ("vs = kv_dtype ? v_scale[g] : 1.0f;\n            int r = attend_one",
-                              "vs = kv_dtype ? k_scale[g] : 1.0f;\n            int r = attend_one"),
-    "prefill V uses k_scale": ("vs = kv_dtype ? v_scale[g] : 1.0f;\n            int r;",
-                               "vs = kv_dtype ? k_scale[g] : 1.0f;\n            int r;"),
+    "decode V uses k_scale": ("vs = kv_dtype ? v_scale[g] : 1.0f;\n            int r = gather_kv",
+                              "vs = kv_dtype ? k_scale[g] : 1.0f;\n            int r = gather_kv"),
+    "prefill V uses k_scale": ("vs = kv_dtype ? v_scale[g] : 1.0f;\n            int64_t C",
+                               "vs = kv_dtype ? k_scale[g] : 1.0f;\n            int64_t C"),
     "swap copies K into V": ("memcpy((char *)dst_v + d * block_bytes, (const char *)src_v + s * block_bytes",
                              "memcpy((char *)dst_v + d * block_bytes, (const char *)src_k + s * block_bytes"),
 }
