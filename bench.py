@@ -1,19 +1,26 @@
 """Benchmark of one paged-attention serving step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--partition replicas|kv_heads]
+                    [--impl ours|reference]
 
-A step is one pass of the hot path over one batch: copy-on-write forks (when the workload
-has shared prefixes), kv_append of every new token, paged decode attention (split-K + LSE
-reduce) and paged prefill (when the workload has prefill chunks).  The default workload is the
-Llama-3-8B-shaped decode batch (64 sequences, 32 query / 8 KV heads, head_dim 128, 16-token
-blocks, contexts uniform in [513, 4097] after the append, blocks shuffled over a pool 1.25x the
-need).  Inputs are seeded synthetic data; every input is resident in HBM before timing and
-the KV pool (about 1.2 GB) is larger than L2, so every step streams the cache from HBM.
+A step is one pass of the hot path over one batch: copy-on-write forks (when the workload has shared
+prefixes), kv_append of every new token, paged decode attention (split-K + LSE reduce) and paged prefill
+(when the workload has prefill chunks).  The default workload is the Llama-3-8B-shaped decode batch (64
+sequences, 32 query / 8 KV heads, head_dim 128, 16-token blocks, contexts uniform in [513, 4097] after the
+append, blocks shuffled over a pool 1.25x the need).  Inputs are seeded synthetic data, resident in HBM
+before timing; every KV pool is larger than the 126 MB L2, so each step streams the cache from HBM.
 
-metric: KV-read HBM GB/s = algorithmic bytes of the decode attention (every cached K and V
-element once, plus q, out, tables and lengths) / step time, summed over ranks.
-One JSON line on rank 0.  With --impl reference the CPU oracle is timed instead on a bounded
-sample of the same workload (rank 0 only).
+metric: KV-read HBM GB/s = algorithmic bytes of the decode attention (every cached K and V element once,
+plus q, out, tables and lengths) / step time, summed over ranks.  One JSON line on rank 0.  At one GPU the
+line also carries, under "workloads", the other three full-size workloads (the continuous-batching mixed
+step, the long-context batch, the MHA batch over an FP8 cache), each timed the same way with its own
+fraction of the roofline.
+
+--gpus N launches N ranks itself (one process per GPU) unless it already runs under torchrun.
+--partition replicas: every rank runs the whole batch on its own pool (weak scaling, no collective);
+kv_heads: rank r holds KV heads [r*Hkv/N, (r+1)*Hkv/N) of every block and the query heads that use them
+(tensor parallelism, strong scaling); attention needs no exchange between ranks either way.
+--impl reference: the CPU oracle timed on a bounded sample of the same workload (rank 0 only).
 """
 from __future__ import annotations
 
@@ -21,6 +28,7 @@ import argparse
 import json
 import os
 import statistics
+import subprocess
 import sys
 import threading
 import time
@@ -33,18 +41,33 @@ sys.path.insert(0, ROOT)
 
 METRIC = "paged-attn decode: KV-read HBM GB/s (% of peak), sequence-steps/s"
 DEFAULT_WORKLOAD = "llama3_8b_decode"
+SUB_WORKLOADS = ("mixed_step", "long_context_decode", "mha_fp8_decode")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ----------------------------------------------------------------------------- helpers
 
-def peaks():
+def _peaks_file():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
-            d = json.load(f)
+            return json.load(f)
+    return None
+
+
+def peaks():
+    d = _peaks_file()
+    if d and "hbm_gbs" in d:
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def bf16_peak():
+    d = _peaks_file()
+    if d and "bf16_tflops" in d:
+        return float(d["bf16_tflops"]), "measured (burst)"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def decode_bytes(batch) -> int:
@@ -70,14 +93,6 @@ def prefill_flops(batch) -> int:
     return 4 * batch.head_dim * batch.num_q_heads * tot
 
 
-def bf16_peak():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
-    return 1590.0, "fallback"
-
-
 def kv_unique_bytes(batch) -> int:
     """Bytes of the distinct cache slots the decode reads: a prefix block shared by several sequences
     counts once (it is stored once in HBM; the other readers can be served from L2)."""
@@ -99,8 +114,19 @@ def kv_bytes(batch) -> int:
     return int(batch.context_lens[:nd].astype(np.int64).sum()) * 2 * batch.num_kv_heads * batch.head_dim * e
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 class ClockSampler:
-    """Polls SM clock, max clock and throttle reasons through NVML while the timed region runs."""
+    """Polls SM clock, max clock and throttle reasons through NVML while the timed regions run."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -108,10 +134,11 @@ class ClockSampler:
         0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
     }
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.max_mhz = [], 0, None
         self.period = period_s
         self._stop = threading.Event()
+        self._on = threading.Event()
         self.ok = False
         try:
             import pynvml
@@ -125,12 +152,25 @@ class ClockSampler:
 
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
-            except Exception:
-                pass
+            if self._on.is_set():
+                try:
+                    self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                    self.reasons |= int(self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+                except Exception:
+                    pass
             time.sleep(self.period)
+
+    def timed(self):
+        """Context manager: sample only while a timed region runs."""
+        sampler = self
+
+        class _T:
+            def __enter__(self):
+                sampler._on.set()
+
+            def __exit__(self, *a):
+                sampler._on.clear()
+        return _T()
 
     def __enter__(self):
         if self.ok:
@@ -169,11 +209,11 @@ def traffic_record(kernel_tag: str):
         return None
 
 
-def combine_over_ranks(times_ms: dict, bytes_per_step: int, world: int, device) -> dict:
+def combine_over_ranks(times_ms: dict, work_per_step: float, world: int, device) -> dict:
     """Whole-job figures from every rank's own timings: each time is the MAX over ranks (the job is
-    as slow as its slowest replica) and the work is the SUM of the ranks' bytes per step."""
+    as slow as its slowest rank) and the work is the SUM of the ranks' work per step."""
     keys = sorted(times_ms)
-    t = torch.tensor([float(times_ms[k]) for k in keys] + [float(bytes_per_step)], dtype=torch.float64,
+    t = torch.tensor([float(times_ms[k]) for k in keys] + [float(work_per_step)], dtype=torch.float64,
                      device=device)
     if world > 1:
         mx = t[:-1].clone()
@@ -184,6 +224,54 @@ def combine_over_ranks(times_ms: dict, bytes_per_step: int, world: int, device) 
     out = {k: float(v) for k, v in zip(keys, t[:-1].tolist())}
     out["bytes"] = float(t[-1])
     return out
+
+
+def graph_steps(K: int) -> int:
+    """Steps per captured CUDA graph: the largest of 10, 8, 5, 4, 2, 1 that divides K."""
+    return next(g for g in (10, 8, 5, 4, 2, 1) if K % g == 0)
+
+
+def capture(fn, G: int, dev):
+    """A CUDA graph of G calls of fn (the library's launches keep their programmatic dependencies), or
+    None if capture is refused."""
+    try:
+        graph = torch.cuda.CUDAGraph()
+        # thread_local: the capture rules apply to this thread only, not to NCCL's helper threads
+        with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev), capture_error_mode="thread_local"):
+            for _ in range(G):
+                fn()
+        torch.cuda.synchronize(dev)
+        for _ in range(2):
+            graph.replay()
+        torch.cuda.synchronize(dev)
+        return graph
+    except RuntimeError as e:
+        print(f"bench: CUDA graph capture failed ({e}); timing stream launches", file=sys.stderr)
+        torch.cuda.synchronize(dev)
+        return None
+
+
+def time_calls(fn, K: int, dev, use_graph: bool, clk) -> tuple:
+    """Average ms of one call of fn over K calls run back to back (from CUDA graphs of several calls when
+    use_graph), timed with CUDA events on the launching stream, synchronised on both sides."""
+    G = graph_steps(K) if use_graph else 0
+    graph = capture(fn, G, dev) if G else None
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    with clk.timed():
+        e0.record(stream)
+        if graph is not None:
+            for _ in range(K // G):
+                graph.replay()
+        else:
+            for _ in range(K):
+                fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+    how = f"CUDA graph of {G} calls, replayed" if graph is not None else "stream launches"
+    del graph
+    return e0.elapsed_time(e1) / K, how
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -199,116 +287,136 @@ def workload_config(name, batch) -> dict:
     }
 
 
-def run_ours(args, rank, world, local_rank):
+def rank_batch(full, rank: int, world: int, partition: str):
+    """The part of the workload rank `rank` of `world` runs: all of it (replicas), or its KV heads of every
+    block and the query heads that use them (kv_heads, tensor parallelism)."""
+    if partition == "kv_heads" and world > 1:
+        from pagedattention_block_table_b200 import sharding
+        return sharding.shard_batch(full, rank, world)
+    if partition not in ("replicas", "kv_heads"):
+        raise ValueError(partition)
+    return full
+
+
+def launches_per_step(st) -> int:
+    """Kernels of this library one step launches: fork, append, decode, LSE reduce, prefill (when present)."""
+    b = st.batch
+    return ((1 if b.cow_pairs.shape[0] else 0) + 1 + (1 if b.num_decode else 0)
+            + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0))
+
+
+def measure(name, dev, K, W, args, rank, world, clk, e2e=False):
+    """Time one workload on this rank: the whole step, the decode call alone and the prefill call alone
+    (each from CUDA graphs of back-to-back calls), and optionally the end-to-end host-fed step."""
     from pagedattention_block_table_b200 import binding as B
     from pagedattention_block_table_b200.inputs import make_batch
-    from pagedattention_block_table_b200.runner import DeviceStep
+    from pagedattention_block_table_b200.runner import DeviceStep, HostPipeline
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    B.lib()
-    batch = make_batch(args.workload, device=dev)
+    full = make_batch(name, device=dev)
+    batch = rank_batch(full, rank, world, args.partition)
     st = DeviceStep(batch, device=dev, split_tokens=args.split or None)
     st.fill_history()
     torch.cuda.synchronize(dev)
-    stream = torch.cuda.current_stream(dev)
-
-    launches = (1 if batch.cow_pairs.shape[0] else 0) + 1 + (1 if batch.num_decode else 0) \
-        + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0)
-
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, W)):
         st.step()
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-
-    K = args.steps
-    ev0 = torch.cuda.Event(enable_timing=True)
-    ev1 = torch.cuda.Event(enable_timing=True)
-    d0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    d1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    p1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    # The step value replays the K steps from CUDA graphs of G steps each, so that the Python launch path
-    # (ctypes marshalling, the GIL shared with the clock sampler) cannot leave gaps between kernels.  The
-    # graph holds the same launches as st.step(), with their programmatic (PDL) dependencies.
-    G = next(g for g in (10, 8, 5, 4, 2, 1) if K % g == 0) if not args.no_graph else 0
-    graph = None
-    if G:
-        try:
-            graph = torch.cuda.CUDAGraph()
-            # thread_local: the capture rules apply to this thread only, not to NCCL's helper threads
-            with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev), capture_error_mode="thread_local"):
-                for _ in range(G):
-                    st.step()
-            torch.cuda.synchronize(dev)
-            for _ in range(2):
-                graph.replay()
-            torch.cuda.synchronize(dev)
-        except RuntimeError as e:            # capture refused: time stream launches instead, and say so
-            print(f"bench: CUDA graph capture failed ({e}); timing stream launches", file=sys.stderr)
-            graph, G = None, 0
-            torch.cuda.synchronize(dev)
-    with ClockSampler(local_rank) as clk:
-        # the step value: K steps back to back, no event between the kernels (an event record between
-        # two launches ends the programmatic overlap of the second with the first)
-        torch.cuda.synchronize(dev)
-        ev0.record(stream)
-        if graph is not None:
-            for _ in range(K // G):
-                graph.replay()
-        else:
-            for i in range(K):
-                st.step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        # the same K steps again with events around each attention call: the kernels' own durations
-        for i in range(K):
-            st.fork()
-            st.append()
-            d0[i].record(stream)
-            st.decode()
-            d1[i].record(stream)
-            st.prefill()
-            p1[i].record(stream)
-        torch.cuda.synchronize(dev)
+    use_graph = not args.no_graph
+    step_ms, launch = time_calls(st.step, K, dev, use_graph, clk)
+    dec_ms = time_calls(st.decode, K, dev, use_graph, clk)[0] if batch.num_decode else 0.0
+    pre_ms = time_calls(st.prefill, K, dev, use_graph, clk)[0] if st.max_q else 0.0
     if world > 1:
         torch.distributed.barrier()
-    step_ms = ev0.elapsed_time(ev1) / K
-    dec_ms = sum(a.elapsed_time(b) for a, b in zip(d0, d1)) / K
-    pre_ms = sum(a.elapsed_time(b) for a, b in zip(d1, p1)) / K
     if B.pa_get_device_error() != B.PA_OK:
-        raise RuntimeError("device error flagged during the timed region")
+        raise RuntimeError(f"device error flagged while timing {name}")
+    res = dict(batch=batch, full=full, st=st, step_ms=step_ms, dec_ms=dec_ms, pre_ms=pre_ms, launch=launch)
+    if e2e:
+        # end to end through the public API: every step copies its inputs in from pinned host memory and
+        # its outputs back out; a copy stream overlaps those copies with the neighbouring steps' compute
+        pipe = HostPipeline(st)
+        for _ in range(max(3, W)):
+            pipe.step()
+        pipe.finish()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        K2 = max(1, min(K, 500))
+        stream = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with clk.timed():
+            e0.record(stream)
+            for _ in range(K2):
+                pipe.step()
+            pipe.finish()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        res.update(e2e_ms=e0.elapsed_time(e1) / K2, h2d=pipe.h2d_bytes, d2h=pipe.d2h_bytes)
+        if B.pa_get_device_error() != B.PA_OK:
+            raise RuntimeError(f"device error flagged in the end-to-end leg of {name}")
+    return res
 
-    # end to end through the public API: every step copies its inputs in from pinned host memory and
-    # its outputs back out; a copy stream overlaps those copies with the neighbouring steps' compute
-    from pagedattention_block_table_b200.runner import HostPipeline
-    pipe = HostPipeline(st)
-    h2d, d2h = pipe.h2d_bytes, pipe.d2h_bytes
-    for _ in range(max(3, args.warmup)):
-        pipe.step()
-    pipe.finish()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        torch.distributed.barrier()
-    K2 = max(1, min(K, 500))
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K2):
-        pipe.step()
-    pipe.finish()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / K2
 
-    dbytes = decode_bytes(batch)
-    kvb = kv_bytes(batch)
-    agg = combine_over_ranks({"step_ms": step_ms, "dec_ms": dec_ms, "e2e_ms": e2e_ms}, dbytes, world, dev)
+def sub_record(name, dev, args, clk):
+    """The workloads sub-record of one more full-size workload at one GPU: decode GB/s (logical and unique
+    bytes) and prefill TFLOP/s, each against its measured peak."""
+    K = max(10, min(args.steps, args.sub_steps))
+    m = measure(name, dev, K, args.warmup, args, 0, 1, clk)
+    batch, st = m["batch"], m["st"]
+    peak, peak_kind = peaks()
+    rec = {"config": {**workload_config(name, batch), "split_tokens": st.split_tokens}, "steps": K,
+           "ms_per_step": round(m["step_ms"], 5), "launch": m["launch"]}
+    if batch.num_decode:
+        db, kvb, kvu = decode_bytes(batch), kv_bytes(batch), kv_unique_bytes(batch)
+        ach = db / (m["dec_ms"] * 1e-3) / 1e9
+        rec["decode"] = {
+            "kernel": "pa_paged_attention (paged_decode_kernel + lse_reduce_kernel)", "bound": "hbm",
+            "unit": "GB/s", "achieved": round(ach, 2), "peak": peak, "peak_kind": peak_kind,
+            "frac": round(ach / peak, 4), "avg_launch_ms": round(m["dec_ms"], 5), "algorithmic_bytes": db,
+            "dtype": {0: "bf16", 1: "fp8_e4m3", 2: "int8"}[batch.kv_dtype],
+        }
+        if kvu != kvb:
+            au = (db - kvb + kvu) / (m["dec_ms"] * 1e-3) / 1e9
+            rec["decode"].update(achieved_unique=round(au, 2), frac_unique=round(au / peak, 4),
+                                 unique_bytes=db - kvb + kvu)
+    if st.max_q:
+        pf = prefill_flops(batch)
+        tp, tk = bf16_peak()
+        ach = pf / (m["pre_ms"] * 1e-3) / 1e12
+        rec["prefill"] = {"kernel": "paged_prefill_kernel (tcgen05)", "bound": "tensor", "unit": "TFLOP/s",
+                          "achieved": round(ach, 2), "peak": tp, "peak_kind": tk, "frac": round(ach / tp, 4),
+                          "flops": pf, "avg_launch_ms": round(m["pre_ms"], 5)}
+    del m, st, batch
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_ours(args, rank, world, local_rank):
+    from pagedattention_block_table_b200 import binding as B
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B.lib()
+    K = args.steps
+    with ClockSampler(local_rank) as clk:
+        m = measure(args.workload, dev, K, args.warmup, args, rank, world, clk, e2e=True)
+        batch, st = m["batch"], m["st"]
+        dbytes = decode_bytes(batch)
+        kvb = kv_bytes(batch)
+        agg = combine_over_ranks({"step_ms": m["step_ms"], "dec_ms": m["dec_ms"], "e2e_ms": m["e2e_ms"],
+                                  "pre_ms": m["pre_ms"]}, dbytes, world, dev)
+        subs = {}
+        if world == 1 and not args.no_workloads and args.workload == DEFAULT_WORKLOAD:
+            for name in SUB_WORKLOADS:
+                subs[name] = sub_record(name, dev, args, clk)
     step_ms, dec_ms, e2e_ms = agg["step_ms"], agg["dec_ms"], agg["e2e_ms"]
     peak, peak_kind = peaks()
     value = agg["bytes"] / (step_ms * 1e-3) / 1e9
     achieved = dbytes / (dec_ms * 1e-3) / 1e9
     tr = traffic_record(f"decode/{args.workload}")
+    kvu = kv_unique_bytes(batch)
+    scaling = "strong" if args.partition == "kv_heads" and world > 1 else "weak"
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -318,45 +426,52 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup,
         "ms_per_step": round(step_ms, 5),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": scaling,
         "vs_baseline": None,
         "dtype": {0: "bf16", 1: "fp8_e4m3 KV, bf16 q/out, fp32 accumulate",
                   2: "int8 KV, bf16 q/out, fp32 accumulate"}[batch.kv_dtype],
         "data": "synthetic",
         "config": {
-            **workload_config(args.workload, batch),
+            **workload_config(args.workload, m["full"]),
             "split_tokens": st.split_tokens,
-            "launch": f"CUDA graph of {G} steps, replayed" if G else "stream launches",
+            "launch": m["launch"],
             "l2": "inputs larger than L2: KV pool %.2f GB vs 126 MB" % (2 * st.k_cache.numel() * st.k_cache.element_size() / 1e9),
-            "parallelism": f"replicas x{world}",
+            "parallelism": (f"kv_heads x{world} (tensor parallel: {batch.num_kv_heads} of "
+                            f"{m['full'].num_kv_heads} KV heads per rank)") if scaling == "strong"
+            else f"replicas x{world}",
         },
         "pct_of_peak": round(100 * value / world / peak, 2),
         "pct_of_spec_8000_gbs": round(100 * value / world / 8000.0, 2),   # B200 HBM3e datasheet figure
-        "seq_steps_per_s": round(world * batch.num_decode / (step_ms * 1e-3), 1),
+        "seq_steps_per_s": round((world if scaling == "weak" else 1) * batch.num_decode / (step_ms * 1e-3), 1),
         "decode_kv_bytes_per_step": kvb,
-        "decode_kv_unique_bytes_per_step": kv_unique_bytes(batch),
+        "decode_kv_unique_bytes_per_step": kvu,
         "roofline": {
             "kernel": "pa_paged_attention (paged_decode_kernel + lse_reduce_kernel)",
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "traffic": None if tr is None else tr.get("bytes_per_launch"),
             "algorithmic_bytes": dbytes, "avg_launch_ms": round(dec_ms, 5),
-            "achieved_unique": round((dbytes - kvb + kv_unique_bytes(batch)) / (dec_ms * 1e-3) / 1e9, 2),
+            "timing": "decode calls alone, " + m["launch"],
+            "achieved_unique": round((dbytes - kvb + kvu) / (dec_ms * 1e-3) / 1e9, 2),
         },
         "e2e": {"value": round(agg["bytes"] / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": launches * K,
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": int(m["h2d"]),
+                "d2h_bytes_per_step": int(m["d2h"])},
+        "gpu_launches": launches_per_step(st) * K,
         "clocks": clk.summary(),
     }
     if st.max_q:
         pf = prefill_flops(batch)
-        tf_peak = bf16_peak()
+        tp, tk = bf16_peak()
+        pre_ms = agg["pre_ms"]
         line["prefill"] = {"kernel": "paged_prefill_kernel (tcgen05)", "bound": "tensor", "unit": "TFLOP/s",
-                           "achieved": round(pf / (pre_ms * 1e-3) / 1e12, 2), "peak": tf_peak[0],
-                           "peak_kind": tf_peak[1], "frac": round(pf / (pre_ms * 1e-3) / 1e12 / tf_peak[0], 4),
-                           "flops": pf, "avg_launch_ms": round(pre_ms, 5)}
+                           "achieved": round(pf / (pre_ms * 1e-3) / 1e12, 2), "peak": tp, "peak_kind": tk,
+                           "frac": round(pf / (pre_ms * 1e-3) / 1e12 / tp, 4), "flops": pf,
+                           "avg_launch_ms": round(pre_ms, 5)}
+    if subs:
+        line["workloads"] = subs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(batch, args.cpu_sample_seqs)
+        line["cpu_baseline"] = cpu_baseline(batch, args.cpu_budget_s)
     return line
 
 
@@ -408,25 +523,39 @@ def _oracle_run(batch, smp):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(batch, nseq, budget_s=15.0):
-    """The oracle on the host cores: append + decode, one (sequence, KV head) unit at a time in order,
-    until `nseq` sequences are done or about `budget_s` seconds of oracle work have been spent."""
+def cpu_baseline(batch, budget_s=4.0):
+    """The oracle on the host cores: append + decode of (sequence, KV head) units in order.  The sample is
+    the units one all-core pass reaches in about `budget_s` seconds; it is run three times on all cores
+    (median reported) and its first 1/cores part once on one core (scaled to the same unit)."""
     from oracle import oracle as O
-    done_bytes, secs, units, tokens = 0, 0.0, 0, 0
-    for s in range(min(nseq, batch.num_decode)):
-        for g in range(batch.num_kv_heads):
-            smp = _oracle_sample(batch, 1, first=s, kv_head=g)
-            secs += _oracle_run(batch, smp)
-            done_bytes += smp["kv_bytes"]
-            units += 1
-            tokens += int(smp["lens"].sum())
-            if secs >= budget_s:
-                break
+    cores = O.num_threads()
+    units = [(s, g) for s in range(batch.num_decode) for g in range(batch.num_kv_heads)]
+    samples = [_oracle_sample(batch, 1, first=s, kv_head=g) for s, g in units[:4096]]
+    n, secs, nbytes = 0, 0.0, 0
+    for smp in samples:                       # pass 1 sizes the sample
+        secs += _oracle_run(batch, smp)
+        nbytes += smp["kv_bytes"]
+        n += 1
         if secs >= budget_s:
             break
-    return {"value": round(done_bytes / secs / 1e9, 4), "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
-            "sample": f"append + decode of the first {units} (sequence, KV head) units of {batch.num_decode} x "
-                      f"{batch.num_kv_heads} ({tokens} token-heads), fp64, {secs:.2f} s of oracle time"}
+    runs = [secs]
+    for _ in range(2):
+        runs.append(sum(_oracle_run(batch, smp) for smp in samples[:n]))
+    med = statistics.median(runs)
+    n1 = max(1, n // max(1, cores))
+    O.set_num_threads(1)
+    try:
+        t1 = sum(_oracle_run(batch, smp) for smp in samples[:n1])
+    finally:
+        O.set_num_threads(cores)
+    b1 = sum(smp["kv_bytes"] for smp in samples[:n1])
+    tokens = int(sum(int(smp["lens"].sum()) for smp in samples[:n]))
+    return {"value": round(nbytes / med / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "cpu_model": cpu_model(), "runs": 3, "run_s": [round(r, 3) for r in runs],
+            "value_1core": round(b1 / t1 / 1e9, 4),
+            "sample": f"append + decode of the first {n} (sequence, KV head) units of {batch.num_decode} x "
+                      f"{batch.num_kv_heads} ({tokens} token-heads), fp64, median of 3 all-core runs; "
+                      f"1 core: the first {n1} units"}
 
 
 def run_reference(args, rank, world):
@@ -454,6 +583,7 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {**workload_config(args.workload, batch), "sample_seqs": len(smp["lens"])},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
+                         "cpu_model": cpu_model(),
                          "sample": f"append + decode of {len(smp['lens'])} of {batch.num_decode} sequences per step"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -506,30 +636,58 @@ def run_swap(args):
             "frac_out": round(t_d2h / t_out, 3), "frac_in": round(t_h2d / t_in, 3), "steps": K}
 
 
-# ----------------------------------------------------------------------------- main
+# ----------------------------------------------------------------------------- launch
 
-def main():
+def _free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def relaunch_command(argv, n: int, port: int) -> list:
+    """The torchrun command that runs this script on n local ranks with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+
+
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--partition", choices=["replicas", "kv_heads"], default="replicas",
+                    help="N>1: whole batch per rank (weak scaling) or KV heads split over the ranks (strong)")
     ap.add_argument("--split", type=int, default=0, help="split_tokens (0 = library default)")
     ap.add_argument("--no-graph", action="store_true", help="time the steps as stream launches, not graph replays")
-    ap.add_argument("--cpu-sample-seqs", type=int, default=16)
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other full-size workloads at N=1")
+    ap.add_argument("--sub-steps", type=int, default=50, help="timed steps of each of the other workloads")
+    ap.add_argument("--cpu-budget-s", type=float, default=4.0)
     ap.add_argument("--ref-sample-seqs", type=int, default=4)
     ap.add_argument("--ref-max-steps", type=int, default=20)
     ap.add_argument("--ref-budget-s", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mode", choices=["step", "swap"], default="step",
                     help="step: the hot-path step (default); swap: KV eviction throughput")
-    args = ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def main():
+    args = parse_args()
     if args.mode == "swap":
         print(json.dumps(run_swap(args)), flush=True)
         return
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # one process per GPU: launch the ranks ourselves
+        if args.gpus > torch.cuda.device_count():
+            raise SystemExit(f"bench: --gpus {args.gpus} but only {torch.cuda.device_count()} CUDA devices visible")
+        cmd = relaunch_command(sys.argv[1:], args.gpus, _free_port())
+        raise SystemExit(subprocess.call(["timeout", "-k", "60", "1800", *cmd]))
+    if args.gpus != world:
+        raise SystemExit(f"bench: --gpus {args.gpus} but WORLD_SIZE={world}")
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":

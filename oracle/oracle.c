@@ -402,3 +402,14 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* run the following calls on n OpenMP threads (for timing the oracle on one core and on all) */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

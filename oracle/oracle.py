@@ -48,6 +48,8 @@ def configure(lib):
     lib.oracle_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, L, I, D, I, P, P]
     lib.oracle_num_threads.restype = I
     lib.oracle_num_threads.argtypes = []
+    lib.oracle_set_num_threads.restype = None
+    lib.oracle_set_num_threads.argtypes = [I]
     return lib
 
 
@@ -77,6 +79,11 @@ def _check(rc, what):
 
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Run later oracle calls on n OpenMP threads."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def kv_cache_bytes(layers, kv_heads, head_dim, seq_len, batch, elem_bytes) -> int:

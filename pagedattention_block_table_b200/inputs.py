@@ -331,8 +331,9 @@ def make_batch(name: str, *, seed: Optional[int] = None, device="cpu", perm_seed
     if kv_dtype:
         # one fp32 scale per KV head (and per K/V tensor): absmax of the seeded data / largest code
         top = E4M3_MAX if kv_dtype == 1 else INT8_MAX
-        k_scale = (tok_k.float().abs().amax(dim=(0, 2)) / top).to(torch.float32)
-        v_scale = (tok_v.float().abs().amax(dim=(0, 2)) / top).to(torch.float32)
+        # (abs and max are exact in bf16, so the absmax is taken before widening to fp32)
+        k_scale = (tok_k.abs().amax(dim=(0, 2)).float() / top).to(torch.float32)
+        v_scale = (tok_v.abs().amax(dim=(0, 2)).float() / top).to(torch.float32)
 
     return PagedBatch(
         name=name, num_q_heads=hq, num_kv_heads=hkv, head_dim=D, num_blocks=num_blocks,

@@ -90,3 +90,32 @@ def oracle_attend_prefix(batch: PagedBatch, s: int, L: int, q_bits: np.ndarray, 
     n = q_bits.shape[0]
     tables = np.tile(np.arange(nblk, dtype=np.int32)[None], (n, 1))
     return O.paged_decode(q_bits, kc, vc, tables, np.full(n, L, np.int32), batch.scale)
+
+
+def oracle_decode_all(batch: PagedBatch, O, kv_dtype=None) -> np.ndarray:
+    """Oracle decode of every decoding sequence, [num_decode][Hq][D] fp64, each from its own token rows in
+    a fresh contiguous cache (the plain definition: no paging, no sharing, no forks)."""
+    return np.stack([oracle_decode_one(batch, s, O, kv_dtype) for s in range(batch.num_decode)])
+
+
+def oracle_prefill_all(batch: PagedBatch, O) -> np.ndarray:
+    """Oracle causal attention of every prefill row, [sum C][Hq][D] fp64: chunk c's rows over its own
+    token rows (history + chunk) in a fresh contiguous bf16 cache."""
+    cu = batch.cu_q_lens
+    ctx = batch.context_lens
+    outs = []
+    for c in range(batch.num_seqs - batch.num_decode):
+        s = batch.num_decode + c
+        L = int(ctx[s])
+        rows = torch.from_numpy(batch.seq_rows(s)[:L]).to(batch.tok_k.device)
+        tk = bf16_bits(batch.tok_k.index_select(0, rows))
+        tv = bf16_bits(batch.tok_v.index_select(0, rows))
+        nblk = max(1, (L + 15) // 16)
+        kc = np.zeros((nblk, batch.num_kv_heads, 16, batch.head_dim), np.uint16)
+        vc = np.zeros_like(kc)
+        O.kv_append(kc, vc, tk, tv, np.arange(L, dtype=np.int64))
+        C = int(cu[c + 1] - cu[c])
+        q = bf16_bits(batch.q_prefill[int(cu[c]):int(cu[c + 1])])
+        outs.append(O.paged_prefill(q, np.array([0, C], np.int32), kc, vc, np.arange(nblk, dtype=np.int32)[None],
+                                    np.array([L], np.int32), batch.scale))
+    return np.concatenate(outs) if outs else np.zeros((0, batch.num_q_heads, batch.head_dim))

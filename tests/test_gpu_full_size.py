@@ -1,0 +1,52 @@
+"""The four full-size workloads against the oracle, every output element.
+
+Each runs on the GPU exactly as bench.py times it (same inputs, same split choice, longest-first launch
+order): the Llama-3-8B-shaped decode batch (64 sequences, 32/8 heads, contexts 513..4097), the
+continuous-batching mixed step (256 prefix-sharing decode sequences with copy-on-write forks plus four
+causal prefill chunks of 512..2048 tokens), the long-context batch (8 x 32768 tokens, split 512) and the
+MHA batch over an FP8 E4M3 cache (32 sequences, 64/64 heads, contexts 2049..8193).  The oracle computes
+every sequence from its own token rows in a fresh contiguous cache (no paging, sharing or forks), so the
+comparison also checks that paging, prefix sharing and copy-on-write change nothing.
+Tolerances: attention max-abs <= 1e-2 and mean-abs <= 1e-3 against the oracle on the same bf16 inputs
+(for the FP8 cache: on the same dequantised codes), and <= 5e-2 max against the oracle on the original
+bf16 K/V for the FP8 cache.
+"""
+import pytest
+import torch
+
+from pagedattention_block_table_b200.inputs import make_batch
+from tests.common import FP8_MAX, assert_close, oracle_decode_all, oracle_prefill_all, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(batch):
+    from pagedattention_block_table_b200.runner import DeviceStep
+    st = DeviceStep(batch, split_tokens=None)
+    st.fill_history()
+    st.step()
+    torch.cuda.synchronize()
+    return st
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context_decode", "mha_fp8_decode"])
+def test_full_size_decode_every_element(O, cuda_lib, name):
+    batch = make_batch(name, device="cuda")
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    if name == "long_context_decode":
+        assert st.split_tokens == 512 and st.dec_max_len == 32768          # 64 splits per sequence
+    got = to_f64(st.out_dec)
+    assert_close(got, oracle_decode_all(batch, O), what=name)
+    if batch.kv_dtype:
+        assert_close(got, oracle_decode_all(batch, O, kv_dtype=0), max_tol=FP8_MAX, mean_tol=None,
+                     what=f"{name} vs the bf16 K/V")
+
+
+def test_full_size_mixed_step_every_element(O, cuda_lib):
+    batch = make_batch("mixed_step", device="cuda")
+    assert batch.cow_pairs.shape[0] > 0 and batch.shared_blocks.shape[0] > 0
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(st.out_dec), oracle_decode_all(batch, O), what="mixed step: 256 decode rows")
+    assert_close(to_f64(st.out_pre), oracle_prefill_all(batch, O), what="mixed step: every prefill row")

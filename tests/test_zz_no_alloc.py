@@ -77,3 +77,28 @@ def test_noalloc_rejects_partials_beyond_the_scratch(cuda_lib):
         B.pa_paged_attention_noalloc(out, st.q_dec, st.k_cache, st.v_cache, st.dec_tables, st.dec_lens,
                                      batch.scale, st.dec_max_len, split_tokens=16)
     assert e.value.status == B.PA_EWORKSPACE
+
+
+def test_noalloc_lengthens_an_auto_split_that_overflows_the_scratch(cuda_lib):
+    """split_tokens = 0 where the auto split's partials would not fit the static scratch: the call lengthens
+    the split until they do, and gives exactly what the workspace call gives at that split."""
+    from pagedattention_block_table_b200.runner import DeviceStep
+    B = cuda_lib
+    cap = 16 * 1024 * 1024
+    batch = make_batch("llama3_8b_decode", seed=75, device="cuda",
+                       overrides=dict(num_seqs=64, num_q_heads=128, num_kv_heads=8, hist=("uniform", 6200, 8000)))
+    st = DeviceStep(batch, split_tokens=512)
+    st.fill_history()
+    st.append()
+    args = (batch.num_decode, batch.num_q_heads, batch.head_dim, st.dec_max_len)
+    S = B.pa_paged_attention_auto_split(batch.num_decode, batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                                        st.dec_max_len)
+    assert B.pa_paged_attention_workspace_size(*args, S) > cap, "the case must overflow at the auto split"
+    while B.pa_paged_attention_workspace_size(*args, S) > cap:
+        S = -(-2 * S // 16) * 16
+    ref = _with_workspace(B, batch, st, S)
+    for call in range(2):
+        out = _no_alloc(B, batch, st, 0)
+        torch.cuda.synchronize()
+        assert B.pa_get_device_error() == B.PA_OK
+        assert torch.equal(out, ref), f"call {call}"
