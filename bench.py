@@ -202,7 +202,7 @@ def traffic_record(kernel_tag: str):
         if not d:
             return None
         from pagedattention_block_table_b200.build import source_digest
-        if d.get("source_digest") != source_digest():
+        if d.get("source_digest") != source_digest(d.get("sources")):
             return None
         return d
     except Exception:

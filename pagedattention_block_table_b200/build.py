@@ -23,12 +23,17 @@ def _sources():
                   + glob.glob(os.path.join(CSRC, "*.cpp")) + [os.path.join(ROOT, "include", "pagedattn.h")])
 
 
-def source_digest() -> str:
-    """sha256 of the CUDA sources (the kernels and their launch code, csrc/*.cu and *.cuh): identifies
-    which kernels a profile was taken on.  Host-only C++ (the block manager) does not enter it."""
+def source_digest(names=None) -> str:
+    """sha256 of CUDA sources: identifies which kernels a profile was taken on.  `names` lists the csrc
+    files a kernel depends on (for example its header, pa_common.cuh and api.cu, which holds its launch
+    code); None takes every csrc/*.cu and *.cuh.  Host-only C++ (the block manager) never enters it."""
     import hashlib
     h = hashlib.sha256()
-    for src in sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
+    if names is None:
+        files = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh")))
+    else:
+        files = [os.path.join(CSRC, n) for n in sorted(names)]
+    for src in files:
         with open(src, "rb") as f:
             h.update(os.path.basename(src).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]

@@ -221,3 +221,18 @@ def test_many_splits_and_a_reused_workspace(O, cuda_lib):
         for s in range(3):
             assert_close(got[s], oracle_decode_one(batch, s, O), what=f"seq {s}, split {split}")
     assert B.pa_get_device_error() == B.PA_OK
+
+
+@pytest.mark.parametrize("e", [-20, 20, 0])
+def test_decode_fp8_any_query_magnitude(O, cuda_lib, e):
+    """The FP8 decode keeps q in f16 after rescaling it by a power of two per query: q * 2^e with the
+    softmax scale * 2^-e gives the same scores far outside f16's range (2^20 overflows it, 2^-20 is
+    subnormal in it), and the output still matches the oracle."""
+    import math
+    batch = make_batch("mha_fp8_decode", seed=63, overrides=dict(num_seqs=3, num_q_heads=8, num_kv_heads=4,
+                                                               hist=("uniform", 100, 900)))
+    batch.q_decode = (batch.q_decode.float() * 2.0 ** e).to(torch.bfloat16)    # exact: a power of two
+    batch.scale = 1.0 / math.sqrt(batch.head_dim) * 2.0 ** -e
+    got = to_f64(_gpu_decode(batch, 256).out_dec)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(got, oracle_step(batch, O)["decode"], what=f"fp8, q * 2^{e}")
