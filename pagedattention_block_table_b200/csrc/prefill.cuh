@@ -152,6 +152,61 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+
+// Groups of K-steps issued from one asm statement.  The issuing thread dispatches one product at a time,
+// so whatever it executes between two products adds to every product's time: a clock64 timeline showed
+// 104-132 cycles per 128x128x16 product when each step computed its shared-memory descriptors in C++
+// (and the PV loop ran with a runtime trip count), against 72-76 for products issued back to back.  Here
+// only immediate adds to the two descriptors sit between products.  The start-address field of a
+// descriptor holds (address >> 4) in 14 bits; shared-memory addresses stay below 2^18 bytes, so the adds
+// never carry out of it.
+//
+// NK steps of D (+)= A*B, both operands in shared memory (K-major, 128-byte swizzle): step kk reads 32 bytes
+// at column (kk % 4) of plane (kk / 4) of each operand; APL / BPL are the plane strides in 16-byte units.
+// The first step overwrites D (the S products start a new tile).
+template <int NK, int APL, int BPL>
+__device__ __forceinline__ void mma_ss_group(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+  static_assert(NK == 4 || NK == 8, "steps per group");
+#define PA_MMA_SS(P) "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, " P ";\n\t"
+#define PA_STEP2 "add.s64 %1, %1, 2;\n\tadd.s64 %2, %2, 2;\n\t"
+  if constexpr (NK == 8) {
+    asm volatile(
+        "{\n\t.reg .pred f, t;\n\tsetp.ne.b32 f, %3, %3;\n\tsetp.eq.b32 t, %3, %3;\n\t"
+        PA_MMA_SS("f") PA_STEP2 PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t")
+        "add.s64 %1, %1, %4;\n\tadd.s64 %2, %2, %5;\n\t"
+        PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t") "}"
+        : "+r"(d_tmem), "+l"(a_desc), "+l"(b_desc)
+        : "r"(idesc), "n"(APL - 6), "n"(BPL - 6)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred f, t;\n\tsetp.ne.b32 f, %3, %3;\n\tsetp.eq.b32 t, %3, %3;\n\t"
+        PA_MMA_SS("f") PA_STEP2 PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t") PA_STEP2 PA_MMA_SS("t") "}"
+        : "+r"(d_tmem), "+l"(a_desc), "+l"(b_desc)
+        : "r"(idesc)
+        : "memory");
+  }
+#undef PA_STEP2
+#undef PA_MMA_SS
+}
+
+// Eight steps of D += A*B with A in TMEM (8 columns = 16 bf16 per lane and step) and B in shared memory
+// (MN-major, 16 rows = 2048 bytes per step); the first step accumulates only when acc0 != 0.
+__device__ __forceinline__ void mma_ts_group8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t acc0) {
+#define PA_MMA_TS(P) "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, " P ";\n\t"
+#define PA_STEPV "add.u32 %1, %1, 8;\n\tadd.s64 %2, %2, 128;\n\t"
+  asm volatile(
+      "{\n\t.reg .pred f, t;\n\tsetp.ne.b32 f, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\t"
+      PA_MMA_TS("f") PA_STEPV PA_MMA_TS("t") PA_STEPV PA_MMA_TS("t") PA_STEPV PA_MMA_TS("t") PA_STEPV
+      PA_MMA_TS("t") PA_STEPV PA_MMA_TS("t") PA_STEPV PA_MMA_TS("t") PA_STEPV PA_MMA_TS("t") "}"
+      : "+r"(d_tmem), "+r"(a_tmem), "+l"(b_desc)
+      : "r"(idesc), "r"(acc0)
+      : "memory");
+#undef PA_STEPV
+#undef PA_MMA_TS
+}
+
 // Store 32 consecutive 32-bit columns of this thread's TMEM lane (no wait).
 __device__ __forceinline__ void tmem_st32u_nowait(uint32_t taddr, const uint32_t *v) {
   asm volatile(
@@ -540,23 +595,23 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         return r;
       };
       auto release = [&](int i) { mma_commit(&bars[kEmpty + i % C::NSLOT]); };
+      const uint64_t qdesc[2] = {sw128_desc(qa, 16, 1024), sw128_desc(qb, 16, 1024)};
       auto issue_s = [&](int X, int j) {
-        const uint32_t qx = X ? qb : qa;
-        const uint32_t kt = smem_u32(slot_of(2 * j));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk & 3) * 32;
-          mma_bf16(tmem + C::s_col(X), sw128_desc(qx + (kk >> 2) * C::Q_PLANE + ko, 16, 1024),
-                   sw128_desc(kt + (kk >> 2) * C::KV_PLANE + ko, 16, 1024), idS, kk > 0);
-        }
+        mma_ss_group<D / 16, C::Q_PLANE / 16, C::KV_PLANE / 16>(
+            tmem + C::s_col(X), qdesc[X], sw128_desc(smem_u32(slot_of(2 * j)), 16, 1024), idS);
         mma_commit(&bars[kSFull + X]);
       };
       auto issue_o = [&](int X, int j) {
         const uint32_t vt = smem_u32(slot_of(2 * j + 1));
         const int nk = j == ntiles - 1 ? last_k16 : C::BN / 16;
-        for (int kk = 0; kk < nk; ++kk)
-          mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
-                      sw128_desc(vt + kk * (16 * 128), C::KV_PLANE, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+        if (nk == C::BN / 16) {
+          mma_ts_group8(tmem + C::o_col(X), tmem + C::s_col(X), sw128_desc(vt, C::KV_PLANE, 1024), idO,
+                        j > 0 ? 1u : 0u);
+        } else {
+          for (int kk = 0; kk < nk; ++kk)
+            mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
+                        sw128_desc(vt + kk * (16 * 128), C::KV_PLANE, 1024), idO, (j > 0 || kk > 0) ? 1u : 0u);
+        }
       };
       bool ok = mbar_wait(&bars[kQReady], 0) && ready(0);
       if (ok) {
