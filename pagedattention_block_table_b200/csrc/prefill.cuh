@@ -28,6 +28,8 @@
 // and rescale its O row in TMEM (tcgen05.ld/st) and its sum l.  O and l always share the reference,
 // so out = O / l is exact whichever reference was used.
 #pragma once
+#include <type_traits>
+
 #include "pa_common.cuh"
 
 #ifndef PA_PREFILL_SPLIT_REGS
@@ -465,48 +467,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       tmem_ld128(s_addr, sr);
       const int kbase = j * C::BN;
       const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
-      // scaled row max of this tile; masked keys (past the row's position) do not take part
-      float mt_ = -INFINITY;
-      if (!diag) {
-        // max of s * qscale: the max of s for a positive scale, the min for a negative one
-        // (three-input max/min: two new keys per instruction, four independent chains)
-        const float s0 = __uint_as_float(sr[0]), s1 = __uint_as_float(sr[1]), s2 = __uint_as_float(sr[2]),
-                    s3 = __uint_as_float(sr[3]), s4 = __uint_as_float(sr[4]), s5 = __uint_as_float(sr[5]),
-                    s6 = __uint_as_float(sr[6]), s7 = __uint_as_float(sr[7]);
-        if (qs >= 0.f) {
-          float e0 = fmaxf(s0, s1), e1 = fmaxf(s2, s3), e2 = fmaxf(s4, s5), e3 = fmaxf(s6, s7);
-#pragma unroll
-          for (int k = 8; k < C::BN; k += 8) {
-            e0 = fmax3(e0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
-            e1 = fmax3(e1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
-            e2 = fmax3(e2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
-            e3 = fmax3(e3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
-          }
-          mt_ = fmax3(fmaxf(e0, e1), e2, e3) * qs;
-        } else {
-          float e0 = fminf(s0, s1), e1 = fminf(s2, s3), e2 = fminf(s4, s5), e3 = fminf(s6, s7);
-#pragma unroll
-          for (int k = 8; k < C::BN; k += 8) {
-            e0 = fmin3(e0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
-            e1 = fmin3(e1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
-            e2 = fmin3(e2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
-            e3 = fmin3(e3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
-          }
-          mt_ = fmin3(fminf(e0, e1), e2, e3) * qs;
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < C::BN; ++k)
-          if (kbase + k <= pos) mt_ = fmaxf(mt_, __uint_as_float(sr[k]) * qs);
-      }
-      // move the reference when the tile's max exceeds it by more than 2^8 (O and l follow below)
-      const bool bump = mt_ > m_ref + kRescale;
-      const bool any_bump = __any_sync(0xffffffffu, bump);
-      float alpha = 1.f;
-      if (bump) {
-        alpha = exp2f(m_ref - mt_);
-        m_ref = mt_;
-      }
       // last key tile: V rows of keys no row may see, up to the last 16-key step the PV product reads,
       // are zeroed (tile A's threads, one row each) once the V tile has landed, so that 0 * (whatever
       // the cache holds past the context) never reaches the MMA
@@ -522,29 +482,96 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
           fence_async_smem();
         }
       }
-      uint64_t ls2 = 0ull;
-      const uint64_t qs2 = f2pack(qs, qs), nm2 = f2pack(-m_ref, -m_ref);
+      if (m_ref == -INFINITY) {
+        // first tile of the row: the reference is the tile's scaled max (masked keys do not take part)
+        float mt_ = -INFINITY;
+        if (!diag) {
+          // max of s * qscale: the max of s for a positive scale, the min for a negative one
+          // (three-input max/min: two new keys per instruction, four independent chains)
+          const float s0 = __uint_as_float(sr[0]), s1 = __uint_as_float(sr[1]), s2 = __uint_as_float(sr[2]),
+                      s3 = __uint_as_float(sr[3]), s4 = __uint_as_float(sr[4]), s5 = __uint_as_float(sr[5]),
+                      s6 = __uint_as_float(sr[6]), s7 = __uint_as_float(sr[7]);
+          if (qs >= 0.f) {
+            float e0 = fmaxf(s0, s1), e1 = fmaxf(s2, s3), e2 = fmaxf(s4, s5), e3 = fmaxf(s6, s7);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+            for (int k = 8; k < C::BN; k += 8) {
+              e0 = fmax3(e0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+              e1 = fmax3(e1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
+              e2 = fmax3(e2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
+              e3 = fmax3(e3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
+            }
+            mt_ = fmax3(fmaxf(e0, e1), e2, e3) * qs;
+          } else {
+            float e0 = fminf(s0, s1), e1 = fminf(s2, s3), e2 = fminf(s4, s5), e3 = fminf(s6, s7);
 #pragma unroll
-        for (int k2 = 0; k2 < 32; ++k2) {
-          const int k = half * 64 + 2 * k2;
-          // x = s * qscale - m_ref for two keys at once; keys past the row's position get p = 0
-          float2 x = f2unpack(ffma2(f2pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), qs2, nm2));
-          if (diag) {
-            if (kbase + k > pos) x.x = -INFINITY;
-            if (kbase + k + 1 > pos) x.y = -INFINITY;
+            for (int k = 8; k < C::BN; k += 8) {
+              e0 = fmin3(e0, __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+              e1 = fmin3(e1, __uint_as_float(sr[k + 2]), __uint_as_float(sr[k + 3]));
+              e2 = fmin3(e2, __uint_as_float(sr[k + 4]), __uint_as_float(sr[k + 5]));
+              e3 = fmin3(e3, __uint_as_float(sr[k + 6]), __uint_as_float(sr[k + 7]));
+            }
+            mt_ = fmin3(fminf(e0, e1), e2, e3) * qs;
           }
-          const float a = ex2(x.x);
-          const float b = ex2(x.y);
-          ls2 = f2add(ls2, f2pack(a, b));
-          pk[k2] = pack_bf16x2(a, b);
+        } else {
+#pragma unroll
+          for (int k = 0; k < C::BN; ++k)
+            if (kbase + k <= pos) mt_ = fmaxf(mt_, __uint_as_float(sr[k]) * qs);
         }
-        tmem_st32u_nowait(s_addr + half * 32, pk);
+        m_ref = mt_;
       }
-      const float2 lsv = f2unpack(ls2);
-      l_run = l_run * alpha + (lsv.x + lsv.y);
+      // p = 2^(s * qscale - m_ref) for the tile's keys into the first 64 columns of S (bf16 pairs), with the
+      // largest exponent; keys past the row's position get p = 0.  Masking is compiled only into the pass
+      // of diagonal tiles.
+      float sum = 0.f;
+      auto pass = [&](auto diag_c) {
+        constexpr bool kDiag = decltype(diag_c)::value;
+        float mx = -INFINITY;
+        uint64_t ls2 = 0ull;
+        const uint64_t qs2 = f2pack(qs, qs), nm2 = f2pack(-m_ref, -m_ref);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int k2 = 0; k2 < 32; ++k2) {
+            const int k = half * 64 + 2 * k2;
+            float2 x = f2unpack(ffma2(f2pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), qs2, nm2));
+            if (kDiag) {
+              if (kbase + k > pos) x.x = -INFINITY;
+              if (kbase + k + 1 > pos) x.y = -INFINITY;
+            }
+            mx = fmax3(mx, x.x, x.y);
+            const float a = ex2(x.x);
+            const float b = ex2(x.y);
+            ls2 = f2add(ls2, f2pack(a, b));
+            pk[k2] = pack_bf16x2(a, b);
+          }
+          tmem_st32u_nowait(s_addr + half * 32, pk);
+        }
+        const float2 lsv = f2unpack(ls2);
+        sum = lsv.x + lsv.y;
+        return mx;
+      };
+      // the pass stores P with warp-collective tcgen05.st, so the choice is made per warp: the masking pass
+      // when any row of the warp has a key past its position (it masks nothing for the other rows)
+      const bool wdiag = __any_sync(0xffffffffu, diag);
+      const float mx = wdiag ? pass(std::true_type{}) : pass(std::false_type{});
+      // The reference moves only when the tile's max exceeds it by more than 2^8: then P is recomputed
+      // against the new one (p of such a tile may even have overflowed), O and l are rescaled below.  The
+      // recompute rewrites P (warp-collective tcgen05.st), so the whole warp takes it when any row does; a
+      // row that keeps its reference rewrites the same values.
+      const bool bump = mx > kRescale;
+      const bool any_bump = __any_sync(0xffffffffu, bump);
+      float alpha = 1.f;
+      if (any_bump) {
+        if (bump) {
+          const float m_new = m_ref + mx;
+          alpha = exp2f(m_ref - m_new);
+          m_ref = m_new;
+        }
+        tmem_wait_st();
+        (void)(wdiag ? pass(std::true_type{}) : pass(std::false_type{}));
+      }
+      l_run = l_run * alpha + sum;
       if (any_bump && j > 0) {
         // rescale this row's O to the new reference (O_X(j-1) is complete; O_X(j) waits for P_X(j))
 #pragma unroll 1
