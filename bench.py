@@ -305,14 +305,26 @@ def launches_per_step(st) -> int:
             + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0))
 
 
+def workload_batch(name, device, num_seqs=0):
+    """The named workload's synthetic batch; num_seqs > 0 keeps its shapes and length distribution but
+    draws that many sequences (a smaller case of the same workload, for profiling)."""
+    from pagedattention_block_table_b200.inputs import WORKLOADS, make_batch
+    ov = None
+    if num_seqs:
+        ov = {"num_seqs": num_seqs}
+        hist = WORKLOADS[name]["hist"]
+        if hist[0] == "fixed":
+            ov["hist"] = ("fixed", list(hist[1])[:num_seqs])
+    return make_batch(name, device=device, overrides=ov)
+
+
 def measure(name, dev, K, W, args, rank, world, clk, e2e=False):
     """Time one workload on this rank: the whole step, the decode call alone and the prefill call alone
     (each from CUDA graphs of back-to-back calls), and optionally the end-to-end host-fed step."""
     from pagedattention_block_table_b200 import binding as B
-    from pagedattention_block_table_b200.inputs import make_batch
     from pagedattention_block_table_b200.runner import DeviceStep, HostPipeline
 
-    full = make_batch(name, device=dev)
+    full = workload_batch(name, dev, args.num_seqs if name == args.workload else 0)
     batch = rank_batch(full, rank, world, args.partition)
     st = DeviceStep(batch, device=dev, split_tokens=args.split or None)
     st.fill_history()
@@ -562,8 +574,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     from oracle import oracle as O
-    from pagedattention_block_table_b200.inputs import make_batch
-    batch = make_batch(args.workload, device="cpu")
+    batch = workload_batch(args.workload, "cpu", args.num_seqs)
     smp = _oracle_sample(batch, args.ref_sample_seqs)
     for _ in range(max(0, min(args.warmup, 1))):
         _oracle_run(batch, smp)
@@ -658,6 +669,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--num-seqs", type=int, default=0,
+                    help="draw this many sequences of the workload instead of its own count (profiling)")
     ap.add_argument("--partition", choices=["replicas", "kv_heads"], default="replicas",
                     help="N>1: whole batch per rank (weak scaling) or KV heads split over the ranks (strong)")
     ap.add_argument("--split", type=int, default=0, help="split_tokens (0 = library default)")

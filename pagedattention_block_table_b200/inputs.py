@@ -2,7 +2,7 @@
 
 This module is the one place both the CUDA path and the CPU oracle get their inputs
 from.  It draws token K/V and queries (N(0,1) rounded to bf16), context lengths with
-the distributions of the five workloads, a seeded random placement of logical blocks
+the distributions of the workloads, a seeded random placement of logical blocks
 in the physical pool, the slot of every token, and -- for the prefix-sharing step --
 which blocks are shared and which copy-on-write pairs a fork needs.  It holds none
 of the method's arithmetic: no attention, no quantisation, no copying of caches.
@@ -27,7 +27,7 @@ BLOCK = 16
 E4M3_MAX = 448.0
 INT8_MAX = 127.0
 
-# The five workloads.  Lengths given here are HISTORIES (tokens already cached);
+# The workloads.  Lengths given here are HISTORIES (tokens already cached);
 # every decode sequence then appends one token, so it attends over history + 1.
 WORKLOADS: Dict[str, dict] = {
     "tiny_decode": dict(num_seqs=4, num_q_heads=8, num_kv_heads=2, head_dim=64,
@@ -42,6 +42,10 @@ WORKLOADS: Dict[str, dict] = {
                                 hist=("fixed", [32767] * 8), split_tokens=512),
     "mha_fp8_decode": dict(num_seqs=32, num_q_heads=64, num_kv_heads=64, head_dim=128,
                            hist=("uniform", 2048, 8192), kv_dtype="fp8"),
+    # eight query heads per KV head (the 64 / 8 head layout of a 70B-class model): a decode CTA takes
+    # four query heads, so each KV tile is fetched by two CTAs; measures whether the second fetch hits L2
+    "gqa8_decode": dict(num_seqs=32, num_q_heads=64, num_kv_heads=8, head_dim=128,
+                        hist=("uniform", 512, 4096)),
 }
 WORKLOAD_SEED = {name: 1001 + i for i, name in enumerate(WORKLOADS)}
 

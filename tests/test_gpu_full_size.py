@@ -1,12 +1,14 @@
-"""The four full-size workloads against the oracle, every output element.
+"""The full-size workloads against the oracle, every output element.
 
 Each runs on the GPU exactly as bench.py times it (same inputs, same split choice, longest-first launch
 order): the Llama-3-8B-shaped decode batch (64 sequences, 32/8 heads, contexts 513..4097), the
 continuous-batching mixed step (256 prefix-sharing decode sequences with copy-on-write forks plus four
-causal prefill chunks of 512..2048 tokens), the long-context batch (8 x 32768 tokens, split 512) and the
-MHA batch over an FP8 E4M3 cache (32 sequences, 64/64 heads, contexts 2049..8193).  The oracle computes
-every sequence from its own token rows in a fresh contiguous cache (no paging, sharing or forks), so the
-comparison also checks that paging, prefix sharing and copy-on-write change nothing.
+causal prefill chunks of 512..2048 tokens), the long-context batch (8 x 32768 tokens, split 512), the
+MHA batch over an FP8 E4M3 cache (32 sequences, 64/64 heads, contexts 2049..8193), and a GQA batch with
+eight query heads per KV head (32 sequences, 64/8 heads, contexts 513..4097), whose KV tiles two CTAs
+each read.  The oracle computes every sequence from its own token rows in a fresh contiguous cache (no
+paging, sharing or forks), so the comparison also checks that paging, prefix sharing and copy-on-write
+change nothing.
 Tolerances: attention max-abs <= 1e-2 and mean-abs <= 1e-3 against the oracle on the same bf16 inputs
 (for the FP8 cache: on the same dequantised codes), and <= 5e-2 max against the oracle on the original
 bf16 K/V for the FP8 cache.
@@ -29,7 +31,7 @@ def _run(batch):
     return st
 
 
-@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context_decode", "mha_fp8_decode"])
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context_decode", "mha_fp8_decode", "gqa8_decode"])
 def test_full_size_decode_every_element(O, cuda_lib, name):
     batch = make_batch(name, device="cuda")
     st = _run(batch)
