@@ -305,6 +305,14 @@ def launches_per_step(st) -> int:
             + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0))
 
 
+def decode_kernel_label(batch) -> str:
+    """Which decode kernel pa_paged_attention runs for this batch (the library decides)."""
+    from pagedattention_block_table_b200 import binding as B
+    tc = B.pa_paged_attention_uses_tensor_cores(batch.num_q_heads, batch.num_kv_heads, batch.kv_dtype)
+    k = "paged_decode_mma_kernel (mma.sync)" if tc == 1 else "paged_decode_kernel"
+    return f"pa_paged_attention ({k} + lse_reduce_kernel)"
+
+
 def workload_batch(name, device, num_seqs=0):
     """The named workload's synthetic batch; num_seqs > 0 keeps its shapes and length distribution but
     draws that many sequences (a smaller case of the same workload, for profiling)."""
@@ -382,7 +390,7 @@ def sub_record(name, dev, args, clk):
         db, kvb, kvu = decode_bytes(batch), kv_bytes(batch), kv_unique_bytes(batch)
         ach = db / (m["dec_ms"] * 1e-3) / 1e9
         rec["decode"] = {
-            "kernel": "pa_paged_attention (paged_decode_kernel + lse_reduce_kernel)", "bound": "hbm",
+            "kernel": decode_kernel_label(batch), "bound": "hbm",
             "unit": "GB/s", "achieved": round(ach, 2), "peak": peak, "peak_kind": peak_kind,
             "frac": round(ach / peak, 4), "avg_launch_ms": round(m["dec_ms"], 5), "algorithmic_bytes": db,
             "dtype": {0: "bf16", 1: "fp8_e4m3", 2: "int8"}[batch.kv_dtype],
@@ -458,7 +466,7 @@ def run_ours(args, rank, world, local_rank):
         "decode_kv_bytes_per_step": kvb,
         "decode_kv_unique_bytes_per_step": kvu,
         "roofline": {
-            "kernel": "pa_paged_attention (paged_decode_kernel + lse_reduce_kernel)",
+            "kernel": decode_kernel_label(batch),
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
             "traffic": None if tr is None else tr.get("bytes_per_launch"),

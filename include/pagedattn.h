@@ -128,6 +128,14 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
                                   int max_context_len, int kv_dtype);
 
 /*
+ * pa_paged_attention_uses_tensor_cores -- 1 when pa_paged_attention runs its products on the tensor
+ * cores for this shape (bf16 cache, at least 4 query heads per KV head, a group of at most 16 heads or
+ * a multiple of 16), 0 when it uses the CUDA-core kernel (one-byte caches, smaller groups), -1 for an
+ * invalid shape.  Both compute the same function; this only names the kernel that runs.
+ */
+int pa_paged_attention_uses_tensor_cores(int num_q_heads, int num_kv_heads, int kv_dtype);
+
+/*
  * pa_paged_attention -- decode attention over the paged cache [Core Concepts §3.2: the kernel reads
  * non-contiguous K/V through the block table; KV Cache to vLLM §1.2: the new token's query attends
  * over all cached keys and takes the weighted sum of values; §2.2 GQA].  For every sequence b and

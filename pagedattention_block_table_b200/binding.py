@@ -31,7 +31,8 @@ PA_KV_INT8 = 2
 # every entry point include/pagedattn.h declares
 EXPORTED = (
     "pa_kv_append", "pa_copy_blocks", "pa_paged_attention_workspace_size",
-    "pa_paged_attention_auto_split", "pa_paged_attention", "pa_paged_prefill",
+    "pa_paged_attention_auto_split", "pa_paged_attention_uses_tensor_cores", "pa_paged_attention",
+    "pa_paged_prefill",
     "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
     "pa_paged_attention_noalloc", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_attention_workspace_size.argtypes = [I, I, I, I, I]
         L.pa_paged_attention_auto_split.restype = I
         L.pa_paged_attention_auto_split.argtypes = [I, I, I, I, I, I]
+        L.pa_paged_attention_uses_tensor_cores.restype = I
+        L.pa_paged_attention_uses_tensor_cores.argtypes = [I, I, I]
         L.pa_paged_attention.restype = I
         L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, I, F, I, P, P, I, I, P, P, SZ, P]
         L.pa_paged_attention_noalloc.restype = I
@@ -228,6 +231,10 @@ def pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                   kv_dtype=PA_KV_BF16) -> int:
     return int(lib().pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                                    max_context_len, kv_dtype))
+
+
+def pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, kv_dtype=PA_KV_BF16) -> int:
+    return int(lib().pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, kv_dtype))
 
 
 def _host_i32(a, n):

@@ -1,0 +1,390 @@
+// decode_mma.cuh -- paged decode attention for GQA groups on the tensor cores (bf16 cache, sm_100a).
+//
+// Same operation and split-K scheme as paged_decode_kernel (decode.cuh): for sequence b and query head
+// h, out = softmax(scale * q . K^T) V over the context, token t read through the block table.  With a
+// group of G query heads per KV head, every K/V element meets G queries, so the CUDA-core kernel's
+// work per byte of KV grows with G; at G = 8 it is compute-bound at about half the HBM bandwidth.  Here
+// the products go to the tensor cores instead (warp-level mma.sync m16n8k16, bf16 in, fp32 out): the
+// CTA's query heads are the 16 rows of the A operand (padded with zeros when G < 16), and a 16-token
+// block is one N=16 QK^T product and one K=16 PV product per warp.
+//
+// Per warp and 16-token block:
+//   S[16 heads][16 tokens] = Q K^T     2 n-tiles of 8 tokens x D/16 k-steps; Q's fragments sit in
+//                                      registers for the whole launch, K's are read from shared memory
+//   online softmax in base 2 on S's fragments (a row's 16 scores are spread over the 4 lanes of a quad)
+//   O[16][D] += P V                    P (bf16) is built from S's fragments in registers; V's fragments
+//                                      come from shared memory with ldmatrix.trans (V is token-major)
+// K and V tiles reach shared memory by 2-D TMA (the cache seen as rows of D elements, one 16-row x
+// 64-element box per 64-element plane, 128-byte swizzle, no multicast), so ldmatrix and the 16-byte K
+// loads are free of bank conflicts.  The dims of a k-step are permuted (the same way for Q and K, which
+// leaves the dot product unchanged) so that each lane's K fragments come from two 16-byte loads.
+#pragma once
+#include "decode.cuh"
+#include "prefill.cuh"   // tensor-map encoding, 2-D TMA load
+
+namespace pa {
+
+template <int D, int NW, int STAGES>
+struct DecodeMmaCfg {
+  static constexpr int PLANES = D / 64;                 // 64-element (128-byte) planes of a row
+  static constexpr int PLANE = kBlock * 128;            // one 16-row plane: 2 KB
+  static constexpr int TILE = PLANES * PLANE;           // one (unit, head) K or V tile
+  static constexpr int KS = D / 16;                     // k-steps of the QK product
+  static constexpr int NT = D / 8;                      // 8-dim n-tiles of the PV product
+  static constexpr int BAR_BYTES = STAGES * 8;
+  // swizzled tiles need 1024-byte alignment: each warp's area is a multiple of 1024
+  static constexpr int WARP_BYTES = ((2 * STAGES * TILE + BAR_BYTES) + 1023) / 1024 * 1024;
+  static constexpr int SMEM = NW * WARP_BYTES + 1024;   // + slack to align the base
+  static constexpr int ML = 16 * D;                     // offset of the (m, l) pairs in a warp's merge area
+  static_assert(D == 64 || D == 128, "head_dim");
+  static_assert((16 * D + 32) * 4 <= 2 * STAGES * TILE, "merge area fits in the warp's tiles");
+};
+
+// 2-D TMA load with an L2 cache hint (the decode reads every KV byte once: evict first).
+__device__ __forceinline__ void tma_load_2d_hint(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// D(16x8, fp32) += A(16x16, bf16, row-major) * B(16x8, bf16, column-major); fragments as in the PTX ISA's
+// m16n8k16 layout (group = lane / 4, pair = lane % 4).
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Byte offset of 16-byte chunk c (0..D/8-1) of row r in a tile of 128-byte-swizzled 64-element planes.
+__device__ __forceinline__ uint32_t sw_chunk(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * (kBlock * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// HI: the CTA serves more than 8 query heads (rows 8-15 of the products are real).
+template <int D, int NW, int STAGES, bool HI, bool ORDERED>
+__global__ void __launch_bounds__(NW * 32)
+    paged_decode_mma_kernel(const DecodeParams P, const __grid_constant__ CUtensorMap kmap,
+                            const __grid_constant__ CUtensorMap vmap, const __grid_constant__ WorkOrder<ORDERED> W) {
+  using C = DecodeMmaCfg<D, NW, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 2, pr = lane & 3;           // fragment row group and pair index
+  const int split = ORDERED ? (W.item[blockIdx.y] >> 16) : static_cast<int>(blockIdx.z);
+  const int b = ORDERED ? (W.item[blockIdx.y] & 0xffff) : static_cast<int>(blockIdx.y);
+  const int hpc = P.group < 16 ? P.group : 16;        // query heads of this CTA (rows of the products)
+  const int sub_groups = P.group / hpc;
+  const int g = blockIdx.x / sub_groups;
+  const int h0 = g * P.group + (blockIdx.x % sub_groups) * hpc;
+  // any input may come from the kernel before this one on the stream (launched with PDL)
+  griddep_wait();
+  griddep_launch();
+
+  // ---- context length, validated: never read past the table row or the launch bound
+  int L = P.context_lens[b];
+  {
+    const int lim = min(P.max_blocks_per_seq * P.block_size, P.max_context_len);
+    if (L < 0 || L > lim) {
+      if (threadIdx.x == 0 && split == 0) flag_error(kErrLength);
+      L = L < 0 ? 0 : lim;
+    }
+  }
+  const int n_splits = (L + P.split_tokens - 1) / P.split_tokens;
+  if (split >= (n_splits > 1 ? n_splits : 1)) return;
+  const bool final_out = n_splits <= 1;
+  const int t0 = split * P.split_tokens;
+  const int t1 = min(L, t0 + P.split_tokens);
+  const int nblk = t1 > t0 ? (t1 - t0 + kBlock - 1) / kBlock : 0;
+  const int blk0 = t0 / kBlock;
+
+  uint8_t *wbase = smem + warp * C::WARP_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + 2 * STAGES * C::TILE);
+  const int nwb = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;  // blocks of this warp
+  if (lane == 0) {
+    for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+
+  // ---- block-table window: lane k holds the 16-row tile index of this warp's unit win*32 + k
+  const int32_t *trow = P.block_tables + (int64_t)b * P.max_blocks_per_seq;
+  const int upb = P.block_size / kBlock;   // 16-token units per block: 1 or 2
+  auto load_window = [&](int win) -> int {
+    const int i = win * 32 + lane;
+    int tile = 0;
+    if (i < nwb) {
+      const int u = blk0 + warp + NW * i;
+      int e = __ldg(trow + u / upb);
+      if (e < 0 || e >= P.num_blocks) {
+        flag_error(kErrBlockId);
+        e = 0;
+      }
+      tile = (e * P.num_kv_heads + g) * upb + u % upb;
+    }
+    return tile;
+  };
+  int tw = load_window(0);
+  const uint64_t pol = l2_evict_first_policy();
+  auto issue = [&](int i) {  // warp-uniform call
+    if (i >= nwb) return;
+    if ((i & 31) == 0 && i > 0) tw = load_window(i >> 5);
+    const int tile = __shfl_sync(0xffffffffu, tw, i & 31);
+    const int s = i % STAGES;
+    if (lane == 0) mbar_arrive_expect_tx(&bars[s], 2 * C::TILE);
+    __syncwarp();
+    if (lane < 2 * C::PLANES) {   // one 16 x 64 box per lane: K planes, then V planes
+      const int pl = lane % C::PLANES;
+      const bool v = lane >= C::PLANES;
+      tma_load_2d_hint(wbase + ((v ? STAGES : 0) + s) * C::TILE + pl * C::PLANE, v ? &vmap : &kmap, pl * 64,
+                       tile * kBlock, &bars[s], pol);
+    }
+  };
+
+  int issued = 0;
+  for (; issued < STAGES && issued < nwb; ++issued) issue(issued);
+
+  // ---- Q fragments (rows h0 + grp and h0 + grp + 8), unscaled bf16; k-step 4t+u of plane t holds dims
+  // 64t + 16*pr + 4u + {0,1} (A[0], A[1]) and + {2,3} (A[2], A[3])
+  uint32_t qlo[C::KS][2], qhi[C::KS][2];
+#pragma unroll
+  for (int t = 0; t < C::PLANES; ++t) {
+    uint4 w[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+    if (grp < hpc) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(P.q + ((int64_t)b * P.num_q_heads + h0 + grp) * D +
+                                                          64 * t + 16 * pr);
+      w[0] = src[0];
+      w[1] = src[1];
+    }
+    const uint32_t ww[8] = {w[0].x, w[0].y, w[0].z, w[0].w, w[1].x, w[1].y, w[1].z, w[1].w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      qlo[4 * t + u][0] = ww[2 * u];
+      qlo[4 * t + u][1] = ww[2 * u + 1];
+    }
+    if constexpr (HI) {
+      uint4 x[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+      if (grp + 8 < hpc) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(P.q + ((int64_t)b * P.num_q_heads + h0 + grp + 8) * D +
+                                                            64 * t + 16 * pr);
+        x[0] = src[0];
+        x[1] = src[1];
+      }
+      const uint32_t xx[8] = {x[0].x, x[0].y, x[0].z, x[0].w, x[1].x, x[1].y, x[1].z, x[1].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        qhi[4 * t + u][0] = xx[2 * u];
+        qhi[4 * t + u][1] = xx[2 * u + 1];
+      }
+    }
+  }
+
+  // ---- running state per row: reference max (log2 units), this lane's share of the sum, O fragments
+  constexpr float kRescale = 8.f;
+  const float qs = P.qscale;
+  float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
+  float o[C::NT][4];
+#pragma unroll
+  for (int j = 0; j < C::NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+
+  const uint32_t wbase_s = smem_u32(wbase);
+  bool ok = true;
+  int i = 0;
+  for (; i < nwb; ++i) {
+    const int s = i % STAGES;
+    const bool got = mbar_wait(&bars[s], (i / STAGES) & 1);
+    if (__any_sync(0xffffffffu, !got)) {
+      ok = false;
+      break;
+    }
+    const int jb = warp + NW * i;                       // block index within the split
+    const int nvalid = min(kBlock, t1 - (t0 + jb * kBlock));
+    const uint32_t Kt = wbase_s + s * C::TILE;
+    const uint32_t Vt = wbase_s + (STAGES + s) * C::TILE;
+    if (nvalid < kBlock) {
+      // V rows past the context are zeroed: P is 0 there, but 0 * (whatever the cache holds) may not be
+      uint8_t *vt = wbase + (STAGES + s) * C::TILE;
+      for (int idx = lane; idx < (kBlock - nvalid) * (D / 8); idx += 32) {
+        const int r = nvalid + idx / (D / 8), c = idx % (D / 8);
+        *reinterpret_cast<uint4 *>(vt + sw_chunk(r, c)) = make_uint4(0, 0, 0, 0);
+      }
+      fence_async_smem();   // before the TMA writes this slot again
+      __syncwarp();
+    }
+
+    // -- S = Q K^T: n-tile nt holds tokens 8nt..8nt+7; lane (grp, pr) reads token 8nt+grp's dims
+    // 64t + 16pr .. +16 (two 16-byte chunks of plane t)
+    float sc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      const int R = 8 * nt + grp;
+#pragma unroll
+      for (int t = 0; t < C::PLANES; ++t) {
+        const uint4 k0 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr));
+        const uint4 k1 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr + 1));
+        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ks = 4 * t + u;
+          mma_16816(sc[nt], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
+                    kw[2 * u + 1]);
+        }
+      }
+    }
+
+    // -- online softmax: lane (grp, pr) holds row grp's tokens 8nt + 2pr + {0,1} (sc[nt][0..1]) and row
+    // grp+8's (sc[nt][2..3]); a row's max comes from the 4 lanes of its quad
+    float x[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int tok = 8 * nt + 2 * pr + (e & 1);
+        x[nt][e] = tok < nvalid ? sc[nt][e] * qs : -INFINITY;
+      }
+    float bm_lo = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+    bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 1));
+    bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 2));
+    // the reference moves only when the block's max exceeds it by more than 2^8 (or on the first block);
+    // O and l are rescaled with it, so O / l is exact whichever reference is used
+    if (bm_lo > m_lo + kRescale) {
+      const float alpha = m_lo == -INFINITY ? 0.f : exp2f(m_lo - bm_lo);
+      m_lo = bm_lo;
+      l_lo *= alpha;
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j) {
+        o[j][0] *= alpha;
+        o[j][1] *= alpha;
+      }
+    }
+    float p[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      p[nt][0] = exp2f(x[nt][0] - m_lo);
+      p[nt][1] = exp2f(x[nt][1] - m_lo);
+      l_lo += p[nt][0] + p[nt][1];
+    }
+    if constexpr (HI) {
+      float bm_hi = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+      bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 1));
+      bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 2));
+      if (bm_hi > m_hi + kRescale) {
+        const float alpha = m_hi == -INFINITY ? 0.f : exp2f(m_hi - bm_hi);
+        m_hi = bm_hi;
+        l_hi *= alpha;
+#pragma unroll
+        for (int j = 0; j < C::NT; ++j) {
+          o[j][2] *= alpha;
+          o[j][3] *= alpha;
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        p[nt][2] = exp2f(x[nt][2] - m_hi);
+        p[nt][3] = exp2f(x[nt][3] - m_hi);
+        l_hi += p[nt][2] + p[nt][3];
+      }
+    }
+    // P as the A operand of the PV product (K = the block's 16 tokens): its fragments are S's
+    const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+    const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+    const uint32_t pa1 = HI ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
+    const uint32_t pa3 = HI ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
+    __syncwarp();
+
+    // -- O += P V: ldmatrix.trans gives the B fragments of two 8-dim n-tiles per call; lane l addresses
+    // row (l/8 % 2)*8 + l%8 (token) of 8-dim chunk 2jj + l/16
+    const int vr = ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+    for (int jj = 0; jj < C::NT / 2; ++jj) {
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_trans(Vt + sw_chunk(vr, 2 * jj + (lane >> 4)), v0, v1, v2, v3);
+      mma_16816(o[2 * jj], pa0, pa1, pa2, pa3, v0, v1);
+      mma_16816(o[2 * jj + 1], pa0, pa1, pa2, pa3, v2, v3);
+    }
+    __syncwarp();
+    if (issued < nwb) issue(issued++);
+  }
+  if (!ok) {
+    // a wait gave up: give the copies this warp still has in flight a bounded chance to land, then drop
+    // this warp's state (the error word already says why)
+    for (int k = i; k < issued; ++k) (void)mbar_wait(&bars[k % STAGES], (k / STAGES) & 1);
+    m_lo = m_hi = -INFINITY;
+    l_lo = l_hi = 0.f;
+#pragma unroll
+    for (int j = 0; j < C::NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  }
+  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+  if constexpr (HI) {
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+  }
+
+  // ---- merge the warps: each writes its rows' (O, m, l) over its consumed tiles, then the CTA combines
+  __syncwarp();
+  float *mrg = reinterpret_cast<float *>(wbase);
+#pragma unroll
+  for (int j = 0; j < C::NT; ++j) {
+    *reinterpret_cast<float2 *>(mrg + grp * D + 8 * j + 2 * pr) = make_float2(o[j][0], o[j][1]);
+    if constexpr (HI) *reinterpret_cast<float2 *>(mrg + (grp + 8) * D + 8 * j + 2 * pr) = make_float2(o[j][2], o[j][3]);
+  }
+  if (pr == 0) {
+    mrg[C::ML + 2 * grp] = m_lo;
+    mrg[C::ML + 2 * grp + 1] = l_lo;
+    if constexpr (HI) {
+      mrg[C::ML + 2 * (grp + 8)] = m_hi;
+      mrg[C::ML + 2 * (grp + 8) + 1] = l_hi;
+    }
+  }
+  __syncthreads();
+
+  for (int idx = threadIdx.x; idx < hpc * D; idx += NW * 32) {
+    const int qi = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, reinterpret_cast<const float *>(smem + w * C::WARP_BYTES)[C::ML + 2 * qi]);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float *mw = reinterpret_cast<const float *>(smem + w * C::WARP_BYTES);
+        const float sc_w = exp2f(mw[C::ML + 2 * qi] - M);
+        Lsum += sc_w * mw[C::ML + 2 * qi + 1];
+        O += sc_w * mw[qi * D + d];
+      }
+    }
+    const int h = h0 + qi;
+    if (final_out) {
+      const float val = Lsum > 0.f ? O / Lsum : 0.f;
+      P.out[((int64_t)b * P.num_q_heads + h) * D + d] = __float2bfloat16_rn(val);
+    } else {
+      const int64_t row = ((int64_t)b * P.num_q_heads + h) * P.max_splits + split;
+      P.ws_o[row * D + d] = O;
+      if (d == 0) {
+        P.ws_ml[row * 2] = M;
+        P.ws_ml[row * 2 + 1] = Lsum;
+      }
+    }
+  }
+}
+
+}  // namespace pa

@@ -56,6 +56,18 @@ def test_status_strings(L):
     assert "sm_100a" in B.pa_version()
 
 
+def test_decode_kernel_choice(L):
+    """bf16 caches with groups of 4 or more query heads decode on the tensor cores (up to 16 heads per
+    CTA, or a multiple of 16); one-byte caches and smaller groups on the CUDA cores."""
+    f = L.pa_paged_attention_uses_tensor_cores
+    f.argtypes = [ctypes.c_int] * 3
+    assert f(32, 8, 0) == 1 and f(64, 8, 0) == 1 and f(32, 2, 0) == 1 and f(32, 1, 0) == 1
+    assert f(32, 8, 1) == 0 and f(32, 8, 2) == 0          # FP8 / INT8 caches
+    assert f(8, 8, 0) == 0 and f(4, 2, 0) == 0 and f(6, 2, 0) == 0
+    assert f(48, 2, 0) == 0                                  # a group of 24: neither <= 16 nor a multiple of 16
+    assert f(32, 3, 0) == -1 and f(0, 8, 0) == -1
+
+
 def test_workspace_size(L):
     assert B.pa_paged_attention_workspace_size(8, 32, 128, 32768, 512) == 8 * 32 * 64 * 130 * 4
     assert B.pa_paged_attention_workspace_size(8, 32, 128, 512, 512) == 0

@@ -33,6 +33,16 @@ SMALL = {
     "gqa4_d128_bs32": ("llama3_8b_decode", dict(num_seqs=5, hist=("fixed", [0, 31, 32, 700, 1500]), block_size=32)),
     "gqa2_d64_bs32": ("tiny_decode", dict(num_seqs=4, num_q_heads=4, num_kv_heads=2, hist=("uniform", 1, 400),
                                           num_blocks=None, block_size=32)),
+    # groups of 8 or more query heads per KV head take the tensor-core kernel: 8 rows, 16 rows, a group
+    # split over two CTAs (32 heads), head_dim 64, 32-token blocks; lengths 0, 1, block edges and splits
+    "gqa8_d128_edges": ("llama3_8b_decode", dict(num_seqs=6, num_q_heads=32, num_kv_heads=4,
+                                                 hist=("fixed", [0, 1, 15, 16, 17, 1301]))),
+    "gqa16_d128": ("llama3_8b_decode", dict(num_seqs=4, num_q_heads=32, num_kv_heads=2, hist=("uniform", 1, 900))),
+    "gqa32_d128": ("llama3_8b_decode", dict(num_seqs=2, num_q_heads=32, num_kv_heads=1, hist=("fixed", [5, 333]))),
+    "gqa8_d64": ("tiny_decode", dict(num_seqs=4, num_q_heads=16, num_kv_heads=2, hist=("uniform", 1, 700),
+                                     num_blocks=None)),
+    "gqa8_d128_bs32": ("llama3_8b_decode", dict(num_seqs=4, num_q_heads=64, num_kv_heads=8, block_size=32,
+                                                hist=("fixed", [31, 32, 33, 777]))),
 }
 
 
@@ -69,8 +79,13 @@ def test_decode_fp8_with_gqa(O, cuda_lib):
     assert_close(to_f64(_gpu_decode(batch).out_dec), oracle_step(batch, O)["decode"], what="fp8 gqa4")
 
 
-def test_placement_invariance_bit_identical(cuda_lib):
-    kw = dict(seed=44, overrides=dict(num_seqs=5, hist=("uniform", 100, 1200)))
+GROUPS = {"g4": dict(num_q_heads=32, num_kv_heads=8), "g8": dict(num_q_heads=64, num_kv_heads=8),
+          "g16": dict(num_q_heads=32, num_kv_heads=2)}
+
+
+@pytest.mark.parametrize("grp", sorted(GROUPS))
+def test_placement_invariance_bit_identical(cuda_lib, grp):
+    kw = dict(seed=44, overrides=dict(num_seqs=5, hist=("uniform", 100, 1200), **GROUPS[grp]))
     outs = [_gpu_decode(make_batch("llama3_8b_decode", perm_seed=p, **kw), 256).out_dec for p in (1, 2, -1)]
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
@@ -85,8 +100,10 @@ def test_split_and_unsplit_agree(O, cuda_lib):
     assert_close(a, b, max_tol=ATOL_MAX, mean_tol=ATOL_MEAN, what="split vs unsplit")
 
 
-def test_one_token_context_returns_v_exactly(cuda_lib):
-    batch = make_batch("llama3_8b_decode", seed=46, overrides=dict(num_seqs=3, hist=("fixed", [0, 0, 0])))
+@pytest.mark.parametrize("grp", sorted(GROUPS))
+def test_one_token_context_returns_v_exactly(cuda_lib, grp):
+    batch = make_batch("llama3_8b_decode", seed=46, overrides=dict(num_seqs=3, hist=("fixed", [0, 0, 0]),
+                                                                   **GROUPS[grp]))
     st = _gpu_decode(batch)
     g = batch.num_q_heads // batch.num_kv_heads
     for s in range(3):
@@ -94,9 +111,11 @@ def test_one_token_context_returns_v_exactly(cuda_lib):
         assert torch.equal(st.out_dec[s], v0.repeat_interleave(g, 0))
 
 
-def test_zero_length_sequence_gives_zero_row(cuda_lib):
+@pytest.mark.parametrize("grp", sorted(GROUPS))
+def test_zero_length_sequence_gives_zero_row(cuda_lib, grp):
     from pagedattention_block_table_b200 import binding as B
-    batch = make_batch("llama3_8b_decode", seed=47, overrides=dict(num_seqs=3, hist=("fixed", [5, 40, 9])))
+    batch = make_batch("llama3_8b_decode", seed=47, overrides=dict(num_seqs=3, hist=("fixed", [5, 40, 9]),
+                                                                   **GROUPS[grp]))
     from pagedattention_block_table_b200.runner import DeviceStep
     st = DeviceStep(batch)
     st.fill_history()
@@ -110,9 +129,10 @@ def test_zero_length_sequence_gives_zero_row(cuda_lib):
     assert torch.isfinite(out.float()).all()
 
 
-def test_bad_block_id_is_flagged_and_stays_in_pool(cuda_lib):
+@pytest.mark.parametrize("hq", [8, 16])
+def test_bad_block_id_is_flagged_and_stays_in_pool(cuda_lib, hq):
     from pagedattention_block_table_b200 import binding as B
-    batch = make_batch("tiny_decode", seed=48)
+    batch = make_batch("tiny_decode", seed=48, overrides=dict(num_q_heads=hq))
     from pagedattention_block_table_b200.runner import DeviceStep
     st = DeviceStep(batch)
     st.fill_history()
@@ -177,13 +197,15 @@ def test_host_pipeline_delivers_the_step_outputs(cuda_lib):
         assert torch.equal(pipe.host_out[s][1], ref.out_pre.cpu())
 
 
+@pytest.mark.parametrize("grp", ["g4", "g8"])
 @pytest.mark.parametrize("split", [64, 256])
-def test_longest_first_order_changes_nothing_but_the_order(O, cuda_lib, split):
+def test_longest_first_order_changes_nothing_but_the_order(O, cuda_lib, split, grp):
     """The host copy of the context lengths only orders the launch (longest (sequence, split) first):
     natural order, the true lengths and deliberately wrong ones all give bit-identical outputs, and
     they match the oracle."""
     from pagedattention_block_table_b200 import binding as B
-    batch = make_batch("llama3_8b_decode", seed=61, overrides=dict(num_seqs=9, hist=("uniform", 0, 1500)))
+    batch = make_batch("llama3_8b_decode", seed=61, overrides=dict(num_seqs=9, hist=("uniform", 0, 1500),
+                                                                   **GROUPS[grp]))
     st = _gpu_decode(batch, split)
     ref = oracle_step(batch, O)["decode"]
     outs = {}
@@ -206,11 +228,13 @@ def test_longest_first_order_changes_nothing_but_the_order(O, cuda_lib, split):
                              host_context_lens=true_lens[:-1])
 
 
-def test_many_splits_and_a_reused_workspace(O, cuda_lib):
+@pytest.mark.parametrize("grp", ["g4", "g8"])
+def test_many_splits_and_a_reused_workspace(O, cuda_lib, grp):
     """79 and 313 splits of one sequence (the reduce kernel loops over more than 32 partials per lane
     group), a second call on the same workspace, and sampled rows against the oracle."""
     from pagedattention_block_table_b200 import binding as B
-    batch = make_batch("llama3_8b_decode", seed=62, overrides=dict(num_seqs=3, hist=("fixed", [20000, 7000, 300])))
+    batch = make_batch("llama3_8b_decode", seed=62, overrides=dict(num_seqs=3, hist=("fixed", [20000, 7000, 300]),
+                                                                   **GROUPS[grp]))
     for split in (256, 64):
         st = _gpu_decode(batch, split)
         first = st.out_dec.clone()
@@ -225,9 +249,9 @@ def test_many_splits_and_a_reused_workspace(O, cuda_lib):
 
 @pytest.mark.parametrize("e", [-20, 20, 0])
 def test_decode_fp8_any_query_magnitude(O, cuda_lib, e):
-    """The FP8 decode keeps q in f16 after rescaling it by a power of two per query: q * 2^e with the
-    softmax scale * 2^-e gives the same scores far outside f16's range (2^20 overflows it, 2^-20 is
-    subnormal in it), and the output still matches the oracle."""
+    """Scores do not depend on how q and the softmax scale share a power of two: q * 2^e with the scale
+    * 2^-e gives the same scores (the FP8 decode folds the scale and the K scale into q in fp32), far
+    outside bf16's usual range of q, and the output still matches the oracle."""
     import math
     batch = make_batch("mha_fp8_decode", seed=63, overrides=dict(num_seqs=3, num_q_heads=8, num_kv_heads=4,
                                                                hist=("uniform", 100, 900)))
