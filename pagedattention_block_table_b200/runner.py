@@ -114,42 +114,94 @@ class DeviceStep:
 class HostPipeline:
     """Serving steps fed from host memory, double-buffered: while the device computes step i, a copy
     stream brings step i+1's inputs (queries, new K/V, slots, tables, lengths) in from pinned host
-    buffers and takes step i-1's outputs back out.  Every step still moves all of its own inputs and
+    memory and takes step i-1's outputs back out.  Every step still moves all of its own inputs and
     outputs across the host link; the copies only overlap the computation instead of preceding it.
+
+    The inputs of a step travel as one packed buffer (one host-to-device copy) and its outputs as one
+    (one device-to-host copy).  Each of the two slots runs its step as a CUDA graph captured once on
+    that slot's buffers (``use_graphs``), so the host issues a handful of calls per step instead of a
+    launch per kernel; the graphs keep the host-side parameters of the :class:`DeviceStep` (maximum
+    length, split, the host copy of the lengths that orders the launch), as the eager launches do.
     """
 
     IN_KEYS = ("q_dec", "k_new", "v_new", "step_slots", "dec_tables", "dec_lens", "q_pre")
+    OUT_KEYS = ("out_dec", "out_pre")
+    ALIGN = 256
 
-    def __init__(self, st: DeviceStep):
+    @classmethod
+    def _layout(cls, st, keys):
+        off, lay = 0, []
+        for k in keys:
+            t = getattr(st, k)
+            n = t.numel() * t.element_size()
+            lay.append((k, off, n, t.dtype, tuple(t.shape)))
+            off += (n + cls.ALIGN - 1) // cls.ALIGN * cls.ALIGN
+        return lay, max(off, cls.ALIGN)
+
+    @staticmethod
+    def _views(buf, lay):
+        return {k: buf[o:o + n].view(dt).view(shape) for k, o, n, dt, shape in lay}
+
+    def __init__(self, st: DeviceStep, use_graphs: bool = True):
         self.st = st
         dev = st.device
-        self.host_in = {k: getattr(st, k).detach().cpu().pin_memory() for k in self.IN_KEYS}
-        self.slots_in = [{k: torch.empty_like(getattr(st, k)) for k in self.IN_KEYS} for _ in range(2)]
-        self.slots_out = [(torch.empty_like(st.out_dec), torch.empty_like(st.out_pre)) for _ in range(2)]
-        self.host_out = [(torch.empty_like(st.out_dec, device="cpu").pin_memory(),
-                          torch.empty_like(st.out_pre, device="cpu").pin_memory()) for _ in range(2)]
+        self.lay_in, nin = self._layout(st, self.IN_KEYS)
+        self.lay_out, nout = self._layout(st, self.OUT_KEYS)
+        self.host_in_buf = torch.empty(nin, dtype=torch.uint8).pin_memory()
+        self.host_in = self._views(self.host_in_buf, self.lay_in)
+        for k in self.IN_KEYS:
+            self.host_in[k].copy_(getattr(st, k).detach().cpu())
+        self.dev_in = [torch.empty(nin, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.slots_in = [self._views(b, self.lay_in) for b in self.dev_in]
+        self.dev_out = [torch.empty(nout, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.slots_out = [self._views(b, self.lay_out) for b in self.dev_out]
+        self.host_out_buf = [torch.empty(nout, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self.host_out = [tuple(self._views(b, self.lay_out)[k] for k in self.OUT_KEYS) for b in self.host_out_buf]
         self.copy = torch.cuda.Stream(device=dev)
         self.comp = torch.cuda.current_stream(dev)
         self.h2d_done = [torch.cuda.Event() for _ in range(2)]
         self.comp_done = [torch.cuda.Event() for _ in range(2)]
         self.d2h_done = [torch.cuda.Event() for _ in range(2)]
+        self.graphs = [self._capture(s) for s in range(2)] if use_graphs else [None, None]
         self.i = 0
 
     @property
     def h2d_bytes(self) -> int:
-        return sum(t.numel() * t.element_size() for t in self.host_in.values())
+        """Bytes copied in per step: the packed input buffer, alignment padding included."""
+        return self.host_in_buf.numel()
 
     @property
     def d2h_bytes(self) -> int:
-        a, b = self.host_out[0]
-        return a.numel() * a.element_size() + b.numel() * b.element_size()
+        """Bytes copied out per step: the packed output buffer."""
+        return self.host_out_buf[0].numel()
+
+    def _bind(self, slot: int):
+        for k, t in self.slots_in[slot].items():
+            setattr(self.st, k, t)
+        for k, t in self.slots_out[slot].items():
+            setattr(self.st, k, t)
+
+    def _capture(self, slot: int):
+        """The step on slot's buffers as a CUDA graph (None if capture is refused: eager launches)."""
+        dev = self.st.device
+        self._bind(slot)
+        self.dev_in[slot].copy_(self.host_in_buf)
+        try:
+            torch.cuda.synchronize(dev)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=torch.cuda.Stream(dev), capture_error_mode="thread_local"):
+                self.st.step()
+            torch.cuda.synchronize(dev)
+            return g
+        except RuntimeError:
+            torch.cuda.synchronize(dev)
+            return None
 
     def _load(self, slot: int):
         with torch.cuda.stream(self.copy):
             if self.i >= 2:
                 self.copy.wait_event(self.comp_done[slot])      # slot's previous step has read its inputs
-            for k, t in self.host_in.items():
-                self.slots_in[slot][k].copy_(t, non_blocking=True)
+            self.dev_in[slot].copy_(self.host_in_buf, non_blocking=True)
             self.h2d_done[slot].record(self.copy)
 
     def step(self):
@@ -157,21 +209,21 @@ class HostPipeline:
         s = self.i % 2
         if self.i == 0:
             self._load(0)
-        st = self.st
         self.comp.wait_event(self.h2d_done[s])
         if self.i >= 2:
             self.comp.wait_event(self.d2h_done[s])              # output slot free again
-        for k, t in self.slots_in[s].items():
-            setattr(st, k, t)
-        st.out_dec, st.out_pre = self.slots_out[s]
-        st.step(self.comp)
+        if self.graphs[s] is not None:
+            with torch.cuda.stream(self.comp):
+                self.graphs[s].replay()
+        else:
+            self._bind(s)
+            self.st.step(self.comp)
         self.comp_done[s].record(self.comp)
         self.i += 1
         self._load(self.i % 2)
         with torch.cuda.stream(self.copy):
             self.copy.wait_event(self.comp_done[s])
-            self.host_out[s][0].copy_(self.slots_out[s][0], non_blocking=True)
-            self.host_out[s][1].copy_(self.slots_out[s][1], non_blocking=True)
+            self.host_out_buf[s].copy_(self.dev_out[s], non_blocking=True)
             self.d2h_done[s].record(self.copy)
 
     def finish(self):

@@ -175,19 +175,23 @@ def test_kv_head_shards_reproduce_the_unsharded_call(O, cuda_lib):
     assert torch.equal(torch.cat(parts, dim=1), full)
 
 
-def test_host_pipeline_delivers_the_step_outputs(cuda_lib):
+@pytest.mark.parametrize("graphs", [True, False])
+def test_host_pipeline_delivers_the_step_outputs(cuda_lib, graphs):
     """The double-buffered host-fed pipeline (inputs copied in and outputs copied out every step,
-    overlapped with compute) returns the same outputs to the host as a plain device step."""
+    overlapped with compute; CUDA graphs per slot or eager launches) returns the same outputs to the
+    host as a plain device step, and a step run after new inputs were written to the host buffer uses
+    those inputs."""
     from pagedattention_block_table_b200.runner import DeviceStep, HostPipeline
     # no shared prefixes: a repeated step is then idempotent (with forks, re-copying a page that its
     # last holder already appended into would change the copy)
-    batch = make_batch("mixed_step", seed=53, overrides=dict(
-        num_seqs=6, hist=("uniform", 20, 300), share_group=0, share_prefix=0, prefill_chunks=2,
-        chunk_len=(30, 150), chunk_hist=(1, 100), num_q_heads=8, num_kv_heads=2))
+    ov = dict(num_seqs=6, hist=("uniform", 20, 300), share_group=0, share_prefix=0, prefill_chunks=2,
+              chunk_len=(30, 150), chunk_hist=(1, 100), num_q_heads=8, num_kv_heads=2)
+    batch = make_batch("mixed_step", seed=53, overrides=ov)
     ref = _gpu_decode(batch, 64)
     st = DeviceStep(batch, split_tokens=64)
     st.fill_history()
-    pipe = HostPipeline(st)
+    pipe = HostPipeline(st, use_graphs=graphs)
+    assert (pipe.graphs[0] is not None) == graphs
     for _ in range(5):
         pipe.step()
     pipe.finish()
@@ -195,6 +199,20 @@ def test_host_pipeline_delivers_the_step_outputs(cuda_lib):
     for s in range(2):
         assert torch.equal(pipe.host_out[s][0], ref.out_dec.cpu())
         assert torch.equal(pipe.host_out[s][1], ref.out_pre.cpu())
+    # new queries through the host buffer (negated: exact).  The next step's inputs are already on the
+    # device, so the two steps after it (one per slot) are the first to read the new ones
+    batch2 = make_batch("mixed_step", seed=53, overrides=ov)
+    batch2.q_decode = -batch2.q_decode
+    ref2 = _gpu_decode(batch2, 64)
+    pipe.host_in["q_dec"].copy_(batch2.q_decode)
+    for _ in range(3):
+        pipe.step()
+    pipe.finish()
+    torch.cuda.synchronize()
+    for s in range(2):
+        assert torch.equal(pipe.host_out[s][0], ref2.out_dec.cpu())
+        assert torch.equal(pipe.host_out[s][1], ref.out_pre.cpu())
+    assert not torch.equal(ref2.out_dec, ref.out_dec)
 
 
 @pytest.mark.parametrize("grp", ["g4", "g8"])
