@@ -23,10 +23,19 @@ def _sources():
                   + glob.glob(os.path.join(CSRC, "*.cpp")) + [os.path.join(ROOT, "include", "pagedattn.h")])
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank lines (what the compiler sees, for the digest)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def source_digest(names=None) -> str:
-    """sha256 of CUDA sources: identifies which kernels a profile was taken on.  `names` lists the csrc
-    files a kernel depends on (for example its header, pa_common.cuh and api.cu, which holds its launch
-    code); None takes every csrc/*.cu and *.cuh.  Host-only C++ (the block manager) never enters it."""
+    """sha256 of CUDA sources, comments left out: identifies which kernels a profile was taken on.
+    `names` lists the csrc files a kernel depends on (for example its header, pa_common.cuh and api.cu,
+    which holds its launch code); None takes every csrc/*.cu and *.cuh.  Host-only C++ (the block
+    manager) never enters it."""
     import hashlib
     h = hashlib.sha256()
     if names is None:
@@ -34,8 +43,8 @@ def source_digest(names=None) -> str:
     else:
         files = [os.path.join(CSRC, n) for n in sorted(names)]
     for src in files:
-        with open(src, "rb") as f:
-            h.update(os.path.basename(src).encode() + b"\0" + f.read())
+        with open(src, encoding="utf-8") as f:
+            h.update(os.path.basename(src).encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

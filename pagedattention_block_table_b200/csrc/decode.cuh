@@ -9,7 +9,7 @@
 // CTA per unit; its warps take the split's 16-token blocks round-robin and each warp runs its
 // own pipeline: lane 0 pulls the (block, head) K tile and V tile -- each one contiguous
 // 16*head_dim run in the [block][head][16][D] layout -- into shared memory with 1-D bulk async
-// copies (cp.async.bulk, mbarrier completion, no multicast), STAGES blocks ahead.  All query
+// copies (mbarrier completion, this CTA's own shared memory only), STAGES blocks ahead.  All query
 // heads of the group are processed against each tile, so every KV byte crosses HBM once.
 // Scores use an fp32 online softmax in base 2 (q is pre-scaled by scale*log2(e)); partial
 // sums are combined with warp shuffles.  Warps of a CTA merge their (max, sum, output) in

@@ -15,7 +15,7 @@
 //   O[16][D] += P V                    P (bf16) is built from S's fragments in registers; V's fragments
 //                                      come from shared memory with ldmatrix.trans (V is token-major)
 // K and V tiles reach shared memory by 2-D TMA (the cache seen as rows of D elements, one 16-row x
-// 64-element box per 64-element plane, 128-byte swizzle, no multicast), so ldmatrix and the 16-byte K
+// 64-element box per 64-element plane, 128-byte swizzle, into this CTA's own shared memory), so ldmatrix and the 16-byte K
 // loads are free of bank conflicts.  The dims of a k-step are permuted (the same way for Q and K, which
 // leaves the dot product unchanged) so that each lane's K fragments come from two 16-byte loads.
 #pragma once

@@ -104,7 +104,7 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
 }
 
 // 1-D bulk async copy global -> this CTA's shared memory, completing `bytes` on `bar`.
-// dst and src 16-byte aligned, bytes a multiple of 16.  No multicast.
+// dst and src 16-byte aligned, bytes a multiple of 16.  The destination is this CTA's own shared memory.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
                                          uint64_t policy) {
   asm volatile(

@@ -15,7 +15,7 @@
 // Keys come in tiles of 128 (8 units of 16 tokens).  K and V tiles take turns in one ring of shared
 // memory slots (K0, V0, K1, V1, ...), filled by TMA with one 16-row x 64-element box per unit and per
 // 64-element plane of head_dim, in the UMMA 128-byte-swizzled layout (tensor map over the cache seen
-// as [num_blocks*Hkv*block_size][head_dim]; no multicast).
+// as [num_blocks*Hkv*block_size][head_dim]; each CTA loads its own copy).
 // TMEM (512 columns): S_A, S_B (128 columns each), O_A, O_B (head_dim columns each).
 // Per key tile j and query tile X:
 //   S_X = Q_X K_j^T        M=128, N=128, both operands in shared memory, fp32 into TMEM

@@ -118,3 +118,12 @@ def test_prefill_rejects_fp8_and_bad_heads(L):
     f = L.pa_paged_prefill
     assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 1, 16, 64, None) == B.PA_EUNSUPPORTED
     assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 16, 0.1, 0, 16, 64, None) == B.PA_EINVAL
+
+
+def test_source_digest_ignores_comments_only():
+    """Profiles are tied to kernel code by a digest of the sources without their comments: a comment
+    edit keeps a committed DRAM measurement valid, any code edit voids it."""
+    strip = build._code_only
+    a = "int f() {  // returns one\n  return 1; /* the\n value */\n}\n"
+    assert strip(a) == strip("int f() {\n  return 1;\n\n}  // changed comment\n")
+    assert strip(a) != strip("int f() {\n  return 2;\n}\n")
