@@ -334,7 +334,7 @@ def measure(name, dev, K, W, args, rank, world, clk, e2e=False):
 
     full = workload_batch(name, dev, args.num_seqs if name == args.workload else 0)
     batch = rank_batch(full, rank, world, args.partition)
-    st = DeviceStep(batch, device=dev, split_tokens=args.split or None)
+    st = DeviceStep(batch, device=dev, split_tokens=args.split or None, overlap=not args.no_overlap)
     st.fill_history()
     torch.cuda.synchronize(dev)
     for _ in range(max(3, W)):
@@ -683,6 +683,8 @@ def parse_args(argv=None):
                     help="N>1: whole batch per rank (weak scaling) or KV heads split over the ranks (strong)")
     ap.add_argument("--split", type=int, default=0, help="split_tokens (0 = library default)")
     ap.add_argument("--no-graph", action="store_true", help="time the steps as stream launches, not graph replays")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run a step's decode and prefill one after the other on one stream")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other full-size workloads at N=1")
     ap.add_argument("--sub-steps", type=int, default=50, help="timed steps of each of the other workloads")
     ap.add_argument("--cpu-budget-s", type=float, default=4.0)

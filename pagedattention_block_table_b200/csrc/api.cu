@@ -375,13 +375,24 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 8) per_sm = 8;
   const int64_t slots = (int64_t)device_sm_count() * per_sm;
-  // Splits of at most 2048 tokens, shortened (powers of two, down to 256) until there are ~4 waves
-  // of work units.  Measured on B200 (pa_paged_attention GB/s by split length, longest-first launch
-  // order): Llama-3-8B decode batch 512: 5182, 1024: 5461, 2048: 5018 (the wave rule picks 1024);
-  // mixed step 512: 5264, 1024: 5807, 2048: 6035; FP8 MHA 512: 4544, 1024: 4736, 2048: 4839.
+  // Splits of at most 2048 tokens, shortened (powers of two, down to 256) until the launch has enough
+  // waves of work units.  Measured on B200 (pa_paged_attention GB/s by split length, longest-first
+  // launch order):
+  //   CUDA-core kernel: Llama-3-8B batch 512: 5182, 1024: 5461, 2048: 5018; FP8 MHA 512: 4544,
+  //     1024: 4736, 2048: 4839  -> about 4 waves;
+  //   tensor-core kernel: Llama-3-8B batch 512: 6173, 1024: 6383, 2048: 6433 (3.5 waves at 2048); GQA-8
+  //     batch 512: 5315, 1024: 5433, 2048: 5725 (1.2 waves); 8 x 32768 tokens 512: 6277, 1024: 6530,
+  //     2048: 6386  -> one wave, and 4 waves once a sequence has 8 or more splits.
   int64_t S = 256;
   while (S < max_context_len && S < 2048) S *= 2;
-  while (S > 256 && units * ceil_div64(max_context_len, S) < 4 * slots) S /= 2;
+  const bool mma = decode_uses_mma(kv_dtype, group);
+  auto enough = [&](int64_t s) {
+    const int64_t splits = ceil_div64(max_context_len, s);
+    const int64_t work = units * splits;
+    if (!mma) return work >= 4 * slots;
+    return work >= slots && (splits < 8 || work >= 4 * slots);
+  };
+  while (S > 256 && !enough(S)) S /= 2;
   return static_cast<int>(S);
 }
 

@@ -209,16 +209,13 @@ __device__ __forceinline__ void mma_ts_group8(uint32_t d_tmem, uint32_t a_tmem, 
 #undef PA_MMA_TS
 }
 
-// Store 32 consecutive 32-bit columns of this thread's TMEM lane (no wait).
-__device__ __forceinline__ void tmem_st32u_nowait(uint32_t taddr, const uint32_t *v) {
+// Store 16 consecutive 32-bit columns of this thread's TMEM lane (no wait).
+__device__ __forceinline__ void tmem_st16u_nowait(uint32_t taddr, const uint32_t *v) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
-      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]),
-      "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]),
-      "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -459,14 +456,18 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     const float qs = P.qscale;
     float m_ref = -INFINITY, l_run = 0.f;
     for (int j = 0; j < ntiles; ++j) {
+      const int kbase = j * C::BN;
+      const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
+      // the passes below store P with warp-collective tcgen05.st, so the choice of pass is made per warp:
+      // the masking pass when any row of the warp has a key past its position (it masks nothing for the
+      // other rows).  Decided before S is ready, off the tile's critical path.
+      const bool wdiag = __any_sync(0xffffffffu, diag);
       // every wait's outcome is made warp-uniform: the tcgen05.ld/st below are warp-collective.
       // S_X(j) complete also means O_X(j-1) complete (issued before it, tracked by the same commit).
       if (!__all_sync(0xffffffffu, mbar_wait(&bars[kSFull + X], j & 1))) { timeout = true; break; }
       tc_fence_after();
       uint32_t sr[C::BN];
       tmem_ld128(s_addr, sr);
-      const int kbase = j * C::BN;
-      const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
       // last key tile: V rows of keys no row may see, up to the last 16-key step the PV product reads,
       // are zeroed (tile A's threads, one row each) once the V tile has landed, so that 0 * (whatever
       // the cache holds past the context) never reaches the MMA
@@ -525,35 +526,38 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       float sum = 0.f;
       auto pass = [&](auto diag_c) {
         constexpr bool kDiag = decltype(diag_c)::value;
-        float mx = -INFINITY;
+        // two independent max chains, P stored in quarters of 32 keys: the last store and the last max
+        // are short when the pass ends
+        float mx = -INFINITY, my = -INFINITY;
         uint64_t ls2 = 0ull;
         const uint64_t qs2 = f2pack(qs, qs), nm2 = f2pack(-m_ref, -m_ref);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+        for (int qq = 0; qq < 4; ++qq) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int k2 = 0; k2 < 32; ++k2) {
-            const int k = half * 64 + 2 * k2;
+          for (int k2 = 0; k2 < 16; ++k2) {
+            const int k = qq * 32 + 2 * k2;
             float2 x = f2unpack(ffma2(f2pack(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), qs2, nm2));
             if (kDiag) {
               if (kbase + k > pos) x.x = -INFINITY;
               if (kbase + k + 1 > pos) x.y = -INFINITY;
             }
-            mx = fmax3(mx, x.x, x.y);
+            if (k2 & 1)
+              my = fmax3(my, x.x, x.y);
+            else
+              mx = fmax3(mx, x.x, x.y);
             const float a = ex2(x.x);
             const float b = ex2(x.y);
             ls2 = f2add(ls2, f2pack(a, b));
             pk[k2] = pack_bf16x2(a, b);
           }
-          tmem_st32u_nowait(s_addr + half * 32, pk);
+          tmem_st16u_nowait(s_addr + qq * 16, pk);
         }
+        mx = fmaxf(mx, my);
         const float2 lsv = f2unpack(ls2);
         sum = lsv.x + lsv.y;
         return mx;
       };
-      // the pass stores P with warp-collective tcgen05.st, so the choice is made per warp: the masking pass
-      // when any row of the warp has a key past its position (it masks nothing for the other rows)
-      const bool wdiag = __any_sync(0xffffffffu, diag);
       const float mx = wdiag ? pass(std::true_type{}) : pass(std::false_type{});
       // The reference moves only when the tile's max exceeds it by more than 2^8: then P is recomputed
       // against the new one (p of such a tile may even have overflowed), O and l are rescaled below.  The
@@ -571,7 +575,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         tmem_wait_st();
         (void)(wdiag ? pass(std::true_type{}) : pass(std::false_type{}));
       }
-      l_run = l_run * alpha + sum;
       if (any_bump && j > 0) {
         // rescale this row's O to the new reference (O_X(j-1) is complete; O_X(j) waits for P_X(j))
 #pragma unroll 1
@@ -586,6 +589,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bars[kPFull + X]);
+      l_run = l_run * alpha + sum;
     }
     // ---- epilogue: out = O / l once the last PV is done
     if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0))) {

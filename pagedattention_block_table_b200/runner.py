@@ -22,9 +22,12 @@ class DeviceStep:
     """Device-resident state (cache, tables, inputs) of one :class:`PagedBatch` step."""
 
     def __init__(self, batch: PagedBatch, device="cuda", split_tokens: Optional[int] = None,
-                 zero_cache: bool = True):
+                 zero_cache: bool = True, overlap: bool = True):
         self.batch = batch
         self.device = torch.device(device)
+        self.overlap = overlap
+        self._side = None
+        self._ev = None
         dev = self.device
         nb, hkv, d = batch.num_blocks, batch.num_kv_heads, batch.head_dim
         self.kv_dtype = batch.kv_dtype
@@ -103,11 +106,28 @@ class DeviceStep:
                            self.pre_lens, self.batch.scale, self.max_q, self.pre_max_len, self.kv_dtype, stream)
 
     def step(self, stream=None):
-        """copy-on-write forks -> append -> decode attention -> prefill attention."""
-        self.fork(stream)
-        self.append(stream)
-        self.decode(stream)
-        self.prefill(stream)
+        """copy-on-write forks -> append -> decode attention and prefill attention.
+
+        Decode and prefill both read the cache the append has just written and write separate outputs,
+        so with ``overlap`` (and both present) the decode runs on a second stream beside the prefill:
+        the HBM-bound decode CTAs fill the SMs the tensor-bound prefill leaves idle in its last waves.
+        """
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        self.fork(s)
+        self.append(s)
+        if self.overlap and self.batch.num_decode and self.max_q:
+            if self._side is None:
+                self._side = torch.cuda.Stream(device=self.device)
+                self._ev = (torch.cuda.Event(), torch.cuda.Event())
+            self._ev[0].record(s)
+            self._side.wait_event(self._ev[0])
+            self.decode(self._side)
+            self.prefill(s)
+            self._ev[1].record(self._side)
+            s.wait_event(self._ev[1])
+        else:
+            self.decode(s)
+            self.prefill(s)
 
 
 
