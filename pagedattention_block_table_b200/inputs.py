@@ -46,6 +46,9 @@ WORKLOADS: Dict[str, dict] = {
     # four query heads, so each KV tile is fetched by two CTAs; measures whether the second fetch hits L2
     "gqa8_decode": dict(num_seqs=32, num_q_heads=64, num_kv_heads=8, head_dim=128,
                         hist=("uniform", 512, 4096)),
+    # the Llama-3-8B decode batch over an FP8 E4M3 cache: four query heads meet every dequantised byte
+    "llama3_8b_fp8_decode": dict(num_seqs=64, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                                 hist=("uniform", 512, 4096), kv_dtype="fp8"),
 }
 WORKLOAD_SEED = {name: 1001 + i for i, name in enumerate(WORKLOADS)}
 
