@@ -308,7 +308,8 @@ def launches_per_step(st) -> int:
 def decode_kernel_label(batch) -> str:
     """Which decode kernel pa_paged_attention runs for this batch (the library decides)."""
     from pagedattention_block_table_b200 import binding as B
-    tc = B.pa_paged_attention_uses_tensor_cores(batch.num_q_heads, batch.num_kv_heads, batch.kv_dtype)
+    tc = B.pa_paged_attention_uses_tensor_cores(batch.num_q_heads, batch.num_kv_heads, batch.head_dim,
+                                                batch.kv_dtype)
     k = "paged_decode_mma_kernel (mma.sync)" if tc == 1 else "paged_decode_kernel"
     return f"pa_paged_attention ({k} + lse_reduce_kernel)"
 

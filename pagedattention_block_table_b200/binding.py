@@ -71,7 +71,7 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_attention_auto_split.restype = I
         L.pa_paged_attention_auto_split.argtypes = [I, I, I, I, I, I]
         L.pa_paged_attention_uses_tensor_cores.restype = I
-        L.pa_paged_attention_uses_tensor_cores.argtypes = [I, I, I]
+        L.pa_paged_attention_uses_tensor_cores.argtypes = [I, I, I, I]
         L.pa_paged_attention.restype = I
         L.pa_paged_attention.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, I, F, I, P, P, I, I, P, P, SZ, P]
         L.pa_paged_attention_noalloc.restype = I
@@ -233,8 +233,8 @@ def pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                                    max_context_len, kv_dtype))
 
 
-def pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, kv_dtype=PA_KV_BF16) -> int:
-    return int(lib().pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, kv_dtype))
+def pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, head_dim=128, kv_dtype=PA_KV_BF16) -> int:
+    return int(lib().pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, head_dim, kv_dtype))
 
 
 def _host_i32(a, n):

@@ -29,8 +29,14 @@
 #ifndef PA_DEC_MMA_MIN_GROUP
 #define PA_DEC_MMA_MIN_GROUP 4
 #endif
+#ifndef PA_DEC_MMA_MIN_GROUP_Q8
+#define PA_DEC_MMA_MIN_GROUP_Q8 4
+#endif
 #ifndef PA_DEC_MMA_STAGES
 #define PA_DEC_MMA_STAGES 2
+#endif
+#ifndef PA_DEC_MMA_STAGES_Q8
+#define PA_DEC_MMA_STAGES_Q8 4   // one-byte tiles are half the size: twice the stages, the same bytes in flight
 #endif
 #ifndef PA_DEC_STAGES_SMALL
 #define PA_DEC_STAGES_SMALL 2
@@ -81,12 +87,20 @@ int queries_per_cta(int group) {
 // use the CUDA-core kernel.  Measured on B200 (pa_paged_attention GB/s, CUDA graphs of calls): the
 // Llama-3-8B batch (G = 4) 6,030-6,090 on the CUDA cores, 6,370 on the tensor cores; the 32-sequence
 // batch with G = 8 (64 / 8 heads) 3,210 and 5,280.
-bool decode_uses_mma(int kv_dtype, int group) {
-  return kv_dtype == PA_KV_BF16 && group >= PA_DEC_MMA_MIN_GROUP && (group <= 16 || group % 16 == 0);
+bool decode_uses_mma(int kv_dtype, int group, int head_dim) {
+  if (!(group <= 16 || group % 16 == 0)) return false;
+  if (kv_dtype == PA_KV_BF16) return group >= PA_DEC_MMA_MIN_GROUP;
+  // one-byte caches: f16 products on dequantised tiles, head_dim 128
+  return head_dim == 128 && group >= PA_DEC_MMA_MIN_GROUP_Q8;
 }
-int decode_heads_per_cta(int kv_dtype, int group) {
-  if (decode_uses_mma(kv_dtype, group)) return group < 16 ? group : 16;
+int decode_heads_per_cta(int kv_dtype, int group, int head_dim) {
+  if (decode_uses_mma(kv_dtype, group, head_dim)) return group < 16 ? group : 16;
   return queries_per_cta(group);
+}
+int decode_mma_smem(int kv_dtype, int head_dim) {
+  if (kv_dtype != PA_KV_BF16) return pa::DecodeMmaCfg<1, 128, PA_DEC_NW, PA_DEC_MMA_STAGES_Q8>::SMEM;
+  return head_dim == 128 ? pa::DecodeMmaCfg<0, 128, PA_DEC_NW, PA_DEC_MMA_STAGES>::SMEM
+                         : pa::DecodeMmaCfg<0, 64, PA_DEC_NW, PA_DEC_MMA_STAGES>::SMEM;
 }
 
 template <typename K>
@@ -180,11 +194,12 @@ pa_status dispatch_decode(int kt, int d, int qpb, const pa::DecodeParams &P, con
   return PA_EUNSUPPORTED;
 }
 
-template <int D, bool HI, bool ORDERED>
+template <int KT, int D, bool HI, bool ORDERED>
 pa_status launch_decode_mma_as(const pa::DecodeParams &P, const CUtensorMap &km, const CUtensorMap &vm,
                                const pa::WorkOrder<ORDERED> &W, dim3 grid, cudaStream_t st) {
-  using C = pa::DecodeMmaCfg<D, PA_DEC_NW, PA_DEC_MMA_STAGES>;
-  auto kern = pa::paged_decode_mma_kernel<D, PA_DEC_NW, PA_DEC_MMA_STAGES, HI, ORDERED>;
+  constexpr int S = KT == 0 ? PA_DEC_MMA_STAGES : PA_DEC_MMA_STAGES_Q8;
+  using C = pa::DecodeMmaCfg<KT, D, PA_DEC_NW, S>;
+  auto kern = pa::paged_decode_mma_kernel<KT, D, PA_DEC_NW, S, HI, ORDERED>;
   pa_status s = set_smem(kern, C::SMEM);
   if (s != PA_OK) return s;
   if (pa::launch_pdl(kern, grid, dim3(PA_DEC_NW * 32), C::SMEM, st, P, km, vm, W) != cudaSuccess)
@@ -192,28 +207,33 @@ pa_status launch_decode_mma_as(const pa::DecodeParams &P, const CUtensorMap &km,
   return launch_status();
 }
 
-template <int D, bool HI>
+template <int KT, int D, bool HI>
 pa_status launch_decode_mma(const pa::DecodeParams &P, const CUtensorMap &km, const CUtensorMap &vm,
                             const pa::WorkOrder<true> *order, int n_order, dim3 grid, cudaStream_t st) {
-  if (order) return launch_decode_mma_as<D, HI, true>(P, km, vm, *order, dim3(grid.x, n_order, 1), st);
-  return launch_decode_mma_as<D, HI, false>(P, km, vm, pa::WorkOrder<false>{}, grid, st);
+  if (order) return launch_decode_mma_as<KT, D, HI, true>(P, km, vm, *order, dim3(grid.x, n_order, 1), st);
+  return launch_decode_mma_as<KT, D, HI, false>(P, km, vm, pa::WorkOrder<false>{}, grid, st);
 }
 
-// Tensor-core decode: tensor maps over the two caches (rows of head_dim bf16 elements), then the launch
-// for head_dim and for whether the CTA's heads reach past 8 rows.
-pa_status dispatch_decode_mma(int d, int hpc, const pa::DecodeParams &P, const pa::WorkOrder<true> *order,
+// Tensor-core decode: tensor maps over the two caches (rows of head_dim elements), then the launch for the
+// cache element, head_dim and whether the CTA's heads reach past 8 rows.
+pa_status dispatch_decode_mma(int kt, int d, int hpc, const pa::DecodeParams &P, const pa::WorkOrder<true> *order,
                               int n_order, dim3 grid, cudaStream_t st) {
   CUtensorMap km, vm;
   const int64_t rows = P.num_blocks * P.num_kv_heads * P.block_size;
-  if (!pa::make_cache_map(&km, P.k_cache, rows, d) || !pa::make_cache_map(&vm, P.v_cache, rows, d)) {
+  const bool maps = kt == PA_KV_BF16
+                        ? pa::make_cache_map(&km, P.k_cache, rows, d) && pa::make_cache_map(&vm, P.v_cache, rows, d)
+                        : pa::make_cache_map_u8(&km, P.k_cache, rows, d) && pa::make_cache_map_u8(&vm, P.v_cache, rows, d);
+  if (!maps) {
     fprintf(stderr, "pagedattn: tensor map encoding for the decode failed\n");
     return PA_ECUDA;
   }
   const bool hi = hpc > 8;
-  if (d == 128) return hi ? launch_decode_mma<128, true>(P, km, vm, order, n_order, grid, st)
-                          : launch_decode_mma<128, false>(P, km, vm, order, n_order, grid, st);
-  if (d == 64) return hi ? launch_decode_mma<64, true>(P, km, vm, order, n_order, grid, st)
-                         : launch_decode_mma<64, false>(P, km, vm, order, n_order, grid, st);
+#define PA_DM(KT, D)                                                                                 \
+  if (kt == KT && d == D)                                                                            \
+    return hi ? launch_decode_mma<KT, D, true>(P, km, vm, order, n_order, grid, st)                  \
+              : launch_decode_mma<KT, D, false>(P, km, vm, order, n_order, grid, st);
+  PA_DM(0, 128) PA_DM(0, 64) PA_DM(1, 128) PA_DM(2, 128)
+#undef PA_DM
   return PA_EUNSUPPORTED;
 }
 
@@ -365,12 +385,10 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
                                   int max_context_len, int kv_dtype) {
   if (num_seqs <= 0 || num_kv_heads <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 16;
   const int group = num_q_heads / num_kv_heads;
-  const int hpc = decode_heads_per_cta(kv_dtype, group > 0 ? group : 1);
+  const int hpc = decode_heads_per_cta(kv_dtype, group > 0 ? group : 1, head_dim);
   const int64_t units = (int64_t)num_seqs * num_kv_heads * (group / hpc > 0 ? group / hpc : 1);
-  const int smem = decode_uses_mma(kv_dtype, group)
-                       ? (head_dim == 128 ? pa::DecodeMmaCfg<128, PA_DEC_NW, PA_DEC_MMA_STAGES>::SMEM
-                                          : pa::DecodeMmaCfg<64, PA_DEC_NW, PA_DEC_MMA_STAGES>::SMEM)
-                       : decode_smem_rt(kv_dtype, head_dim, hpc);
+  const int smem = decode_uses_mma(kv_dtype, group, head_dim) ? decode_mma_smem(kv_dtype, head_dim)
+                                                              : decode_smem_rt(kv_dtype, head_dim, hpc);
   int per_sm = smem > 0 ? (227 * 1024) / (smem + 1024) : 1;
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 8) per_sm = 8;
@@ -385,7 +403,7 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
   //     2048: 6386  -> one wave, and 4 waves once a sequence has 8 or more splits.
   int64_t S = 256;
   while (S < max_context_len && S < 2048) S *= 2;
-  const bool mma = decode_uses_mma(kv_dtype, group);
+  const bool mma = decode_uses_mma(kv_dtype, group, head_dim);
   auto enough = [&](int64_t s) {
     const int64_t splits = ceil_div64(max_context_len, s);
     const int64_t work = units * splits;
@@ -396,9 +414,11 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
   return static_cast<int>(S);
 }
 
-int pa_paged_attention_uses_tensor_cores(int num_q_heads, int num_kv_heads, int kv_dtype) {
+int pa_paged_attention_uses_tensor_cores(int num_q_heads, int num_kv_heads, int head_dim, int kv_dtype) {
   if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return -1;
-  return decode_uses_mma(kv_dtype, num_q_heads / num_kv_heads) ? 1 : 0;
+  if (head_dim != 64 && head_dim != 128) return -1;
+  if (kv_dtype != PA_KV_BF16 && kv_dtype != PA_KV_FP8_E4M3 && kv_dtype != PA_KV_INT8) return -1;
+  return decode_uses_mma(kv_dtype, num_q_heads / num_kv_heads, head_dim) ? 1 : 0;
 }
 
 size_t pa_paged_attention_workspace_size(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
@@ -430,8 +450,8 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
   if (kv_dtype != PA_KV_BF16 && (!k_scale || !v_scale)) return PA_EINVAL;
   const int group = num_q_heads / num_kv_heads;
-  const bool mma = decode_uses_mma(kv_dtype, group);
-  const int qpb = decode_heads_per_cta(kv_dtype, group);
+  const bool mma = decode_uses_mma(kv_dtype, group, head_dim);
+  const int qpb = decode_heads_per_cta(kv_dtype, group, head_dim);
   if ((int64_t)num_kv_heads * (group / qpb) > (int64_t(1) << 31) - 1) return PA_EINVAL;
   int S = split_tokens;
   if (S == 0) S = pa_paged_attention_auto_split(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, kv_dtype);
@@ -474,7 +494,7 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
   const int n_order = host_context_lens ? build_work_order(host_context_lens, num_seqs, S, max_context_len,
                                                            static_cast<int>(max_splits), order.item)
                                         : 0;
-  pa_status s = mma ? dispatch_decode_mma(head_dim, qpb, P, n_order ? &order : nullptr, n_order, grid, st)
+  pa_status s = mma ? dispatch_decode_mma(kv_dtype, head_dim, qpb, P, n_order ? &order : nullptr, n_order, grid, st)
                     : dispatch_decode(kv_dtype, head_dim, qpb, P, n_order ? &order : nullptr, n_order, grid, st);
   if (s != PA_OK || max_splits <= 1) return s;
   dim3 rgrid(static_cast<unsigned>((num_q_heads + 3) / 4), static_cast<unsigned>(num_seqs));

@@ -15,29 +15,44 @@
 //   O[16][D] += P V                    P (bf16) is built from S's fragments in registers; V's fragments
 //                                      come from shared memory with ldmatrix.trans (V is token-major)
 // K and V tiles reach shared memory by 2-D TMA (the cache seen as rows of D elements, one 16-row x
-// 64-element box per 64-element plane, 128-byte swizzle, into this CTA's own shared memory), so ldmatrix and the 16-byte K
-// loads are free of bank conflicts.  The dims of a k-step are permuted (the same way for Q and K, which
-// leaves the dot product unchanged) so that each lane's K fragments come from two 16-byte loads.
+// 128-byte box per 128-byte plane, 128-byte swizzle, into this CTA's own shared memory), so ldmatrix and
+// the 16-byte K loads are free of bank conflicts.  The dims of a k-step are permuted (the same way for Q
+// and K, which leaves the dot product unchanged) so that each lane's K fragments come from two 16-byte
+// loads.
+//
+// One-byte caches (FP8 E4M3, INT8; head_dim 128): the products run in f16 (m16n8k16, f32 accumulate).
+// Every E4M3 and INT8 code is exact in f16.  Q is scaled per row by a power of two into [1, 2) before it
+// is rounded to f16 (exact for every bf16 entry within 2^-14 of the row's largest), and that power, the
+// softmax scale and the K scale multiply the scores; the V scale multiplies the output.  A lane converts
+// the 32 bytes [32p, 32p+32) of a K row into 16 f16 pairs (k-step s takes pairs 2s and 2s+1, and Q uses
+// the same dims).  V needs pairs along tokens, so a lane converts its V row's 32 bytes into 16 pairs of
+// adjacent dims and `movmatrix.trans` turns each 8x8 block (8 tokens x the 8 dims {32p' + 2j, +1}) into
+// the B fragment of n-tile j; n-tile j of the output then holds dims 32p + 2j, +1, so a lane's 16 n-tiles
+// cover its 32 contiguous dims.
 #pragma once
 #include "decode.cuh"
 #include "prefill.cuh"   // tensor-map encoding, 2-D TMA load
 
 namespace pa {
 
-template <int D, int NW, int STAGES>
+template <int KT, int D, int NW, int STAGES>
 struct DecodeMmaCfg {
-  static constexpr int PLANES = D / 64;                 // 64-element (128-byte) planes of a row
+  static constexpr int E = KT == 0 ? 2 : 1;             // bytes per cache element
+  static constexpr int ROWB = D * E;                    // bytes of one token row of one head
+  static constexpr int PLANES = ROWB / 128;             // 128-byte planes of a row
   static constexpr int PLANE = kBlock * 128;            // one 16-row plane: 2 KB
   static constexpr int TILE = PLANES * PLANE;           // one (unit, head) K or V tile
   static constexpr int KS = D / 16;                     // k-steps of the QK product
   static constexpr int NT = D / 8;                      // 8-dim n-tiles of the PV product
   static constexpr int BAR_BYTES = STAGES * 8;
-  // swizzled tiles need 1024-byte alignment: each warp's area is a multiple of 1024
-  static constexpr int WARP_BYTES = ((2 * STAGES * TILE + BAR_BYTES) + 1023) / 1024 * 1024;
-  static constexpr int SMEM = NW * WARP_BYTES + 1024;   // + slack to align the base
   static constexpr int ML = 16 * D;                     // offset of the (m, l) pairs in a warp's merge area
+  // a warp's tiles, reused at the end as its merge area (16 rows of O and their (m, l)), then its barriers
+  static constexpr int DATA = 2 * STAGES * TILE > (ML + 32) * 4 ? 2 * STAGES * TILE : (ML + 32) * 4;
+  // swizzled tiles need 1024-byte alignment: each warp's area is a multiple of 1024
+  static constexpr int WARP_BYTES = ((DATA + BAR_BYTES) + 1023) / 1024 * 1024;
+  static constexpr int SMEM = NW * WARP_BYTES + 1024;   // + slack to align the base
   static_assert(D == 64 || D == 128, "head_dim");
-  static_assert((16 * D + 32) * 4 <= 2 * STAGES * TILE, "merge area fits in the warp's tiles");
+  static_assert(KT == 0 || D == 128, "one-byte caches: head_dim 128");
 };
 
 // 2-D TMA load with an L2 cache hint (the decode reads every KV byte once: evict first).
@@ -61,6 +76,48 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// The same with f16 operands.
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8x8 matrix of 16-bit elements held one pair per lane (lane l: row l/4, columns
+// 2(l%4), +1), returned in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Four one-byte codes (element 0 in the low byte) -> two f16 pairs (0,1) and (2,3), exact.  KT 1: OCP
+// E4M3 through the hardware e4m3x2 -> f16x2 conversion.  KT 2: signed INT8: each byte, biased to unsigned,
+// becomes the low byte of the f16 1024 + b (byte permute), and 1024 + 128 is subtracted (packed).
+template <int KT>
+__device__ __forceinline__ void bytes4_to_h2(uint32_t w, uint32_t &p01, uint32_t &p23) {
+  if constexpr (KT == 1) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu), __NV_E4M3);
+    const __half2_raw c = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+    p01 = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    p23 = static_cast<uint32_t>(c.x) | (static_cast<uint32_t>(c.y) << 16);
+  } else {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t bias = 0x64806480u;   // (1152, 1152) in f16
+    const uint32_t x01 = __byte_perm(u, 0x64646464u, 0x4140), x23 = __byte_perm(u, 0x64646464u, 0x4342);
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p01) : "r"(x01), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p23) : "r"(x23), "r"(bias));
+  }
+}
+
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -78,12 +135,13 @@ __device__ __forceinline__ uint32_t sw_chunk(int r, int c) {
   return static_cast<uint32_t>((c >> 3) * (kBlock * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
-// HI: the CTA serves more than 8 query heads (rows 8-15 of the products are real).
-template <int D, int NW, int STAGES, bool HI, bool ORDERED>
+// KT: cache element (0 bf16, 1 FP8 E4M3, 2 INT8).  HI: the CTA serves more than 8 query heads (rows 8-15
+// of the products are real).
+template <int KT, int D, int NW, int STAGES, bool HI, bool ORDERED>
 __global__ void __launch_bounds__(NW * 32)
     paged_decode_mma_kernel(const DecodeParams P, const __grid_constant__ CUtensorMap kmap,
                             const __grid_constant__ CUtensorMap vmap, const __grid_constant__ WorkOrder<ORDERED> W) {
-  using C = DecodeMmaCfg<D, NW, STAGES>;
+  using C = DecodeMmaCfg<KT, D, NW, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -116,7 +174,7 @@ __global__ void __launch_bounds__(NW * 32)
   const int blk0 = t0 / kBlock;
 
   uint8_t *wbase = smem + warp * C::WARP_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + 2 * STAGES * C::TILE);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + C::DATA);
   const int nwb = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;  // blocks of this warp
   if (lane == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&bars[s], 1);
@@ -150,20 +208,62 @@ __global__ void __launch_bounds__(NW * 32)
     const int s = i % STAGES;
     if (lane == 0) mbar_arrive_expect_tx(&bars[s], 2 * C::TILE);
     __syncwarp();
-    if (lane < 2 * C::PLANES) {   // one 16 x 64 box per lane: K planes, then V planes
+    if (lane < 2 * C::PLANES) {   // one 16-row x 128-byte box per lane: K planes, then V planes
       const int pl = lane % C::PLANES;
       const bool v = lane >= C::PLANES;
-      tma_load_2d_hint(wbase + ((v ? STAGES : 0) + s) * C::TILE + pl * C::PLANE, v ? &vmap : &kmap, pl * 64,
-                       tile * kBlock, &bars[s], pol);
+      tma_load_2d_hint(wbase + ((v ? STAGES : 0) + s) * C::TILE + pl * C::PLANE, v ? &vmap : &kmap,
+                       pl * (128 / C::E), tile * kBlock, &bars[s], pol);
     }
   };
 
   int issued = 0;
   for (; issued < STAGES && issued < nwb; ++issued) issue(issued);
 
-  // ---- Q fragments (rows h0 + grp and h0 + grp + 8), unscaled bf16; k-step 4t+u of plane t holds dims
-  // 64t + 16*pr + 4u + {0,1} (A[0], A[1]) and + {2,3} (A[2], A[3])
+  // ---- Q fragments (rows h0 + grp and h0 + grp + 8).  bf16 cache: unscaled bf16; k-step 4t+u of plane t
+  // holds dims 64t + 16*pr + 4u + {0,1} (A[0], A[1]) and + {2,3} (A[2], A[3]).  One-byte caches: f16 scaled
+  // per row; k-step s holds dims 32*pr + 4s + {0,1} and + {2,3}; qsc_* multiplies the row's scores.
   uint32_t qlo[C::KS][2], qhi[C::KS][2];
+  float qsc_lo = P.qscale, qsc_hi = P.qscale;
+  if constexpr (KT != 0) {
+    const float ks = P.k_scale[g];
+    auto load_row = [&](int row, uint32_t (&qf)[C::KS][2], float &qsc) {
+      float v[32];
+      if (row < hpc) {
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(P.q + ((int64_t)b * P.num_q_heads + h0 + row) * D + 32 * pr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = src[c];
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            v[8 * c + 2 * t] = bf16lo(ww[t]);
+            v[8 * c + 2 * t + 1] = bf16hi(ww[t]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(v[e]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      // the row's largest |q| has binary exponent ex; q * 2^-ex lies within (-2, 2)
+      int ex = amax > 0.f ? static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127 : 0;
+      ex = ex < -126 ? -126 : (ex > 126 ? 126 : ex);
+      const float down = __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+      qsc = __uint_as_float(static_cast<uint32_t>(127 + ex) << 23) * (P.qscale * ks);
+#pragma unroll
+      for (int s2 = 0; s2 < C::KS; ++s2) {
+        qf[s2][0] = pack_f16x2(v[4 * s2] * down, v[4 * s2 + 1] * down);
+        qf[s2][1] = pack_f16x2(v[4 * s2 + 2] * down, v[4 * s2 + 3] * down);
+      }
+    };
+    load_row(grp, qlo, qsc_lo);
+    if constexpr (HI) load_row(grp + 8, qhi, qsc_hi);
+  } else {
 #pragma unroll
   for (int t = 0; t < C::PLANES; ++t) {
     uint4 w[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
@@ -195,10 +295,10 @@ __global__ void __launch_bounds__(NW * 32)
       }
     }
   }
+  }
 
   // ---- running state per row: reference max (log2 units), this lane's share of the sum, O fragments
   constexpr float kRescale = 8.f;
-  const float qs = P.qscale;
   float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
   float o[C::NT][4];
 #pragma unroll
@@ -221,8 +321,9 @@ __global__ void __launch_bounds__(NW * 32)
     if (nvalid < kBlock) {
       // V rows past the context are zeroed: P is 0 there, but 0 * (whatever the cache holds) may not be
       uint8_t *vt = wbase + (STAGES + s) * C::TILE;
-      for (int idx = lane; idx < (kBlock - nvalid) * (D / 8); idx += 32) {
-        const int r = nvalid + idx / (D / 8), c = idx % (D / 8);
+      constexpr int CPR = C::ROWB / 16;   // 16-byte chunks per row
+      for (int idx = lane; idx < (kBlock - nvalid) * CPR; idx += 32) {
+        const int r = nvalid + idx / CPR, c = idx % CPR;
         *reinterpret_cast<uint4 *>(vt + sw_chunk(r, c)) = make_uint4(0, 0, 0, 0);
       }
       fence_async_smem();   // before the TMA writes this slot again
@@ -236,16 +337,29 @@ __global__ void __launch_bounds__(NW * 32)
     for (int nt = 0; nt < 2; ++nt) {
       sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
       const int R = 8 * nt + grp;
+      if constexpr (KT == 0) {
 #pragma unroll
-      for (int t = 0; t < C::PLANES; ++t) {
-        const uint4 k0 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr));
-        const uint4 k1 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr + 1));
+        for (int t = 0; t < C::PLANES; ++t) {
+          const uint4 k0 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr));
+          const uint4 k1 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr + 1));
+          const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int ks = 4 * t + u;
+            mma_16816(sc[nt], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
+                      kw[2 * u + 1]);
+          }
+        }
+      } else {
+        // the row's bytes [32pr, 32pr + 32): 16 f16 pairs, k-step s takes pairs 2s and 2s + 1
+        const uint4 k0 = lds128(Kt + sw_chunk(R, 2 * pr));
+        const uint4 k1 = lds128(Kt + sw_chunk(R, 2 * pr + 1));
         const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int ks = 4 * t + u;
-          mma_16816(sc[nt], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
-                    kw[2 * u + 1]);
+        for (int s2 = 0; s2 < C::KS; ++s2) {
+          uint32_t b0, b1;
+          bytes4_to_h2<KT>(kw[s2], b0, b1);
+          mma_16816_f16(sc[nt], qlo[s2][0], HI ? qhi[s2][0] : 0u, qlo[s2][1], HI ? qhi[s2][1] : 0u, b0, b1);
         }
       }
     }
@@ -258,7 +372,7 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int tok = 8 * nt + 2 * pr + (e & 1);
-        x[nt][e] = tok < nvalid ? sc[nt][e] * qs : -INFINITY;
+        x[nt][e] = tok < nvalid ? sc[nt][e] * (e < 2 ? qsc_lo : qsc_hi) : -INFINITY;
       }
     float bm_lo = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
     bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 1));
@@ -304,21 +418,46 @@ __global__ void __launch_bounds__(NW * 32)
       }
     }
     // P as the A operand of the PV product (K = the block's 16 tokens): its fragments are S's
-    const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
-    const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
-    const uint32_t pa1 = HI ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
-    const uint32_t pa3 = HI ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
-    __syncwarp();
+    if constexpr (KT == 0) {
+      const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+      const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+      const uint32_t pa1 = HI ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
+      const uint32_t pa3 = HI ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
+      __syncwarp();
 
-    // -- O += P V: ldmatrix.trans gives the B fragments of two 8-dim n-tiles per call; lane l addresses
-    // row (l/8 % 2)*8 + l%8 (token) of 8-dim chunk 2jj + l/16
-    const int vr = ((lane >> 3) & 1) * 8 + (lane & 7);
+      // -- O += P V: ldmatrix.trans gives the B fragments of two 8-dim n-tiles per call; lane l addresses
+      // row (l/8 % 2)*8 + l%8 (token) of 8-dim chunk 2jj + l/16
+      const int vr = ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
-    for (int jj = 0; jj < C::NT / 2; ++jj) {
-      uint32_t v0, v1, v2, v3;
-      ldsm_x4_trans(Vt + sw_chunk(vr, 2 * jj + (lane >> 4)), v0, v1, v2, v3);
-      mma_16816(o[2 * jj], pa0, pa1, pa2, pa3, v0, v1);
-      mma_16816(o[2 * jj + 1], pa0, pa1, pa2, pa3, v2, v3);
+      for (int jj = 0; jj < C::NT / 2; ++jj) {
+        uint32_t v0, v1, v2, v3;
+        ldsm_x4_trans(Vt + sw_chunk(vr, 2 * jj + (lane >> 4)), v0, v1, v2, v3);
+        mma_16816(o[2 * jj], pa0, pa1, pa2, pa3, v0, v1);
+        mma_16816(o[2 * jj + 1], pa0, pa1, pa2, pa3, v2, v3);
+      }
+    } else {
+      // P in f16 (p <= 2^8)
+      const uint32_t pa0 = pack_f16x2(p[0][0], p[0][1]);
+      const uint32_t pa2 = pack_f16x2(p[1][0], p[1][1]);
+      const uint32_t pa1 = HI ? pack_f16x2(p[0][2], p[0][3]) : 0u;
+      const uint32_t pa3 = HI ? pack_f16x2(p[1][2], p[1][3]) : 0u;
+      __syncwarp();
+      // -- O += P V: lane (grp, pr) converts V row (8h + grp)'s bytes [32pr, 32pr + 32) into 16 pairs of
+      // adjacent dims; pair j, transposed across the warp, is the B fragment of n-tile j (dims
+      // {32p' + 2j, +1}) for the 8 tokens of half h
+      uint32_t vh[2][16];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int R = 8 * h + grp;
+        const uint4 v0 = lds128(Vt + sw_chunk(R, 2 * pr));
+        const uint4 v1 = lds128(Vt + sw_chunk(R, 2 * pr + 1));
+        const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int t = 0; t < 8; ++t) bytes4_to_h2<KT>(vw[t], vh[h][2 * t], vh[h][2 * t + 1]);
+      }
+#pragma unroll
+      for (int j = 0; j < C::NT; ++j)
+        mma_16816_f16(o[j], pa0, pa1, pa2, pa3, movmatrix_trans(vh[0][j]), movmatrix_trans(vh[1][j]));
     }
     __syncwarp();
     if (issued < nwb) issue(issued++);
@@ -344,8 +483,10 @@ __global__ void __launch_bounds__(NW * 32)
   float *mrg = reinterpret_cast<float *>(wbase);
 #pragma unroll
   for (int j = 0; j < C::NT; ++j) {
-    *reinterpret_cast<float2 *>(mrg + grp * D + 8 * j + 2 * pr) = make_float2(o[j][0], o[j][1]);
-    if constexpr (HI) *reinterpret_cast<float2 *>(mrg + (grp + 8) * D + 8 * j + 2 * pr) = make_float2(o[j][2], o[j][3]);
+    // n-tile j of this lane holds dims 8j + 2pr, +1 (bf16 cache) or 32pr + 2j, +1 (one-byte caches)
+    const int col = KT == 0 ? 8 * j + 2 * pr : 32 * pr + 2 * j;
+    *reinterpret_cast<float2 *>(mrg + grp * D + col) = make_float2(o[j][0], o[j][1]);
+    if constexpr (HI) *reinterpret_cast<float2 *>(mrg + (grp + 8) * D + col) = make_float2(o[j][2], o[j][3]);
   }
   if (pr == 0) {
     mrg[C::ML + 2 * grp] = m_lo;
@@ -357,6 +498,7 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncthreads();
 
+  const float vs = KT != 0 ? P.v_scale[g] : 1.f;
   for (int idx = threadIdx.x; idx < hpc * D; idx += NW * 32) {
     const int qi = idx / D, d = idx % D;
     float M = -INFINITY;
@@ -374,11 +516,11 @@ __global__ void __launch_bounds__(NW * 32)
     }
     const int h = h0 + qi;
     if (final_out) {
-      const float val = Lsum > 0.f ? O / Lsum : 0.f;
+      const float val = Lsum > 0.f ? O / Lsum * vs : 0.f;
       P.out[((int64_t)b * P.num_q_heads + h) * D + d] = __float2bfloat16_rn(val);
     } else {
       const int64_t row = ((int64_t)b * P.num_q_heads + h) * P.max_splits + split;
-      P.ws_o[row * D + d] = O;
+      P.ws_o[row * D + d] = O * vs;
       if (d == 0) {
         P.ws_ml[row * 2] = M;
         P.ws_ml[row * 2 + 1] = Lsum;

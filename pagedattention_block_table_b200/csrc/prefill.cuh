@@ -773,6 +773,19 @@ inline bool make_cache_map(CUtensorMap *map, const void *base, int64_t rows, int
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same over a one-byte cache (FP8 E4M3 or INT8 codes): box = 16 rows x 128 bytes, 128-byte swizzle.
+inline bool make_cache_map_u8(CUtensorMap *map, const void *base, int64_t rows, int D) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (!fn || D != 128) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D)};
+  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(kBlock)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D>
 int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_cache, int num_chunks, int max_q_len,
                      cudaStream_t st) {

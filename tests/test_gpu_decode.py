@@ -79,6 +79,53 @@ def test_decode_fp8_with_gqa(O, cuda_lib):
     assert_close(to_f64(_gpu_decode(batch).out_dec), oracle_step(batch, O)["decode"], what="fp8 gqa4")
 
 
+# one-byte caches with groups of 4 or more query heads take the tensor-core kernel at head_dim 128 (f16
+# products on codes converted in registers): groups of 4, 8 (two CTAs' worth of rows), 16, a group split
+# over two CTAs, 32-token blocks, lengths at block edges, several splits
+ONE_BYTE_MMA = {
+    "g4": dict(num_seqs=5, num_q_heads=32, num_kv_heads=8, hist=("fixed", [0, 15, 16, 700, 1500])),
+    "g8": dict(num_seqs=3, num_q_heads=64, num_kv_heads=8, hist=("uniform", 30, 900)),
+    "g16": dict(num_seqs=3, num_q_heads=32, num_kv_heads=2, hist=("uniform", 1, 900)),
+    "g32": dict(num_seqs=2, num_q_heads=32, num_kv_heads=1, hist=("fixed", [5, 333])),
+    "g4_bs32": dict(num_seqs=4, num_q_heads=32, num_kv_heads=8, hist=("fixed", [31, 32, 33, 777]), block_size=32),
+}
+
+
+@pytest.mark.parametrize("kv", ["fp8", "int8"])
+@pytest.mark.parametrize("case", sorted(ONE_BYTE_MMA))
+@pytest.mark.parametrize("split", [None, 128])
+def test_one_byte_gqa_decode_on_tensor_cores(O, cuda_lib, kv, case, split):
+    from pagedattention_block_table_b200 import binding as B
+    ov = dict(ONE_BYTE_MMA[case], kv_dtype=kv)
+    batch = make_batch("mha_fp8_decode", seed=71, overrides=ov)
+    assert B.pa_paged_attention_uses_tensor_cores(batch.num_q_heads, batch.num_kv_heads, 128, batch.kv_dtype) == 1
+    got = to_f64(_gpu_decode(batch, split).out_dec)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(got, oracle_step(batch, O)["decode"], what=f"{kv} {case} vs dequantised")
+    # against the original bf16 K/V: the quantisation error of a one-byte code (up to 2^-4 relative for
+    # E4M3) averages out only over many tokens, so sequences of at least 64 tokens
+    b16 = make_batch("mha_fp8_decode", seed=71, overrides=dict(ov, kv_dtype=None))
+    long_ = batch.context_lens[:batch.num_decode] >= 64
+    assert long_.any()
+    assert_close(got[long_], oracle_step(b16, O)["decode"][long_], max_tol=FP8_MAX, mean_tol=None,
+                 what=f"{kv} {case} vs bf16")
+
+
+@pytest.mark.parametrize("e", [-20, 20, 0])
+def test_one_byte_gqa_decode_any_query_magnitude(O, cuda_lib, e):
+    """The tensor-core path rounds q to f16 after scaling each row by a power of two into [1, 2): q * 2^e
+    with the softmax scale * 2^-e gives the same scores far outside f16's range (2^20 overflows it, 2^-20
+    is below its normal range), and the output still matches the oracle."""
+    import math
+    batch = make_batch("mha_fp8_decode", seed=72, overrides=dict(num_seqs=3, num_q_heads=32, num_kv_heads=8,
+                                                               hist=("uniform", 100, 900)))
+    batch.q_decode = (batch.q_decode.float() * 2.0 ** e).to(torch.bfloat16)    # exact: a power of two
+    batch.scale = 1.0 / math.sqrt(batch.head_dim) * 2.0 ** -e
+    got = to_f64(_gpu_decode(batch, 256).out_dec)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(got, oracle_step(batch, O)["decode"], what=f"fp8 gqa, q * 2^{e}")
+
+
 GROUPS = {"g4": dict(num_q_heads=32, num_kv_heads=8), "g8": dict(num_q_heads=64, num_kv_heads=8),
           "g16": dict(num_q_heads=32, num_kv_heads=2)}
 

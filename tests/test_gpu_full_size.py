@@ -4,9 +4,9 @@ Each runs on the GPU exactly as bench.py times it (same inputs, same split choic
 order): the Llama-3-8B-shaped decode batch (64 sequences, 32/8 heads, contexts 513..4097), the
 continuous-batching mixed step (256 prefix-sharing decode sequences with copy-on-write forks plus four
 causal prefill chunks of 512..2048 tokens), the long-context batch (8 x 32768 tokens, split 512), the
-MHA batch over an FP8 E4M3 cache (32 sequences, 64/64 heads, contexts 2049..8193), and a GQA batch with
-eight query heads per KV head (32 sequences, 64/8 heads, contexts 513..4097), whose KV tiles two CTAs
-each read.  The oracle computes every sequence from its own token rows in a fresh contiguous cache (no
+MHA batch over an FP8 E4M3 cache (32 sequences, 64/64 heads, contexts 2049..8193), a GQA batch with
+eight query heads per KV head (32 sequences, 64/8 heads, contexts 513..4097) and the Llama-3-8B batch over
+an FP8 cache.  The oracle computes every sequence from its own token rows in a fresh contiguous cache (no
 paging, sharing or forks), so the comparison also checks that paging, prefix sharing and copy-on-write
 change nothing.
 Tolerances: attention max-abs <= 1e-2 and mean-abs <= 1e-3 against the oracle on the same bf16 inputs
@@ -31,7 +31,8 @@ def _run(batch):
     return st
 
 
-@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context_decode", "mha_fp8_decode", "gqa8_decode"])
+@pytest.mark.parametrize("name", ["llama3_8b_decode", "long_context_decode", "mha_fp8_decode", "gqa8_decode",
+                                  "llama3_8b_fp8_decode"])
 def test_full_size_decode_every_element(O, cuda_lib, name):
     batch = make_batch(name, device="cuda")
     st = _run(batch)
