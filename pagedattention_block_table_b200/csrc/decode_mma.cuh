@@ -105,10 +105,7 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 template <int KT>
 __device__ __forceinline__ void bytes4_to_h2(uint32_t w, uint32_t &p01, uint32_t &p23) {
   if constexpr (KT == 1) {
-    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu), __NV_E4M3);
-    const __half2_raw c = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
-    p01 = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
-    p23 = static_cast<uint32_t>(c.x) | (static_cast<uint32_t>(c.y) << 16);
+    e4m3x4_to_h2x2(w, p01, p23);
   } else {
     const uint32_t u = w ^ 0x80808080u;
     const uint32_t bias = 0x64806480u;   // (1152, 1152) in f16

@@ -148,23 +148,35 @@ __device__ __forceinline__ uint64_t f2add(uint64_t a, uint64_t b) {
 // bf16x2 word -> packed fp32 pair (element 0 low).
 __device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2pack(bf16lo(w), bf16hi(w)); }
 
-// Two E4M3 codes (low 16 bits of w, element 0 in the low byte) -> two floats (exact).
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t w) {
-  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w), __NV_E4M3);
-  return __half22float2(*reinterpret_cast<__half2 *>(&h));
+// Four E4M3 codes (element 0 in the low byte of w) -> f16 pairs (0,1) and (2,3), exact: the hardware
+// e4m3x2 -> f16x2 conversion on each 16-bit half of w (one instruction per pair, no repacking).
+__device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t w, uint32_t &p01, uint32_t &p23) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+      : "=r"(p01), "=r"(p23)
+      : "r"(w));
+}
+// f16 pair (element 0 low) -> packed fp32 pair, exact.
+__device__ __forceinline__ uint64_t h2_to_f2(uint32_t h) {
+  uint64_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t.reg .f32 a, b;\n\tmov.b32 {lo, hi}, %1;\n\t"
+      "cvt.f32.f16 a, lo;\n\tcvt.f32.f16 b, hi;\n\tmov.b64 %0, {a, b};\n\t}"
+      : "=l"(r)
+      : "r"(h));
+  return r;
 }
 
 // Four one-byte KV codes (element 0 in the low byte) -> two packed fp32 pairs (0,1) and (2,3), exact.
-// KT 1: OCP E4M3 through the hardware e4m3x2 -> f16x2 conversion.  KT 2: signed INT8: each byte,
+// KT 1: OCP E4M3 through the hardware e4m3x2 -> f16x2 conversion, then f16 -> f32.  KT 2: signed INT8: each byte,
 // biased to unsigned, is placed in the mantissa of 2^23 (byte permute), and 2^23 + 128 is then
 // subtracted (packed), which is exact for every value.
 template <int KT>
 __device__ __forceinline__ void bytes4_to_f2(uint32_t w, uint64_t &p01, uint64_t &p23) {
   if constexpr (KT == 1) {
-    const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w & 0xffffu));
-    const float2 b = e4m3x2_to_float2(static_cast<uint16_t>(w >> 16));
-    p01 = f2pack(a.x, a.y);
-    p23 = f2pack(b.x, b.y);
+    uint32_t h01, h23;
+    e4m3x4_to_h2x2(w, h01, h23);
+    p01 = h2_to_f2(h01);
+    p23 = h2_to_f2(h23);
   } else {
     const uint32_t u = w ^ 0x80808080u;
     const float f0 = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650));
