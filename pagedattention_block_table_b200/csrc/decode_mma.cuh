@@ -25,10 +25,10 @@
 // is rounded to f16 (exact for every bf16 entry within 2^-14 of the row's largest), and that power, the
 // softmax scale and the K scale multiply the scores; the V scale multiplies the output.  A lane converts
 // the 32 bytes [32p, 32p+32) of a K row into 16 f16 pairs (k-step s takes pairs 2s and 2s+1, and Q uses
-// the same dims).  V needs pairs along tokens, so a lane converts its V row's 32 bytes into 16 pairs of
-// adjacent dims and `movmatrix.trans` turns each 8x8 block (8 tokens x the 8 dims {32p' + 2j, +1}) into
-// the B fragment of n-tile j; n-tile j of the output then holds dims 32p + 2j, +1, so a lane's 16 n-tiles
-// cover its 32 contiguous dims.
+// the same dims).  V needs pairs along tokens: a lane reads 16 dims [16g, 16g + 16) of two token rows
+// and a byte permute pairs the two rows' codes of each dim before the conversion, which gives the B
+// fragment of n-tile e (column g = dim 16g + e); n-tile e of the output then holds dims 32p + e and
+// 32p + 16 + e.
 #pragma once
 #include "decode.cuh"
 #include "prefill.cuh"   // tensor-map encoding, 2-D TMA load
@@ -84,14 +84,6 @@ __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Transpose of an 8x8 matrix of 16-bit elements held one pair per lane (lane l: row l/4, columns
-// 2(l%4), +1), returned in the same layout.
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
-  uint32_t d;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
-  return d;
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -442,19 +434,23 @@ __global__ void __launch_bounds__(NW * 32)
       // -- O += P V: lane (grp, pr) converts V row (8h + grp)'s bytes [32pr, 32pr + 32) into 16 pairs of
       // adjacent dims; pair j, transposed across the warp, is the B fragment of n-tile j (dims
       // {32p' + 2j, +1}) for the 8 tokens of half h
-      uint32_t vh[2][16];
+      // lane (grp, pr) reads dims [16grp, 16grp + 16) of token rows 2pr, 2pr + 1 (half h = 0) and 8 + 2pr,
+      // 9 + 2pr (h = 1); a byte permute pairs the two rows' codes of one dim, which is the B fragment of
+      // n-tile e (column grp = dim 16grp + e) for tokens (2pr, 2pr + 1) + 8h
+      uint32_t vb[2][16];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int R = 8 * h + grp;
-        const uint4 v0 = lds128(Vt + sw_chunk(R, 2 * pr));
-        const uint4 v1 = lds128(Vt + sw_chunk(R, 2 * pr + 1));
-        const uint32_t vw[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        const uint4 r0 = lds128(Vt + sw_chunk(8 * h + 2 * pr, grp));
+        const uint4 r1 = lds128(Vt + sw_chunk(8 * h + 2 * pr + 1, grp));
+        const uint32_t a[4] = {r0.x, r0.y, r0.z, r0.w}, c[4] = {r1.x, r1.y, r1.z, r1.w};
 #pragma unroll
-        for (int t = 0; t < 8; ++t) bytes4_to_h2<KT>(vw[t], vh[h][2 * t], vh[h][2 * t + 1]);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          bytes4_to_h2<KT>(__byte_perm(a[q4], c[q4], 0x5140), vb[h][4 * q4], vb[h][4 * q4 + 1]);
+          bytes4_to_h2<KT>(__byte_perm(a[q4], c[q4], 0x7362), vb[h][4 * q4 + 2], vb[h][4 * q4 + 3]);
+        }
       }
 #pragma unroll
-      for (int j = 0; j < C::NT; ++j)
-        mma_16816_f16(o[j], pa0, pa1, pa2, pa3, movmatrix_trans(vh[0][j]), movmatrix_trans(vh[1][j]));
+      for (int e = 0; e < C::NT; ++e) mma_16816_f16(o[e], pa0, pa1, pa2, pa3, vb[0][e], vb[1][e]);
     }
     __syncwarp();
     if (issued < nwb) issue(issued++);
@@ -480,10 +476,20 @@ __global__ void __launch_bounds__(NW * 32)
   float *mrg = reinterpret_cast<float *>(wbase);
 #pragma unroll
   for (int j = 0; j < C::NT; ++j) {
-    // n-tile j of this lane holds dims 8j + 2pr, +1 (bf16 cache) or 32pr + 2j, +1 (one-byte caches)
-    const int col = KT == 0 ? 8 * j + 2 * pr : 32 * pr + 2 * j;
-    *reinterpret_cast<float2 *>(mrg + grp * D + col) = make_float2(o[j][0], o[j][1]);
-    if constexpr (HI) *reinterpret_cast<float2 *>(mrg + (grp + 8) * D + col) = make_float2(o[j][2], o[j][3]);
+    if constexpr (KT == 0) {
+      // n-tile j of this lane holds dims 8j + 2pr, +1
+      *reinterpret_cast<float2 *>(mrg + grp * D + 8 * j + 2 * pr) = make_float2(o[j][0], o[j][1]);
+      if constexpr (HI)
+        *reinterpret_cast<float2 *>(mrg + (grp + 8) * D + 8 * j + 2 * pr) = make_float2(o[j][2], o[j][3]);
+    } else {
+      // one-byte caches: n-tile j of this lane holds dims 32pr + j and 32pr + 16 + j
+      mrg[grp * D + 32 * pr + j] = o[j][0];
+      mrg[grp * D + 32 * pr + 16 + j] = o[j][1];
+      if constexpr (HI) {
+        mrg[(grp + 8) * D + 32 * pr + j] = o[j][2];
+        mrg[(grp + 8) * D + 32 * pr + 16 + j] = o[j][3];
+      }
+    }
   }
   if (pr == 0) {
     mrg[C::ML + 2 * grp] = m_lo;
