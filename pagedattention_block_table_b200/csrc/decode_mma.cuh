@@ -1,10 +1,10 @@
-// decode_mma.cuh -- paged decode attention for GQA groups on the tensor cores (bf16 cache, sm_100a).
+// decode_mma.cuh -- paged decode attention for GQA groups on the tensor cores (sm_100a).
 //
 // Same operation and split-K scheme as paged_decode_kernel (decode.cuh): for sequence b and query head
 // h, out = softmax(scale * q . K^T) V over the context, token t read through the block table.  With a
 // group of G query heads per KV head, every K/V element meets G queries, so the CUDA-core kernel's
 // work per byte of KV grows with G; at G = 8 it is compute-bound at about half the HBM bandwidth.  Here
-// the products go to the tensor cores instead (warp-level mma.sync m16n8k16, bf16 in, fp32 out): the
+// the products go to the tensor cores instead (warp-level mma.sync m16n8k16, fp32 accumulate): the
 // CTA's query heads are the 16 rows of the A operand (padded with zeros when G < 16), and a 16-token
 // block is one N=16 QK^T product and one K=16 PV product per warp.
 //
@@ -14,11 +14,11 @@
 //   online softmax in base 2 on S's fragments (a row's 16 scores are spread over the 4 lanes of a quad)
 //   O[16][D] += P V                    P (bf16) is built from S's fragments in registers; V's fragments
 //                                      come from shared memory with ldmatrix.trans (V is token-major)
-// K and V tiles reach shared memory by 2-D TMA (the cache seen as rows of D elements, one 16-row x
-// 128-byte box per 128-byte plane, 128-byte swizzle, into this CTA's own shared memory), so ldmatrix and
-// the 16-byte K loads are free of bank conflicts.  The dims of a k-step are permuted (the same way for Q
-// and K, which leaves the dot product unchanged) so that each lane's K fragments come from two 16-byte
-// loads.
+// bf16 caches: bf16 products.  K and V tiles reach shared memory by 2-D TMA (the cache seen as rows of D
+// elements, one 16-row x 128-byte box per 128-byte plane, 128-byte swizzle, into this CTA's own shared
+// memory), so ldmatrix and the 16-byte K loads are free of bank conflicts.  The dims of a k-step are
+// permuted (the same way for Q and K, which leaves the dot product unchanged) so that each lane's K
+// fragments come from two 16-byte loads.
 //
 // One-byte caches (FP8 E4M3, INT8; head_dim 128): the products run in f16 (m16n8k16, f32 accumulate).
 // Every E4M3 and INT8 code is exact in f16.  Q is scaled per row by a power of two into [1, 2) before it
