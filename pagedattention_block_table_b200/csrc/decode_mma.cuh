@@ -321,10 +321,12 @@ __global__ void __launch_bounds__(NW * 32)
 
     // -- S = Q K^T: n-tile nt holds tokens 8nt..8nt+7; lane (grp, pr) reads token 8nt+grp's dims
     // 64t + 16pr .. +16 (two 16-byte chunks of plane t)
+    // (two accumulators per n-tile, even and odd k-steps, so that the dependent chain of products on one
+    // accumulator is half as long)
     float sc[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       const int R = 8 * nt + grp;
       if constexpr (KT == 0) {
 #pragma unroll
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int ks = 4 * t + u;
-            mma_16816(sc[nt], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
+            mma_16816(acc[ks & 1], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
                       kw[2 * u + 1]);
           }
         }
@@ -348,9 +350,11 @@ __global__ void __launch_bounds__(NW * 32)
         for (int s2 = 0; s2 < C::KS; ++s2) {
           uint32_t b0, b1;
           bytes4_to_h2<KT>(kw[s2], b0, b1);
-          mma_16816_f16(sc[nt], qlo[s2][0], HI ? qhi[s2][0] : 0u, qlo[s2][1], HI ? qhi[s2][1] : 0u, b0, b1);
+          mma_16816_f16(acc[s2 & 1], qlo[s2][0], HI ? qhi[s2][0] : 0u, qlo[s2][1], HI ? qhi[s2][1] : 0u, b0, b1);
         }
       }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[nt][e] = acc[0][e] + acc[1][e];
     }
 
     // -- online softmax: lane (grp, pr) holds row grp's tokens 8nt + 2pr + {0,1} (sc[nt][0..1]) and row
