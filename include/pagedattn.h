@@ -206,16 +206,20 @@ pa_status pa_paged_attention_noalloc(void *out, const void *q, const void *k_cac
  *   cu_q_lens    : int32 [num_chunks + 1] on the device, non-decreasing, cu_q_lens[0] = 0
  *   block_tables : int32 [num_chunks][max_blocks_per_seq];  context_lens : int32 [num_chunks]
  *   max_q_len    : host-side upper bound of C_c;  max_context_len : upper bound of context_lens.
+ *   kv_dtype     : PA_KV_BF16 (head_dim 64 or 128), or PA_KV_FP8_E4M3 / PA_KV_INT8 (head_dim 128), with
+ *                  k_scale / v_scale fp32 [num_kv_heads] on the device as for pa_paged_attention (NULL for
+ *                  bf16): K[t] = code * k_scale[h/G], V[t] = code * v_scale[h/G]  [KV Cache to vLLM §2.2].
  * A chunk whose C_c exceeds max_q_len, or whose context exceeds max_context_len or its table row,
  * sets the device error word (PA_EDEVICE_OOB from pa_get_device_error) and its rows are not written.
- * bf16 caches only (kv_dtype must be PA_KV_BF16).  Runs on the tcgen05 tensor cores.
+ * bf16 caches run on the tcgen05 tensor cores; one-byte caches on warp-level tensor-core products in
+ * f16 over codes converted in registers.  A one-byte cache at head_dim 64 returns PA_EUNSUPPORTED.
  */
 pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks,
                            const void *k_cache, const void *v_cache, const int32_t *block_tables,
                            int max_blocks_per_seq, const int32_t *context_lens, int num_q_heads,
                            int num_kv_heads, int head_dim, int64_t num_blocks, int block_size,
-                           float scale, int kv_dtype, int max_q_len, int max_context_len,
-                           pa_stream_t stream);
+                           float scale, int kv_dtype, const float *k_scale, const float *v_scale,
+                           int max_q_len, int max_context_len, pa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------------------
  * Host block manager: the control plane that produces block tables, slot mappings and copy-on-write

@@ -77,7 +77,7 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_attention_noalloc.restype = I
         L.pa_paged_attention_noalloc.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P]
         L.pa_paged_prefill.restype = I
-        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, I, F, I, I, I, P]
+        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, I, F, I, P, P, I, I, P]
         L.pa_get_device_error.restype = I
         L.pa_get_device_error.argtypes = [P]
         L.pa_selftest_bounded_wait.restype = I
@@ -297,7 +297,7 @@ def pa_paged_attention_noalloc(out, q, k_cache, v_cache, block_tables, context_l
 
 
 def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, max_q_len,
-                     max_context_len, kv_dtype=PA_KV_BF16, stream=None):
+                     max_context_len, kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, stream=None):
     nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     tq, hq, dq = q.shape
@@ -311,7 +311,8 @@ def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_
         _ptr(cu_q_lens, "cu_q_lens", (torch.int32,)), n, _ptr(k_cache, "k_cache", cd),
         _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
         int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), hq, hkv, d, nb, bs,
-        float(scale), int(kv_dtype), int(max_q_len), int(max_context_len), _stream(stream))
+        float(scale), int(kv_dtype), _ptr(k_scale, "k_scale", (torch.float32,)),
+        _ptr(v_scale, "v_scale", (torch.float32,)), int(max_q_len), int(max_context_len), _stream(stream))
     _check(st, "pa_paged_prefill")
 
 

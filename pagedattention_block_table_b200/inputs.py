@@ -49,6 +49,11 @@ WORKLOADS: Dict[str, dict] = {
     # the Llama-3-8B decode batch over an FP8 E4M3 cache: four query heads meet every dequantised byte
     "llama3_8b_fp8_decode": dict(num_seqs=64, num_q_heads=32, num_kv_heads=8, head_dim=128,
                                  hist=("uniform", 512, 4096), kv_dtype="fp8"),
+    # the continuous-batching mixed step over an FP8 E4M3 cache (prefill and decode both read one-byte K/V)
+    "mixed_step_fp8": dict(num_seqs=256, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                           hist=("lognormal", 800.0, 1.0, 16, 8192),
+                           share_group=8, share_prefix=1024,
+                           prefill_chunks=4, chunk_len=(512, 2048), chunk_hist=(1, 4095), kv_dtype="fp8"),
 }
 WORKLOAD_SEED = {name: 1001 + i for i, name in enumerate(WORKLOADS)}
 

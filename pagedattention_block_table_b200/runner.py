@@ -103,7 +103,8 @@ class DeviceStep:
         if self.max_q == 0:
             return
         B.pa_paged_prefill(self.out_pre, self.q_pre, self.cu_q, self.k_cache, self.v_cache, self.pre_tables,
-                           self.pre_lens, self.batch.scale, self.max_q, self.pre_max_len, self.kv_dtype, stream)
+                           self.pre_lens, self.batch.scale, self.max_q, self.pre_max_len, self.kv_dtype,
+                           k_scale=self.k_scale, v_scale=self.v_scale, stream=stream)
 
     def step(self, stream=None):
         """copy-on-write forks -> append -> decode attention and prefill attention.

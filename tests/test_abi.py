@@ -115,11 +115,19 @@ def test_empty_batch_is_a_no_op(L):
     assert L.pa_kv_append(P(16), P(16), P(16), P(16), P(16), 4, 8, 128, 10, 24, 0, None, None, None) == B.PA_EUNSUPPORTED
 
 
-def test_prefill_rejects_fp8_and_bad_heads(L):
+def test_prefill_argument_checks(L):
     P = ctypes.c_void_p
     f = L.pa_paged_prefill
-    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 1, 16, 64, None) == B.PA_EUNSUPPORTED
-    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 16, 0.1, 0, 16, 64, None) == B.PA_EINVAL
+    # one-byte caches: head_dim 128 only, and both scales required
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 64, 10, 16, 0.1, 1, P(16), P(16), 16, 64,
+             None) == B.PA_EUNSUPPORTED
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 1, None, P(16), 16, 64,
+             None) == B.PA_EINVAL
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 5, P(16), P(16), 16, 64,
+             None) == B.PA_EUNSUPPORTED
+    # heads not a multiple of the KV heads
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 16, 0.1, 0, None, None, 16, 64,
+             None) == B.PA_EINVAL
 
 
 def test_source_digest_ignores_comments_only():

@@ -1,4 +1,5 @@
-"""GPU parity of the tcgen05 paged prefill (and of the whole mixed step) against the oracle."""
+"""GPU parity of the paged prefill (tcgen05 for bf16 caches, warp-level tensor cores for one-byte caches) and
+of the whole mixed step against the oracle."""
 import numpy as np
 import pytest
 import torch
@@ -100,3 +101,32 @@ def test_prefill_chunk_longer_than_max_q_is_flagged(cuda_lib):
                               batch.scale, 100, st.pre_max_len)
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_EDEVICE_OOB
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK          # reading the word clears it
+
+
+ONE_BYTE = {k: CASES[k] for k in ("gqa4_d128", "gqa4_d128_long", "mha_d128", "tiny_chunks", "gqa8_d128", "gqa3_d128",
+                                  "gqa4_d128_bs32")}
+ONE_BYTE["gqa16_d128"] = _chunks(num_q_heads=16, num_kv_heads=1, chunk_len=(5, 90))
+
+
+@pytest.mark.parametrize("kv", ["fp8", "int8"])
+@pytest.mark.parametrize("case", sorted(ONE_BYTE))
+def test_one_byte_prefill_matches_oracle(O, cuda_lib, case, kv):
+    """Prefill over FP8 / INT8 caches (f16 products on codes converted in registers) against the oracle on
+    the same codes and scales; the step's decode rows ride along."""
+    batch = make_batch("mixed_step", seed=54, overrides=dict(ONE_BYTE[case], kv_dtype=kv))
+    ref = oracle_step(batch, O)
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(st.out_pre), ref["prefill"], what=f"{kv} prefill {case}")
+    assert_close(to_f64(st.out_dec), ref["decode"], what=f"{kv} decode {case}")
+
+
+def test_one_byte_prefill_long_chunk_over_long_history(O, cuda_lib):
+    """1000-row FP8 chunks with GQA 4, one starting a request and one over a 2000-token history: many row
+    tiles, every key unit, the causal edge inside the last units."""
+    ov = _chunks(prefill_chunks=2, chunk_len=(1000, 1000), chunk_hist=(2000, 2000), kv_dtype="fp8")
+    batch = make_batch("mixed_step", seed=55, overrides=ov)
+    ref = oracle_step(batch, O)["prefill"]
+    st = _run(batch)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(st.out_pre), ref, what="fp8 long chunk")
