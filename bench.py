@@ -314,6 +314,13 @@ def decode_kernel_label(batch) -> str:
     return f"pa_paged_attention ({k} + lse_reduce_kernel)"
 
 
+def prefill_kernel_label(batch) -> str:
+    """The prefill kernel pa_paged_prefill runs for this batch's cache."""
+    if batch.kv_dtype:
+        return "paged_prefill_mma_kernel (mma.sync, f16 products on one-byte codes)"
+    return "paged_prefill_kernel (tcgen05)"
+
+
 def workload_batch(name, device, num_seqs=0):
     """The named workload's synthetic batch; num_seqs > 0 keeps its shapes and length distribution but
     draws that many sequences (a smaller case of the same workload, for profiling)."""
@@ -404,7 +411,7 @@ def sub_record(name, dev, args, clk):
         pf = prefill_flops(batch)
         tp, tk = bf16_peak()
         ach = pf / (m["pre_ms"] * 1e-3) / 1e12
-        rec["prefill"] = {"kernel": "paged_prefill_kernel (tcgen05)", "bound": "tensor", "unit": "TFLOP/s",
+        rec["prefill"] = {"kernel": prefill_kernel_label(batch), "bound": "tensor", "unit": "TFLOP/s",
                           "achieved": round(ach, 2), "peak": tp, "peak_kind": tk, "frac": round(ach / tp, 4),
                           "flops": pf, "avg_launch_ms": round(m["pre_ms"], 5)}
     del m, st, batch
@@ -485,7 +492,7 @@ def run_ours(args, rank, world, local_rank):
         pf = prefill_flops(batch)
         tp, tk = bf16_peak()
         pre_ms = agg["pre_ms"]
-        line["prefill"] = {"kernel": "paged_prefill_kernel (tcgen05)", "bound": "tensor", "unit": "TFLOP/s",
+        line["prefill"] = {"kernel": prefill_kernel_label(batch), "bound": "tensor", "unit": "TFLOP/s",
                            "achieved": round(pf / (pre_ms * 1e-3) / 1e12, 2), "peak": tp, "peak_kind": tk,
                            "frac": round(pf / (pre_ms * 1e-3) / 1e12 / tp, 4), "flops": pf,
                            "avg_launch_ms": round(pre_ms, 5)}

@@ -100,9 +100,14 @@ def oracle_decode_all(batch: PagedBatch, O, kv_dtype=None) -> np.ndarray:
 
 def oracle_prefill_all(batch: PagedBatch, O) -> np.ndarray:
     """Oracle causal attention of every prefill row, [sum C][Hq][D] fp64: chunk c's rows over its own
-    token rows (history + chunk) in a fresh contiguous bf16 cache."""
+    token rows (history + chunk) in a fresh contiguous cache of the batch's element type."""
     cu = batch.cu_q_lens
     ctx = batch.context_lens
+    kv_dtype = batch.kv_dtype
+    dt = {0: np.uint16, 1: np.uint8, 2: np.int8}[kv_dtype]
+    ks = vs = None
+    if kv_dtype:
+        ks, vs = batch.k_scale.cpu().numpy(), batch.v_scale.cpu().numpy()
     outs = []
     for c in range(batch.num_seqs - batch.num_decode):
         s = batch.num_decode + c
@@ -111,11 +116,11 @@ def oracle_prefill_all(batch: PagedBatch, O) -> np.ndarray:
         tk = bf16_bits(batch.tok_k.index_select(0, rows))
         tv = bf16_bits(batch.tok_v.index_select(0, rows))
         nblk = max(1, (L + 15) // 16)
-        kc = np.zeros((nblk, batch.num_kv_heads, 16, batch.head_dim), np.uint16)
+        kc = np.zeros((nblk, batch.num_kv_heads, 16, batch.head_dim), dt)
         vc = np.zeros_like(kc)
-        O.kv_append(kc, vc, tk, tv, np.arange(L, dtype=np.int64))
+        O.kv_append(kc, vc, tk, tv, np.arange(L, dtype=np.int64), kv_dtype, ks, vs)
         C = int(cu[c + 1] - cu[c])
         q = bf16_bits(batch.q_prefill[int(cu[c]):int(cu[c + 1])])
         outs.append(O.paged_prefill(q, np.array([0, C], np.int32), kc, vc, np.arange(nblk, dtype=np.int32)[None],
-                                    np.array([L], np.int32), batch.scale))
+                                    np.array([L], np.int32), batch.scale, kv_dtype, ks, vs))
     return np.concatenate(outs) if outs else np.zeros((0, batch.num_q_heads, batch.head_dim))

@@ -6,7 +6,7 @@ continuous-batching mixed step (256 prefix-sharing decode sequences with copy-on
 causal prefill chunks of 512..2048 tokens), the long-context batch (8 x 32768 tokens, split 512), the
 MHA batch over an FP8 E4M3 cache (32 sequences, 64/64 heads, contexts 2049..8193), a GQA batch with
 eight query heads per KV head (32 sequences, 64/8 heads, contexts 513..4097) and the Llama-3-8B batch over
-an FP8 cache.  The oracle computes every sequence from its own token rows in a fresh contiguous cache (no
+an FP8 cache, and the mixed step over an FP8 cache.  The oracle computes every sequence from its own token rows in a fresh contiguous cache (no
 paging, sharing or forks), so the comparison also checks that paging, prefix sharing and copy-on-write
 change nothing.
 Tolerances: attention max-abs <= 1e-2 and mean-abs <= 1e-3 against the oracle on the same bf16 inputs
@@ -46,10 +46,11 @@ def test_full_size_decode_every_element(O, cuda_lib, name):
                      what=f"{name} vs the bf16 K/V")
 
 
-def test_full_size_mixed_step_every_element(O, cuda_lib):
-    batch = make_batch("mixed_step", device="cuda")
+@pytest.mark.parametrize("name", ["mixed_step", "mixed_step_fp8"])
+def test_full_size_mixed_step_every_element(O, cuda_lib, name):
+    batch = make_batch(name, device="cuda")
     assert batch.cow_pairs.shape[0] > 0 and batch.shared_blocks.shape[0] > 0
     st = _run(batch)
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
-    assert_close(to_f64(st.out_dec), oracle_decode_all(batch, O), what="mixed step: 256 decode rows")
-    assert_close(to_f64(st.out_pre), oracle_prefill_all(batch, O), what="mixed step: every prefill row")
+    assert_close(to_f64(st.out_dec), oracle_decode_all(batch, O), what=f"{name}: 256 decode rows")
+    assert_close(to_f64(st.out_pre), oracle_prefill_all(batch, O), what=f"{name}: every prefill row")
