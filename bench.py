@@ -317,7 +317,7 @@ def decode_kernel_label(batch) -> str:
 def prefill_kernel_label(batch) -> str:
     """The prefill kernel pa_paged_prefill runs for this batch's cache."""
     if batch.kv_dtype:
-        return "paged_prefill_mma_kernel (mma.sync, f16 products on one-byte codes)"
+        return "paged_prefill_kernel (tcgen05, f16 products on converted one-byte codes)"
     return "paged_prefill_kernel (tcgen05)"
 
 

@@ -13,7 +13,6 @@
 #include "kv_append.cuh"
 #include "prefill.cuh"
 #include "decode_mma.cuh"
-#include "prefill_mma.cuh"
 
 // Launch shapes of the decode kernel (warps per CTA, pipeline stages per warp); overridable
 // at build time for tuning sweeps.  Two stages for the small tiles (one-byte caches, head_dim 64):
@@ -523,23 +522,11 @@ pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, i
   if (num_chunks == 0 || max_q_len == 0) return PA_OK;
   if (!out || !q || !cu_q_lens || !k_cache || !v_cache || !block_tables || !context_lens) return PA_EINVAL;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
-  if (kv_dtype != PA_KV_BF16) {
-    if (!k_scale || !v_scale) return PA_EINVAL;
-    if (num_blocks * num_kv_heads * block_size >= (int64_t(1) << 31)) return PA_EINVAL;
-    const int r = pa::launch_prefill_mma(kv_dtype, out, q, cu_q_lens, num_chunks, k_cache, v_cache, block_tables,
-                                         max_blocks_per_seq, context_lens, num_q_heads, num_kv_heads, num_blocks,
-                                         block_size, scale, k_scale, v_scale, max_q_len, max_context_len,
-                                         reinterpret_cast<cudaStream_t>(stream));
-    if (r == -1) return PA_EINVAL;
-    if (r != 0) {
-      (void)launch_status();   // reports the CUDA error, if any
-      return PA_ECUDA;
-    }
-    return launch_status();
-  }
+  if (kv_dtype != PA_KV_BF16 && (!k_scale || !v_scale)) return PA_EINVAL;
   return pa::launch_prefill(out, q, cu_q_lens, num_chunks, k_cache, v_cache, block_tables, max_blocks_per_seq,
                             context_lens, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
-                            max_q_len, max_context_len, reinterpret_cast<cudaStream_t>(stream));
+                            kv_dtype, k_scale, v_scale, max_q_len, max_context_len,
+                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

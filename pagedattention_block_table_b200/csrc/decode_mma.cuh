@@ -86,27 +86,6 @@ __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// Four one-byte codes (element 0 in the low byte) -> two f16 pairs (0,1) and (2,3), exact.  KT 1: OCP
-// E4M3 through the hardware e4m3x2 -> f16x2 conversion.  KT 2: signed INT8: each byte, biased to unsigned,
-// becomes the low byte of the f16 1024 + b (byte permute), and 1024 + 128 is subtracted (packed).
-template <int KT>
-__device__ __forceinline__ void bytes4_to_h2(uint32_t w, uint32_t &p01, uint32_t &p23) {
-  if constexpr (KT == 1) {
-    e4m3x4_to_h2x2(w, p01, p23);
-  } else {
-    const uint32_t u = w ^ 0x80808080u;
-    const uint32_t bias = 0x64806480u;   // (1152, 1152) in f16
-    const uint32_t x01 = __byte_perm(u, 0x64646464u, 0x4140), x23 = __byte_perm(u, 0x64646464u, 0x4342);
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p01) : "r"(x01), "r"(bias));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p23) : "r"(x23), "r"(bias));
-  }
-}
-
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)

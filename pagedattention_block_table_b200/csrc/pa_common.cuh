@@ -156,6 +156,27 @@ __device__ __forceinline__ void e4m3x4_to_h2x2(uint32_t w, uint32_t &p01, uint32
       : "=r"(p01), "=r"(p23)
       : "r"(w));
 }
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// Four one-byte codes (element 0 in the low byte) -> two f16 pairs (0,1) and (2,3), exact.  KT 1: OCP
+// E4M3 through the hardware e4m3x2 -> f16x2 conversion.  KT 2: signed INT8: each byte, biased to unsigned,
+// becomes the low byte of the f16 1024 + b (byte permute), and 1024 + 128 is subtracted (packed).
+template <int KT>
+__device__ __forceinline__ void bytes4_to_h2(uint32_t w, uint32_t &p01, uint32_t &p23) {
+  if constexpr (KT == 1) {
+    e4m3x4_to_h2x2(w, p01, p23);
+  } else {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t bias = 0x64806480u;   // (1152, 1152) in f16
+    const uint32_t x01 = __byte_perm(u, 0x64646464u, 0x4140), x23 = __byte_perm(u, 0x64646464u, 0x4342);
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p01) : "r"(x01), "r"(bias));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(p23) : "r"(x23), "r"(bias));
+  }
+}
+
 // f16 pair (element 0 low) -> packed fp32 pair, exact.
 __device__ __forceinline__ uint64_t h2_to_f2(uint32_t h) {
   uint64_t r;

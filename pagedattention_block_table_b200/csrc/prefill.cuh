@@ -27,6 +27,14 @@
 // reference max; only when a tile's max exceeds it by more than 2^8 does the row move the reference
 // and rescale its O row in TMEM (tcgen05.ld/st) and its sum l.  O and l always share the reference,
 // so out = O / l is exact whichever reference was used.
+//
+// One-byte caches (FP8 E4M3 or INT8 codes with a scale per KV head, head_dim 128; vLLM "Quantized KV
+// Cache" page).  The products run in f16 (kind::f16 with f16 operands): TMA brings each unit's codes
+// (16 rows x 128 bytes) into a two-item staging ring, warps 10-11 convert them into f16 tiles of the
+// same swizzled layout in the K/V ring (exact for every code: E4M3 and INT8 values are f16 values), and
+// the MMA and softmax warps run unchanged.  Each Q row is scaled by a power of two into f16 range
+// (exact for its elements down to 2^-22 of its largest), P is written as f16 (it is at most 2^8), the
+// K scale and the power of two fold into the row's softmax scale and the V scale into 1 / l.
 #pragma once
 #include <type_traits>
 
@@ -247,6 +255,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
+// The same with f16 A and B (format fields 0).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -270,11 +283,14 @@ struct PrefillParams {
   int max_context_len;
   int num_chunks;
   float qscale;         // scale * log2(e)
+  const float *k_scale; // one-byte caches: per-KV-head scales of the codes (else unused)
+  const float *v_scale;
 };
 
 constexpr int kOrderedChunks = 64;   // chunks the prefill grid orders by context length
 
-template <int D>
+// KT: cache element type (0 bf16, 1 FP8 E4M3, 2 INT8; one-byte types at head_dim 128 only)
+template <int D, int KT = 0>
 struct PrefillCfg {
   static constexpr int BM = 128;                  // rows per query tile (= TMEM lanes)
   static constexpr int BN = 128;                  // keys per key tile (8 units of 16 tokens)
@@ -283,11 +299,15 @@ struct PrefillCfg {
   static constexpr int Q_BYTES = DH * Q_PLANE;
   static constexpr int KV_PLANE = BN * 128;       // 16 KB
   static constexpr int SLOT_BYTES = DH * KV_PLANE;  // one K or V tile
-  static constexpr int NSLOT = D == 128 ? 5 : 8;  // ring of K/V tiles (K and V alternate)
+  // ring of K/V tiles (K and V alternate); one-byte caches give a slot to the staging ring of codes
+  static constexpr int NSLOT = KT != 0 ? 4 : (D == 128 ? 5 : 8);
+  static constexpr int NU8 = KT != 0 ? 2 : 0;     // staging ring of one-byte K or V tiles
+  static constexpr int U8_BYTES = BN * 128;       // 16 KB: 128 keys x 128 one-byte codes
   static constexpr int OFF_QA = 0;
   static constexpr int OFF_QB = OFF_QA + Q_BYTES;
   static constexpr int OFF_KV = OFF_QB + Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NSLOT * SLOT_BYTES;
+  static constexpr int OFF_U8 = OFF_KV + NSLOT * SLOT_BYTES;
+  static constexpr int OFF_BAR = OFF_U8 + NU8 * U8_BYTES;
   static constexpr int NBAR = 32;
   static constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;  // + slack to align the base to 1024
   static constexpr uint32_t TMEM_COLS = 512;
@@ -295,17 +315,19 @@ struct PrefillCfg {
   __host__ __device__ static constexpr uint32_t s_col(int X) { return 128u * X; }
   __host__ __device__ static constexpr uint32_t o_col(int X) { return 256u + static_cast<uint32_t>(D) * X; }
 #if PA_PREFILL_SPLIT_REGS
-  // three warpgroups: softmax A, softmax B, and one holding the MMA and TMA warps (plus two idle warps)
-  // that hands registers to the softmax warpgroups with setmaxnreg
+  // three warpgroups: softmax A, softmax B, and one holding the MMA and TMA warps (plus two warps that
+  // convert one-byte codes, idle over a bf16 cache) that hands registers to the softmax warpgroups with
+  // setmaxnreg
   static constexpr int THREADS = 384;
   static constexpr int REGS_LAUNCH = 168;         // 65536 / 384, rounded down to a multiple of 8
   static constexpr int REGS_SOFTMAX = 216;
   static constexpr int REGS_PRODUCER = 64;
   static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_PRODUCER <= THREADS * REGS_LAUNCH, "register split");
 #else
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = KT != 0 ? 384 : 320;
 #endif
   static_assert(D == 64 || D == 128, "head_dim");
+  static_assert(KT == 0 || D == 128, "one-byte caches at head_dim 128");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -317,7 +339,9 @@ enum : int {
   kPFull = kSFull + 2,
   kQReady = kPFull + 2,
   kDone = kQReady + 1,
-  kNumBars = kDone + 1
+  kU8Full = kDone + 1,   // one-byte staging ring: codes landed / codes converted
+  kU8Empty = kU8Full + 2,
+  kNumBars = kU8Empty + 2
 };
 
 // Three-input max / min (sm_100).
@@ -338,12 +362,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <int D>
-__global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
+template <int D, int KT>
+__global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                          const PrefillParams P) {
-  using C = PrefillCfg<D>;
-  static_assert(kNumBars <= C::NBAR && C::NSLOT <= 8, "barrier slots");
+  using C = PrefillCfg<D, KT>;
+  static_assert(kNumBars <= C::NBAR && C::NSLOT <= 8 && C::NU8 <= 2, "barrier slots");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -402,8 +426,12 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   }
   if (tid == 0) {
     for (int i = 0; i < C::NSLOT; ++i) {
-      mbar_init(&bars[kFull + i], 1);
+      mbar_init(&bars[kFull + i], KT != 0 ? 64 : 1);   // one-byte: the 64 converting threads
       mbar_init(&bars[kEmpty + i], 1);
+    }
+    for (int i = 0; i < C::NU8; ++i) {
+      mbar_init(&bars[kU8Full + i], 1);
+      mbar_init(&bars[kU8Empty + i], 64);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars[kSFull + i], 1);
@@ -433,8 +461,38 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     const bool row_ok = pos_i < Cn;
     const int pos = row_ok ? H + pos_i : kv_len - 1;  // padding rows behave like the last row
     uint8_t *sQ = smem + (X ? C::OFF_QB : C::OFF_QA);
+    float qs = P.qscale;
     // Q row into the K-major 128-byte-swizzled tile (chunk ch of row r at ch ^ (r % 8))
-    {
+    if constexpr (KT != 0) {
+      // f16 row scaled by 2^e so that its largest magnitude lies in [2^8, 2^9); 2^-e and the K scale
+      // join the row's softmax scale
+      uint8_t *rowp = sQ + r * 128;
+      uint4 w[D / 8];
+      float amax = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        w[ch] = row_ok ? reinterpret_cast<const uint4 *>(P.q + ((int64_t)(q0 + pos_i) * P.num_q_heads + h) * D)[ch]
+                       : make_uint4(0, 0, 0, 0);
+        const uint32_t ww[4] = {w[ch].x, w[ch].y, w[ch].z, w[ch].w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) amax = fmax3(amax, fabsf(bf16lo(ww[t])), fabsf(bf16hi(ww[t])));
+      }
+      int ex = amax > 0.f ? static_cast<int>((__float_as_uint(amax) >> 23) & 0xff) - 127 : 0;
+      ex = ex < -118 ? -118 : (ex > 126 ? 126 : ex);
+      const float up = __uint_as_float(static_cast<uint32_t>(127 + 8 - ex) << 23);   // 2^(8 - ex)
+      qs = __uint_as_float(static_cast<uint32_t>(127 + ex - 8) << 23) * (P.qscale * P.k_scale[g]);
+#pragma unroll
+      for (int ch = 0; ch < D / 8; ++ch) {
+        const uint32_t ww[4] = {w[ch].x, w[ch].y, w[ch].z, w[ch].w};
+        uint32_t hw[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) hw[t] = pack_f16x2(bf16lo(ww[t]) * up, bf16hi(ww[t]) * up);
+        *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::Q_PLANE + (((ch & 7) ^ (r & 7)) << 4)) =
+            make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      }
+      fence_async_smem();
+      mbar_arrive(&bars[kQReady]);
+    } else {
       uint8_t *rowp = sQ + r * 128;
       if (row_ok) {
         const uint4 *src = reinterpret_cast<const uint4 *>(P.q + ((int64_t)(q0 + pos_i) * P.num_q_heads + h) * D);
@@ -453,7 +511,6 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     const uint32_t s_addr = tmem + lane_base + C::s_col(X);
     const uint32_t o_addr = tmem + lane_base + C::o_col(X);
     constexpr float kRescale = 8.f;
-    const float qs = P.qscale;
     float m_ref = -INFINITY, l_run = 0.f;
     for (int j = 0; j < ntiles; ++j) {
       const int kbase = j * C::BN;
@@ -471,7 +528,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       // last key tile: V rows of keys no row may see, up to the last 16-key step the PV product reads,
       // are zeroed (tile A's threads, one row each) once the V tile has landed, so that 0 * (whatever
       // the cache holds past the context) never reaches the MMA
-      if (X == 0 && j == ntiles - 1 && kbase + r >= kv_len && r < last_k16 * 16) {
+      // (one-byte caches: the converting warps write those rows as zeros)
+      if (KT == 0 && X == 0 && j == ntiles - 1 && kbase + r >= kv_len && r < last_k16 * 16) {
         const int it = 2 * j + 1;
         if (mbar_wait(&bars[kFull + it % C::NSLOT], (it / C::NSLOT) & 1)) {
           uint8_t *vt = slot_of(it);
@@ -549,7 +607,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
             const float a = ex2(x.x);
             const float b = ex2(x.y);
             ls2 = f2add(ls2, f2pack(a, b));
-            pk[k2] = pack_bf16x2(a, b);
+            pk[k2] = KT != 0 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
           }
           tmem_st16u_nowait(s_addr + qq * 16, pk);
         }
@@ -594,7 +652,7 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     // ---- epilogue: out = O / l once the last PV is done
     if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0))) {
       tc_fence_after();
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = l_run > 0.f ? (KT != 0 ? P.v_scale[g] : 1.f) / l_run : 0.f;
       uint4 *dst = reinterpret_cast<uint4 *>(P.out + ((int64_t)(q0 + (row_ok ? pos_i : 0)) * P.num_q_heads + h) * D);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -617,8 +675,8 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
   if (warp == 8) {
     // ===================================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, C::BN, false);
-      constexpr uint32_t idO = idesc_bf16(128, D, true);
+      constexpr uint32_t idS = KT != 0 ? idesc_f16(128, C::BN, false) : idesc_bf16(128, C::BN, false);
+      constexpr uint32_t idO = KT != 0 ? idesc_f16(128, D, true) : idesc_bf16(128, D, true);
       const uint32_t qa = smem_u32(smem + C::OFF_QA), qb = smem_u32(smem + C::OFF_QB);
       auto ready = [&](int i) {
         const bool r = mbar_wait(&bars[kFull + i % C::NSLOT], (i / C::NSLOT) & 1);
@@ -677,15 +735,23 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
     // One copy per lane: a key tile is UPT units x DH planes for K and as many for V (32 copies at
     // head_dim 128), so lane l copies plane l % DH of unit (l / DH) % UPT of K (first half of the
     // warp) or V (second half).  Each lane loads its unit's block-table entry two tiles ahead.
+    // One-byte caches: one 128-byte plane per unit, into the staging ring.
     {
       const int32_t *trow = P.block_tables + (int64_t)c * P.max_blocks_per_seq;
       const int ush = P.block_size == 32 ? 1 : 0;   // log2(16-row units per physical block)
       constexpr int UPT = C::BN / kBlock;             // units per key tile
-      constexpr int PER = UPT * C::DH;                // copies per K or V tile
+      constexpr int NPL = KT != 0 ? 1 : C::DH;        // 128-byte planes per unit row
+      constexpr int PER = UPT * NPL;                  // copies per K or V tile
+      constexpr int NRING = KT != 0 ? C::NU8 : C::NSLOT;
+      constexpr int FULL = KT != 0 ? kU8Full : kFull, EMPTY = KT != 0 ? kU8Empty : kEmpty;
+      constexpr int PLANE_BYTES = KT != 0 ? C::U8_BYTES : C::KV_PLANE;
       static_assert(2 * PER <= 32, "one copy per lane");
       const int w_lane = lane / PER;                  // 0: K, 1: V, 2+: idle
-      const int bb = (lane / C::DH) % UPT;            // unit of the tile
-      const int hh = lane % C::DH;                    // 64-element plane
+      const int bb = (lane / NPL) % UPT;              // unit of the tile
+      const int hh = lane % NPL;                      // 128-byte plane
+      auto ring_of = [&](int i) {
+        return KT != 0 ? smem + C::OFF_U8 + (i % NRING) * C::U8_BYTES : slot_of(i);
+      };
       auto row_of = [&](int j) {                      // cache row of this lane's unit of key tile j
         const int u = j * UPT + bb;
         int e = 0;
@@ -704,19 +770,20 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
         const int y2 = row_of(j + 2);
         const int nu = min(UPT, (kv_len - j * C::BN + kBlock - 1) / kBlock);
         for (int w = 0; w < 2; ++w) {                 // K, then V of tile j
-          const int it = 2 * j + w, slot = it % C::NSLOT;
+          const int it = 2 * j + w, slot = it % NRING;
           int ok = 1;
           if (lane == 0) {
-            if (it >= C::NSLOT) ok = mbar_wait(&bars[kEmpty + slot], ((it / C::NSLOT) - 1) & 1);
-            if (ok) mbar_arrive_expect_tx(&bars[kFull + slot], nu * C::DH * (kBlock * 128));
+            if (it >= NRING) ok = mbar_wait(&bars[EMPTY + slot], ((it / NRING) - 1) & 1);
+            if (ok) mbar_arrive_expect_tx(&bars[FULL + slot], nu * NPL * (kBlock * 128));
           }
           if (!__shfl_sync(0xffffffffu, ok, 0)) {
             timeout = true;
             break;
           }
+          // x: element 64 * hh of the bf16 row, or byte 0 of the one-byte row (16-byte aligned)
           if (w_lane == w && bb < nu)
-            tma_load_2d(slot_of(it) + hh * C::KV_PLANE + bb * (kBlock * 128), w ? &vmap : &kmap, hh * 64, y0,
-                        &bars[kFull + slot]);
+            tma_load_2d(ring_of(it) + hh * PLANE_BYTES + bb * (kBlock * 128), w ? &vmap : &kmap, hh * 64, y0,
+                        &bars[FULL + slot]);
           issued = it + 1;
         }
         y0 = y1;
@@ -725,8 +792,49 @@ __global__ void __launch_bounds__(PrefillCfg<D>::THREADS, 1)
       // before leaving, the last tiles this warp issued must have landed (a no-op when the MMA warp
       // consumed them; bounded when a wait elsewhere gave up)
       if (lane == 0)
-        for (int k = max(0, issued - C::NSLOT); k < issued; ++k)
-          (void)mbar_wait(&bars[kFull + (k % C::NSLOT)], (k / C::NSLOT) & 1);
+        for (int k = max(0, issued - NRING); k < issued; ++k)
+          (void)mbar_wait(&bars[FULL + (k % NRING)], (k / NRING) & 1);
+    }
+  } else if (warp >= 10) {
+    if constexpr (KT != 0) {
+      // ===================================================================== one-byte codes -> f16 tiles
+      // Warp 10 converts dims 0-63 (plane 0 of the f16 tile), warp 11 dims 64-127.  Per instruction a warp
+      // takes 8 rows (lane % 8) x 4 chunks of 16 codes (lane / 8): the 8 lanes of a quarter-warp share a
+      // chunk and cover 8 consecutive rows, so both the 16-byte reads and the two 16-byte writes of each
+      // lane fall in 8 distinct bank groups (the swizzle XORs the chunk with row % 8).  Rows past the
+      // context, including units the producer did not load, are written as zeros: their K columns are
+      // masked, and their V rows meet p = 0, which must not meet a NaN code.
+      const int w = warp - 10, r8 = lane & 7, cq = lane >> 3;
+      const int c = 4 * w + cq;                         // chunk of 16 codes = dims [16c, 16c + 16)
+      for (int it = 0; it < 2 * ntiles; ++it) {
+        const int su = it % C::NU8, slot = it % C::NSLOT;
+        const bool ok = mbar_wait(&bars[kU8Full + su], (it / C::NU8) & 1) &&
+                        (it < C::NSLOT || mbar_wait(&bars[kEmpty + slot], ((it / C::NSLOT) - 1) & 1));
+        if (!__all_sync(0xffffffffu, ok)) {
+          timeout = true;
+          break;
+        }
+        const uint8_t *src = smem + C::OFF_U8 + su * C::U8_BYTES;
+        uint8_t *dst = slot_of(it) + w * C::KV_PLANE;
+        const int nvalid = kv_len - (it >> 1) * C::BN;  // rows of this tile that hold keys (may exceed BN)
+#pragma unroll 4
+        for (int i = 0; i < C::BN / 8; ++i) {
+          const int R = 8 * i + r8;
+          uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
+          if (R < nvalid) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(src + R * 128 + ((c ^ r8) << 4));
+            bytes4_to_h2<KT>(v.x, lo.x, lo.y);
+            bytes4_to_h2<KT>(v.y, lo.z, lo.w);
+            bytes4_to_h2<KT>(v.z, hi.x, hi.y);
+            bytes4_to_h2<KT>(v.w, hi.z, hi.w);
+          }
+          *reinterpret_cast<uint4 *>(dst + R * 128 + (((2 * cq) ^ r8) << 4)) = lo;
+          *reinterpret_cast<uint4 *>(dst + R * 128 + (((2 * cq + 1) ^ r8) << 4)) = hi;
+        }
+        fence_async_smem();
+        mbar_arrive(&bars[kU8Empty + su]);
+        mbar_arrive(&bars[kFull + slot]);
+      }
     }
   }
   }
@@ -786,21 +894,23 @@ inline bool make_cache_map_u8(CUtensorMap *map, const void *base, int64_t rows, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, int KT>
 int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_cache, int num_chunks, int max_q_len,
                      cudaStream_t st) {
-  using C = PrefillCfg<D>;
+  using C = PrefillCfg<D, KT>;
   CUtensorMap km, vm;
   const int64_t rows = P.num_blocks * P.num_kv_heads * P.block_size;
-  if (!make_cache_map(&km, k_cache, rows, D) || !make_cache_map(&vm, v_cache, rows, D)) return -3;
-  if (cudaFuncSetAttribute(paged_prefill_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+  if (KT != 0 ? (!make_cache_map_u8(&km, k_cache, rows, D) || !make_cache_map_u8(&vm, v_cache, rows, D))
+              : (!make_cache_map(&km, k_cache, rows, D) || !make_cache_map(&vm, v_cache, rows, D)))
+    return -3;
+  if (cudaFuncSetAttribute(paged_prefill_kernel<D, KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return -3;
 #if PA_PREFILL_SPLIT_REGS
   // setmaxnreg.inc waits until the block's launch allocation can cover the new split: never launch a
   // build whose register count per thread would not
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, paged_prefill_kernel<D>) != cudaSuccess ||
+  if (cudaFuncGetAttributes(&fa, paged_prefill_kernel<D, KT>) != cudaSuccess ||
       fa.numRegs * C::THREADS < 2 * 128 * C::REGS_SOFTMAX + 128 * C::REGS_PRODUCER)
     return -3;
 #endif
@@ -808,14 +918,15 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
   const int tiles = (max_q_len + 2 * ppt - 1) / (2 * ppt);
   if (tiles > 65535) return -1;
   dim3 grid(P.num_q_heads / P.hpr, tiles, num_chunks);
-  return launch_pdl(paged_prefill_kernel<D>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;
+  return launch_pdl(paged_prefill_kernel<D, KT>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;
 }
 
+// kv_dtype: 0 bf16, 1 FP8 E4M3, 2 INT8 (one-byte types: head_dim 128, k_scale / v_scale per KV head)
 inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
                           const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                           const int32_t *context_lens, int num_q_heads, int num_kv_heads, int head_dim,
-                          int64_t num_blocks, int block_size, float scale, int max_q_len, int max_context_len,
-                          cudaStream_t st) {
+                          int64_t num_blocks, int block_size, float scale, int kv_dtype, const float *k_scale,
+                          const float *v_scale, int max_q_len, int max_context_len, cudaStream_t st) {
   if (num_chunks > 65535 || num_q_heads > 65535) return -1;
   if (num_blocks * num_kv_heads * block_size >= (int64_t(1) << 31)) return -2;
   PrefillParams P;
@@ -834,8 +945,13 @@ inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, in
   P.max_context_len = max_context_len;
   P.num_chunks = num_chunks;
   P.qscale = scale * 1.4426950408889634f;
-  return head_dim == 128 ? launch_prefill_d<128>(P, k_cache, v_cache, num_chunks, max_q_len, st)
-                         : launch_prefill_d<64>(P, k_cache, v_cache, num_chunks, max_q_len, st);
+  P.k_scale = k_scale;
+  P.v_scale = v_scale;
+  if (kv_dtype != 0 && (head_dim != 128 || k_scale == nullptr || v_scale == nullptr)) return -1;
+  if (kv_dtype == 1) return launch_prefill_d<128, 1>(P, k_cache, v_cache, num_chunks, max_q_len, st);
+  if (kv_dtype == 2) return launch_prefill_d<128, 2>(P, k_cache, v_cache, num_chunks, max_q_len, st);
+  return head_dim == 128 ? launch_prefill_d<128, 0>(P, k_cache, v_cache, num_chunks, max_q_len, st)
+                         : launch_prefill_d<64, 0>(P, k_cache, v_cache, num_chunks, max_q_len, st);
 }
 
 }  // namespace pa
