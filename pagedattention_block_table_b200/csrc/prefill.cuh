@@ -321,7 +321,7 @@ struct PrefillCfg {
   static constexpr int THREADS = 384;
   static constexpr int REGS_LAUNCH = 168;         // 65536 / 384, rounded down to a multiple of 8
   static constexpr int REGS_SOFTMAX = 216;
-  static constexpr int REGS_PRODUCER = 64;
+  static constexpr int REGS_PRODUCER = 72;        // the rest of the launch allocation (one-byte converters)
   static_assert(2 * 128 * REGS_SOFTMAX + 128 * REGS_PRODUCER <= THREADS * REGS_LAUNCH, "register split");
 #else
   static constexpr int THREADS = KT != 0 ? 384 : 320;
@@ -817,20 +817,36 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
         const uint8_t *src = smem + C::OFF_U8 + su * C::U8_BYTES;
         uint8_t *dst = slot_of(it) + w * C::KV_PLANE;
         const int nvalid = kv_len - (it >> 1) * C::BN;  // rows of this tile that hold keys (may exceed BN)
-#pragma unroll 4
-        for (int i = 0; i < C::BN / 8; ++i) {
-          const int R = 8 * i + r8;
-          uint4 lo = make_uint4(0, 0, 0, 0), hi = make_uint4(0, 0, 0, 0);
-          if (R < nvalid) {
-            const uint4 v = *reinterpret_cast<const uint4 *>(src + R * 128 + ((c ^ r8) << 4));
-            bytes4_to_h2<KT>(v.x, lo.x, lo.y);
-            bytes4_to_h2<KT>(v.y, lo.z, lo.w);
-            bytes4_to_h2<KT>(v.z, hi.x, hi.y);
-            bytes4_to_h2<KT>(v.w, hi.z, hi.w);
+        // eight 16-byte reads in flight per lane, then their conversions and writes; the row test is
+        // compiled only into the last tile's pass (a test per read keeps the reads from batching)
+        auto convert = [&](auto partial_c) {
+          constexpr bool kPartial = decltype(partial_c)::value;
+#pragma unroll 1
+          for (int i0 = 0; i0 < C::BN / 8; i0 += 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int R = 8 * (i0 + k) + r8;
+              v[k] = (!kPartial || R < nvalid) ? *reinterpret_cast<const uint4 *>(src + R * 128 + ((c ^ r8) << 4))
+                                               : make_uint4(0, 0, 0, 0);   // code 0 is +0 in both types
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int R = 8 * (i0 + k) + r8;
+              uint4 lo, hi;
+              bytes4_to_h2<KT>(v[k].x, lo.x, lo.y);
+              bytes4_to_h2<KT>(v[k].y, lo.z, lo.w);
+              bytes4_to_h2<KT>(v[k].z, hi.x, hi.y);
+              bytes4_to_h2<KT>(v[k].w, hi.z, hi.w);
+              *reinterpret_cast<uint4 *>(dst + R * 128 + (((2 * cq) ^ r8) << 4)) = lo;
+              *reinterpret_cast<uint4 *>(dst + R * 128 + (((2 * cq + 1) ^ r8) << 4)) = hi;
+            }
           }
-          *reinterpret_cast<uint4 *>(dst + R * 128 + (((2 * cq) ^ r8) << 4)) = lo;
-          *reinterpret_cast<uint4 *>(dst + R * 128 + (((2 * cq + 1) ^ r8) << 4)) = hi;
-        }
+        };
+        if (nvalid >= C::BN)
+          convert(std::false_type{});
+        else
+          convert(std::true_type{});
         fence_async_smem();
         mbar_arrive(&bars[kU8Empty + su]);
         mbar_arrive(&bars[kFull + slot]);
