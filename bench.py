@@ -302,7 +302,8 @@ def launches_per_step(st) -> int:
     """Kernels of this library one step launches: fork, append, decode, LSE reduce, prefill (when present)."""
     b = st.batch
     return ((1 if b.cow_pairs.shape[0] else 0) + 1 + (1 if b.num_decode else 0)
-            + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0))
+            + (1 if st.workspace is not None else 0) + (1 if st.max_q else 0)
+            + (1 if st.max_q and st.pre_workspace is not None else 0))
 
 
 def decode_kernel_label(batch) -> str:
@@ -314,11 +315,11 @@ def decode_kernel_label(batch) -> str:
     return f"pa_paged_attention ({k} + lse_reduce_kernel)"
 
 
-def prefill_kernel_label(batch) -> str:
-    """The prefill kernel pa_paged_prefill runs for this batch's cache."""
-    if batch.kv_dtype:
-        return "paged_prefill_kernel (tcgen05, f16 products on converted one-byte codes)"
-    return "paged_prefill_kernel (tcgen05)"
+def prefill_kernel_label(batch, split=False) -> str:
+    """The prefill kernel pa_paged_prefill runs for this batch's cache (and the merge of split key ranges)."""
+    k = ("paged_prefill_kernel (tcgen05, f16 products on converted one-byte codes)" if batch.kv_dtype
+         else "paged_prefill_kernel (tcgen05)")
+    return k + (" + prefill_combine_kernel" if split else "")
 
 
 def workload_batch(name, device, num_seqs=0):
@@ -411,7 +412,8 @@ def sub_record(name, dev, args, clk):
         pf = prefill_flops(batch)
         tp, tk = bf16_peak()
         ach = pf / (m["pre_ms"] * 1e-3) / 1e12
-        rec["prefill"] = {"kernel": prefill_kernel_label(batch), "bound": "tensor", "unit": "TFLOP/s",
+        rec["prefill"] = {"kernel": prefill_kernel_label(batch, st.pre_workspace is not None), "bound": "tensor",
+                          "unit": "TFLOP/s",
                           "achieved": round(ach, 2), "peak": tp, "peak_kind": tk, "frac": round(ach / tp, 4),
                           "flops": pf, "avg_launch_ms": round(m["pre_ms"], 5)}
     del m, st, batch
@@ -492,7 +494,8 @@ def run_ours(args, rank, world, local_rank):
         pf = prefill_flops(batch)
         tp, tk = bf16_peak()
         pre_ms = agg["pre_ms"]
-        line["prefill"] = {"kernel": prefill_kernel_label(batch), "bound": "tensor", "unit": "TFLOP/s",
+        line["prefill"] = {"kernel": prefill_kernel_label(batch, st.pre_workspace is not None), "bound": "tensor",
+                           "unit": "TFLOP/s",
                            "achieved": round(pf / (pre_ms * 1e-3) / 1e12, 2), "peak": tp, "peak_kind": tk,
                            "frac": round(pf / (pre_ms * 1e-3) / 1e12 / tp, 4), "flops": pf,
                            "avg_launch_ms": round(pre_ms, 5)}

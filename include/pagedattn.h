@@ -211,15 +211,35 @@ pa_status pa_paged_attention_noalloc(void *out, const void *q, const void *k_cac
  *                  bf16): K[t] = code * k_scale[h/G], V[t] = code * v_scale[h/G]  [KV Cache to vLLM §2.2].
  * A chunk whose C_c exceeds max_q_len, or whose context exceeds max_context_len or its table row,
  * sets the device error word (PA_EDEVICE_OOB from pa_get_device_error) and its rows are not written.
- * bf16 caches run on the tcgen05 tensor cores; one-byte caches on warp-level tensor-core products in
- * f16 over codes converted in registers.  A one-byte cache at head_dim 64 returns PA_EUNSUPPORTED.
+ * All cache types run on the tcgen05 tensor cores (one-byte codes are converted to f16 tiles in shared
+ * memory inside the kernel).  A one-byte cache at head_dim 64 returns PA_EUNSUPPORTED.
+ *   host_cu_q_lens, host_context_lens : optional host copies of cu_q_lens / context_lens (both or
+ *                  neither; they must hold the same values as the device arrays).  With them the call
+ *                  plans its launch: work items longest first, and a CTA whose key range is long next to
+ *                  the launch's work per SM is cut into pieces whose partial results a second kernel
+ *                  merges (the same log-sum-exp merge as the decode's split-K).  The plan changes the
+ *                  schedule only, not the result beyond rounding.  Without them the launch is ordered on
+ *                  the device by context length and nothing is split.
+ *   workspace    : device memory of at least pa_paged_prefill_workspace_size(...) bytes, 16-byte aligned,
+ *                  for the pieces' partials (NULL when that size is 0); owned by the caller, reusable
+ *                  once the call has completed on the stream.  Too small: PA_EWORKSPACE, nothing launched.
  */
 pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks,
                            const void *k_cache, const void *v_cache, const int32_t *block_tables,
                            int max_blocks_per_seq, const int32_t *context_lens, int num_q_heads,
                            int num_kv_heads, int head_dim, int64_t num_blocks, int block_size,
                            float scale, int kv_dtype, const float *k_scale, const float *v_scale,
-                           int max_q_len, int max_context_len, pa_stream_t stream);
+                           int max_q_len, int max_context_len, const int32_t *host_cu_q_lens,
+                           const int32_t *host_context_lens, void *workspace, size_t workspace_bytes,
+                           pa_stream_t stream);
+
+/* pa_paged_prefill_workspace_size -- bytes of workspace a pa_paged_prefill call with these host lengths
+ * needs (0: the plan splits nothing, or no host lengths).  Deterministic for given arguments on a given
+ * device model (the plan depends on its SM count). */
+size_t pa_paged_prefill_workspace_size(int num_chunks, const int32_t *host_cu_q_lens,
+                                       const int32_t *host_context_lens, int num_q_heads, int num_kv_heads,
+                                       int head_dim, int max_blocks_per_seq, int block_size, int max_q_len,
+                                       int max_context_len);
 
 /* ------------------------------------------------------------------------------------------------
  * Host block manager: the control plane that produces block tables, slot mappings and copy-on-write

@@ -32,7 +32,7 @@ PA_KV_INT8 = 2
 EXPORTED = (
     "pa_kv_append", "pa_copy_blocks", "pa_paged_attention_workspace_size",
     "pa_paged_attention_auto_split", "pa_paged_attention_uses_tensor_cores", "pa_paged_attention",
-    "pa_paged_prefill",
+    "pa_paged_prefill", "pa_paged_prefill_workspace_size",
     "pa_get_device_error", "pa_status_string", "pa_kv_cache_bytes", "pa_version",
     "pa_paged_attention_noalloc", "pa_swap_blocks",
     "pa_bm_create", "pa_bm_destroy", "pa_bm_num_free", "pa_bm_add", "pa_bm_fork", "pa_bm_append", "pa_bm_free",
@@ -77,7 +77,9 @@ def lib() -> ctypes.CDLL:
         L.pa_paged_attention_noalloc.restype = I
         L.pa_paged_attention_noalloc.argtypes = [P, P, P, P, P, I, P, I, I, I, I, I64, F, I, P, P, I, I, P]
         L.pa_paged_prefill.restype = I
-        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, I, F, I, P, P, I, I, P]
+        L.pa_paged_prefill.argtypes = [P, P, P, I, P, P, P, I, P, I, I, I, I64, I, F, I, P, P, I, I, P, P, P, SZ, P]
+        L.pa_paged_prefill_workspace_size.restype = SZ
+        L.pa_paged_prefill_workspace_size.argtypes = [I, P, P, I, I, I, I, I, I, I]
         L.pa_get_device_error.restype = I
         L.pa_get_device_error.argtypes = [P]
         L.pa_selftest_bounded_wait.restype = I
@@ -237,17 +239,17 @@ def pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, head_dim=128
     return int(lib().pa_paged_attention_uses_tensor_cores(num_q_heads, num_kv_heads, head_dim, kv_dtype))
 
 
-def _host_i32(a, n):
+def _host_i32(a, n, name="host_context_lens"):
     """Host pointer of an int32 array of n elements (numpy or CPU tensor), or None."""
     if a is None:
         return None
     if isinstance(a, torch.Tensor):
         if a.device.type != "cpu" or a.dtype != torch.int32 or not a.is_contiguous() or a.numel() != n:
-            raise ValueError("host_context_lens must be a contiguous int32 CPU tensor of num_seqs elements")
+            raise ValueError(f"{name} must be a contiguous int32 CPU tensor of {n} elements")
         return a.data_ptr()
     import numpy as np
     if not isinstance(a, np.ndarray) or a.dtype != np.int32 or not a.flags["C_CONTIGUOUS"] or a.size != n:
-        raise ValueError("host_context_lens must be a contiguous int32 array of num_seqs elements")
+        raise ValueError(f"{name} must be a contiguous int32 array of {n} elements")
     return a.ctypes.data
 
 
@@ -296,8 +298,22 @@ def pa_paged_attention_noalloc(out, q, k_cache, v_cache, block_tables, context_l
     _check(st, "pa_paged_attention_noalloc")
 
 
+def pa_paged_prefill_workspace_size(host_cu_q_lens, host_context_lens, num_q_heads, num_kv_heads, head_dim,
+                                    max_blocks_per_seq, block_size, max_q_len, max_context_len) -> int:
+    """Workspace bytes pa_paged_prefill needs with these host lengths (int32 numpy arrays or CPU tensors)."""
+    n = len(host_context_lens)
+    return int(lib().pa_paged_prefill_workspace_size(
+        n, _host_i32(host_cu_q_lens, n + 1, "host_cu_q_lens"), _host_i32(host_context_lens, n), int(num_q_heads),
+        int(num_kv_heads), int(head_dim), int(max_blocks_per_seq), int(block_size), int(max_q_len),
+        int(max_context_len)))
+
+
 def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_lens, scale, max_q_len,
-                     max_context_len, kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, stream=None):
+                     max_context_len, kv_dtype=PA_KV_BF16, k_scale=None, v_scale=None, stream=None,
+                     host_cu_q_lens=None, host_context_lens=None, workspace=None):
+    """host_cu_q_lens / host_context_lens: optional host copies of the length arrays (int32 numpy arrays or CPU
+    tensors, the same values); with them the launch is planned, and `workspace` (a CUDA tensor of at least
+    pa_paged_prefill_workspace_size bytes) holds the partials of split key ranges."""
     nb, hkv, d, bs = _cache_geometry(k_cache)
     cd = _CACHE_DTYPES[kv_dtype]
     tq, hq, dq = q.shape
@@ -312,7 +328,10 @@ def pa_paged_prefill(out, q, cu_q_lens, k_cache, v_cache, block_tables, context_
         _ptr(v_cache, "v_cache", cd), _ptr(block_tables, "block_tables", (torch.int32,)),
         int(block_tables.shape[1]), _ptr(context_lens, "context_lens", (torch.int32,)), hq, hkv, d, nb, bs,
         float(scale), int(kv_dtype), _ptr(k_scale, "k_scale", (torch.float32,)),
-        _ptr(v_scale, "v_scale", (torch.float32,)), int(max_q_len), int(max_context_len), _stream(stream))
+        _ptr(v_scale, "v_scale", (torch.float32,)), int(max_q_len), int(max_context_len),
+        _host_i32(host_cu_q_lens, n + 1, "host_cu_q_lens"), _host_i32(host_context_lens, n),
+        _ptr(workspace, "workspace"), 0 if workspace is None else workspace.numel() * workspace.element_size(),
+        _stream(stream))
     _check(st, "pa_paged_prefill")
 
 

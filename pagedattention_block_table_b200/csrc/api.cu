@@ -505,11 +505,44 @@ pa_status pa_paged_attention(void *out, const void *q, const void *k_cache, cons
   return launch_status();
 }
 
+namespace {
+// The plan of a prefill call whose lengths the caller also has on the host (see plan_prefill); false
+// when none applies.  Both the workspace query and the call build it the same way.
+bool prefill_plan_for(int num_chunks, const int32_t *host_cu_q_lens, const int32_t *host_context_lens,
+                      int num_q_heads, int num_kv_heads, int max_blocks_per_seq, int block_size, int max_q_len,
+                      int max_context_len, pa::PrefillPlanHost &plan) {
+  if (!host_cu_q_lens || !host_context_lens || num_chunks <= 0 || num_kv_heads <= 0 ||
+      num_q_heads % num_kv_heads != 0)
+    return false;
+  const int group = num_q_heads / num_kv_heads;
+  const int hpr = (group <= 128 && 128 % group == 0) ? group : 1;
+  const int64_t lim = std::min<int64_t>((int64_t)max_blocks_per_seq * block_size, max_context_len);
+  return pa::plan_prefill(host_cu_q_lens, host_context_lens, num_chunks, hpr, num_q_heads / hpr, device_sm_count(),
+                          max_q_len, static_cast<int>(lim), plan);
+}
+thread_local pa::PrefillPlanHost g_prefill_plan;   // 20 KB: kept off the stack
+}  // namespace
+
+size_t pa_paged_prefill_workspace_size(int num_chunks, const int32_t *host_cu_q_lens, const int32_t *host_context_lens,
+                                       int num_q_heads, int num_kv_heads, int head_dim, int max_blocks_per_seq,
+                                       int block_size, int max_q_len, int max_context_len) {
+  if (head_dim != 64 && head_dim != 128) return 0;
+  pa::PrefillPlanHost &plan = g_prefill_plan;
+  if (!prefill_plan_for(num_chunks, host_cu_q_lens, host_context_lens, num_q_heads, num_kv_heads, max_blocks_per_seq,
+                        block_size, max_q_len, max_context_len, plan))
+    return 0;
+  const int group = num_q_heads / num_kv_heads;
+  const int hpr = (group <= 128 && 128 % group == 0) ? group : 1;
+  return pa::prefill_plan_workspace(plan, num_q_heads / hpr, head_dim);
+}
+
 pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
                            const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                            const int32_t *context_lens, int num_q_heads, int num_kv_heads, int head_dim,
                            int64_t num_blocks, int block_size, float scale, int kv_dtype, const float *k_scale,
-                           const float *v_scale, int max_q_len, int max_context_len, pa_stream_t stream) {
+                           const float *v_scale, int max_q_len, int max_context_len, const int32_t *host_cu_q_lens,
+                           const int32_t *host_context_lens, void *workspace, size_t workspace_bytes,
+                           pa_stream_t stream) {
   if (num_chunks < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
     return PA_EINVAL;
   if (!block_size_ok(block_size)) return PA_EUNSUPPORTED;
@@ -519,14 +552,31 @@ pa_status pa_paged_prefill(void *out, const void *q, const int32_t *cu_q_lens, i
   if (kv_dtype != PA_KV_BF16 && head_dim != 128) return PA_EUNSUPPORTED;
   if (max_q_len < 0 || max_context_len < 0) return PA_EINVAL;
   if (!(scale == scale) || isinf(scale)) return PA_EINVAL;
+  if ((host_cu_q_lens == nullptr) != (host_context_lens == nullptr)) return PA_EINVAL;
   if (num_chunks == 0 || max_q_len == 0) return PA_OK;
   if (!out || !q || !cu_q_lens || !k_cache || !v_cache || !block_tables || !context_lens) return PA_EINVAL;
   if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return PA_EINVAL;
   if (kv_dtype != PA_KV_BF16 && (!k_scale || !v_scale)) return PA_EINVAL;
-  return pa::launch_prefill(out, q, cu_q_lens, num_chunks, k_cache, v_cache, block_tables, max_blocks_per_seq,
-                            context_lens, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
-                            kv_dtype, k_scale, v_scale, max_q_len, max_context_len,
-                            reinterpret_cast<cudaStream_t>(stream));
+  pa::PrefillPlanHost &plan = g_prefill_plan;
+  const bool planned = prefill_plan_for(num_chunks, host_cu_q_lens, host_context_lens, num_q_heads, num_kv_heads,
+                                        max_blocks_per_seq, block_size, max_q_len, max_context_len, plan);
+  if (planned) {
+    const int group = num_q_heads / num_kv_heads;
+    const int hpr = (group <= 128 && 128 % group == 0) ? group : 1;
+    const size_t need = pa::prefill_plan_workspace(plan, num_q_heads / hpr, head_dim);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_EWORKSPACE;
+  }
+  const int r = pa::launch_prefill(out, q, cu_q_lens, num_chunks, k_cache, v_cache, block_tables, max_blocks_per_seq,
+                                   context_lens, num_q_heads, num_kv_heads, head_dim, num_blocks, block_size, scale,
+                                   kv_dtype, k_scale, v_scale, max_q_len, max_context_len,
+                                   planned ? &plan : nullptr, workspace, reinterpret_cast<cudaStream_t>(stream));
+  if (r == -1) return PA_EINVAL;
+  if (r == -2) return PA_EUNSUPPORTED;
+  if (r != 0) {
+    (void)launch_status();   // reports the CUDA error, if any
+    return PA_ECUDA;
+  }
+  return launch_status();
 }
 
 }  // extern "C"

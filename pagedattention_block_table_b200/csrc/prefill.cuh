@@ -36,7 +36,11 @@
 // (exact for its elements down to 2^-22 of its largest), P is written as f16 (it is at most 2^8), the
 // K scale and the power of two fold into the row's softmax scale and the V scale into 1 / l.
 #pragma once
+#include <algorithm>
+#include <functional>
+#include <queue>
 #include <type_traits>
+#include <vector>
 
 #include "pa_common.cuh"
 
@@ -285,9 +289,34 @@ struct PrefillParams {
   float qscale;         // scale * log2(e)
   const float *k_scale; // one-byte caches: per-KV-head scales of the codes (else unused)
   const float *v_scale;
+  float *ws_o;          // planned launches with split key ranges: partial O rows [slot][x][256][D]
+  float *ws_ml;         // and their (reference max, sum) [slot][x][256][2]
 };
 
 constexpr int kOrderedChunks = 64;   // chunks the prefill grid orders by context length
+constexpr int kPlanItems = 1024;     // work items of a planned launch (kernel-parameter list)
+constexpr int kPlanChunks = 1024;    // chunks a planned launch can carry
+
+// A planned launch (the caller passed the lengths on the host too): grid row y serves work item y, in
+// the order a longest-processing-time-first schedule gives.  An item is a query-tile pair of a chunk
+// and a range of its key tiles: a CTA whose key range is long next to the launch's average is cut into
+// pieces of `per` key tiles that run as separate CTAs and leave partial (O, max, sum) rows in the
+// workspace; prefill_combine_kernel merges them.
+//   item[y][0] = chunk | pair << 16   (pair 0 = the chunk's last query-tile pair, which sees the most keys)
+//   item[y][1] = piece | pieces << 8 | per << 16
+//   slot[y]    = workspace slot of the piece's partials (pieces > 1)
+//   pairs[c]   = query-tile pairs the plan launched for chunk c (a longer chunk on the device is flagged)
+template <bool PLANNED>
+struct PrefillPlan {
+  int32_t item[PLANNED ? kPlanItems : 1][2];
+  int32_t slot[PLANNED ? kPlanItems : 1];
+  int32_t pairs[PLANNED ? kPlanChunks : 1];
+};
+// The split items of a plan, for the combine: item[i][0] = chunk | pair << 16; item[i][1] = pieces | first
+// slot << 8.
+struct PrefillCombineList {
+  int32_t item[kPlanItems][2];
+};
 
 // KT: cache element type (0 bf16, 1 FP8 E4M3, 2 INT8; one-byte types at head_dim 128 only)
 template <int D, int KT = 0>
@@ -362,10 +391,10 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <int D, int KT>
+template <int D, int KT, bool PLANNED>
 __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                         const PrefillParams P) {
+                         const PrefillParams P, const __grid_constant__ PrefillPlan<PLANNED> W) {
   using C = PrefillCfg<D, KT>;
   static_assert(kNumBars <= C::NBAR && C::NSLOT <= 8 && C::NU8 <= 2, "barrier slots");
   extern __shared__ uint8_t smem_raw[];
@@ -378,12 +407,24 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
   griddep_wait();
   griddep_launch();
 
-  // Longest work first (CTAs are dispatched in index order): chunk rank blockIdx.z serves the chunk
-  // with the rank-th longest context (ties by index), and within a chunk blockIdx.y counts query
-  // tiles down from the last one, which sees the most keys.  Up to kOrderedChunks chunks; beyond
-  // that, blockIdx.z is the chunk.
-  int c = blockIdx.z;
-  if (P.num_chunks <= kOrderedChunks) {
+  // Longest work first (CTAs are dispatched in index order).  Planned launch: grid row y is work item y.
+  // Otherwise chunk rank blockIdx.z serves the chunk with the rank-th longest context (ties by index),
+  // and within a chunk blockIdx.y counts query-tile pairs down from the last one, which sees the most
+  // keys (up to kOrderedChunks chunks; beyond that, blockIdx.z is the chunk).
+  int c = blockIdx.z, pair = blockIdx.y, piece = 0, pieces = 1, per = 0, slot = 0;
+  if constexpr (PLANNED) {
+    const int32_t w0 = W.item[blockIdx.y][0], w1 = W.item[blockIdx.y][1];
+    c = w0 & 0xffff;
+    pair = (w0 >> 16) & 0xffff;
+    piece = w1 & 0xff;
+    pieces = (w1 >> 8) & 0xff;
+    per = (w1 >> 16) & 0xffff;
+    slot = W.slot[blockIdx.y];
+    if (c >= P.num_chunks || pieces < 1 || (pieces > 1 && per < 1)) {
+      if (tid == 0 && blockIdx.x == 0) flag_error(kErrLength);
+      return;
+    }
+  } else if (P.num_chunks <= kOrderedChunks) {
     int *s_chunk = reinterpret_cast<int *>(smem + C::OFF_BAR + C::NBAR * 8 + 8);
     if (tid < P.num_chunks) {
       const int mine = P.context_lens[tid];
@@ -406,17 +447,43 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
     return;
   }
   const int nx = (Cn + 2 * ppt - 1) / (2 * ppt);      // CTAs (pairs of query tiles) of this chunk
-  if (nx > static_cast<int>(gridDim.y)) {             // chunk longer than the max_q_len launched for
+  if (!PLANNED && nx > static_cast<int>(gridDim.y)) { // chunk longer than the max_q_len launched for
     if (tid == 0 && blockIdx.x == 0 && blockIdx.y == 0) flag_error(kErrLength);
     return;
   }
-  if (static_cast<int>(blockIdx.y) >= nx) return;
-  const int p0 = (nx - 1 - static_cast<int>(blockIdx.y)) * 2 * ppt;   // first position of tile A
+  if constexpr (PLANNED) {
+    // the device chunk needs query-tile pairs the plan did not launch (host lengths shorter than the
+    // device's): reported like a chunk longer than max_q_len, and those rows are not written
+    if (nx > W.pairs[c] && pair == 0 && piece == 0) {
+      if (tid == 0 && blockIdx.x == 0) flag_error(kErrLength);
+    }
+  }
+  if (pair >= nx) return;                             // (planned: the plan's chunk was longer)
+  const int p0 = (nx - 1 - pair) * 2 * ppt;           // first position of tile A
   const int p_end = min(Cn, p0 + 2 * ppt);
   const int kv_len = H + p_end;                       // keys visible to some row of this CTA
-  const int ntiles = (kv_len + C::BN - 1) / C::BN;
-  // 16-key steps of the last tile that hold a visible key (the PV product stops there)
-  const int last_k16 = (kv_len - (ntiles - 1) * C::BN + 15) / 16;
+  const int all_tiles = (kv_len + C::BN - 1) / C::BN;
+  // this CTA's key tiles [tl0, tl0 + ntiles): all of them, or one piece (the last piece always runs to
+  // the end, so the keys are covered whatever lengths the plan was made for)
+  int tl0 = 0, tl1 = all_tiles;
+  if (pieces > 1) {
+    tl0 = min(piece * per, all_tiles);
+    tl1 = piece == pieces - 1 ? all_tiles : min(all_tiles, tl0 + per);
+  }
+  const int ntiles = tl1 - tl0;
+  // rows of this CTA in the workspace (split items): [slot][blockIdx.x][256 rows]
+  const int64_t ws_row0 = ((int64_t)slot * gridDim.x + blockIdx.x) * 256;
+  if (ntiles <= 0) {
+    // an empty piece (the chunk is shorter than the plan's): its rows contribute nothing to the merge
+    if (pieces > 1 && tid < 256) {
+      P.ws_ml[(ws_row0 + tid) * 2] = -INFINITY;
+      P.ws_ml[(ws_row0 + tid) * 2 + 1] = 0.f;
+    }
+    return;
+  }
+  // 16-key steps of the last tile that hold a visible key (the PV product stops there; a piece that
+  // ends before the CTA's last tile has only full tiles)
+  const int last_k16 = tl1 == all_tiles ? (kv_len - (all_tiles - 1) * C::BN + 15) / 16 : C::BN / 16;
 
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
@@ -513,7 +580,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
     constexpr float kRescale = 8.f;
     float m_ref = -INFINITY, l_run = 0.f;
     for (int j = 0; j < ntiles; ++j) {
-      const int kbase = j * C::BN;
+      const int kbase = (tl0 + j) * C::BN;
       const bool diag = kbase + C::BN - 1 > pos;       // some key of this tile is past the row
       // the passes below store P with warp-collective tcgen05.st, so the choice of pass is made per warp:
       // the masking pass when any row of the warp has a key past its position (it masks nothing for the
@@ -649,8 +716,26 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
       mbar_arrive(&bars[kPFull + X]);
       l_run = l_run * alpha + sum;
     }
-    // ---- epilogue: out = O / l once the last PV is done
-    if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0))) {
+    // ---- epilogue: out = O / l once the last PV is done; a piece of a split key range leaves its
+    // unnormalised O row and (reference, sum) for the merge instead
+    if (pieces > 1) {
+      if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0))) {
+        tc_fence_after();
+        const int64_t wrow = ws_row0 + X * 128 + r;
+        float4 *dst = reinterpret_cast<float4 *>(P.ws_o + wrow * D);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float ov[32];
+          tmem_ld32(o_addr + cc * 32, ov);
+          if (row_ok) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              dst[cc * 8 + q4] = make_float4(ov[4 * q4], ov[4 * q4 + 1], ov[4 * q4 + 2], ov[4 * q4 + 3]);
+          }
+        }
+        if (row_ok) *reinterpret_cast<float2 *>(P.ws_ml + wrow * 2) = make_float2(m_ref, l_run);
+      }
+    } else if (!timeout && __all_sync(0xffffffffu, mbar_wait(&bars[kDone], 0))) {
       tc_fence_after();
       const float inv = l_run > 0.f ? (KT != 0 ? P.v_scale[g] : 1.f) / l_run : 0.f;
       uint4 *dst = reinterpret_cast<uint4 *>(P.out + ((int64_t)(q0 + (row_ok ? pos_i : 0)) * P.num_q_heads + h) * D);
@@ -752,8 +837,8 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
       auto ring_of = [&](int i) {
         return KT != 0 ? smem + C::OFF_U8 + (i % NRING) * C::U8_BYTES : slot_of(i);
       };
-      auto row_of = [&](int j) {                      // cache row of this lane's unit of key tile j
-        const int u = j * UPT + bb;
+      auto row_of = [&](int j) {                      // cache row of this lane's unit of key tile tl0 + j
+        const int u = (tl0 + j) * UPT + bb;
         int e = 0;
         if (w_lane < 2 && j < ntiles && u * kBlock < kv_len) {
           e = __ldg(trow + (u >> ush));
@@ -768,7 +853,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
       int issued = 0;                                 // ring items whose copies are in flight
       for (int j = 0; j < ntiles && !timeout; ++j) {
         const int y2 = row_of(j + 2);
-        const int nu = min(UPT, (kv_len - j * C::BN + kBlock - 1) / kBlock);
+        const int nu = min(UPT, (kv_len - (tl0 + j) * C::BN + kBlock - 1) / kBlock);
         for (int w = 0; w < 2; ++w) {                 // K, then V of tile j
           const int it = 2 * j + w, slot = it % NRING;
           int ok = 1;
@@ -816,7 +901,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
         }
         const uint8_t *src = smem + C::OFF_U8 + su * C::U8_BYTES;
         uint8_t *dst = slot_of(it) + w * C::KV_PLANE;
-        const int nvalid = kv_len - (it >> 1) * C::BN;  // rows of this tile that hold keys (may exceed BN)
+        const int nvalid = kv_len - (tl0 + (it >> 1)) * C::BN;  // rows of this tile holding keys (may exceed BN)
         // eight 16-byte reads in flight per lane, then their conversions and writes; the row test is
         // compiled only into the last tile's pass (a test per read keeps the reads from batching)
         auto convert = [&](auto partial_c) {
@@ -863,6 +948,194 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// ----------------------------------------------------------------------------- merge of split key ranges
+// For each split work item of a plan and head group: every row (position, head) of the item's query-tile
+// pair combines its pieces' partials,  out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s  (M = max_s m_s;
+// a piece in which the row saw no key has m = -inf, l = 0 and is left out), times the V scale of a
+// one-byte cache.  One warp per row; lane l holds dims [l D/32, (l + 1) D/32).
+template <int D, bool ONE_BYTE>
+__global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillParams P,
+                                                              const __grid_constant__ PrefillCombineList L) {
+  griddep_wait();  // the partials come from the prefill kernel just before this one
+  griddep_launch();
+  const int32_t w0 = L.item[blockIdx.y][0], w1 = L.item[blockIdx.y][1];
+  const int c = w0 & 0xffff, pair = (w0 >> 16) & 0xffff, pieces = w1 & 0xff, slot0 = (w1 >> 8) & 0xffffff;
+  if (c >= P.num_chunks) return;
+  const int q0 = P.cu_q_lens[c];
+  const int Cn = P.cu_q_lens[c + 1] - q0;
+  const int ppt = 128 / P.hpr;
+  const int nx = (Cn + 2 * ppt - 1) / (2 * ppt);
+  if (Cn <= 0 || pair >= nx) return;
+  const int p0 = (nx - 1 - pair) * 2 * ppt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hg0 = blockIdx.x * P.hpr;
+  const float vs = ONE_BYTE ? P.v_scale[hg0 / P.group] : 1.f;
+  constexpr int DPL = D / 32;
+  for (int rr = warp; rr < 256; rr += 8) {
+    const int r = rr & 127;
+    const int pos_i = p0 + (rr >> 7) * ppt + r / P.hpr;
+    if (pos_i >= Cn) continue;                        // a padding row (the same for the whole warp)
+    auto row_of = [&](int s) { return ((int64_t)(slot0 + s) * gridDim.x + blockIdx.x) * 256 + rr; };
+    float M = -INFINITY;
+    for (int s = lane; s < pieces; s += 32) M = fmaxf(M, P.ws_ml[row_of(s) * 2]);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float acc[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+    float den = 0.f;
+    for (int s = 0; s < pieces; ++s) {
+      const int64_t row = row_of(s);
+      const float m = P.ws_ml[row * 2];
+      if (m == -INFINITY) continue;                   // no key of this piece reached the row
+      const float w = exp2f(m - M);
+      den = fmaf(w, P.ws_ml[row * 2 + 1], den);
+      const float *op = P.ws_o + row * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(op);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+        acc[2] = fmaf(w, v.z, acc[2]);
+        acc[3] = fmaf(w, v.w, acc[3]);
+      } else {
+        const float2 v = *reinterpret_cast<const float2 *>(op);
+        acc[0] = fmaf(w, v.x, acc[0]);
+        acc[1] = fmaf(w, v.y, acc[1]);
+      }
+    }
+    const float inv = den > 0.f ? vs / den : 0.f;
+    __nv_bfloat16 *orow = P.out + ((int64_t)(q0 + pos_i) * P.num_q_heads + hg0 + r % P.hpr) * D + lane * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; e += 2)
+      *reinterpret_cast<__nv_bfloat162 *>(orow + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+  }
+}
+
+// ----------------------------------------------------------------------------- host plan
+// The launch order and key-range split of a prefill call, from the host copies of its lengths.  Work is
+// counted in key tiles per CTA (a query-tile pair of one head group); a CTA runs on one SM.  Candidate
+// piece lengths (fractions of the work per SM, and no split) are scored by the makespan of a
+// longest-first greedy schedule on the SMs, each piece of a split CTA costing one more tile of set-up;
+// the shortest schedule wins, ties to fewer pieces.
+struct PrefillPlanHost {
+  PrefillPlan<true> plan;
+  PrefillCombineList combine;
+  int n_items = 0;
+  int n_combine = 0;
+  int n_slots = 0;   // workspace slots (pieces of split items)
+};
+
+// Greedy schedule cost: pieces (lengths in tiles, `copies` CTAs each) longest first onto `sms` SMs.
+inline int64_t lpt_makespan(std::vector<int> len, int copies, int sms) {
+  std::sort(len.begin(), len.end(), std::greater<int>());
+  std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> load;
+  for (int i = 0; i < sms; ++i) load.push(0);
+  int64_t worst = 0;
+  for (const int t : len)
+    for (int k = 0; k < copies; ++k) {
+      const int64_t v = load.top() + t;
+      load.pop();
+      load.push(v);
+      worst = std::max(worst, v);
+    }
+  return worst;
+}
+
+// Returns false when the lengths are out of range (the kernel would flag them) or the work does not fit
+// the plan's lists; the caller then launches unplanned.
+inline bool plan_prefill(const int32_t *hcu, const int32_t *hctx, int num_chunks, int hpr, int groups_x, int sm_count,
+                         int max_q_len, int ctx_limit, PrefillPlanHost &out) {
+  if (num_chunks <= 0 || num_chunks > kPlanChunks || groups_x <= 0 || sm_count <= 0) return false;
+  const int ppt = 128 / hpr;
+  struct Pair {
+    int c, k, T;
+  };
+  std::vector<Pair> pairs;
+  int64_t W = 0;
+  for (int c = 0; c < num_chunks; ++c) {
+    const int Cn = hcu[c + 1] - hcu[c], ctx = hctx[c], H = ctx - Cn;
+    if (Cn < 0 || H < 0 || ctx > ctx_limit || Cn > max_q_len) return false;
+    const int nx = (Cn + 2 * ppt - 1) / (2 * ppt);
+    if (nx > 65535) return false;
+    out.plan.pairs[c] = nx;
+    for (int k = 0; k < nx; ++k) {
+      const int p0 = (nx - 1 - k) * 2 * ppt, p_end = std::min(Cn, p0 + 2 * ppt);
+      const int T = (H + p_end + 127) / 128;
+      pairs.push_back({c, k, T});
+      W += T;
+    }
+  }
+  if (pairs.empty() || pairs.size() > static_cast<size_t>(kPlanItems)) return false;
+  auto n_pieces = [](int T, int per) { return (per <= 0 || T <= per) ? 1 : std::min(255, (T + per - 1) / per); };
+  auto pieces_for = [&](int per, std::vector<int> *len) {
+    int total = 0;
+    for (const Pair &p : pairs) {
+      const int n = n_pieces(p.T, per);
+      const int q = (p.T + n - 1) / n;
+      for (int s = 0; s < n; ++s)
+        if (len) len->push_back(std::min(q, p.T - s * q) + (n > 1 ? 1 : 0));
+      total += n;
+    }
+    return total;
+  };
+  // candidate piece lengths; splitting is only weighed while the schedule stays cheap to score
+  int best_per = 0;
+  {
+    std::vector<int> len;
+    pieces_for(0, &len);
+    int64_t best = lpt_makespan(len, groups_x, sm_count);
+    const double per_sm = static_cast<double>(W) * groups_x / sm_count;
+    if (static_cast<int64_t>(pairs.size()) * groups_x <= 16384) {
+      for (int f10 = 3; f10 <= 10; ++f10) {
+        const int per = std::max(4, static_cast<int>(per_sm * f10 / 10.0 + 0.999));
+        if (pieces_for(per, nullptr) > kPlanItems) continue;
+        len.clear();
+        pieces_for(per, &len);
+        const int64_t ms = lpt_makespan(len, groups_x, sm_count);
+        if (ms < best) {
+          best = ms;
+          best_per = per;
+        }
+      }
+    }
+  }
+  // items, longest piece first (ties in chunk, pair, piece order); slots for the split pairs
+  struct Item {
+    int c, k, s, n, q, len, slot;
+  };
+  std::vector<Item> items;
+  int slots = 0, n_comb = 0;
+  for (const Pair &p : pairs) {
+    const int n = n_pieces(p.T, best_per);
+    const int q = (p.T + n - 1) / n;
+    if (q > 65535) return false;
+    if (n > 1) {
+      out.combine.item[n_comb][0] = p.c | (p.k << 16);
+      out.combine.item[n_comb][1] = n | (slots << 8);
+      ++n_comb;
+    }
+    for (int s = 0; s < n; ++s) items.push_back({p.c, p.k, s, n, q, std::min(q, p.T - s * q), n > 1 ? slots + s : 0});
+    if (n > 1) slots += n;
+  }
+  if (slots >= (1 << 23)) return false;
+  std::stable_sort(items.begin(), items.end(), [](const Item &a, const Item &b) { return a.len > b.len; });
+  for (size_t i = 0; i < items.size(); ++i) {
+    const Item &it = items[i];
+    out.plan.item[i][0] = it.c | (it.k << 16);
+    out.plan.item[i][1] = it.s | (it.n << 8) | (it.q << 16);
+    out.plan.slot[i] = it.slot;
+  }
+  out.n_items = static_cast<int>(items.size());
+  out.n_combine = n_comb;
+  out.n_slots = slots;
+  return true;
+}
+
+// Workspace bytes of a plan: the partial rows of every piece of its split items.
+inline size_t prefill_plan_workspace(const PrefillPlanHost &pl, int groups_x, int head_dim) {
+  return static_cast<size_t>(pl.n_slots) * groups_x * 256 * (head_dim + 2) * sizeof(float);
 }
 
 // ----------------------------------------------------------------------------- host launch
@@ -912,37 +1185,57 @@ inline bool make_cache_map_u8(CUtensorMap *map, const void *base, int64_t rows, 
 
 template <int D, int KT>
 int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_cache, int num_chunks, int max_q_len,
-                     cudaStream_t st) {
+                     const PrefillPlanHost *plan, cudaStream_t st) {
   using C = PrefillCfg<D, KT>;
   CUtensorMap km, vm;
   const int64_t rows = P.num_blocks * P.num_kv_heads * P.block_size;
   if (KT != 0 ? (!make_cache_map_u8(&km, k_cache, rows, D) || !make_cache_map_u8(&vm, v_cache, rows, D))
               : (!make_cache_map(&km, k_cache, rows, D) || !make_cache_map(&vm, v_cache, rows, D)))
     return -3;
-  if (cudaFuncSetAttribute(paged_prefill_kernel<D, KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
-      cudaSuccess)
-    return -3;
+  auto prepare = [&](auto kernel) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return false;
 #if PA_PREFILL_SPLIT_REGS
-  // setmaxnreg.inc waits until the block's launch allocation can cover the new split: never launch a
-  // build whose register count per thread would not
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, paged_prefill_kernel<D, KT>) != cudaSuccess ||
-      fa.numRegs * C::THREADS < 2 * 128 * C::REGS_SOFTMAX + 128 * C::REGS_PRODUCER)
-    return -3;
+    // setmaxnreg.inc waits until the block's launch allocation can cover the new split: never launch a
+    // build whose register count per thread would not
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess ||
+        fa.numRegs * C::THREADS < 2 * 128 * C::REGS_SOFTMAX + 128 * C::REGS_PRODUCER)
+      return false;
 #endif
+    return true;
+  };
+  const unsigned gx = static_cast<unsigned>(P.num_q_heads / P.hpr);
+  if (plan != nullptr) {
+    if (!prepare(paged_prefill_kernel<D, KT, true>)) return -3;
+    if (launch_pdl(paged_prefill_kernel<D, KT, true>, dim3(gx, static_cast<unsigned>(plan->n_items)),
+                   dim3(C::THREADS), C::SMEM, st, km, vm, P, plan->plan) != cudaSuccess)
+      return -3;
+    if (plan->n_combine > 0 &&
+        launch_pdl(prefill_combine_kernel<D, (KT != 0)>, dim3(gx, static_cast<unsigned>(plan->n_combine)), dim3(256),
+                   0, st, P, plan->combine) != cudaSuccess)
+      return -3;
+    return 0;
+  }
+  if (!prepare(paged_prefill_kernel<D, KT, false>)) return -3;
   const int ppt = C::BM / P.hpr;
   const int tiles = (max_q_len + 2 * ppt - 1) / (2 * ppt);
   if (tiles > 65535) return -1;
-  dim3 grid(P.num_q_heads / P.hpr, tiles, num_chunks);
-  return launch_pdl(paged_prefill_kernel<D, KT>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P) == cudaSuccess ? 0 : -3;
+  dim3 grid(gx, tiles, num_chunks);
+  return launch_pdl(paged_prefill_kernel<D, KT, false>, grid, dim3(C::THREADS), C::SMEM, st, km, vm, P,
+                    PrefillPlan<false>{}) == cudaSuccess
+             ? 0
+             : -3;
 }
 
-// kv_dtype: 0 bf16, 1 FP8 E4M3, 2 INT8 (one-byte types: head_dim 128, k_scale / v_scale per KV head)
+// kv_dtype: 0 bf16, 1 FP8 E4M3, 2 INT8 (one-byte types: head_dim 128, k_scale / v_scale per KV head).
+// plan (optional): the planned order and split of the launch, its partials in ws (plan's workspace bytes).
 inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, int num_chunks, const void *k_cache,
                           const void *v_cache, const int32_t *block_tables, int max_blocks_per_seq,
                           const int32_t *context_lens, int num_q_heads, int num_kv_heads, int head_dim,
                           int64_t num_blocks, int block_size, float scale, int kv_dtype, const float *k_scale,
-                          const float *v_scale, int max_q_len, int max_context_len, cudaStream_t st) {
+                          const float *v_scale, int max_q_len, int max_context_len, const PrefillPlanHost *plan,
+                          void *ws, cudaStream_t st) {
   if (num_chunks > 65535 || num_q_heads > 65535) return -1;
   if (num_blocks * num_kv_heads * block_size >= (int64_t(1) << 31)) return -2;
   PrefillParams P;
@@ -963,11 +1256,16 @@ inline int launch_prefill(void *out, const void *q, const int32_t *cu_q_lens, in
   P.qscale = scale * 1.4426950408889634f;
   P.k_scale = k_scale;
   P.v_scale = v_scale;
+  P.ws_o = static_cast<float *>(ws);
+  P.ws_ml = plan != nullptr && ws != nullptr
+                ? P.ws_o + static_cast<int64_t>(plan->n_slots) * (num_q_heads / P.hpr) * 256 * head_dim
+                : nullptr;
   if (kv_dtype != 0 && (head_dim != 128 || k_scale == nullptr || v_scale == nullptr)) return -1;
-  if (kv_dtype == 1) return launch_prefill_d<128, 1>(P, k_cache, v_cache, num_chunks, max_q_len, st);
-  if (kv_dtype == 2) return launch_prefill_d<128, 2>(P, k_cache, v_cache, num_chunks, max_q_len, st);
-  return head_dim == 128 ? launch_prefill_d<128, 0>(P, k_cache, v_cache, num_chunks, max_q_len, st)
-                         : launch_prefill_d<64, 0>(P, k_cache, v_cache, num_chunks, max_q_len, st);
+  if (plan != nullptr && plan->n_slots > 0 && ws == nullptr) return -1;
+  if (kv_dtype == 1) return launch_prefill_d<128, 1>(P, k_cache, v_cache, num_chunks, max_q_len, plan, st);
+  if (kv_dtype == 2) return launch_prefill_d<128, 2>(P, k_cache, v_cache, num_chunks, max_q_len, plan, st);
+  return head_dim == 128 ? launch_prefill_d<128, 0>(P, k_cache, v_cache, num_chunks, max_q_len, plan, st)
+                         : launch_prefill_d<64, 0>(P, k_cache, v_cache, num_chunks, max_q_len, plan, st);
 }
 
 }  // namespace pa

@@ -22,7 +22,7 @@ class DeviceStep:
     """Device-resident state (cache, tables, inputs) of one :class:`PagedBatch` step."""
 
     def __init__(self, batch: PagedBatch, device="cuda", split_tokens: Optional[int] = None,
-                 zero_cache: bool = True, overlap: bool = True):
+                 zero_cache: bool = True, overlap: bool = True, plan_prefill: bool = True):
         self.batch = batch
         self.device = torch.device(device)
         self.overlap = overlap
@@ -46,7 +46,9 @@ class DeviceStep:
         self.dec_lens = torch.from_numpy(self.dec_lens_host).to(dev)
         self.dec_max_len = int(ctx[:nd].max()) if nd else 0
         self.pre_tables = torch.from_numpy(batch.prefill_tables).to(dev)
-        self.pre_lens = torch.from_numpy(np.ascontiguousarray(ctx[nd:])).to(dev)
+        self.pre_lens_host = np.ascontiguousarray(ctx[nd:], dtype=np.int32)   # plan the prefill launch
+        self.pre_cu_host = np.ascontiguousarray(batch.cu_q_lens, dtype=np.int32)
+        self.pre_lens = torch.from_numpy(self.pre_lens_host.copy()).to(dev)
         self.pre_max_len = int(ctx[nd:].max()) if ctx.shape[0] > nd else 0
         self.cu_q = torch.from_numpy(batch.cu_q_lens).to(dev)
         self.max_q = int(batch.new_lens[nd:].max()) if ctx.shape[0] > nd else 0
@@ -68,6 +70,12 @@ class DeviceStep:
         self.split_tokens = split_tokens
         ws = B.pa_paged_attention_workspace_size(nd, hq, d, self.dec_max_len, split_tokens) if nd else 0
         self.workspace = torch.empty(max(ws, 16) // 4 + 4, dtype=torch.float32, device=dev) if ws else None
+        self.plan_prefill = plan_prefill and self.max_q > 0
+        pws = 0
+        if self.plan_prefill:
+            pws = B.pa_paged_prefill_workspace_size(self.pre_cu_host, self.pre_lens_host, hq, hkv, d,
+                                                    batch.prefill_tables.shape[1], bs, self.max_q, self.pre_max_len)
+        self.pre_workspace = torch.empty(pws // 4 + 4, dtype=torch.float32, device=dev) if pws else None
 
     # ------------------------------------------------------------------ set-up (not part of a step)
     def fill_history(self, chunk_tokens: int = 1 << 16):
@@ -102,9 +110,13 @@ class DeviceStep:
     def prefill(self, stream=None):
         if self.max_q == 0:
             return
+        plan = self.plan_prefill
         B.pa_paged_prefill(self.out_pre, self.q_pre, self.cu_q, self.k_cache, self.v_cache, self.pre_tables,
                            self.pre_lens, self.batch.scale, self.max_q, self.pre_max_len, self.kv_dtype,
-                           k_scale=self.k_scale, v_scale=self.v_scale, stream=stream)
+                           k_scale=self.k_scale, v_scale=self.v_scale, stream=stream,
+                           host_cu_q_lens=self.pre_cu_host if plan else None,
+                           host_context_lens=self.pre_lens_host if plan else None,
+                           workspace=self.pre_workspace if plan else None)
 
     def step(self, stream=None):
         """copy-on-write forks -> append -> decode attention and prefill attention.

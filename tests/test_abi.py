@@ -5,6 +5,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 from pagedattention_block_table_b200 import binding as B
@@ -118,16 +119,56 @@ def test_empty_batch_is_a_no_op(L):
 def test_prefill_argument_checks(L):
     P = ctypes.c_void_p
     f = L.pa_paged_prefill
+    tail = (None, None, None, 0, None)   # host lengths, workspace, workspace bytes, stream
     # one-byte caches: head_dim 128 only, and both scales required
     assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 64, 10, 16, 0.1, 1, P(16), P(16), 16, 64,
-             None) == B.PA_EUNSUPPORTED
+             *tail) == B.PA_EUNSUPPORTED
     assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 1, None, P(16), 16, 64,
-             None) == B.PA_EINVAL
+             *tail) == B.PA_EINVAL
     assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 5, P(16), P(16), 16, 64,
-             None) == B.PA_EUNSUPPORTED
+             *tail) == B.PA_EUNSUPPORTED
     # heads not a multiple of the KV heads
     assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 7, 2, 128, 10, 16, 0.1, 0, None, None, 16, 64,
-             None) == B.PA_EINVAL
+             *tail) == B.PA_EINVAL
+    # host lengths come in pairs
+    cu = np.array([0, 16], np.int32)
+    assert f(P(16), P(16), P(16), 1, P(16), P(16), P(16), 4, P(16), 8, 2, 128, 10, 16, 0.1, 0, None, None, 16, 64,
+             cu.ctypes.data, None, None, 0, None) == B.PA_EINVAL
+
+
+def _plan_case(chunks):
+    """cu_q_lens / context_lens (host int32) of prefill chunks given as (new tokens, history) pairs."""
+    c = np.array([n for n, _ in chunks], np.int32)
+    cu = np.concatenate([[0], np.cumsum(c)]).astype(np.int32)
+    ctx = np.array([n + h for n, h in chunks], np.int32)
+    return cu, ctx
+
+
+def test_prefill_plan_workspace():
+    """The prefill plan splits the key ranges of CTAs that are long next to the launch's work per SM and
+    asks for workspace for their partials; a launch of even CTAs needs none; a call that would split
+    without enough workspace is refused before anything is launched."""
+    ws = B.pa_paged_prefill_workspace_size
+    # two long histories in a small launch: the long CTAs are split
+    cu, ctx = _plan_case([(512, 8000), (256, 6000)])
+    need = ws(cu, ctx, 32, 8, 128, 1024, 16, 512, 8512)
+    assert need > 0 and need % (256 * 130 * 4) == 0
+    # no host lengths: nothing planned
+    assert L_ws_none() == 0
+    # many equal CTAs: balanced, nothing to split
+    cu2, ctx2 = _plan_case([(2048, 0)] * 40)
+    assert ws(cu2, ctx2, 32, 8, 128, 128, 16, 2048, 2048) == 0
+    # lengths the kernel would reject (context past max_context_len): no plan
+    assert ws(cu, ctx, 32, 8, 128, 1024, 16, 512, 4096) == 0
+    P = ctypes.c_void_p
+    lib = B.lib()
+    st = lib.pa_paged_prefill(P(16), P(16), P(16), 2, P(16), P(16), P(16), 1024, P(16), 32, 8, 128, 10, 16, 0.1, 0,
+                              None, None, 512, 8512, cu.ctypes.data, ctx.ctypes.data, None, 0, None)
+    assert st == B.PA_EWORKSPACE
+
+
+def L_ws_none():
+    return int(B.lib().pa_paged_prefill_workspace_size(2, None, None, 32, 8, 128, 1024, 16, 512, 8512))
 
 
 def test_source_digest_ignores_comments_only():

@@ -130,3 +130,105 @@ def test_one_byte_prefill_long_chunk_over_long_history(O, cuda_lib):
     st = _run(batch)
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
     assert_close(to_f64(st.out_pre), ref, what="fp8 long chunk")
+
+
+# ---------------------------------------------------------------------------------------------- planned launches
+# With host copies of the lengths the call plans its launch: longest work first, and a CTA whose key range
+# is long next to the launch's work per SM runs as pieces whose partials a merge kernel combines.
+
+PLAN_CASES = {
+    # two long histories in a small launch: the long CTAs are cut into pieces
+    "long_histories": _chunks(prefill_chunks=2, chunk_len=(300, 600), chunk_hist=(3000, 5000)),
+    # one chunk starting a request next to a long one: uneven CTAs
+    "uneven": _chunks(prefill_chunks=3, chunk_len=(64, 900), chunk_hist=(1, 6000)),
+    "gqa8_bs32": _chunks(num_q_heads=16, num_kv_heads=2, block_size=32, prefill_chunks=2, chunk_len=(100, 400),
+                         chunk_hist=(2000, 4000)),
+    "mha_d64": _chunks(num_q_heads=4, num_kv_heads=4, head_dim=64, prefill_chunks=2, chunk_len=(200, 300),
+                       chunk_hist=(2500, 3500)),
+}
+
+
+def _unplanned(st, cuda_lib):
+    out = torch.empty_like(st.out_pre)
+    cuda_lib.pa_paged_prefill(out, st.q_pre, st.cu_q, st.k_cache, st.v_cache, st.pre_tables, st.pre_lens,
+                              st.batch.scale, st.max_q, st.pre_max_len, st.kv_dtype, k_scale=st.k_scale,
+                              v_scale=st.v_scale)
+    torch.cuda.synchronize()
+    return out
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+@pytest.mark.parametrize("case", sorted(PLAN_CASES))
+def test_planned_prefill_matches_oracle(O, cuda_lib, case, kv):
+    """The planned launch splits key ranges (it asks for workspace) and still equals the oracle, and the
+    unplanned launch of the same call, up to the rounding of the merge."""
+    ov = dict(PLAN_CASES[case])
+    if kv == "fp8":
+        if ov["head_dim"] != 128:
+            pytest.skip("one-byte caches need head_dim 128")
+        ov["kv_dtype"] = "fp8"
+    batch = make_batch("mixed_step", seed=57, overrides=ov)
+    ref = oracle_step(batch, O)["prefill"]
+    st = _run(batch)
+    assert st.pre_workspace is not None, "the plan was expected to split this launch"
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(st.out_pre), ref, what=f"planned {kv} prefill {case}")
+    plain = _unplanned(st, cuda_lib)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    assert_close(to_f64(plain), ref, what=f"unplanned {kv} prefill {case}")
+    d = (st.out_pre.float() - plain.float()).abs()
+    assert float(d.max()) <= 2e-2 and float(d.mean()) <= 1e-3
+
+
+def _planned_call(st, cuda_lib, host_cu, host_ctx, max_q, max_ctx):
+    ws_bytes = cuda_lib.pa_paged_prefill_workspace_size(host_cu, host_ctx, st.batch.num_q_heads,
+                                                        st.batch.num_kv_heads, st.batch.head_dim,
+                                                        st.pre_tables.shape[1], st.batch.block_size, max_q, max_ctx)
+    ws = torch.empty(ws_bytes // 4 + 4, dtype=torch.float32, device="cuda") if ws_bytes else None
+    out = torch.zeros_like(st.out_pre)
+    cuda_lib.pa_paged_prefill(out, st.q_pre, st.cu_q, st.k_cache, st.v_cache, st.pre_tables, st.pre_lens,
+                              st.batch.scale, max_q, max_ctx, st.kv_dtype, k_scale=st.k_scale, v_scale=st.v_scale,
+                              host_cu_q_lens=host_cu, host_context_lens=host_ctx, workspace=ws)
+    torch.cuda.synchronize()
+    return out, ws_bytes
+
+
+def test_planned_prefill_with_longer_host_histories(O, cuda_lib):
+    """Host lengths longer than the device's (within the table rows): the plan has pieces past the device's
+    keys, which leave empty partials, and the output still equals the oracle for the device lengths."""
+    batch = make_batch("mixed_step", seed=58, overrides=_chunks(prefill_chunks=2, chunk_len=(300, 300),
+                                                                chunk_hist=(1000, 4000)))
+    st = _run(batch)
+    ref = oracle_step(batch, O)["prefill"]
+    cap = st.pre_tables.shape[1] * batch.block_size
+    host_ctx = np.minimum(st.pre_lens_host + 2500, cap).astype(np.int32)
+    out, ws_bytes = _planned_call(st, cuda_lib, st.pre_cu_host, host_ctx, st.max_q, int(host_ctx.max()))
+    assert ws_bytes > 0
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    # Rows near the start of the chunk that starts a request see a handful of keys, so the bf16 roundings
+    # are not averaged away: P rounded to bf16 (relative 2^-9 per weight, weights summing to 1) moves out
+    # by at most 2^-9 max|v|, and the bf16 output by half an ulp, 2^-9 |out|.
+    vmax = float(batch.tok_v.float().abs().max())
+    bound = 2.0 ** -9 * (vmax + float(np.abs(ref).max())) + 1e-3
+    assert_close(to_f64(out), ref, max_tol=bound, what="planned with longer host histories")
+    # the same arithmetic as the launch planned for the true lengths, up to the merge's rounding
+    d = (out.float() - st.out_pre.float()).abs()
+    assert float(d.max()) <= 2e-2 and float(d.mean()) <= 1e-4
+
+
+def test_planned_prefill_with_shorter_host_chunk_is_flagged(cuda_lib):
+    """Host lengths that give a chunk fewer new tokens than the device's leave query tiles unplanned: the
+    call reports it in the device error word instead of silently skipping rows."""
+    batch = make_batch("mixed_step", seed=59, overrides=_chunks(prefill_chunks=2, chunk_len=(600, 600),
+                                                                chunk_hist=(500, 900)))
+    st = _run(batch)
+    host_cu = st.pre_cu_host.copy()
+    host_cu[1:] -= 300                                 # chunk 0 three hundred rows short on the host
+    host_ctx = st.pre_lens_host.copy()
+    host_ctx[0] -= 300
+    assert cuda_lib.pa_paged_prefill_workspace_size(host_cu, host_ctx, batch.num_q_heads, batch.num_kv_heads,
+                                                    batch.head_dim, st.pre_tables.shape[1], batch.block_size,
+                                                    st.max_q, st.pre_max_len) > 0   # the call is planned
+    _planned_call(st, cuda_lib, host_cu, host_ctx, st.max_q, st.pre_max_len)
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_EDEVICE_OOB
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
