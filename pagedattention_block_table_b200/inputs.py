@@ -54,6 +54,12 @@ WORKLOADS: Dict[str, dict] = {
                            hist=("lognormal", 800.0, 1.0, 16, 8192),
                            share_group=8, share_prefix=1024,
                            prefill_chunks=4, chunk_len=(512, 2048), chunk_hist=(1, 4095), kv_dtype="fp8"),
+    # chunked prefill of a long prompt: two 512-token chunks, one starting a prompt and one 32,256 tokens
+    # into it (Llama-3-8B heads); 64 query-tile pairs x head groups, far fewer CTAs than SMs unless the
+    # long key ranges are split
+    "chunked_prefill_long": dict(num_seqs=2, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                                 hist=("fixed", [100, 200]), prefill_chunks=2, chunk_len=(512, 512),
+                                 chunk_hist=(32256, 32256)),
 }
 WORKLOAD_SEED = {name: 1001 + i for i, name in enumerate(WORKLOADS)}
 

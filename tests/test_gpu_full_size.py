@@ -13,6 +13,7 @@ Tolerances: attention max-abs <= 1e-2 and mean-abs <= 1e-3 against the oracle on
 (for the FP8 cache: on the same dequantised codes), and <= 5e-2 max against the oracle on the original
 bf16 K/V for the FP8 cache.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -54,3 +55,23 @@ def test_full_size_mixed_step_every_element(O, cuda_lib, name):
     assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
     assert_close(to_f64(st.out_dec), oracle_decode_all(batch, O), what=f"{name}: 256 decode rows")
     assert_close(to_f64(st.out_pre), oracle_prefill_all(batch, O), what=f"{name}: every prefill row")
+
+
+def test_full_size_chunked_long_prompt_every_element(O, cuda_lib):
+    """Chunked prefill of a long prompt (a 512-token chunk 32,256 tokens into a prompt, beside one that
+    starts a prompt): far fewer query-tile CTAs than SMs, so the planned launch splits the long key
+    ranges and merges them; every prefill row equals the oracle."""
+    batch = make_batch("chunked_prefill_long", device="cuda")
+    st = _run(batch)
+    assert st.pre_workspace is not None, "the long key ranges were expected to be split"
+    assert cuda_lib.pa_get_device_error() == cuda_lib.PA_OK
+    got, ref = to_f64(st.out_pre), oracle_prefill_all(batch, O)
+    cu = batch.cu_q_lens
+    # the chunk 32,256 tokens in (its key ranges split and merged): the default tolerance
+    assert_close(got[cu[1]:cu[2]], ref[cu[1]:cu[2]], what="chunk over the long history")
+    # the chunk that starts a prompt: its first rows see a handful of keys, so the bf16 roundings are not
+    # averaged away: P rounded to bf16 (relative 2^-9 per weight, weights summing to 1) moves out by at
+    # most 2^-9 max|v|, and the bf16 output by half an ulp, 2^-9 |out|
+    vmax = float(batch.tok_v.float().abs().max())
+    bound = 2.0 ** -9 * (vmax + float(np.abs(ref).max())) + 1e-3
+    assert_close(got[:cu[1]], ref[:cu[1]], max_tol=bound, what="chunk starting a prompt")
