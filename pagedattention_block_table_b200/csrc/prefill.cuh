@@ -954,7 +954,11 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
 // For each split work item of a plan and head group: every row (position, head) of the item's query-tile
 // pair combines its pieces' partials,  out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s  (M = max_s m_s;
 // a piece in which the row saw no key has m = -inf, l = 0 and is left out), times the V scale of a
-// one-byte cache.  One warp per row; lane l holds dims [l D/32, (l + 1) D/32).
+// one-byte cache.  One warp per row, eight rows per CTA (grid z = the item's 32 groups of eight rows, so
+// the merge has as many CTAs in flight as the partials need); lane s holds piece s's (m, l), and each lane
+// sums its D/32 dims over the pieces with up to kMergeBatch independent vector loads in flight.
+constexpr int kMergeBatch = 8;
+
 template <int D, bool ONE_BYTE>
 __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillParams P,
                                                               const __grid_constant__ PrefillCombineList L) {
@@ -969,48 +973,66 @@ __global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillParam
   const int nx = (Cn + 2 * ppt - 1) / (2 * ppt);
   if (Cn <= 0 || pair >= nx) return;
   const int p0 = (nx - 1 - pair) * 2 * ppt;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31;
+  const int rr = blockIdx.z * 8 + (threadIdx.x >> 5);   // row of the item's 256 (tile A: 0-127, B: 128-255)
+  const int r = rr & 127;
+  const int pos_i = p0 + (rr >> 7) * ppt + r / P.hpr;
+  if (pos_i >= Cn) return;                               // a padding row (the same for the whole warp)
   const int hg0 = blockIdx.x * P.hpr;
-  const float vs = ONE_BYTE ? P.v_scale[hg0 / P.group] : 1.f;
+  auto row_of = [&](int s) { return ((int64_t)(slot0 + s) * gridDim.x + blockIdx.x) * 256 + rr; };
   constexpr int DPL = D / 32;
-  for (int rr = warp; rr < 256; rr += 8) {
-    const int r = rr & 127;
-    const int pos_i = p0 + (rr >> 7) * ppt + r / P.hpr;
-    if (pos_i >= Cn) continue;                        // a padding row (the same for the whole warp)
-    auto row_of = [&](int s) { return ((int64_t)(slot0 + s) * gridDim.x + blockIdx.x) * 256 + rr; };
-    float M = -INFINITY;
-    for (int s = lane; s < pieces; s += 32) M = fmaxf(M, P.ws_ml[row_of(s) * 2]);
+  float acc[DPL];
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float acc[DPL];
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  float M = -INFINITY;
+  for (int s = lane; s < pieces; s += 32) M = fmaxf(M, P.ws_ml[row_of(s) * 2]);
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    float den = 0.f;
-    for (int s = 0; s < pieces; ++s) {
-      const int64_t row = row_of(s);
-      const float m = P.ws_ml[row * 2];
-      if (m == -INFINITY) continue;                   // no key of this piece reached the row
-      const float w = exp2f(m - M);
-      den = fmaf(w, P.ws_ml[row * 2 + 1], den);
-      const float *op = P.ws_o + row * D + lane * DPL;
-      if constexpr (DPL == 4) {
-        const float4 v = *reinterpret_cast<const float4 *>(op);
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1] = fmaf(w, v.y, acc[1]);
-        acc[2] = fmaf(w, v.z, acc[2]);
-        acc[3] = fmaf(w, v.w, acc[3]);
-      } else {
-        const float2 v = *reinterpret_cast<const float2 *>(op);
-        acc[0] = fmaf(w, v.x, acc[0]);
-        acc[1] = fmaf(w, v.y, acc[1]);
+  for (int off = 16; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  float den = 0.f;
+  for (int s0 = 0; s0 < pieces; s0 += 32) {
+    // lane k: weight of piece s0 + k (0 for a piece the row saw no key of)
+    float w = 0.f;
+    if (s0 + lane < pieces) {
+      const float2 ml = *reinterpret_cast<const float2 *>(P.ws_ml + row_of(s0 + lane) * 2);
+      if (ml.x != -INFINITY) {
+        w = exp2f(ml.x - M);
+        den = fmaf(w, ml.y, den);
       }
     }
-    const float inv = den > 0.f ? vs / den : 0.f;
-    __nv_bfloat16 *orow = P.out + ((int64_t)(q0 + pos_i) * P.num_q_heads + hg0 + r % P.hpr) * D + lane * DPL;
+    const int cnt = min(32, pieces - s0);
+    for (int k0 = 0; k0 < cnt; k0 += kMergeBatch) {
+      float ov[kMergeBatch][DPL];
 #pragma unroll
-    for (int e = 0; e < DPL; e += 2)
-      *reinterpret_cast<__nv_bfloat162 *>(orow + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+      for (int k = 0; k < kMergeBatch; ++k) {
+        if (k0 + k < cnt) {
+          const float *op = P.ws_o + row_of(s0 + k0 + k) * D + lane * DPL;
+          if constexpr (DPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(op);
+            ov[k][0] = v.x; ov[k][1] = v.y; ov[k][2] = v.z; ov[k][3] = v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2 *>(op);
+            ov[k][0] = v.x; ov[k][1] = v.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kMergeBatch; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, w, (k0 + k) & 31);
+        if (k0 + k < cnt && wk > 0.f) {
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) acc[e] = fmaf(wk, ov[k][e], acc[e]);
+        }
+      }
+    }
   }
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+  const float vs = ONE_BYTE ? P.v_scale[hg0 / P.group] : 1.f;
+  const float inv = den > 0.f ? vs / den : 0.f;
+  __nv_bfloat16 *orow = P.out + ((int64_t)(q0 + pos_i) * P.num_q_heads + hg0 + r % P.hpr) * D + lane * DPL;
+#pragma unroll
+  for (int e = 0; e < DPL; e += 2)
+    *reinterpret_cast<__nv_bfloat162 *>(orow + e) = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
 }
 
 // ----------------------------------------------------------------------------- host plan
@@ -1212,8 +1234,8 @@ int launch_prefill_d(const PrefillParams &P, const void *k_cache, const void *v_
                    dim3(C::THREADS), C::SMEM, st, km, vm, P, plan->plan) != cudaSuccess)
       return -3;
     if (plan->n_combine > 0 &&
-        launch_pdl(prefill_combine_kernel<D, (KT != 0)>, dim3(gx, static_cast<unsigned>(plan->n_combine)), dim3(256),
-                   0, st, P, plan->combine) != cudaSuccess)
+        launch_pdl(prefill_combine_kernel<D, (KT != 0)>, dim3(gx, static_cast<unsigned>(plan->n_combine), 32),
+                   dim3(256), 0, st, P, plan->combine) != cudaSuccess)
       return -3;
     return 0;
   }
