@@ -560,17 +560,18 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
       fence_async_smem();
       mbar_arrive(&bars[kQReady]);
     } else {
+      // all of the row's loads are issued before any store: a store between them would order each load
+      // behind the previous store (the compiler cannot tell the global row from shared memory), and the
+      // row would take one memory latency per 16 bytes
       uint8_t *rowp = sQ + r * 128;
-      if (row_ok) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(P.q + ((int64_t)(q0 + pos_i) * P.num_q_heads + h) * D);
+      uint4 w[D / 8];
+      const uint4 *src =
+          reinterpret_cast<const uint4 *>(P.q + ((int64_t)(q0 + (row_ok ? pos_i : 0)) * P.num_q_heads + h) * D);
 #pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch)
-          *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::Q_PLANE + (((ch & 7) ^ (r & 7)) << 4)) = src[ch];
-      } else {
+      for (int ch = 0; ch < D / 8; ++ch) w[ch] = row_ok ? __ldg(src + ch) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch)
-          *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::Q_PLANE + (ch & 7) * 16) = make_uint4(0, 0, 0, 0);
-      }
+      for (int ch = 0; ch < D / 8; ++ch)
+        *reinterpret_cast<uint4 *>(rowp + (ch >> 3) * C::Q_PLANE + (((ch & 7) ^ (r & 7)) << 4)) = w[ch];
       fence_async_smem();
       mbar_arrive(&bars[kQReady]);
     }
