@@ -86,6 +86,14 @@ __device__ __forceinline__ void mma_16816_f16(float (&d)[4], uint32_t a0, uint32
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// An 8x8 matrix of 16-bit values held as m16n8k16 C-fragment pairs (lane (g, t): row g, columns 2t, 2t + 1),
+// transposed across the warp: lane (g, t) gets row g, columns 2t, 2t + 1 of the transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+  return d;
+}
+
 __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
@@ -230,7 +238,14 @@ __global__ void __launch_bounds__(NW * 32)
       }
     };
     load_row(grp, qlo, qsc_lo);
-    if constexpr (HI) load_row(grp + 8, qhi, qsc_hi);
+    if constexpr (HI) {
+      load_row(grp + 8, qhi, qsc_hi);
+    } else {
+      // transposed products: this lane's score columns are queries 2pr and 2pr + 1
+      const float s0 = __shfl_sync(0xffffffffu, qsc_lo, 8 * pr), s1 = __shfl_sync(0xffffffffu, qsc_lo, 8 * pr + 4);
+      qsc_lo = s0;
+      qsc_hi = s1;
+    }
   } else {
 #pragma unroll
   for (int t = 0; t < C::PLANES; ++t) {
@@ -298,142 +313,235 @@ __global__ void __launch_bounds__(NW * 32)
       __syncwarp();
     }
 
-    // -- S = Q K^T: n-tile nt holds tokens 8nt..8nt+7; lane (grp, pr) reads token 8nt+grp's dims
-    // 64t + 16pr .. +16 (two 16-byte chunks of plane t)
-    // (two accumulators per n-tile, even and odd k-steps, so that the dependent chain of products on one
-    // accumulator is half as long)
-    float sc[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      const int R = 8 * nt + grp;
-      if constexpr (KT == 0) {
-#pragma unroll
-        for (int t = 0; t < C::PLANES; ++t) {
-          const uint4 k0 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr));
-          const uint4 k1 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr + 1));
-          const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int ks = 4 * t + u;
-            mma_16816(acc[ks & 1], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
-                      kw[2 * u + 1]);
-          }
-        }
-      } else {
-        // the row's bytes [32pr, 32pr + 32): 16 f16 pairs, k-step s takes pairs 2s and 2s + 1
-        const uint4 k0 = lds128(Kt + sw_chunk(R, 2 * pr));
-        const uint4 k1 = lds128(Kt + sw_chunk(R, 2 * pr + 1));
-        const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    if constexpr (KT != 0 && !HI) {
+      // ---- one-byte caches, up to 8 query heads: the products are transposed so that the block's 16
+      // tokens fill the M side of m16n8k16 and the (at most 8) query heads its N side, which halves the
+      // products per block.  S^T = K Q^T: the A fragments are K's converted codes (lane (grp, pr): tokens
+      // grp and grp + 8, bytes [32pr, 32pr + 32) of their rows; k-step s takes dims 32pr + 4s + {0,1} and
+      // {2,3}, the dims Q's fragments use), the B fragments Q's rows.  Lane (grp, pr) then holds the scores
+      // of tokens grp, grp + 8 for queries 2pr, 2pr + 1.
+      float sc[4];
+      {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const uint4 k0 = lds128(Kt + sw_chunk(grp, 2 * pr));
+        const uint4 k1 = lds128(Kt + sw_chunk(grp, 2 * pr + 1));
+        const uint4 k2 = lds128(Kt + sw_chunk(grp + 8, 2 * pr));
+        const uint4 k3 = lds128(Kt + sw_chunk(grp + 8, 2 * pr + 1));
+        const uint32_t klo[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+        const uint32_t khi[8] = {k2.x, k2.y, k2.z, k2.w, k3.x, k3.y, k3.z, k3.w};
 #pragma unroll
         for (int s2 = 0; s2 < C::KS; ++s2) {
-          uint32_t b0, b1;
-          bytes4_to_h2<KT>(kw[s2], b0, b1);
-          mma_16816_f16(acc[s2 & 1], qlo[s2][0], HI ? qhi[s2][0] : 0u, qlo[s2][1], HI ? qhi[s2][1] : 0u, b0, b1);
+          uint32_t a0, a1, a2, a3;
+          bytes4_to_h2<KT>(klo[s2], a0, a2);
+          bytes4_to_h2<KT>(khi[s2], a1, a3);
+          mma_16816_f16(acc[s2 & 1], a0, a1, a2, a3, qlo[s2][0], qlo[s2][1]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sc[e] = acc[0][e] + acc[1][e];
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc[nt][e] = acc[0][e] + acc[1][e];
-    }
-
-    // -- online softmax: lane (grp, pr) holds row grp's tokens 8nt + 2pr + {0,1} (sc[nt][0..1]) and row
-    // grp+8's (sc[nt][2..3]); a row's max comes from the 4 lanes of its quad
-    float x[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+      // -- online softmax per query column: a column's 16 scores sit with the 8 lanes of one pr
+      float x[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int tok = 8 * nt + 2 * pr + (e & 1);
-        x[nt][e] = tok < nvalid ? sc[nt][e] * (e < 2 ? qsc_lo : qsc_hi) : -INFINITY;
+        const int tok = grp + ((e & 2) ? 8 : 0);
+        x[e] = tok < nvalid ? sc[e] * ((e & 1) ? qsc_hi : qsc_lo) : -INFINITY;
       }
-    float bm_lo = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-    bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 1));
-    bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 2));
-    // the reference moves only when the block's max exceeds it by more than 2^8 (or on the first block);
-    // O and l are rescaled with it, so O / l is exact whichever reference is used
-    if (bm_lo > m_lo + kRescale) {
-      const float alpha = m_lo == -INFINITY ? 0.f : exp2f(m_lo - bm_lo);
-      m_lo = bm_lo;
-      l_lo *= alpha;
+      float bm0 = fmaxf(x[0], x[2]), bm1 = fmaxf(x[1], x[3]);
 #pragma unroll
-      for (int j = 0; j < C::NT; ++j) {
-        o[j][0] *= alpha;
-        o[j][1] *= alpha;
+      for (int off = 4; off <= 16; off <<= 1) {
+        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
       }
-    }
-    float p[2][4];
+      // the reference of a column moves only when the block's max exceeds it by more than 2^8 (or on the
+      // first block); O and l are rescaled with it, so O / l is exact whichever reference is used
+      if (bm0 > m_lo + kRescale) {
+        const float alpha = m_lo == -INFINITY ? 0.f : exp2f(m_lo - bm0);
+        m_lo = bm0;
+        l_lo *= alpha;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      p[nt][0] = exp2f(x[nt][0] - m_lo);
-      p[nt][1] = exp2f(x[nt][1] - m_lo);
-      l_lo += p[nt][0] + p[nt][1];
-    }
-    if constexpr (HI) {
-      float bm_hi = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-      bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 1));
-      bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 2));
-      if (bm_hi > m_hi + kRescale) {
-        const float alpha = m_hi == -INFINITY ? 0.f : exp2f(m_hi - bm_hi);
-        m_hi = bm_hi;
+        for (int j = 0; j < C::NT / 2; ++j) {
+          o[j][0] *= alpha;
+          o[j][2] *= alpha;
+        }
+      }
+      if (bm1 > m_hi + kRescale) {
+        const float alpha = m_hi == -INFINITY ? 0.f : exp2f(m_hi - bm1);
+        m_hi = bm1;
         l_hi *= alpha;
 #pragma unroll
-        for (int j = 0; j < C::NT; ++j) {
-          o[j][2] *= alpha;
+        for (int j = 0; j < C::NT / 2; ++j) {
+          o[j][1] *= alpha;
           o[j][3] *= alpha;
         }
       }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        p[nt][2] = exp2f(x[nt][2] - m_hi);
-        p[nt][3] = exp2f(x[nt][3] - m_hi);
-        l_hi += p[nt][2] + p[nt][3];
-      }
-    }
-    // P as the A operand of the PV product (K = the block's 16 tokens): its fragments are S's
-    if constexpr (KT == 0) {
-      const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
-      const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
-      const uint32_t pa1 = HI ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
-      const uint32_t pa3 = HI ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
+      const float p0 = exp2f(x[0] - m_lo), p1 = exp2f(x[1] - m_hi), p2 = exp2f(x[2] - m_lo),
+                  p3 = exp2f(x[3] - m_hi);
+      l_lo += p0 + p2;
+      l_hi += p1 + p3;
+      // P^T as the B operand of O^T += V^T P^T: the C layout of tokens 0-7 (and 8-15) x queries, transposed
+      // across the warp by movmatrix, is the B fragment (tokens 2pr, 2pr + 1 (+ 8) of query grp)
+      const uint32_t pb0 = movmatrix_trans(pack_f16x2(p0, p1));
+      const uint32_t pb1 = movmatrix_trans(pack_f16x2(p2, p3));
       __syncwarp();
-
-      // -- O += P V: ldmatrix.trans gives the B fragments of two 8-dim n-tiles per call; lane l addresses
-      // row (l/8 % 2)*8 + l%8 (token) of 8-dim chunk 2jj + l/16
-      const int vr = ((lane >> 3) & 1) * 8 + (lane & 7);
-#pragma unroll
-      for (int jj = 0; jj < C::NT / 2; ++jj) {
-        uint32_t v0, v1, v2, v3;
-        ldsm_x4_trans(Vt + sw_chunk(vr, 2 * jj + (lane >> 4)), v0, v1, v2, v3);
-        mma_16816(o[2 * jj], pa0, pa1, pa2, pa3, v0, v1);
-        mma_16816(o[2 * jj + 1], pa0, pa1, pa2, pa3, v2, v3);
-      }
-    } else {
-      // P in f16 (p <= 2^8)
-      const uint32_t pa0 = pack_f16x2(p[0][0], p[0][1]);
-      const uint32_t pa2 = pack_f16x2(p[1][0], p[1][1]);
-      const uint32_t pa1 = HI ? pack_f16x2(p[0][2], p[0][3]) : 0u;
-      const uint32_t pa3 = HI ? pack_f16x2(p[1][2], p[1][3]) : 0u;
-      __syncwarp();
-      // -- O += P V: lane (grp, pr) converts V row (8h + grp)'s bytes [32pr, 32pr + 32) into 16 pairs of
-      // adjacent dims; pair j, transposed across the warp, is the B fragment of n-tile j (dims
-      // {32p' + 2j, +1}) for the 8 tokens of half h
-      // lane (grp, pr) reads dims [16grp, 16grp + 16) of token rows 2pr, 2pr + 1 (half h = 0) and 8 + 2pr,
-      // 9 + 2pr (h = 1); a byte permute pairs the two rows' codes of one dim, which is the B fragment of
-      // n-tile e (column grp = dim 16grp + e) for tokens (2pr, 2pr + 1) + 8h
-      uint32_t vb[2][16];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4 r0 = lds128(Vt + sw_chunk(8 * h + 2 * pr, grp));
-        const uint4 r1 = lds128(Vt + sw_chunk(8 * h + 2 * pr + 1, grp));
-        const uint32_t a[4] = {r0.x, r0.y, r0.z, r0.w}, c[4] = {r1.x, r1.y, r1.z, r1.w};
+      // -- O^T += V^T P^T: m-tile j holds dims 16grp + 2j (rows grp) and 16grp + 2j + 1 (rows grp + 8).  Lane
+      // (grp, pr) reads dims [16grp, 16grp + 16) of token rows 2pr, 2pr + 1 and 2pr + 8, 2pr + 9; a byte
+      // permute pairs two rows' codes of one dim, which is an A fragment register
+      {
+        const uint4 r0 = lds128(Vt + sw_chunk(2 * pr, grp));
+        const uint4 r1 = lds128(Vt + sw_chunk(2 * pr + 1, grp));
+        const uint4 r2 = lds128(Vt + sw_chunk(2 * pr + 8, grp));
+        const uint4 r3 = lds128(Vt + sw_chunk(2 * pr + 9, grp));
+        const uint32_t va[4] = {r0.x, r0.y, r0.z, r0.w}, vc[4] = {r1.x, r1.y, r1.z, r1.w};
+        const uint32_t vd[4] = {r2.x, r2.y, r2.z, r2.w}, vf[4] = {r3.x, r3.y, r3.z, r3.w};
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          bytes4_to_h2<KT>(__byte_perm(a[q4], c[q4], 0x5140), vb[h][4 * q4], vb[h][4 * q4 + 1]);
-          bytes4_to_h2<KT>(__byte_perm(a[q4], c[q4], 0x7362), vb[h][4 * q4 + 2], vb[h][4 * q4 + 3]);
+          uint32_t a0, a1, a2, a3;
+          bytes4_to_h2<KT>(__byte_perm(va[q4], vc[q4], 0x5140), a0, a1);   // dims 4q4, 4q4 + 1
+          bytes4_to_h2<KT>(__byte_perm(vd[q4], vf[q4], 0x5140), a2, a3);
+          mma_16816_f16(o[2 * q4], a0, a1, a2, a3, pb0, pb1);
+          bytes4_to_h2<KT>(__byte_perm(va[q4], vc[q4], 0x7362), a0, a1);   // dims 4q4 + 2, 4q4 + 3
+          bytes4_to_h2<KT>(__byte_perm(vd[q4], vf[q4], 0x7362), a2, a3);
+          mma_16816_f16(o[2 * q4 + 1], a0, a1, a2, a3, pb0, pb1);
         }
       }
-#pragma unroll
-      for (int e = 0; e < C::NT; ++e) mma_16816_f16(o[e], pa0, pa1, pa2, pa3, vb[0][e], vb[1][e]);
+    } else {
+      // -- S = Q K^T: n-tile nt holds tokens 8nt..8nt+7; lane (grp, pr) reads token 8nt+grp's dims
+      // 64t + 16pr .. +16 (two 16-byte chunks of plane t)
+      // (two accumulators per n-tile, even and odd k-steps, so that the dependent chain of products on one
+      // accumulator is half as long)
+      float sc[2][4];
+  #pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const int R = 8 * nt + grp;
+        if constexpr (KT == 0) {
+  #pragma unroll
+          for (int t = 0; t < C::PLANES; ++t) {
+            const uint4 k0 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr));
+            const uint4 k1 = lds128(Kt + sw_chunk(R, 8 * t + 2 * pr + 1));
+            const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+  #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int ks = 4 * t + u;
+              mma_16816(acc[ks & 1], qlo[ks][0], HI ? qhi[ks][0] : 0u, qlo[ks][1], HI ? qhi[ks][1] : 0u, kw[2 * u],
+                        kw[2 * u + 1]);
+            }
+          }
+        } else {
+          // the row's bytes [32pr, 32pr + 32): 16 f16 pairs, k-step s takes pairs 2s and 2s + 1
+          const uint4 k0 = lds128(Kt + sw_chunk(R, 2 * pr));
+          const uint4 k1 = lds128(Kt + sw_chunk(R, 2 * pr + 1));
+          const uint32_t kw[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+  #pragma unroll
+          for (int s2 = 0; s2 < C::KS; ++s2) {
+            uint32_t b0, b1;
+            bytes4_to_h2<KT>(kw[s2], b0, b1);
+            mma_16816_f16(acc[s2 & 1], qlo[s2][0], HI ? qhi[s2][0] : 0u, qlo[s2][1], HI ? qhi[s2][1] : 0u, b0, b1);
+          }
+        }
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) sc[nt][e] = acc[0][e] + acc[1][e];
+      }
+
+      // -- online softmax: lane (grp, pr) holds row grp's tokens 8nt + 2pr + {0,1} (sc[nt][0..1]) and row
+      // grp+8's (sc[nt][2..3]); a row's max comes from the 4 lanes of its quad
+      float x[2][4];
+  #pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int tok = 8 * nt + 2 * pr + (e & 1);
+          x[nt][e] = tok < nvalid ? sc[nt][e] * (e < 2 ? qsc_lo : qsc_hi) : -INFINITY;
+        }
+      float bm_lo = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+      bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 1));
+      bm_lo = fmaxf(bm_lo, __shfl_xor_sync(0xffffffffu, bm_lo, 2));
+      // the reference moves only when the block's max exceeds it by more than 2^8 (or on the first block);
+      // O and l are rescaled with it, so O / l is exact whichever reference is used
+      if (bm_lo > m_lo + kRescale) {
+        const float alpha = m_lo == -INFINITY ? 0.f : exp2f(m_lo - bm_lo);
+        m_lo = bm_lo;
+        l_lo *= alpha;
+  #pragma unroll
+        for (int j = 0; j < C::NT; ++j) {
+          o[j][0] *= alpha;
+          o[j][1] *= alpha;
+        }
+      }
+      float p[2][4];
+  #pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        p[nt][0] = exp2f(x[nt][0] - m_lo);
+        p[nt][1] = exp2f(x[nt][1] - m_lo);
+        l_lo += p[nt][0] + p[nt][1];
+      }
+      if constexpr (HI) {
+        float bm_hi = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+        bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 1));
+        bm_hi = fmaxf(bm_hi, __shfl_xor_sync(0xffffffffu, bm_hi, 2));
+        if (bm_hi > m_hi + kRescale) {
+          const float alpha = m_hi == -INFINITY ? 0.f : exp2f(m_hi - bm_hi);
+          m_hi = bm_hi;
+          l_hi *= alpha;
+  #pragma unroll
+          for (int j = 0; j < C::NT; ++j) {
+            o[j][2] *= alpha;
+            o[j][3] *= alpha;
+          }
+        }
+  #pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          p[nt][2] = exp2f(x[nt][2] - m_hi);
+          p[nt][3] = exp2f(x[nt][3] - m_hi);
+          l_hi += p[nt][2] + p[nt][3];
+        }
+      }
+      // P as the A operand of the PV product (K = the block's 16 tokens): its fragments are S's
+      if constexpr (KT == 0) {
+        const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+        const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+        const uint32_t pa1 = HI ? pack_bf16x2(p[0][2], p[0][3]) : 0u;
+        const uint32_t pa3 = HI ? pack_bf16x2(p[1][2], p[1][3]) : 0u;
+        __syncwarp();
+
+        // -- O += P V: ldmatrix.trans gives the B fragments of two 8-dim n-tiles per call; lane l addresses
+        // row (l/8 % 2)*8 + l%8 (token) of 8-dim chunk 2jj + l/16
+        const int vr = ((lane >> 3) & 1) * 8 + (lane & 7);
+  #pragma unroll
+        for (int jj = 0; jj < C::NT / 2; ++jj) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_trans(Vt + sw_chunk(vr, 2 * jj + (lane >> 4)), v0, v1, v2, v3);
+          mma_16816(o[2 * jj], pa0, pa1, pa2, pa3, v0, v1);
+          mma_16816(o[2 * jj + 1], pa0, pa1, pa2, pa3, v2, v3);
+        }
+      } else {
+        // P in f16 (p <= 2^8)
+        const uint32_t pa0 = pack_f16x2(p[0][0], p[0][1]);
+        const uint32_t pa2 = pack_f16x2(p[1][0], p[1][1]);
+        const uint32_t pa1 = HI ? pack_f16x2(p[0][2], p[0][3]) : 0u;
+        const uint32_t pa3 = HI ? pack_f16x2(p[1][2], p[1][3]) : 0u;
+        __syncwarp();
+        // -- O += P V: lane (grp, pr) converts V row (8h + grp)'s bytes [32pr, 32pr + 32) into 16 pairs of
+        // adjacent dims; pair j, transposed across the warp, is the B fragment of n-tile j (dims
+        // {32p' + 2j, +1}) for the 8 tokens of half h
+        // lane (grp, pr) reads dims [16grp, 16grp + 16) of token rows 2pr, 2pr + 1 (half h = 0) and 8 + 2pr,
+        // 9 + 2pr (h = 1); a byte permute pairs the two rows' codes of one dim, which is the B fragment of
+        // n-tile e (column grp = dim 16grp + e) for tokens (2pr, 2pr + 1) + 8h
+        uint32_t vb[2][16];
+  #pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 r0 = lds128(Vt + sw_chunk(8 * h + 2 * pr, grp));
+          const uint4 r1 = lds128(Vt + sw_chunk(8 * h + 2 * pr + 1, grp));
+          const uint32_t a[4] = {r0.x, r0.y, r0.z, r0.w}, c[4] = {r1.x, r1.y, r1.z, r1.w};
+  #pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            bytes4_to_h2<KT>(__byte_perm(a[q4], c[q4], 0x5140), vb[h][4 * q4], vb[h][4 * q4 + 1]);
+            bytes4_to_h2<KT>(__byte_perm(a[q4], c[q4], 0x7362), vb[h][4 * q4 + 2], vb[h][4 * q4 + 3]);
+          }
+        }
+  #pragma unroll
+        for (int e = 0; e < C::NT; ++e) mma_16816_f16(o[e], pa0, pa1, pa2, pa3, vb[0][e], vb[1][e]);
+      }
     }
     __syncwarp();
     if (issued < nwb) issue(issued++);
@@ -447,16 +555,41 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
     for (int j = 0; j < C::NT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   }
-  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
-  l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
-  if constexpr (HI) {
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
-    l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+  constexpr bool kTr = KT != 0 && !HI;               // transposed products (one-byte, up to 8 heads)
+  if constexpr (kTr) {
+    // a column's sum is spread over the 8 lanes of one pr
+#pragma unroll
+    for (int off = 4; off <= 16; off <<= 1) {
+      l_lo += __shfl_xor_sync(0xffffffffu, l_lo, off);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, off);
+    }
+  } else {
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
+    l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 2);
+    if constexpr (HI) {
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 1);
+      l_hi += __shfl_xor_sync(0xffffffffu, l_hi, 2);
+    }
   }
 
   // ---- merge the warps: each writes its rows' (O, m, l) over its consumed tiles, then the CTA combines
   __syncwarp();
   float *mrg = reinterpret_cast<float *>(wbase);
+  if constexpr (kTr) {
+    // m-tile j of this lane: queries 2pr, 2pr + 1 at dims 16grp + 2j (o[j][0..1]) and + 1 (o[j][2..3])
+#pragma unroll
+    for (int j = 0; j < C::NT / 2; ++j) {
+      const int d0 = 16 * grp + 2 * j;
+      *reinterpret_cast<float2 *>(mrg + (2 * pr) * D + d0) = make_float2(o[j][0], o[j][2]);
+      *reinterpret_cast<float2 *>(mrg + (2 * pr + 1) * D + d0) = make_float2(o[j][1], o[j][3]);
+    }
+    if (grp == 0) {
+      mrg[C::ML + 2 * (2 * pr)] = m_lo;
+      mrg[C::ML + 2 * (2 * pr) + 1] = l_lo;
+      mrg[C::ML + 2 * (2 * pr + 1)] = m_hi;
+      mrg[C::ML + 2 * (2 * pr + 1) + 1] = l_hi;
+    }
+  } else {
 #pragma unroll
   for (int j = 0; j < C::NT; ++j) {
     if constexpr (KT == 0) {
@@ -481,6 +614,7 @@ __global__ void __launch_bounds__(NW * 32)
       mrg[C::ML + 2 * (grp + 8)] = m_hi;
       mrg[C::ML + 2 * (grp + 8) + 1] = l_hi;
     }
+  }
   }
   __syncthreads();
 
