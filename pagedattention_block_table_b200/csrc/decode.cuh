@@ -15,8 +15,9 @@
 // sums are combined with warp shuffles.  Warps of a CTA merge their (max, sum, output) in
 // shared memory; a sequence covering several splits writes fp32 partials that
 // `lse_reduce_kernel` combines:  out = sum_p 2^(m_p-M) o_p / sum_p 2^(m_p-M) l_p.
-// This CUDA-core kernel serves one-byte caches and groups of fewer than 4 query heads; bf16 caches
-// with larger groups use the tensor-core kernel of decode_mma.cuh (same work units, same partials).
+// This CUDA-core kernel serves bf16 groups of fewer than 4 query heads, one query head per KV head over a
+// one-byte cache, and one-byte caches at head_dim 64; larger groups use the tensor-core kernel of
+// decode_mma.cuh (same work units, same partials).
 #pragma once
 #include "pa_common.cuh"
 

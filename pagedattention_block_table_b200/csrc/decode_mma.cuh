@@ -28,7 +28,11 @@
 // the same dims).  V needs pairs along tokens: a lane reads 16 dims [16g, 16g + 16) of two token rows
 // and a byte permute pairs the two rows' codes of each dim before the conversion, which gives the B
 // fragment of n-tile e (column g = dim 16g + e); n-tile e of the output then holds dims 32p + e and
-// 32p + 16 + e.
+// 32p + 16 + e.  With up to 8 query heads (the rows 8-15 of the products above would stay empty) the
+// one-byte products are transposed instead: S^T = K Q^T puts the block's 16 tokens on M and the heads on
+// N, O^T += V^T P^T the dims on M, so each block takes 8 + 8 products instead of 16 + 16; the scores'
+// C fragments are turned into P^T's B fragments by movmatrix, and a head's softmax column spans the 8
+// lanes of one pair index.
 #pragma once
 #include "decode.cuh"
 #include "prefill.cuh"   // tensor-map encoding, 2-D TMA load

@@ -79,10 +79,11 @@ def test_decode_fp8_with_gqa(O, cuda_lib):
     assert_close(to_f64(_gpu_decode(batch).out_dec), oracle_step(batch, O)["decode"], what="fp8 gqa4")
 
 
-# one-byte caches with groups of 4 or more query heads take the tensor-core kernel at head_dim 128 (f16
-# products on codes converted in registers): groups of 4, 8 (two CTAs' worth of rows), 16, a group split
-# over two CTAs, 32-token blocks, lengths at block edges, several splits
+# one-byte caches with groups of 2 or more query heads take the tensor-core kernel at head_dim 128 (f16
+# products on codes converted in registers; up to 8 heads the products are transposed, tokens on M): groups
+# of 2, 4, 8, 16, a group split over two CTAs, 32-token blocks, lengths at block edges, several splits
 ONE_BYTE_MMA = {
+    "g2": dict(num_seqs=4, num_q_heads=16, num_kv_heads=8, hist=("fixed", [1, 16, 17, 1200])),
     "g4": dict(num_seqs=5, num_q_heads=32, num_kv_heads=8, hist=("fixed", [0, 15, 16, 700, 1500])),
     "g8": dict(num_seqs=3, num_q_heads=64, num_kv_heads=8, hist=("uniform", 30, 900)),
     "g16": dict(num_seqs=3, num_q_heads=32, num_kv_heads=2, hist=("uniform", 1, 900)),
