@@ -30,7 +30,9 @@
 #define PA_DEC_MMA_MIN_GROUP 4
 #endif
 #ifndef PA_DEC_MMA_MIN_GROUP_Q8
-#define PA_DEC_MMA_MIN_GROUP_Q8 2   // one-byte caches: G = 2 ran at 5.67 TB/s on the tensor cores, 3.88 on CUDA cores
+// one-byte caches: every group at head_dim 128 (transposed products): G = 2 ran at 5.76 TB/s on the tensor
+// cores against 3.88 on the CUDA cores, the MHA FP8 batch (G = 1) at 7.29 against 6.42-6.51
+#define PA_DEC_MMA_MIN_GROUP_Q8 1
 #endif
 #ifndef PA_DEC_MMA_STAGES
 #define PA_DEC_MMA_STAGES 2

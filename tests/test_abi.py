@@ -59,15 +59,16 @@ def test_status_strings(L):
 
 def test_decode_kernel_choice(L):
     """Groups of 4 or more query heads per KV head decode on the tensor cores over bf16 caches (up to 16 heads
-    per CTA, or a multiple of 16), groups of 2 or more over one-byte caches at head_dim 128; the rest on the
-    CUDA cores."""
+    per CTA, or a multiple of 16), every group over one-byte caches at head_dim 128; the rest on the CUDA
+    cores."""
     f = L.pa_paged_attention_uses_tensor_cores
     f.argtypes = [ctypes.c_int] * 4
     assert f(32, 8, 128, 0) == 1 and f(64, 8, 128, 0) == 1 and f(32, 2, 128, 0) == 1 and f(32, 1, 128, 0) == 1
     assert f(32, 8, 64, 0) == 1
     assert f(32, 8, 128, 1) == 1 and f(32, 8, 128, 2) == 1   # FP8 / INT8 caches at head_dim 128
-    assert f(16, 8, 128, 1) == 1 and f(16, 8, 128, 2) == 1   # ... from two query heads per KV head
-    assert f(32, 8, 64, 1) == 0 and f(64, 64, 128, 1) == 0   # ... not at 64, nor for one query per KV head
+    assert f(16, 8, 128, 1) == 1 and f(16, 8, 128, 2) == 1   # ... two query heads per KV head
+    assert f(64, 64, 128, 1) == 1 and f(64, 64, 128, 2) == 1 # ... one query per KV head too
+    assert f(32, 8, 64, 1) == 0                              # ... not at head_dim 64
     assert f(8, 8, 128, 0) == 0 and f(4, 2, 128, 0) == 0 and f(6, 2, 128, 0) == 0
     assert f(48, 2, 128, 0) == 0                             # a group of 24: neither <= 16 nor a multiple of 16
     assert f(32, 3, 128, 0) == -1 and f(0, 8, 128, 0) == -1 and f(32, 8, 96, 0) == -1 and f(32, 8, 128, 5) == -1

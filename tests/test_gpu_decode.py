@@ -79,10 +79,11 @@ def test_decode_fp8_with_gqa(O, cuda_lib):
     assert_close(to_f64(_gpu_decode(batch).out_dec), oracle_step(batch, O)["decode"], what="fp8 gqa4")
 
 
-# one-byte caches with groups of 2 or more query heads take the tensor-core kernel at head_dim 128 (f16
-# products on codes converted in registers; up to 8 heads the products are transposed, tokens on M): groups
-# of 2, 4, 8, 16, a group split over two CTAs, 32-token blocks, lengths at block edges, several splits
+# one-byte caches take the tensor-core kernel at head_dim 128 (f16 products on codes converted in
+# registers; up to 8 heads the products are transposed, tokens on M): groups of 1, 2, 4, 8, 16, a group
+# split over two CTAs, 32-token blocks, lengths at block edges, several splits
 ONE_BYTE_MMA = {
+    "g1": dict(num_seqs=4, num_q_heads=8, num_kv_heads=8, hist=("fixed", [2, 16, 500, 2100])),
     "g2": dict(num_seqs=4, num_q_heads=16, num_kv_heads=8, hist=("fixed", [1, 16, 17, 1200])),
     "g4": dict(num_seqs=5, num_q_heads=32, num_kv_heads=8, hist=("fixed", [0, 15, 16, 700, 1500])),
     "g8": dict(num_seqs=3, num_q_heads=64, num_kv_heads=8, hist=("uniform", 30, 900)),
@@ -195,6 +196,15 @@ def test_bad_block_id_is_flagged_and_stays_in_pool(cuda_lib, hq):
                          batch.max_blocks_per_seq * 16 + 5)
     assert B.pa_get_device_error() == B.PA_EDEVICE_OOB
     assert B.pa_get_device_error() == B.PA_OK
+
+
+def test_one_byte_decode_at_head_dim_64_on_cuda_cores(O, cuda_lib):
+    """One-byte caches at head_dim 64 stay on the CUDA-core kernel (FP8 here; INT8 below)."""
+    from pagedattention_block_table_b200 import binding as B
+    assert B.pa_paged_attention_uses_tensor_cores(4, 2, 64, B.PA_KV_FP8_E4M3) == 0
+    ov = dict(num_seqs=4, num_q_heads=4, num_kv_heads=2, head_dim=64, hist=("uniform", 1, 700), kv_dtype="fp8")
+    batch = make_batch("mha_fp8_decode", seed=48, overrides=ov)
+    assert_close(to_f64(_gpu_decode(batch, 256).out_dec), oracle_step(batch, O)["decode"], what="fp8 d64")
 
 
 @pytest.mark.parametrize("d,hq,hkv", [(128, 8, 8), (128, 16, 4), (64, 4, 2)])
