@@ -129,10 +129,10 @@ int pa_paged_attention_auto_split(int num_seqs, int num_q_heads, int num_kv_head
 
 /*
  * pa_paged_attention_uses_tensor_cores -- 1 when pa_paged_attention runs its products on the tensor
- * cores for this shape (at least 4 query heads per KV head, a group of at most 16 heads or a multiple of
- * 16; a bf16 cache, or a one-byte cache at head_dim 128), 0 when it uses the CUDA-core kernel (smaller
- * groups, one-byte caches at head_dim 64), -1 for an invalid shape.  Both kernels compute the same
- * function; this only names the one that runs.
+ * cores for this shape (a group of at most 16 heads or a multiple of 16, and either a bf16 cache with at
+ * least 4 query heads per KV head or a one-byte cache at head_dim 128), 0 when it uses the CUDA-core
+ * kernel (smaller bf16 groups, one-byte caches at head_dim 64), -1 for an invalid shape.  Both kernels
+ * compute the same function; this only names the one that runs.
  */
 int pa_paged_attention_uses_tensor_cores(int num_q_heads, int num_kv_heads, int head_dim, int kv_dtype);
 

@@ -89,11 +89,12 @@ int queries_per_cta(int group) {
   return 1;
 }
 
-// Groups of at least PA_DEC_MMA_MIN_GROUP query heads per KV head over a bf16 cache decode on the tensor
-// cores (decode_mma.cuh): one CTA takes up to 16 heads of a group.  Smaller groups and one-byte caches
-// use the CUDA-core kernel.  Measured on B200 (pa_paged_attention GB/s, CUDA graphs of calls): the
-// Llama-3-8B batch (G = 4) 6,030-6,090 on the CUDA cores, 6,370 on the tensor cores; the 32-sequence
-// batch with G = 8 (64 / 8 heads) 3,210 and 5,280.
+// Groups of at least PA_DEC_MMA_MIN_GROUP query heads per KV head over a bf16 cache, and groups of at
+// least PA_DEC_MMA_MIN_GROUP_Q8 over a one-byte cache at head_dim 128, decode on the tensor cores
+// (decode_mma.cuh): one CTA takes up to 16 heads of a group.  The rest use the CUDA-core kernel.
+// Measured on B200 (pa_paged_attention GB/s, CUDA graphs of calls): the Llama-3-8B batch (G = 4)
+// 6,030-6,090 on the CUDA cores, 6,370 on the tensor cores; the 32-sequence batch with G = 8 (64 / 8
+// heads) 3,210 and 5,280.
 bool decode_uses_mma(int kv_dtype, int group, int head_dim) {
   if (!(group <= 16 || group % 16 == 0)) return false;
   if (kv_dtype == PA_KV_BF16) return group >= PA_DEC_MMA_MIN_GROUP;
