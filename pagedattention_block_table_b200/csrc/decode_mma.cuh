@@ -136,6 +136,17 @@ __global__ void __launch_bounds__(NW * 32)
   griddep_wait();
   griddep_launch();
 
+  // ---- this warp's first block-table entries, read beside the context length instead of after it (the
+  // window's units do not depend on the length; entries past the context are not used or checked)
+  const int32_t *trow = P.block_tables + (int64_t)b * P.max_blocks_per_seq;
+  const int upb = P.block_size / kBlock;   // 16-token units per block: 1 or 2
+  const int blk0 = split * P.split_tokens / kBlock;
+  int e0 = 0;
+  {
+    const int u = blk0 + warp + NW * lane;
+    if (u / upb < P.max_blocks_per_seq) e0 = __ldg(trow + u / upb);
+  }
+
   // ---- context length, validated: never read past the table row or the launch bound
   int L = P.context_lens[b];
   {
@@ -151,7 +162,6 @@ __global__ void __launch_bounds__(NW * 32)
   const int t0 = split * P.split_tokens;
   const int t1 = min(L, t0 + P.split_tokens);
   const int nblk = t1 > t0 ? (t1 - t0 + kBlock - 1) / kBlock : 0;
-  const int blk0 = t0 / kBlock;
 
   uint8_t *wbase = smem + warp * C::WARP_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + C::DATA);
@@ -162,15 +172,14 @@ __global__ void __launch_bounds__(NW * 32)
   }
   __syncwarp();
 
-  // ---- block-table window: lane k holds the 16-row tile index of this warp's unit win*32 + k
-  const int32_t *trow = P.block_tables + (int64_t)b * P.max_blocks_per_seq;
-  const int upb = P.block_size / kBlock;   // 16-token units per block: 1 or 2
+  // ---- block-table window: lane k holds the 16-row tile index of this warp's unit win*32 + k (window 0
+  // from the entries read above)
   auto load_window = [&](int win) -> int {
     const int i = win * 32 + lane;
     int tile = 0;
     if (i < nwb) {
       const int u = blk0 + warp + NW * i;
-      int e = __ldg(trow + u / upb);
+      int e = win == 0 ? e0 : __ldg(trow + u / upb);
       if (e < 0 || e >= P.num_blocks) {
         flag_error(kErrBlockId);
         e = 0;
