@@ -485,6 +485,21 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
   // ends before the CTA's last tile has only full tiles)
   const int last_k16 = tl1 == all_tiles ? (kv_len - (all_tiles - 1) * C::BN + 15) / 16 : C::BN / 16;
 
+  // the producer lanes' block-table entries of the first two key tiles, read before the CTA's set-up so
+  // that their latency overlaps it (the first K tile's copy waits on them; checked where they are used).
+  // bf16 caches only: on the mixed step it moved bf16 from 902 to 913 TFLOP/s and FP8 from 894 to 880.
+  int pre_e0 = 0, pre_e1 = 0;
+  const bool pre_read = KT == 0;
+  if (pre_read && warp == 9) {
+    constexpr int UPT = C::BN / kBlock, NPL = KT != 0 ? 1 : C::DH;
+    const int w_lane = lane / (UPT * NPL), bb = (lane / NPL) % UPT;
+    const int ush = P.block_size == 32 ? 1 : 0;
+    const int32_t *trow = P.block_tables + (int64_t)c * P.max_blocks_per_seq;
+    const int u0 = tl0 * UPT + bb, u1 = u0 + UPT;
+    if (w_lane < 2 && u0 * kBlock < kv_len) pre_e0 = __ldg(trow + (u0 >> ush));
+    if (w_lane < 2 && 1 < ntiles && u1 * kBlock < kv_len) pre_e1 = __ldg(trow + (u1 >> ush));
+  }
+
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + C::NBAR);
   if (warp == 8) {
@@ -842,7 +857,7 @@ __global__ void __launch_bounds__(PrefillCfg<D, KT>::THREADS, 1)
         const int u = (tl0 + j) * UPT + bb;
         int e = 0;
         if (w_lane < 2 && j < ntiles && u * kBlock < kv_len) {
-          e = __ldg(trow + (u >> ush));
+          e = (pre_read && j < 2) ? (j == 0 ? pre_e0 : pre_e1) : __ldg(trow + (u >> ush));
           if (e < 0 || e >= P.num_blocks) {
             flag_error(kErrBlockId);
             e = 0;
